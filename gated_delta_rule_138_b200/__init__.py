@@ -1,0 +1,13 @@
+"""B200-native KDA (Kimi Delta Attention) forward pass and decode step.
+
+The compute path is the C-ABI library ``libkda.so`` built from ``csrc/``
+(hand-written sm_100a CUDA kernels); ``kda.py`` is a thin ctypes binding with
+the same entry-point names.  PyTorch is used only for device memory and
+streams.  Importing this package does not load the CUDA library; the first
+call does, and it raises if the library is missing.
+"""
+from .kda import (KdaError, kda_forward, kda_decode_step, kda_status_string,  # noqa: F401
+                  kda_forward_workspace_bytes, library_path, load_library)
+
+__all__ = ["KdaError", "kda_forward", "kda_decode_step", "kda_status_string",
+           "kda_forward_workspace_bytes", "library_path", "load_library"]

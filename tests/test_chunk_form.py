@@ -1,0 +1,143 @@
+"""The chunk-parallel algebra the CUDA kernels use, restated in fp64 numpy and
+checked against the token-by-token oracle.
+
+"FlashKDA parallelizes token processing inside each chunk ... and uses
+prefix-scan operations ... to reconstruct correct sequential states" (the
+worldcybernews article "Kimi K3 Open Model Surpasses Closed GPT and Anthropic
+Systems on Independent Benchmarks", paragraph 3).  The page gives no algebra;
+this file writes out the one the kernels implement, so that the algebra is
+known to be exact (to fp64 rounding) before any kernel runs:
+
+Per chunk of C tokens (positions r = 0..C-1) with start state S0, a = clamp(alpha):
+  decay from token j (exclusive) to token r (inclusive), per key channel:
+      D(r, j) = prod_{s=j+1..r} a_s
+  A[r, j] = beta_r sum_c k_rc k_jc D(r, j)_c        (j < r, else 0)
+  P[r, j] =        sum_c q_rc k_jc D(r, j)_c        (j <= r, else 0)
+  T  = (I + A)^-1
+  K~ = k * gamma, Q~ = q * gamma, gamma_r = prod_{s<=r} a_s
+  K^ = k * eta,   eta_j = prod_{s>j} a_s
+  W  = T diag(beta) K~,   U~ = T diag(beta) V
+  U  = U~ - W S0
+  O  = Q~ S0 + P U  =  (Q~ - P W) S0 + P U~
+  S_C = Diag(gamma_{C-1}) S0 + K^^T U
+
+D(r, j) is never formed as a ratio of long products (those leave the fp32
+range: a >= e^-5 over 64 tokens reaches e^-320).  It is split at 16-token
+sub-chunk boundaries, where a product stays >= e^-80 > the fp32 minimum:
+  phi_r = prod_{s=start(I)..r} a_s,   psi_j = prod_{s=j+1..end(J)} a_s,
+  pi_I  = prod over sub-chunk I,     Delta_IJ = prod_{J<M<I} pi_M
+  I > J:  D(r, j) = (phi_r Delta_IJ) * psi_j
+  I = J:  D(r, j) = (phi_r / pi_I) * psi_j      (j <= r)
+so A and P are products of a left operand x_r phi_r Delta'_IJ and one right
+operand k_j psi_j, with no factor above e^80.
+"""
+import numpy as np
+import pytest
+
+import oracle
+
+SUB = 16
+
+
+def _clamp(alpha):
+    lo = np.float64(np.float32(np.exp(-5.0)))
+    return np.clip(alpha.astype(np.float32).astype(np.float64), lo, 1.0)
+
+
+def chunk_forward_one(q, k, v, alpha, beta, S0, C):
+    """One (sequence, head): q, k, alpha [T, dk]; v [T, dv]; beta [T]; S0 [dk, dv]."""
+    T, dk = q.shape
+    dv = v.shape[1]
+    a_all = _clamp(alpha)
+    S = S0.astype(np.float64).copy()
+    out = np.zeros((T, dv))
+    for t0 in range(0, T, C):
+        L = min(C, T - t0)
+        # masked tail rows: k = q = v = 0, beta = 0, a = 1
+        Q = np.zeros((C, dk)); K = np.zeros((C, dk)); V = np.zeros((C, dv))
+        a = np.ones((C, dk)); b = np.zeros(C)
+        Q[:L], K[:L], V[:L], a[:L], b[:L] = (q[t0:t0 + L], k[t0:t0 + L], v[t0:t0 + L],
+                                             a_all[t0:t0 + L], beta[t0:t0 + L])
+        nsub = C // SUB
+        phi = np.empty((C, dk)); psi = np.empty((C, dk)); pi = np.empty((nsub, dk))
+        for I in range(nsub):
+            s, e = I * SUB, (I + 1) * SUB
+            phi[s:e] = np.cumprod(a[s:e], axis=0)
+            rev = np.ones((SUB, dk))
+            for r in range(SUB - 2, -1, -1):
+                rev[r] = rev[r + 1] * a[s + r + 1]
+            psi[s:e] = rev
+            pi[I] = phi[e - 1]
+        # left/right operands and A, P by sub-chunk blocks
+        R = K * psi
+        A = np.zeros((C, C)); P = np.zeros((C, C))
+        for I in range(nsub):
+            rs = slice(I * SUB, (I + 1) * SUB)
+            for J in range(I + 1):
+                js = slice(J * SUB, (J + 1) * SUB)
+                if I == J:
+                    dprime = 1.0 / pi[I]
+                else:
+                    dprime = np.prod(pi[J + 1:I], axis=0) if I > J + 1 else np.ones(dk)
+                A[rs, js] = (K[rs] * phi[rs] * dprime) @ R[js].T
+                P[rs, js] = (Q[rs] * phi[rs] * dprime) @ R[js].T
+        A = np.tril(A, -1) * b[:, None]
+        P = np.tril(P, 0)
+        Tm = np.linalg.inv(np.eye(C) + A)
+        # chunk-level decays from the sub-chunk products
+        gamma = np.empty((C, dk)); eta = np.empty((C, dk))
+        for I in range(nsub):
+            rs = slice(I * SUB, (I + 1) * SUB)
+            before = np.prod(pi[:I], axis=0) if I > 0 else np.ones(dk)
+            after = np.prod(pi[I + 1:], axis=0) if I < nsub - 1 else np.ones(dk)
+            gamma[rs] = before * phi[rs]
+            eta[rs] = psi[rs] * after
+        Kt, Qt, Kh = K * gamma, Q * gamma, K * eta
+        W = Tm @ (b[:, None] * Kt)
+        Ut = Tm @ (b[:, None] * V)
+        U = Ut - W @ S
+        O1 = Qt @ S + P @ U
+        O2 = (Qt - P @ W) @ S + P @ Ut
+        assert np.allclose(O1, O2, rtol=1e-10, atol=1e-12)
+        out[t0:t0 + L] = O1[:L]
+        S = gamma[C - 1][:, None] * S + Kh.T @ U
+    return out, S
+
+
+def _case(seed, T, dk, dv, extreme=False):
+    rng = np.random.default_rng(seed)
+    f32 = lambda x: np.asarray(x, np.float32)
+    q = rng.standard_normal((T, dk)); q /= np.linalg.norm(q, axis=1, keepdims=True)
+    k = rng.standard_normal((T, dk)); k /= np.linalg.norm(k, axis=1, keepdims=True)
+    v = rng.standard_normal((T, dv))
+    beta = 1 / (1 + np.exp(-rng.standard_normal(T)))
+    alpha = np.exp(-np.log1p(np.exp(rng.standard_normal((T, dk)))))
+    if extreme:
+        # whole channels pinned at the clamp's bounds and below it
+        alpha[:, : dk // 4] = 1.0
+        alpha[:, dk // 4: dk // 2] = 1e-4
+    S0 = 0.1 * rng.standard_normal((dk, dv))
+    return f32(q), f32(k), f32(v), f32(alpha), f32(beta), f32(S0)
+
+
+@pytest.mark.parametrize("C", [16, 32, 64])
+@pytest.mark.parametrize("T,extreme", [(1, False), (37, False), (130, False), (200, True)])
+def test_chunk_form_equals_oracle(C, T, extreme):
+    dk, dv = 32, 16
+    q, k, v, al, be, S0 = _case(1000 + T + C, T, dk, dv, extreme)
+    ref_o, ref_S = oracle.forward(q[None, :, None], k[None, :, None], v[None, :, None],
+                                  al[None, :, None], be[None, :, None], S0[None, None])
+    o, S = chunk_forward_one(*(x.astype(np.float64) for x in (q, k, v, al, be, S0)), C)
+    np.testing.assert_allclose(o, ref_o[0, :, 0], rtol=1e-11, atol=1e-12)
+    np.testing.assert_allclose(S, ref_S[0, 0], rtol=1e-11, atol=1e-12)
+
+
+def test_subchunk_factors_stay_in_fp32_range():
+    """With every gate at the clamp's floor the factors used for A and P stay
+    inside the fp32 range: phi, psi >= e^-80 and 1/pi <= e^80."""
+    lo = np.float64(np.float32(np.exp(-5.0)))
+    phi_min = lo ** SUB
+    assert phi_min > np.finfo(np.float32).tiny
+    assert 1.0 / phi_min < np.finfo(np.float32).max
+    # one token more per sub-chunk would still fit, two sub-chunks would not
+    assert lo ** (2 * SUB) < np.finfo(np.float32).tiny
