@@ -1,0 +1,546 @@
+#!/usr/bin/env python
+"""KDA forward benchmark on B200: tokens/s and TFLOP/s against the HBM roofline.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME] [--impl ours|reference]
+
+One step = one kda_forward call (the whole chunk-parallel forward, one kernel
+launch) over one batch of seeded synthetic inputs already resident in HBM.
+For N > 1 (launched with torch.distributed.run, one process per GPU) every
+rank runs its own batch (independent sequences, no data-path collective:
+weak scaling); the time is the max over ranks and `value` counts all ranks'
+tokens.  Rank 0 prints ONE JSON line.
+
+--impl reference times the CPU oracle (fp64, token by token) as it stands on
+the host cores, on a bounded sample of the same workload.
+"""
+from __future__ import annotations
+
+import argparse
+import datetime
+import hashlib
+import json
+import os
+import statistics
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+METRIC = "KDA fwd tokens/s and TFLOP/s (% roofline) at H=32, d=128, 1 B200"
+DEFAULT_WORKLOAD = "bf16_B8_T4096_H32_d128"
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+
+
+# ---------------------------------------------------------------- work model
+
+def esize(dtype: str) -> int:
+    return 4 if dtype == "f32" else 2
+
+
+def forward_bytes(w, n_token_heads: int, n_seq_heads: int, has_s0: bool) -> int:
+    """Algorithmic HBM bytes of one forward: q, k, alpha, v, beta read and o
+    written once per (token, head); S0 read and S_final written once per
+    (sequence, head)."""
+    ei, eo = esize(w.dtype), esize(w.out_dtype)
+    per_th = ei * (3 * w.dk + w.dv + 1) + eo * w.dv
+    per_sh = 4 * w.dk * w.dv * ((1 if has_s0 else 0) + 1)
+    return per_th * n_token_heads + per_sh * n_seq_heads
+
+
+def forward_flops(w, n_token_heads: int) -> int:
+    """Chunk-form flops per (token, head): 6 dk dv + 2 C (3 dk + 2 dv)."""
+    return (6 * w.dk * w.dv + 2 * w.chunk * (3 * w.dk + 2 * w.dv)) * n_token_heads
+
+
+def decode_bytes(w, n_seq_heads: int) -> int:
+    ei, eo = esize(w.dtype), esize(w.out_dtype)
+    return n_seq_heads * (8 * w.dk * w.dv + ei * (3 * w.dk + w.dv + 1) + eo * w.dv)
+
+
+def decode_flops(w, n_seq_heads: int) -> int:
+    return n_seq_heads * 6 * w.dk * w.dv
+
+
+def load_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as fh:
+            p = json.load(fh)
+        return {k: float(p[k]) for k in FALLBACK_PEAKS}, "measured"
+    except (OSError, KeyError, ValueError):
+        return dict(FALLBACK_PEAKS), "fallback"
+
+
+def kernel_source_digest(name: str) -> str:
+    path = os.path.join(ROOT, "gated_delta_rule_138_b200", "csrc", name)
+    with open(path, "rb") as fh:
+        return hashlib.sha256(fh.read()).hexdigest()[:16]
+
+
+def recorded_traffic(kernel: str, workload: str):
+    """dram read+write bytes per launch from the committed ncu summary, if it
+    was taken on the kernel source as it is now (else None)."""
+    path = os.path.join(ROOT, "profiles", "dram_traffic.txt")
+    try:
+        lines = open(path).read().splitlines()
+    except OSError:
+        return None
+    for ln in lines:
+        if ln.startswith("#") or not ln.strip():
+            continue
+        f = ln.split()
+        # kernel workload source_file source_sha bytes_per_launch
+        if len(f) >= 5 and f[0] == kernel and f[1] == workload:
+            try:
+                if kernel_source_digest(f[2]) == f[3]:
+                    return float(f[4])
+            except OSError:
+                return None
+    return None
+
+
+# ---------------------------------------------------------------- clocks
+
+class ClockSampler:
+    """Samples SM clock and clock-event reasons through NVML while running."""
+
+    REASONS = {0x4: "sw_power_cap", 0x8: "hw_slowdown", 0x20: "sw_thermal_slowdown",
+               0x40: "hw_thermal_slowdown", 0x80: "hw_power_brake_slowdown",
+               0x2: "applications_clocks_setting", 0x1: "gpu_idle"}
+
+    def __init__(self, device_index: int, period_s: float = 0.005):
+        self.samples = []
+        self.max_mhz = None
+        self._stop = threading.Event()
+        self._period = period_s
+        self._h = None
+        try:
+            import pynvml
+            pynvml.nvmlInit()
+            self._nv = pynvml
+            import torch
+            uuid = str(torch.cuda.get_device_properties(device_index).uuid)
+            try:
+                self._h = pynvml.nvmlDeviceGetHandleByUUID(
+                    uuid if uuid.startswith("GPU-") else "GPU-" + uuid)
+            except Exception:
+                self._h = pynvml.nvmlDeviceGetHandleByIndex(device_index)
+            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(self._h, pynvml.NVML_CLOCK_SM)
+        except Exception as exc:  # pragma: no cover - depends on the box
+            self.error = repr(exc)
+        self._t = threading.Thread(target=self._run, daemon=True)
+
+    def _run(self):
+        nv = self._nv
+        while not self._stop.is_set():
+            try:
+                mhz = nv.nvmlDeviceGetClockInfo(self._h, nv.NVML_CLOCK_SM)
+                try:
+                    rs = nv.nvmlDeviceGetCurrentClocksEventReasons(self._h)
+                except AttributeError:
+                    rs = nv.nvmlDeviceGetCurrentClocksThrottleReasons(self._h)
+                self.samples.append((time.monotonic(), mhz, rs))
+            except Exception:
+                pass
+            time.sleep(self._period)
+
+    def start(self):
+        if self._h is not None:
+            self._t.start()
+        return self
+
+    def stop(self):
+        self._stop.set()
+        if self._t.is_alive():
+            self._t.join(timeout=2)
+
+    def summary(self, t0: float, t1: float):
+        win = [s for s in self.samples if t0 <= s[0] <= t1]
+        if not win and self.samples:   # region shorter than the period: nearest
+            mid = 0.5 * (t0 + t1)
+            win = [min(self.samples, key=lambda s: abs(s[0] - mid))]
+        if not win:
+            return {"sm_mhz": None, "sm_max_mhz": self.max_mhz, "reasons": [],
+                    "samples": 0, "note": getattr(self, "error", "no samples")}
+        reasons = set()
+        for _, _, rs in win:
+            for bit, name in self.REASONS.items():
+                if rs & bit and name != "gpu_idle":
+                    reasons.add(name)
+        return {"sm_mhz": statistics.median(s[1] for s in win), "sm_max_mhz": self.max_mhz,
+                "reasons": sorted(reasons), "samples": len(win)}
+
+
+# ---------------------------------------------------------------- helpers
+
+def dist_setup(n_gpus: int):
+    import torch
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world != n_gpus:
+        raise SystemExit("--gpus %d but WORLD_SIZE=%d (launch N>1 with torch.distributed.run)"
+                         % (n_gpus, world))
+    torch.cuda.set_device(local)
+    if world > 1:
+        import torch.distributed as dist
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300),
+                                device_id=torch.device("cuda", local))
+    return rank, world, local
+
+
+def barrier(world):
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+
+
+def max_over_ranks(x: float, world: int) -> float:
+    if world == 1:
+        return x
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([x], dtype=torch.float64, device="cuda")
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def sum_over_ranks(x: float, world: int) -> float:
+    if world == 1:
+        return x
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([x], dtype=torch.float64, device="cuda")
+    dist.all_reduce(t, op=dist.ReduceOp.SUM)
+    return float(t.item())
+
+
+def make_inputs(w, device, seed_offset: int):
+    from gated_delta_rule_138_b200 import inputs as gen
+    import dataclasses
+    w2 = dataclasses.replace(w, seed=w.seed + seed_offset)
+    return gen.draw_workload(w2, device=device)
+
+
+def counts(w, inp):
+    """(tokens, token-heads, sequence-heads) of one forward step."""
+    if w.kind == "varlen":
+        tokens = int(inp["q"].shape[1])
+        nseq = int(inp["cu_seqlens"].numel() - 1)
+    elif w.kind == "decode":
+        tokens = w.B
+        nseq = w.B
+    else:
+        tokens = w.B * w.T
+        nseq = w.B
+    return tokens, tokens * w.H, nseq * w.H
+
+
+# ---------------------------------------------------------------- CPU oracle timing
+
+def time_oracle(w, inp, budget_s: float, cores: int):
+    """Time the fp64 oracle on a bounded sample of this workload's inputs.
+
+    The sample is the first P (sequence, head) pairs over their first Ts tokens,
+    grown until one timed run takes about `budget_s` or covers the workload.
+    Returns (tokens_per_s, seconds, description).
+    """
+    import numpy as np
+    import oracle
+    f = lambda t: t.detach().float().cpu().numpy()
+    if w.kind == "decode":
+        # one decode step of P (sequence, head) pairs is T = 1 of the forward
+        q, k, v, al, be = (inp[n][0] for n in ("q", "k", "v", "alpha", "beta"))
+        S = inp["S"]
+        total_pairs = S.shape[0] * S.shape[1]
+        P = min(total_pairs, 64)
+        while True:
+            n_seq = max(1, P // w.H)
+            t0 = time.perf_counter()
+            oracle.decode_steps(f(q[None, :n_seq]), f(k[None, :n_seq]), f(v[None, :n_seq]),
+                                f(al[None, :n_seq]), f(be[None, :n_seq]), f(S[:n_seq]),
+                                nthreads=cores)
+            dt = time.perf_counter() - t0
+            if dt >= 0.5 * budget_s or n_seq >= S.shape[0]:
+                return n_seq / dt, dt, "%d sequences x %d heads, one decode step" % (n_seq, w.H)
+            P = min(total_pairs, int(P * max(2.0, budget_s / max(dt, 1e-3))))
+
+    if w.kind == "varlen":
+        cu = inp["cu_seqlens"].cpu().numpy()
+        starts, lens = cu[:-1], np.diff(cu)
+    else:
+        starts = np.arange(w.B) * w.T
+        lens = np.full(w.B, w.T)
+    Tmax = int(lens.max()) if len(lens) else 0
+    flat = {n: inp[n].reshape(-1, *inp[n].shape[2:]) for n in ("q", "k", "v", "alpha", "beta")}
+    S0 = inp.get("S0")
+    pairs = [(s, h) for s in range(len(lens)) for h in range(w.H)]
+    P, Ts = min(len(pairs), 2 * cores), min(Tmax, 1024)
+    while True:
+        sel = pairs[:P]
+        qs, ks, vs, als, bes, s0s = [], [], [], [], [], []
+        for s, h in sel:
+            a = int(starts[s])
+            L = min(int(lens[s]), Ts)
+            pad = Ts - L
+            sl = lambda x: np.pad(f(x[a:a + L, h]), [(0, pad)] + [(0, 0)] * (x.dim() - 2))
+            qs.append(sl(flat["q"])); ks.append(sl(flat["k"])); vs.append(sl(flat["v"]))
+            als.append(sl(flat["alpha"])); bes.append(sl(flat["beta"]))
+            s0s.append(f(S0[s, h]) if S0 is not None else np.zeros((w.dk, w.dv), np.float32))
+        st = lambda xs: np.stack(xs)[:, :, None]
+        t0 = time.perf_counter()
+        oracle.forward(st(qs), st(ks), st(vs), st(als), np.stack(bes)[:, :, None],
+                       np.stack(s0s)[:, None], nthreads=cores)
+        dt = time.perf_counter() - t0
+        covered = P == len(pairs) and Ts == Tmax
+        if dt >= 0.5 * budget_s or covered:
+            tok_heads = P * Ts
+            desc = "%d (sequence, head) pairs x first %d tokens (%d token-heads of %d)" % (
+                P, Ts, tok_heads, int(lens.sum()) * w.H)
+            return (tok_heads / w.H) / dt, dt, desc
+        grow = max(2.0, min(8.0, budget_s / max(dt, 1e-3)))
+        if Ts < Tmax:
+            Ts = min(Tmax, int(Ts * grow))
+        else:
+            P = min(len(pairs), int(P * grow))
+
+
+# ---------------------------------------------------------------- arms
+
+def run_reference(args, w):
+    """The CPU oracle as the reference arm: rank 0 only, host cores."""
+    if int(os.environ.get("RANK", "0")) != 0:
+        return
+    import oracle
+    import torch
+    cores = oracle.available_cores()
+    inp = make_inputs(w, "cpu", 0) if w.kind != "forward" or w.T <= 8192 else None
+    if inp is None:   # long sequences: draw only the first slice of tokens
+        from gated_delta_rule_138_b200 import inputs as gen
+        inp = gen.draw_forward(w.B, 8192, w.H, w.dk, w.dv, w.dtype, w.seed, device="cpu",
+                               s0=w.s0, special_alpha=w.special_alpha)
+    per_step = max(1.0, min(10.0, 150.0 / max(1, args.steps + args.warmup)))
+    for _ in range(args.warmup):
+        time_oracle(w, inp, per_step * 0.25, cores)
+    rates, secs, desc = [], 0.0, ""
+    for _ in range(args.steps):
+        r, dt, desc = time_oracle(w, inp, per_step, cores)
+        rates.append(r)
+        secs += dt
+    value = statistics.median(rates) if rates else 0.0
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": "tokens/s",
+        "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": 1e3 * secs / max(1, args.steps), "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": config_of(w, args.gpus),
+        "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": cores, "kind": "oracle",
+                         "sample": desc},
+        "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0,
+                "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+    del torch
+
+
+def config_of(w, n_gpus):
+    c = {"workload": w.name, "H": w.H, "d_k": w.dk, "d_v": w.dv, "chunk": w.chunk,
+         "in_dtype": w.dtype, "out_dtype": w.out_dtype, "state": "fp32",
+         "parallelism": "replicas x%d (independent sequences per GPU)" % n_gpus}
+    if w.kind == "forward":
+        c.update({"B": w.B, "T": w.T, "global_batch": w.B * n_gpus, "seq_len": w.T})
+    elif w.kind == "varlen":
+        c.update({"num_seqs": w.nseq, "len_range": [w.min_len, w.max_len]})
+    else:
+        c.update({"N": w.B, "steps_per_run": w.steps})
+    return c
+
+
+def run_ours(args, w):
+    import torch
+    import gated_delta_rule_138_b200 as kda
+
+    rank, world, local = dist_setup(args.gpus)
+    dev = torch.device("cuda", local)
+    inp = make_inputs(w, dev, 1000 * rank)
+    tokens, n_th, n_sh = counts(w, inp)
+    peaks, peak_src = load_peaks()
+    stream = torch.cuda.current_stream()
+
+    if w.kind == "decode":
+        S = inp["S"].clone()
+        out = torch.empty(w.B, w.H, w.dv, dtype=torch.bfloat16, device=dev)
+        n_steps_avail = inp["q"].shape[0]
+        state = {"i": 0}
+
+        def step():
+            i = state["i"] % n_steps_avail
+            state["i"] += 1
+            kda.kda_decode_step(inp["q"][i], inp["k"][i], inp["v"][i], inp["alpha"][i],
+                                inp["beta"][i], S, out=out)
+        kname = "decode_f32state"
+        algo_bytes = decode_bytes(w, n_sh)
+        algo_flops = decode_flops(w, n_sh)
+        src_file = "kda_decode.cu"
+    else:
+        cu = inp.get("cu_seqlens")
+        B, T = inp["q"].shape[0], inp["q"].shape[1]
+        out = torch.empty(B, T, w.H, w.dv, dtype=torch.bfloat16 if w.out_dtype == "bf16"
+                          else torch.float32, device=dev)
+        nseq = B if cu is None else cu.numel() - 1
+        Sf = torch.empty(nseq, w.H, w.dk, w.dv, dtype=torch.float32, device=dev)
+
+        def step():
+            kda.kda_forward(inp["q"], inp["k"], inp["v"], inp["alpha"], inp["beta"], inp["S0"],
+                            cu_seqlens=cu, out=out, S_final=Sf, chunk=w.chunk)
+        kname = kda.kda_forward_kernel_name(w.dk, w.dv, w.chunk, inp["q"].dtype, out.dtype)
+        algo_bytes = forward_bytes(w, n_th, n_sh, inp["S0"] is not None)
+        algo_flops = forward_flops(w, n_th)
+        src_file = "kda_chunk_tc.cu" if kname == "chunk_tc_bf16" else "kda_chunk_simt.cu"
+
+    warm = max(3, args.warmup)
+    for _ in range(warm):
+        step()
+    torch.cuda.synchronize()
+
+    sampler = ClockSampler(local).start()
+    time.sleep(0.05)
+    barrier(world)
+    torch.cuda.synchronize()
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+          for _ in range(args.steps)]
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    n0 = kda.kda_launch_count()
+    h0 = time.monotonic()
+    e0.record(stream)
+    for i in range(args.steps):
+        ev[i][0].record(stream)
+        step()
+        ev[i][1].record(stream)
+    e1.record(stream)
+    torch.cuda.synchronize()
+    h1 = time.monotonic()
+    barrier(world)
+    launches = kda.kda_launch_count() - n0
+    sampler.stop()
+    clocks = sampler.summary(h0, h1)
+    elapsed_ms = max_over_ranks(e0.elapsed_time(e1), world)
+    kern_ms = statistics.mean(a.elapsed_time(b) for a, b in ev)
+    kern_ms = max_over_ranks(kern_ms, world)
+    total_tokens = sum_over_ranks(tokens * args.steps, world)
+    value = total_tokens / (elapsed_ms * 1e-3)
+    ms_per_step = elapsed_ms / args.steps
+
+    # end to end: pinned host inputs -> device -> kda_forward -> host results
+    e2e = run_e2e(args, w, inp, dev, stream, world) if w.kind != "decode" else None
+
+    if rank == 0:
+        achieved = algo_bytes / (kern_ms * 1e-3) / 1e9
+        tflops = algo_flops / (kern_ms * 1e-3) / 1e12
+        line = {
+            "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world,
+            "steps": args.steps, "warmup": warm, "ms_per_step": ms_per_step,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+            "dtype": "bf16" if kname == "chunk_tc_bf16" else "f32",
+            "data": "synthetic (seeded generators, the workload's shapes and distributions)",
+            "config": dict(config_of(w, world),
+                           l2="no flush: inputs %.2f GB per step > 126 MB L2"
+                              % (algo_bytes / 1e9)),
+            "tflops": tflops,
+            "roofline": {"bound": "hbm", "achieved": achieved, "peak": peaks["hbm_gbs"],
+                         "unit": "GB/s", "frac": achieved / peaks["hbm_gbs"],
+                         "traffic": recorded_traffic(kname, w.name),
+                         "kernel": kname, "algorithmic_bytes": algo_bytes,
+                         "kernel_ms": kern_ms, "peak_source": peak_src},
+            "tensor": {"achieved_tflops": tflops, "peak": peaks["bf16_tflops"],
+                       "frac": tflops / peaks["bf16_tflops"], "flops_per_step": algo_flops},
+            "clocks": clocks,
+            "gpu_launches": int(launches),
+            "e2e": e2e,
+        }
+        if world == 1 and not args.no_cpu_baseline:
+            import oracle
+            cores = oracle.available_cores()
+            r, dt, desc = time_oracle(w, inp, args.cpu_budget, cores)
+            line["cpu_baseline"] = {"value": r, "unit": "tokens/s", "cores": cores,
+                                    "kind": "oracle", "sample": desc, "seconds": dt}
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        import torch.distributed as dist
+        dist.destroy_process_group()
+
+
+def run_e2e(args, w, inp, dev, stream, world):
+    """Same metric through the public API with host buffers: every step copies
+    its inputs from pinned host memory and reads its result back."""
+    import torch
+    import gated_delta_rule_138_b200 as kda
+    names = [n for n in ("q", "k", "v", "alpha", "beta", "S0", "cu_seqlens")
+             if inp.get(n) is not None]
+    try:
+        host = {n: inp[n].cpu().pin_memory() for n in names}
+    except RuntimeError as exc:
+        return {"value": None, "unit": "tokens/s", "note": "pinned host alloc failed: %s" % exc}
+    devb = {n: torch.empty_like(inp[n]) for n in names}
+    cu = devb.get("cu_seqlens")
+    B, T = inp["q"].shape[0], inp["q"].shape[1]
+    nseq = B if cu is None else cu.numel() - 1
+    out = torch.empty(B, T, w.H, w.dv, dtype=torch.bfloat16 if w.out_dtype == "bf16"
+                      else torch.float32, device=dev)
+    Sf = torch.empty(nseq, w.H, w.dk, w.dv, dtype=torch.float32, device=dev)
+    out_h = torch.empty(out.shape, dtype=out.dtype).pin_memory()
+    Sf_h = torch.empty(Sf.shape, dtype=Sf.dtype).pin_memory()
+    h2d = sum(host[n].numel() * host[n].element_size() for n in names)
+    d2h = out_h.numel() * out_h.element_size() + Sf_h.numel() * Sf_h.element_size()
+
+    def step():
+        for n in names:
+            devb[n].copy_(host[n], non_blocking=True)
+        kda.kda_forward(devb["q"], devb["k"], devb["v"], devb["alpha"], devb["beta"],
+                        devb.get("S0"), cu_seqlens=cu, out=out, S_final=Sf, chunk=w.chunk)
+        out_h.copy_(out, non_blocking=True)
+        Sf_h.copy_(Sf, non_blocking=True)
+
+    n = max(2, min(args.steps, 10))
+    for _ in range(2):
+        step()
+    torch.cuda.synchronize()
+    barrier(world)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(n):
+        step()
+    e1.record(stream)
+    torch.cuda.synchronize()
+    barrier(world)
+    ms = max_over_ranks(e0.elapsed_time(e1), world)
+    tokens, _, _ = counts(w, inp)
+    total = sum_over_ranks(tokens * n, world)
+    return {"value": total / (ms * 1e-3), "unit": "tokens/s", "h2d_bytes_per_step": int(h2d),
+            "d2h_bytes_per_step": int(d2h), "steps": n}
+
+
+def main():
+    ap = argparse.ArgumentParser(description=__doc__.split("\n")[0])
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=50)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--workload", default=DEFAULT_WORKLOAD)
+    ap.add_argument("--cpu-budget", type=float, default=15.0,
+                    help="seconds of oracle time for the cpu_baseline sample")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    from gated_delta_rule_138_b200 import inputs as gen
+    w = gen.WORKLOADS[args.workload]
+    if args.impl == "reference":
+        run_reference(args, w)
+    else:
+        run_ours(args, w)
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,118 @@
+// C ABI of libkda.so (declared in include/kda.h): argument validation and
+// dispatch to the kernels.  No entry point allocates on the caller's behalf
+// beyond the library-owned workspace, synchronises the device, or throws.
+#include <atomic>
+#include <cstdio>
+#include <cstring>
+
+#include "../../include/kda.h"
+#include "kda_common.cuh"
+
+namespace kda {
+cudaError_t launch_chunk_simt(int in_bf16, int out_bf16, int chunk, const void* q, const void* k,
+                              const void* v, const void* alpha, const void* beta, const float* S0,
+                              const int32_t* cu, int nseq, void* out, float* S_final, int64_t T,
+                              int H, int DK, int DV, cudaStream_t s);
+cudaError_t launch_decode(int in_bf16, int out_bf16, const void* q, const void* k, const void* v,
+                          const void* alpha, const void* beta, float* S, void* out, int64_t NH,
+                          int DK, int DV, cudaStream_t s);
+}  // namespace kda
+
+namespace {
+
+thread_local char g_last_error[256] = "";
+std::atomic<uint64_t> g_launches{0};
+
+kda_status_t cuda_status(cudaError_t e) {
+    if (e == cudaSuccess) return KDA_OK;
+    std::snprintf(g_last_error, sizeof(g_last_error), "%s: %s", cudaGetErrorName(e),
+                  cudaGetErrorString(e));
+    return KDA_ERR_CUDA;
+}
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+bool is_dtype(kda_dtype_t d) { return d == KDA_F32 || d == KDA_BF16; }
+bool head_dim_ok(int32_t d) { return d == 64 || d == 128; }
+
+}  // namespace
+
+extern "C" {
+
+const char* kda_status_string(kda_status_t status) {
+    switch (status) {
+        case KDA_OK: return "KDA_OK";
+        case KDA_ERR_INVALID_ARG: return "KDA_ERR_INVALID_ARG";
+        case KDA_ERR_UNSUPPORTED: return "KDA_ERR_UNSUPPORTED";
+        case KDA_ERR_CUDA: return "KDA_ERR_CUDA";
+        case KDA_ERR_DEVICE_TIMEOUT: return "KDA_ERR_DEVICE_TIMEOUT";
+    }
+    return "KDA_ERR_UNKNOWN";
+}
+
+const char* kda_last_error(void) { return g_last_error; }
+
+uint64_t kda_launch_count(void) { return g_launches.load(std::memory_order_relaxed); }
+
+const char* kda_forward_kernel_name(int32_t d_k, int32_t d_v, int32_t chunk,
+                                    kda_dtype_t in_dtype, kda_dtype_t out_dtype) {
+    if (!is_dtype(in_dtype) || !is_dtype(out_dtype)) return nullptr;
+    if (!head_dim_ok(d_k) || !head_dim_ok(d_v)) return nullptr;
+    if (chunk != 16 && chunk != 32 && chunk != 64) return nullptr;
+    return "chunk_simt_f32";
+}
+
+size_t kda_forward_workspace_bytes(int32_t B, int64_t T, int32_t H, int32_t d_k, int32_t d_v,
+                                   int32_t chunk) {
+    (void)B; (void)T; (void)H; (void)d_k; (void)d_v; (void)chunk;
+    return 0;
+}
+
+kda_status_t kda_forward(const void* q, const void* k, const void* v, const void* alpha,
+                         const void* beta, const float* S0, const int32_t* cu_seqlens,
+                         int32_t num_seqs, void* out, float* S_final, int32_t B, int64_t T,
+                         int32_t H, int32_t d_k, int32_t d_v, int32_t chunk,
+                         kda_dtype_t in_dtype, kda_dtype_t out_dtype, kda_stream_t stream) {
+    if (B < 0 || T < 0 || H <= 0 || !is_dtype(in_dtype) || !is_dtype(out_dtype))
+        return KDA_ERR_INVALID_ARG;
+    if (cu_seqlens != nullptr && (B != 1 || num_seqs < 0)) return KDA_ERR_INVALID_ARG;
+    const int64_t nseq = cu_seqlens ? (int64_t)num_seqs : (int64_t)B;
+    const bool has_tokens = (int64_t)B * T > 0;
+    if (has_tokens && (!q || !k || !v || !alpha || !beta || !out)) return KDA_ERR_INVALID_ARG;
+    const void* ptrs[] = {q, k, v, alpha, beta, S0, cu_seqlens, out, S_final};
+    for (const void* p : ptrs)
+        if (p && !aligned16(p)) return KDA_ERR_INVALID_ARG;
+    if (!head_dim_ok(d_k) || !head_dim_ok(d_v)) return KDA_ERR_UNSUPPORTED;
+    if (chunk != 16 && chunk != 32 && chunk != 64) return KDA_ERR_UNSUPPORTED;
+    if (nseq > 65535 || H > 65535) return KDA_ERR_UNSUPPORTED;  // grid y/z limits
+    if (nseq == 0) return KDA_OK;
+    g_last_error[0] = '\0';
+    const cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    const int in_bf16 = in_dtype == KDA_BF16, out_bf16 = out_dtype == KDA_BF16;
+    g_launches.fetch_add(1, std::memory_order_relaxed);
+    return cuda_status(kda::launch_chunk_simt(in_bf16, out_bf16, chunk, q, k, v, alpha, beta, S0,
+                                              cu_seqlens, (int)nseq, out, S_final, T, H, d_k, d_v,
+                                              s));
+}
+
+kda_status_t kda_decode_step(const void* q, const void* k, const void* v, const void* alpha,
+                             const void* beta, float* S, void* out, int32_t N, int32_t H,
+                             int32_t d_k, int32_t d_v, kda_dtype_t in_dtype,
+                             kda_dtype_t out_dtype, kda_stream_t stream) {
+    if (N < 0 || H <= 0 || !is_dtype(in_dtype) || !is_dtype(out_dtype))
+        return KDA_ERR_INVALID_ARG;
+    if (N > 0 && (!q || !k || !v || !alpha || !beta || !S || !out)) return KDA_ERR_INVALID_ARG;
+    const void* ptrs[] = {q, k, v, alpha, beta, S, out};
+    for (const void* p : ptrs)
+        if (p && !aligned16(p)) return KDA_ERR_INVALID_ARG;
+    if (!head_dim_ok(d_k) || !head_dim_ok(d_v)) return KDA_ERR_UNSUPPORTED;
+    const int64_t NH = (int64_t)N * H;
+    if (NH > 0x7fffffffLL) return KDA_ERR_UNSUPPORTED;
+    if (NH == 0) return KDA_OK;
+    g_last_error[0] = '\0';
+    const cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    g_launches.fetch_add(1, std::memory_order_relaxed);
+    return cuda_status(kda::launch_decode(in_dtype == KDA_BF16, out_dtype == KDA_BF16, q, k, v,
+                                          alpha, beta, S, out, NH, d_k, d_v, s));
+}
+
+}  // extern "C"

@@ -1,0 +1,324 @@
+// KDA chunked forward on CUDA cores, fp32 throughout.
+//
+// This is the path for fp32 inputs (the fp32 relative-L2 bar of 1e-5 is below
+// what bf16 or tf32 tensor-core operands can reach) and for every size the
+// tensor-core kernel does not cover.  It implements the same chunk algebra as
+// the tensor-core kernel:
+//
+//   per chunk of C tokens with start state S (d_k x d_v), a = clamp(alpha):
+//     D(r, j)  = prod_{s=j+1..r} a_s                    (per key channel)
+//     A[r, j]  = beta_r sum_c k_rc k_jc D(r, j)_c        j <  r
+//     P[r, j]  =        sum_c q_rc k_jc D(r, j)_c        j <= r
+//     Tinv     = (I + A)^-1
+//     W        = Tinv diag(beta) (k * gamma),  U~ = Tinv diag(beta) V
+//     U        = U~ - W S
+//     O        = (q * gamma - P W) S + P U~
+//     S       <- Diag(gamma_C) S + (k * eta)^T U
+//   gamma_r = prod_{s<=r} a_s, eta_j = prod_{s>j} a_s, gamma_C = prod over the chunk.
+//
+// The worldcybernews article "Kimi K3 Open Model Surpasses Closed GPT and
+// Anthropic Systems on Independent Benchmarks", paragraph 3: tokens inside a
+// chunk are processed in parallel, states are carried across chunks.
+//
+// D(r, j) is split at 16-token sub-chunk boundaries so that no factor leaves
+// the fp32 range (a 64-token product of gates >= e^-5 can reach e^-320):
+//   phi_r = prod_{s=start(I)..r} a_s, psi_j = prod_{s=j+1..end(J)} a_s,
+//   pi_I = prod over sub-chunk I >= e^-80, Delta'_IJ = prod_{J<M<I} pi_M (I > J)
+//   or 1/pi_I (I == J) <= e^80, and D(r, j) = phi_r Delta'_IJ psi_j.
+//
+// One CTA of 256 threads owns one (sequence, head, slice of NV value columns)
+// and walks its chunks in order; the state slice lives in shared memory.
+#include "kda_common.cuh"
+
+namespace kda {
+
+constexpr int kSimtThreads = 256;
+constexpr int kSub = 16;
+
+template <int DK, int NV, int C>
+struct SimtSmem {
+    static constexpr int NSUB = C / kSub;
+    static constexpr int NPAIR = NSUB * (NSUB + 1) / 2;
+    static constexpr int DKP = DK + 1, CP = C + 1, NVP = NV + 1;
+    static constexpr int floats = 3 * C * DKP + 3 * C * CP + 3 * C * NVP + DK * NVP +
+                                  3 * NSUB * DK + NPAIR * DK + C;
+    static constexpr size_t bytes = sizeof(float) * (size_t)floats;
+};
+
+template <typename Tin, typename Tout, int DK, int NV, int C>
+__global__ void __launch_bounds__(kSimtThreads)
+kda_chunk_simt_kernel(const Tin* __restrict__ q, const Tin* __restrict__ k,
+                      const Tin* __restrict__ v, const Tin* __restrict__ alpha,
+                      const Tin* __restrict__ beta, const float* S0,
+                      const int32_t* __restrict__ cu_seqlens, Tout* __restrict__ out,
+                      float* S_final, int64_t T, int H, int DV) {
+    using L = SimtSmem<DK, NV, C>;
+    constexpr int NSUB = L::NSUB, DKP = L::DKP, CP = L::CP, NVP = L::NVP;
+    extern __shared__ float smem[];
+    float* kphi = smem;                 // [C][DKP]  k*phi       -> W
+    float* qphi = kphi + C * DKP;       // [C][DKP]  q*phi       -> Q~ - P W
+    float* kpsi = qphi + C * DKP;       // [C][DKP]  gate stage  -> k*psi -> K^ = k*eta
+    float* Am = kpsi + C * DKP;         // [C][CP]   A
+    float* Pm = Am + C * CP;            // [C][CP]   P
+    float* Tm = Pm + C * CP;            // [C][CP]   (I + A)^-1
+    float* vs = Tm + C * CP;            // [C][NVP]  V slice
+    float* Ut = vs + C * NVP;           // [C][NVP]  U~
+    float* Us = Ut + C * NVP;           // [C][NVP]  U
+    float* Ss = Us + C * NVP;           // [DK][NVP] state slice
+    float* pis = Ss + DK * NVP;         // [NSUB][DK]
+    float* before = pis + NSUB * DK;    // [NSUB][DK] prod_{M<I} pi_M
+    float* after = before + NSUB * DK;  // [NSUB][DK] prod_{M>I} pi_M
+    float* dpr = after + NSUB * DK;     // [NPAIR][DK] Delta'_IJ
+    float* bs = dpr + L::NPAIR * DK;    // [C] beta
+
+    const int tid = threadIdx.x;
+    const int j0 = blockIdx.x * NV, h = blockIdx.y, n = blockIdx.z;
+    int64_t bos, len;
+    seq_range(cu_seqlens, n, T, bos, len);
+    const size_t sbase = ((size_t)n * H + h) * (size_t)DK * DV + j0;
+
+    for (int i = tid; i < DK * NV; i += kSimtThreads) {
+        const int c = i / NV, jj = i % NV;
+        Ss[c * NVP + jj] = S0 ? S0[sbase + (size_t)c * DV + jj] : 0.0f;
+    }
+    __syncthreads();
+
+    for (int64_t t0 = 0; t0 < len; t0 += C) {
+        const int Lc = (int)((len - t0) < C ? (len - t0) : C);
+        const int64_t row0 = bos + t0;  // first token of the chunk in [B*T]
+
+        // ---- gates: sub-chunk products per key channel; V and beta staging
+        if (tid < DK) {
+            const int c = tid;
+            float phi = 1.0f;
+#pragma unroll 8
+            for (int r = 0; r < C; ++r) {
+                float a = 1.0f, kk = 0.0f, qq = 0.0f;
+                if (r < Lc) {
+                    const size_t g = ((size_t)(row0 + r) * H + h) * DK + c;
+                    a = clamp_gate(to_f32(alpha[g]));
+                    kk = to_f32(k[g]);
+                    qq = to_f32(q[g]);
+                }
+                phi = (r % kSub == 0) ? a : phi * a;
+                kphi[r * DKP + c] = kk * phi;
+                qphi[r * DKP + c] = qq * phi;
+                kpsi[r * DKP + c] = a;
+                if (r % kSub == kSub - 1) pis[(r / kSub) * DK + c] = phi;
+            }
+            float psi = 1.0f, a_next = 1.0f;
+#pragma unroll 8
+            for (int r = C - 1; r >= 0; --r) {
+                const float a_r = kpsi[r * DKP + c];
+                psi = (r % kSub == kSub - 1) ? 1.0f : psi * a_next;
+                float kk = 0.0f;
+                if (r < Lc) kk = to_f32(k[((size_t)(row0 + r) * H + h) * DK + c]);
+                kpsi[r * DKP + c] = kk * psi;
+                a_next = a_r;
+            }
+            float acc = 1.0f;
+            for (int I = 0; I < NSUB; ++I) {
+                before[I * DK + c] = acc;
+                acc *= pis[I * DK + c];
+            }
+            acc = 1.0f;
+            for (int I = NSUB - 1; I >= 0; --I) {
+                after[I * DK + c] = acc;
+                acc *= pis[I * DK + c];
+            }
+            for (int I = 0; I < NSUB; ++I) {
+                float between = 1.0f;
+                for (int J = I; J >= 0; --J) {
+                    const int p = I * (I + 1) / 2 + J;
+                    if (J == I) {
+                        dpr[p * DK + c] = 1.0f / pis[I * DK + c];
+                    } else {
+                        dpr[p * DK + c] = between;
+                        between *= pis[J * DK + c];
+                    }
+                }
+            }
+        } else {
+            for (int i = tid - DK; i < C * NV; i += kSimtThreads - DK) {
+                const int r = i / NV, jj = i % NV;
+                vs[r * NVP + jj] =
+                    r < Lc ? to_f32(v[((size_t)(row0 + r) * H + h) * DV + j0 + jj]) : 0.0f;
+            }
+            for (int r = tid - DK; r < C; r += kSimtThreads - DK)
+                bs[r] = r < Lc ? to_f32(beta[(size_t)(row0 + r) * H + h]) : 0.0f;
+        }
+        __syncthreads();
+
+        // ---- A (strictly lower, beta-scaled rows) and P (lower, with diagonal)
+        for (int idx = tid; idx < C * C; idx += kSimtThreads) {
+            const int r = idx / C, j = idx % C;
+            float sa = 0.0f, sp = 0.0f;
+            if (j <= r) {
+                const int I = r / kSub, J = j / kSub;
+                const float* dp = dpr + (I * (I + 1) / 2 + J) * DK;
+                const float* kr = kphi + r * DKP;
+                const float* qr = qphi + r * DKP;
+                const float* kj = kpsi + j * DKP;
+#pragma unroll 8
+                for (int c = 0; c < DK; ++c) {
+                    const float w = kj[c] * dp[c];
+                    sa = fmaf(kr[c], w, sa);
+                    sp = fmaf(qr[c], w, sp);
+                }
+            }
+            Am[r * CP + j] = (j < r) ? bs[r] * sa : 0.0f;
+            Pm[r * CP + j] = sp;
+        }
+        __syncthreads();
+
+        // ---- (I + A)^-1 by forward substitution, one column per thread
+        if (tid < C) {
+            const int m = tid;
+            for (int r = 0; r < C; ++r) {
+                float t;
+                if (r < m) {
+                    t = 0.0f;
+                } else if (r == m) {
+                    t = 1.0f;
+                } else {
+                    float s = 0.0f;
+                    for (int j = m; j < r; ++j) s = fmaf(Am[r * CP + j], Tm[j * CP + m], s);
+                    t = -s;
+                }
+                Tm[r * CP + m] = t;
+            }
+        }
+        __syncthreads();
+
+        // ---- W = Tinv diag(beta) (k*gamma) into registers; U~ = Tinv diag(beta) V
+        {
+            constexpr int RG = kSimtThreads / DK;  // row groups
+            constexpr int RPT = C / RG;            // rows per thread
+            const int c = tid % DK, rg = tid / DK;
+            float acc[RPT];
+#pragma unroll
+            for (int i = 0; i < RPT; ++i) acc[i] = 0.0f;
+            for (int j = 0; j < C; ++j) {
+                const float kt = kphi[j * DKP + c] * before[(j / kSub) * DK + c] * bs[j];
+#pragma unroll
+                for (int i = 0; i < RPT; ++i) {
+                    const int r = rg + RG * i;
+                    if (j <= r) acc[i] = fmaf(Tm[r * CP + j], kt, acc[i]);
+                }
+            }
+            for (int i = tid; i < C * NV; i += kSimtThreads) {
+                const int r = i / NV, jj = i % NV;
+                float s = 0.0f;
+                for (int j = 0; j <= r; ++j) s = fmaf(Tm[r * CP + j] * bs[j], vs[j * NVP + jj], s);
+                Ut[r * NVP + jj] = s;
+            }
+            __syncthreads();
+#pragma unroll
+            for (int i = 0; i < RPT; ++i) kphi[(rg + RG * i) * DKP + c] = acc[i];
+            __syncthreads();
+
+            // Q' = q*gamma - P W  (registers, then over qphi); K^ = k*psi*after in place
+#pragma unroll
+            for (int i = 0; i < RPT; ++i) {
+                const int r = rg + RG * i;
+                float s = qphi[r * DKP + c] * before[(r / kSub) * DK + c];
+                for (int j = 0; j <= r; ++j) s = fmaf(-Pm[r * CP + j], kphi[j * DKP + c], s);
+                acc[i] = s;
+            }
+            __syncthreads();
+#pragma unroll
+            for (int i = 0; i < RPT; ++i) {
+                const int r = rg + RG * i;
+                qphi[r * DKP + c] = acc[i];
+                kpsi[r * DKP + c] *= after[(r / kSub) * DK + c];
+            }
+        }
+        __syncthreads();
+
+        // ---- U = U~ - W S ;  O = Q' S + P U~
+        for (int i = tid; i < C * NV; i += kSimtThreads) {
+            const int r = i / NV, jj = i % NV;
+            float su = Ut[r * NVP + jj], so = 0.0f;
+            const float* wr = kphi + r * DKP;
+            const float* qr = qphi + r * DKP;
+#pragma unroll 8
+            for (int c = 0; c < DK; ++c) {
+                const float s = Ss[c * NVP + jj];
+                su = fmaf(-wr[c], s, su);
+                so = fmaf(qr[c], s, so);
+            }
+            for (int j = 0; j <= r; ++j) so = fmaf(Pm[r * CP + j], Ut[j * NVP + jj], so);
+            Us[r * NVP + jj] = su;
+            if (r < Lc) out[((size_t)(row0 + r) * H + h) * DV + j0 + jj] = from_f32<Tout>(so);
+        }
+        __syncthreads();
+
+        // ---- S <- Diag(gamma_C) S + K^T U
+        for (int i = tid; i < DK * NV; i += kSimtThreads) {
+            const int c = i / NV, jj = i % NV;
+            const float gC = before[(NSUB - 1) * DK + c] * pis[(NSUB - 1) * DK + c];
+            float s = gC * Ss[c * NVP + jj];
+#pragma unroll 8
+            for (int j = 0; j < C; ++j) s = fmaf(kpsi[j * DKP + c], Us[j * NVP + jj], s);
+            Ss[c * NVP + jj] = s;
+        }
+        __syncthreads();
+    }
+
+    if (S_final) {
+        for (int i = tid; i < DK * NV; i += kSimtThreads) {
+            const int c = i / NV, jj = i % NV;
+            S_final[sbase + (size_t)c * DV + jj] = Ss[c * NVP + jj];
+        }
+    }
+}
+
+// ---------------------------------------------------------------- launcher
+
+template <typename Tin, typename Tout, int DK, int NV, int C>
+static cudaError_t launch_simt_t(const void* q, const void* k, const void* v, const void* alpha,
+                                 const void* beta, const float* S0, const int32_t* cu_seqlens,
+                                 int nseq, void* out, float* S_final, int64_t T, int H, int DV,
+                                 cudaStream_t stream) {
+    using L = SimtSmem<DK, NV, C>;
+    auto kern = kda_chunk_simt_kernel<Tin, Tout, DK, NV, C>;
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         (int)L::bytes);
+    if (e != cudaSuccess) return e;
+    dim3 grid(DV / NV, H, nseq);
+    kern<<<grid, kSimtThreads, L::bytes, stream>>>(
+        (const Tin*)q, (const Tin*)k, (const Tin*)v, (const Tin*)alpha, (const Tin*)beta, S0,
+        cu_seqlens, (Tout*)out, S_final, T, H, DV);
+    return cudaGetLastError();
+}
+
+template <typename Tin, typename Tout, int DK>
+static cudaError_t launch_simt_dk(int chunk, const void* q, const void* k, const void* v,
+                                  const void* alpha, const void* beta, const float* S0,
+                                  const int32_t* cu, int nseq, void* out, float* S_final,
+                                  int64_t T, int H, int DV, cudaStream_t s) {
+    switch (chunk) {
+        case 16: return launch_simt_t<Tin, Tout, DK, 32, 16>(q, k, v, alpha, beta, S0, cu, nseq, out, S_final, T, H, DV, s);
+        case 32: return launch_simt_t<Tin, Tout, DK, 32, 32>(q, k, v, alpha, beta, S0, cu, nseq, out, S_final, T, H, DV, s);
+        default: return launch_simt_t<Tin, Tout, DK, 32, 64>(q, k, v, alpha, beta, S0, cu, nseq, out, S_final, T, H, DV, s);
+    }
+}
+
+// Entry used by the C ABI: in/out dtype codes 0 = fp32, 1 = bf16.
+cudaError_t launch_chunk_simt(int in_bf16, int out_bf16, int chunk, const void* q, const void* k,
+                              const void* v, const void* alpha, const void* beta, const float* S0,
+                              const int32_t* cu, int nseq, void* out, float* S_final, int64_t T,
+                              int H, int DK, int DV, cudaStream_t s) {
+#define KDA_SIMT_CASE(TI, TO)                                                                  \
+    return DK == 64 ? launch_simt_dk<TI, TO, 64>(chunk, q, k, v, alpha, beta, S0, cu, nseq, out, \
+                                                 S_final, T, H, DV, s)                       \
+                    : launch_simt_dk<TI, TO, 128>(chunk, q, k, v, alpha, beta, S0, cu, nseq,   \
+                                                  out, S_final, T, H, DV, s);
+    if (!in_bf16 && !out_bf16) { KDA_SIMT_CASE(float, float) }
+    if (!in_bf16 && out_bf16) { KDA_SIMT_CASE(float, __nv_bfloat16) }
+    if (in_bf16 && !out_bf16) { KDA_SIMT_CASE(__nv_bfloat16, float) }
+    KDA_SIMT_CASE(__nv_bfloat16, __nv_bfloat16)
+#undef KDA_SIMT_CASE
+}
+
+}  // namespace kda

@@ -1,0 +1,51 @@
+// Device helpers shared by the KDA kernels in this directory.
+#pragma once
+
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+namespace kda {
+
+// Lower bound of the forget gate: e^-5 rounded to the nearest fp32.  The
+// worldcybernews article "Kimi K3 Open Model Surpasses Closed GPT and Anthropic
+// Systems on Independent Benchmarks", paragraph 2, holds alpha between e^-5
+// and 1 so that BF16 arithmetic neither underflows nor overflows.
+constexpr float kAlphaMin = 0x1.b993fep-8f;
+
+// clamp(alpha, e^-5, 1), taken on the fp32 value of the input
+__device__ __forceinline__ float clamp_gate(float a) {
+    a = a < kAlphaMin ? kAlphaMin : a;
+    return a > 1.0f ? 1.0f : a;
+}
+
+template <typename T> __device__ __forceinline__ float to_f32(T x);
+template <> __device__ __forceinline__ float to_f32<float>(float x) { return x; }
+template <> __device__ __forceinline__ float to_f32<__nv_bfloat16>(__nv_bfloat16 x) {
+    return __bfloat162float(x);
+}
+
+template <typename T> __device__ __forceinline__ T from_f32(float x);
+template <> __device__ __forceinline__ float from_f32<float>(float x) { return x; }
+template <> __device__ __forceinline__ __nv_bfloat16 from_f32<__nv_bfloat16>(float x) {
+    return __float2bfloat16_rn(x);  // round to nearest even
+}
+
+// Sequence n's token range [bos, bos + len) in the flattened [B*T] token axis.
+// A packed table is clamped into [0, T] so a malformed one cannot send a
+// kernel out of bounds.
+__device__ __forceinline__ void seq_range(const int32_t* __restrict__ cu_seqlens, int n, int64_t T,
+                                          int64_t& bos, int64_t& len) {
+    if (cu_seqlens == nullptr) {
+        bos = (int64_t)n * T;
+        len = T;
+        return;
+    }
+    int64_t a = cu_seqlens[n], b = cu_seqlens[n + 1];
+    a = a < 0 ? 0 : (a > T ? T : a);
+    b = b < a ? a : (b > T ? T : b);
+    bos = a;
+    len = b - a;
+}
+
+}  // namespace kda

@@ -1,0 +1,134 @@
+// KDA single-token decode step: the fixed-size state replaces the KV cache
+// (worldcybernews article "Kimi K3 Open Model Surpasses Closed GPT and
+// Anthropic Systems on Independent Benchmarks", paragraph 2).
+//
+// For each (sequence, head), with a = clamp(alpha, e^-5, 1):
+//   S_t = (I - beta k k^T) Diag(a) S + beta k v^T,   o = S_t^T q
+// is computed in ONE pass over S (read once, written once):
+//   x = S^T (a*k),  y = S^T (a*q)           (column sums over key channels)
+//   u = beta (v - x)
+//   o = y + u (k . q)
+//   S <- Diag(a) S + k u^T
+// which expands to the same S_t (Diag(a)S - beta k (k^T Diag(a) S) + beta k v^T)
+// and o_t = S_t^T q = (Diag(a) S)^T q + u (k^T q).
+//
+// The state is fp32 and HBM-bound: one CTA per (sequence, head) streams its
+// d_k x d_v slab with 16-byte loads and stores, keeping it in registers between
+// the reduction and the update.
+#include "kda_common.cuh"
+
+namespace kda {
+
+template <typename Tin, typename Tout, int DK, int DV>
+__global__ void __launch_bounds__(256)
+kda_decode_kernel(const Tin* __restrict__ q, const Tin* __restrict__ k,
+                  const Tin* __restrict__ v, const Tin* __restrict__ alpha,
+                  const Tin* __restrict__ beta, float* __restrict__ S, Tout* __restrict__ out) {
+    constexpr int NT = 256;
+    constexpr int TX = DV / 4;       // threads across a row (float4 each)
+    constexpr int TY = NT / TX;      // rows per pass
+    constexpr int RPT = DK / TY;     // rows per thread
+    static_assert(DV % 4 == 0 && NT % TX == 0 && DK % TY == 0, "tile");
+    __shared__ float ka[DK], qa[DK], kk[DK], ga[DK];
+    __shared__ float red_x[TY][DV], red_y[TY][DV];
+    __shared__ float us[DV];
+    __shared__ float kq_part[NT / 32];
+
+    const int tid = threadIdx.x, tx = tid % TX, ty = tid / TX;
+    const size_t nh = blockIdx.x;                 // (sequence, head) flattened
+    const size_t kb = nh * DK, vb = nh * DV;
+    float4* Sv = reinterpret_cast<float4*>(S + nh * (size_t)DK * DV);
+
+    // issue the state loads first: they are the HBM traffic
+    float4 s[RPT];
+#pragma unroll
+    for (int i = 0; i < RPT; ++i) s[i] = Sv[(size_t)(ty + TY * i) * TX + tx];
+
+    float kqp = 0.0f;
+    if (tid < DK) {
+        const float a = clamp_gate(to_f32(alpha[kb + tid]));
+        const float kv = to_f32(k[kb + tid]), qv = to_f32(q[kb + tid]);
+        ga[tid] = a;
+        ka[tid] = a * kv;
+        qa[tid] = a * qv;
+        kk[tid] = kv;
+        kqp = kv * qv;
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) kqp += __shfl_xor_sync(0xffffffffu, kqp, o);
+    if ((tid & 31) == 0) kq_part[tid >> 5] = kqp;
+    __syncthreads();
+
+    float4 px = make_float4(0.f, 0.f, 0.f, 0.f), py = px;
+#pragma unroll
+    for (int i = 0; i < RPT; ++i) {
+        const int c = ty + TY * i;
+        const float wk = ka[c], wq = qa[c];
+        px.x = fmaf(s[i].x, wk, px.x); px.y = fmaf(s[i].y, wk, px.y);
+        px.z = fmaf(s[i].z, wk, px.z); px.w = fmaf(s[i].w, wk, px.w);
+        py.x = fmaf(s[i].x, wq, py.x); py.y = fmaf(s[i].y, wq, py.y);
+        py.z = fmaf(s[i].z, wq, py.z); py.w = fmaf(s[i].w, wq, py.w);
+    }
+    *reinterpret_cast<float4*>(&red_x[ty][4 * tx]) = px;
+    *reinterpret_cast<float4*>(&red_y[ty][4 * tx]) = py;
+    __syncthreads();
+
+    if (tid < DV) {
+        float x = 0.0f, y = 0.0f;
+#pragma unroll
+        for (int i = 0; i < TY; ++i) { x += red_x[i][tid]; y += red_y[i][tid]; }
+        float kq = 0.0f;
+#pragma unroll
+        for (int i = 0; i < NT / 32; ++i) kq += kq_part[i];
+        const float b = to_f32(beta[nh]);
+        const float u = b * (to_f32(v[vb + tid]) - x);
+        us[tid] = u;
+        out[vb + tid] = from_f32<Tout>(fmaf(u, kq, y));
+    }
+    __syncthreads();
+
+    const float4 u4 = *reinterpret_cast<const float4*>(&us[4 * tx]);
+#pragma unroll
+    for (int i = 0; i < RPT; ++i) {
+        const int c = ty + TY * i;
+        const float a = ga[c];
+        const float kc = kk[c];
+        float4 r;
+        r.x = fmaf(a, s[i].x, kc * u4.x);
+        r.y = fmaf(a, s[i].y, kc * u4.y);
+        r.z = fmaf(a, s[i].z, kc * u4.z);
+        r.w = fmaf(a, s[i].w, kc * u4.w);
+        Sv[(size_t)c * TX + tx] = r;
+    }
+}
+
+template <typename Tin, typename Tout, int DK, int DV>
+static cudaError_t launch_decode_t(const void* q, const void* k, const void* v, const void* alpha,
+                                   const void* beta, float* S, void* out, int64_t NH,
+                                   cudaStream_t stream) {
+    kda_decode_kernel<Tin, Tout, DK, DV><<<(unsigned)NH, 256, 0, stream>>>(
+        (const Tin*)q, (const Tin*)k, (const Tin*)v, (const Tin*)alpha, (const Tin*)beta, S,
+        (Tout*)out);
+    return cudaGetLastError();
+}
+
+template <typename Tin, typename Tout>
+static cudaError_t launch_decode_d(int DK, int DV, const void* q, const void* k, const void* v,
+                                   const void* alpha, const void* beta, float* S, void* out,
+                                   int64_t NH, cudaStream_t s) {
+    if (DK == 64 && DV == 64) return launch_decode_t<Tin, Tout, 64, 64>(q, k, v, alpha, beta, S, out, NH, s);
+    if (DK == 64 && DV == 128) return launch_decode_t<Tin, Tout, 64, 128>(q, k, v, alpha, beta, S, out, NH, s);
+    if (DK == 128 && DV == 64) return launch_decode_t<Tin, Tout, 128, 64>(q, k, v, alpha, beta, S, out, NH, s);
+    return launch_decode_t<Tin, Tout, 128, 128>(q, k, v, alpha, beta, S, out, NH, s);
+}
+
+cudaError_t launch_decode(int in_bf16, int out_bf16, const void* q, const void* k, const void* v,
+                          const void* alpha, const void* beta, float* S, void* out, int64_t NH,
+                          int DK, int DV, cudaStream_t s) {
+    if (!in_bf16 && !out_bf16) return launch_decode_d<float, float>(DK, DV, q, k, v, alpha, beta, S, out, NH, s);
+    if (!in_bf16 && out_bf16) return launch_decode_d<float, __nv_bfloat16>(DK, DV, q, k, v, alpha, beta, S, out, NH, s);
+    if (in_bf16 && !out_bf16) return launch_decode_d<__nv_bfloat16, float>(DK, DV, q, k, v, alpha, beta, S, out, NH, s);
+    return launch_decode_d<__nv_bfloat16, __nv_bfloat16>(DK, DV, q, k, v, alpha, beta, S, out, NH, s);
+}
+
+}  // namespace kda

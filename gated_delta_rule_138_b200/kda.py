@@ -1,0 +1,194 @@
+"""Thin ctypes binding of libkda.so (include/kda.h), same entry-point names.
+
+Argument marshalling only: shapes and dtypes are read off torch tensors, the
+device pointers and the current CUDA stream are passed to the C ABI, and a
+non-OK status raises KdaError.  Every step of the computation runs in the
+library's CUDA kernels; there is no other implementation to fall back to.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+from typing import Optional, Tuple
+
+import torch
+
+HERE = os.path.dirname(os.path.abspath(__file__))
+_LIB_NAME = "libkda.so"
+
+KDA_F32, KDA_BF16 = 0, 1
+_STATUS = {0: "KDA_OK", 1: "KDA_ERR_INVALID_ARG", 2: "KDA_ERR_UNSUPPORTED",
+           3: "KDA_ERR_CUDA", 4: "KDA_ERR_DEVICE_TIMEOUT"}
+
+
+class KdaError(RuntimeError):
+    def __init__(self, fn: str, status: int, detail: str = ""):
+        self.status = status
+        msg = "%s failed: %s" % (fn, _STATUS.get(status, "status %d" % status))
+        if detail:
+            msg += " (%s)" % detail
+        super().__init__(msg)
+
+
+_lib = None
+
+
+def library_path() -> str:
+    return os.path.join(HERE, _LIB_NAME)
+
+
+def load_library(build_if_missing: bool = True) -> ctypes.CDLL:
+    """Load libkda.so, building it first if it is absent and nvcc is present.
+
+    Raises KdaError if the library cannot be found or built: there is no
+    non-CUDA path.
+    """
+    global _lib
+    if _lib is not None:
+        return _lib
+    path = library_path()
+    if build_if_missing:
+        try:
+            from . import build as _build
+            path = _build.build()
+        except (OSError, FileNotFoundError) as exc:
+            if not os.path.exists(path):
+                raise KdaError("load_library", -1, "libkda.so missing and not buildable: %s" % exc)
+    if not os.path.exists(path):
+        raise KdaError("load_library", -1, "libkda.so not found at %s" % path)
+    lib = ctypes.CDLL(path)
+    vp, i32, i64 = ctypes.c_void_p, ctypes.c_int32, ctypes.c_int64
+    lib.kda_forward.restype = ctypes.c_int
+    lib.kda_forward.argtypes = [vp, vp, vp, vp, vp, vp, vp, i32, vp, vp,
+                                i32, i64, i32, i32, i32, i32, ctypes.c_int, ctypes.c_int, vp]
+    lib.kda_decode_step.restype = ctypes.c_int
+    lib.kda_decode_step.argtypes = [vp, vp, vp, vp, vp, vp, vp, i32, i32, i32, i32,
+                                    ctypes.c_int, ctypes.c_int, vp]
+    lib.kda_status_string.restype = ctypes.c_char_p
+    lib.kda_status_string.argtypes = [ctypes.c_int]
+    lib.kda_forward_workspace_bytes.restype = ctypes.c_size_t
+    lib.kda_forward_workspace_bytes.argtypes = [i32, i64, i32, i32, i32, i32]
+    lib.kda_last_error.restype = ctypes.c_char_p
+    lib.kda_last_error.argtypes = []
+    lib.kda_forward_kernel_name.restype = ctypes.c_char_p
+    lib.kda_forward_kernel_name.argtypes = [i32, i32, i32, ctypes.c_int, ctypes.c_int]
+    lib.kda_launch_count.restype = ctypes.c_uint64
+    lib.kda_launch_count.argtypes = []
+    _lib = lib
+    return lib
+
+
+def _dt(t: torch.Tensor) -> int:
+    if t.dtype == torch.float32:
+        return KDA_F32
+    if t.dtype == torch.bfloat16:
+        return KDA_BF16
+    raise TypeError("unsupported dtype %s (fp32 or bf16)" % t.dtype)
+
+
+def _ptr(t: Optional[torch.Tensor]):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _stream(stream) -> ctypes.c_void_p:
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    return ctypes.c_void_p(stream.cuda_stream)
+
+
+def _check(fn: str, status: int):
+    if status != 0:
+        lib = load_library(False)
+        raise KdaError(fn, status, lib.kda_last_error().decode())
+
+
+def kda_status_string(status: int) -> str:
+    return load_library().kda_status_string(int(status)).decode()
+
+
+def kda_forward_workspace_bytes(B: int, T: int, H: int, d_k: int, d_v: int, chunk: int = 64) -> int:
+    return int(load_library().kda_forward_workspace_bytes(B, T, H, d_k, d_v, chunk))
+
+
+def kda_forward_kernel_name(d_k: int, d_v: int, chunk: int, in_dtype: torch.dtype,
+                            out_dtype: Optional[torch.dtype] = None) -> Optional[str]:
+    """Kernel kda_forward would run for these sizes and dtypes (None = rejected)."""
+    code = lambda d: KDA_F32 if d == torch.float32 else KDA_BF16
+    r = load_library().kda_forward_kernel_name(d_k, d_v, chunk, code(in_dtype),
+                                                code(out_dtype or in_dtype))
+    return None if r is None else r.decode()
+
+
+def kda_launch_count() -> int:
+    """Kernels launched by the library so far in this process."""
+    return int(load_library().kda_launch_count())
+
+
+def _contig(name, t):
+    if t is not None and not t.is_contiguous():
+        raise ValueError("%s must be contiguous" % name)
+
+
+def kda_forward(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, alpha: torch.Tensor,
+                beta: torch.Tensor, S0: Optional[torch.Tensor] = None,
+                cu_seqlens: Optional[torch.Tensor] = None, out: Optional[torch.Tensor] = None,
+                S_final: Optional[torch.Tensor] = None, chunk: int = 64,
+                out_dtype: Optional[torch.dtype] = None, want_state: bool = True,
+                stream=None) -> Tuple[torch.Tensor, Optional[torch.Tensor]]:
+    """KDA forward (chunk-parallel) through the C ABI.
+
+    q, k, alpha [B, T, H, d_k]; v [B, T, H, d_v]; beta [B, T, H] (fp32 or bf16,
+    one dtype); S0 fp32 [N, H, d_k, d_v] or None; cu_seqlens int32 [N + 1] or
+    None (packed batch, B == 1).  Returns (out [B, T, H, d_v], S_final or None).
+    """
+    lib = load_library()
+    B, T, H, dk = q.shape
+    dv = v.shape[-1]
+    if k.shape != q.shape or alpha.shape != q.shape or v.shape != (B, T, H, dv) \
+            or beta.shape != (B, T, H):
+        raise ValueError("inconsistent shapes")
+    dts = {q.dtype, k.dtype, v.dtype, alpha.dtype, beta.dtype}
+    if len(dts) != 1:
+        raise TypeError("q, k, v, alpha, beta must share one dtype")
+    for name, t in (("q", q), ("k", k), ("v", v), ("alpha", alpha), ("beta", beta),
+                    ("S0", S0), ("cu_seqlens", cu_seqlens)):
+        _contig(name, t)
+    nseq = B if cu_seqlens is None else cu_seqlens.numel() - 1
+    if cu_seqlens is not None and cu_seqlens.dtype != torch.int32:
+        raise TypeError("cu_seqlens must be int32")
+    if S0 is not None and (S0.dtype != torch.float32 or tuple(S0.shape) != (nseq, H, dk, dv)):
+        raise ValueError("S0 must be fp32 [N, H, d_k, d_v]")
+    od = out_dtype or q.dtype
+    if out is None:
+        out = torch.empty(B, T, H, dv, dtype=od, device=q.device)
+    if S_final is None and want_state:
+        S_final = torch.empty(nseq, H, dk, dv, dtype=torch.float32, device=q.device)
+    st = lib.kda_forward(_ptr(q), _ptr(k), _ptr(v), _ptr(alpha), _ptr(beta), _ptr(S0),
+                         _ptr(cu_seqlens), int(nseq), _ptr(out), _ptr(S_final),
+                         int(B), int(T), int(H), int(dk), int(dv), int(chunk),
+                         _dt(q), _dt(out), _stream(stream))
+    _check("kda_forward", st)
+    return out, S_final
+
+
+def kda_decode_step(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, alpha: torch.Tensor,
+                    beta: torch.Tensor, S: torch.Tensor, out: Optional[torch.Tensor] = None,
+                    out_dtype: Optional[torch.dtype] = None, stream=None) -> torch.Tensor:
+    """One decode step through the C ABI; S (fp32 [N, H, d_k, d_v]) is updated in place.
+
+    q, k, alpha [N, H, d_k]; v [N, H, d_v]; beta [N, H].  Returns out [N, H, d_v].
+    """
+    lib = load_library()
+    N, H, dk = q.shape
+    dv = v.shape[-1]
+    if S.dtype != torch.float32 or tuple(S.shape) != (N, H, dk, dv):
+        raise ValueError("S must be fp32 [N, H, d_k, d_v]")
+    for name, t in (("q", q), ("k", k), ("v", v), ("alpha", alpha), ("beta", beta), ("S", S)):
+        _contig(name, t)
+    if out is None:
+        out = torch.empty(N, H, dv, dtype=out_dtype or q.dtype, device=q.device)
+    st = lib.kda_decode_step(_ptr(q), _ptr(k), _ptr(v), _ptr(alpha), _ptr(beta), _ptr(S),
+                             _ptr(out), int(N), int(H), int(dk), int(dv), _dt(q), _dt(out),
+                             _stream(stream))
+    _check("kda_decode_step", st)
+    return out

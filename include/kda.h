@@ -1,0 +1,143 @@
+/*
+ * kda.h -- C ABI of libkda.so: the KDA (Kimi Delta Attention) forward pass and
+ * single-token decode step on NVIDIA B200 (sm_100a).
+ *
+ * The method.  The worldcybernews article "Kimi K3 Open Model Surpasses Closed
+ * GPT and Anthropic Systems on Independent Benchmarks", paragraph 2, replaces
+ * the KV cache by a fixed-size state matrix S per head, updated by the delta
+ * rule with a write strength beta and a forgetting coefficient alpha that is
+ * clamped between e^-5 and 1.  Paragraph 3 of the same article processes the
+ * tokens of a chunk in parallel and reconstructs the sequential states across
+ * chunks with a prefix scan.  The page prints no equation; this library
+ * computes, per sequence and head, with alpha per key channel:
+ *
+ *     a_t = clamp(alpha_t, e^-5, 1)                               [d_k]
+ *     S_t = (I - beta_t k_t k_t^T) Diag(a_t) S_{t-1} + beta_t k_t v_t^T   [d_k x d_v]
+ *     o_t = S_t^T q_t                                             [d_v]
+ *
+ * No query scale and no normalisation are applied: q and k are used as given.
+ *
+ * Conventions shared by every entry point:
+ *   - All tensor pointers are DEVICE pointers owned by the caller; the library
+ *     never frees or retains them beyond the call.
+ *   - Row-major layouts, innermost dimension last, no padding.
+ *   - Calls are asynchronous on `stream` (NULL = legacy default stream); no
+ *     entry point synchronises the device except where stated.
+ *   - Arguments are validated before anything is launched; a rejected call has
+ *     no side effects.  Nothing is thrown across the ABI.
+ *   - Every pointer must be 16-byte aligned.
+ */
+#ifndef KDA_H_
+#define KDA_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* Same handle type as cudaStream_t / CUstream. */
+typedef struct CUstream_st* kda_stream_t;
+
+typedef enum {
+    KDA_F32 = 0,   /* IEEE binary32 */
+    KDA_BF16 = 1   /* bfloat16 */
+} kda_dtype_t;
+
+typedef enum {
+    KDA_OK = 0,
+    KDA_ERR_INVALID_ARG = 1,     /* a NULL, misaligned or inconsistent argument */
+    KDA_ERR_UNSUPPORTED = 2,     /* valid, but a size or dtype this build has no kernel for */
+    KDA_ERR_CUDA = 3,            /* a CUDA runtime error (launch or device) */
+    KDA_ERR_DEVICE_TIMEOUT = 4   /* a bounded device-side wait gave up */
+} kda_status_t;
+
+/*
+ * kda_forward -- chunk-parallel KDA forward over whole sequences (prefill).
+ * Article paragraph 2 (the update) and paragraph 3 (chunk-parallel processing
+ * with sequential states reconstructed across chunks).
+ *
+ *   q, k, alpha : [B, T, H, d_k]   in_dtype
+ *   v           : [B, T, H, d_v]   in_dtype
+ *   beta        : [B, T, H]        in_dtype
+ *   S0          : NULL (zero initial state) or fp32 [N, H, d_k, d_v]
+ *   cu_seqlens  : NULL for a dense batch (N = B sequences of T tokens), or
+ *                 int32 [num_seqs + 1] for a packed batch: B must be 1,
+ *                 N = num_seqs, sequence n owns tokens [cu_seqlens[n],
+ *                 cu_seqlens[n+1]), cu_seqlens[0] = 0, cu_seqlens[num_seqs] = T,
+ *                 non-decreasing.  cu_seqlens is device memory and only the
+ *                 kernels read it; each kernel clamps the offsets it reads into
+ *                 [0, T] (a malformed table gives wrong results, never an
+ *                 out-of-bounds access).
+ *   out         : [B, T, H, d_v]   out_dtype (written for every token)
+ *   S_final     : NULL or fp32 [N, H, d_k, d_v]; the state after each
+ *                 sequence's last token.  May alias S0 exactly (in-place update);
+ *                 any other overlap is undefined.
+ *   chunk       : tokens per chunk: 64 (16 and 32 are accepted by the fp32 path).
+ *   in_dtype    : KDA_F32 or KDA_BF16 for q, k, v, alpha, beta.
+ *   out_dtype   : KDA_F32 or KDA_BF16.
+ *
+ * Supported: d_k, d_v in {64, 128}; H >= 1; T >= 0 (T = 0 only writes S_final
+ * = S0).  bf16 inputs with d_k = d_v = 128 and chunk 64 run on the
+ * tensor-core (tcgen05) kernel; every other supported combination runs on the
+ * fp32 CUDA-core kernel.
+ * Returns KDA_OK, KDA_ERR_INVALID_ARG, KDA_ERR_UNSUPPORTED or KDA_ERR_CUDA.
+ */
+kda_status_t kda_forward(const void* q, const void* k, const void* v,
+                         const void* alpha, const void* beta, const float* S0,
+                         const int32_t* cu_seqlens, int32_t num_seqs,
+                         void* out, float* S_final,
+                         int32_t B, int64_t T, int32_t H, int32_t d_k, int32_t d_v,
+                         int32_t chunk, kda_dtype_t in_dtype, kda_dtype_t out_dtype,
+                         kda_stream_t stream);
+
+/*
+ * kda_decode_step -- one token for each of N sequences, the state updated in
+ * place (the fixed-size state that replaces the KV cache, article paragraph 2).
+ *
+ *   q, k, alpha : [N, H, d_k]      in_dtype
+ *   v           : [N, H, d_v]      in_dtype
+ *   beta        : [N, H]           in_dtype
+ *   S           : fp32 [N, H, d_k, d_v], read and overwritten with S_t
+ *   out         : [N, H, d_v]      out_dtype, o_t = S_t^T q_t
+ *
+ * Supported: d_k, d_v in {64, 128}.  Returns as kda_forward.
+ */
+kda_status_t kda_decode_step(const void* q, const void* k, const void* v,
+                             const void* alpha, const void* beta, float* S, void* out,
+                             int32_t N, int32_t H, int32_t d_k, int32_t d_v,
+                             kda_dtype_t in_dtype, kda_dtype_t out_dtype,
+                             kda_stream_t stream);
+
+/* A static, human-readable name for a status code (never NULL). */
+const char* kda_status_string(kda_status_t status);
+
+/*
+ * Bytes of device workspace kda_forward uses for these sizes.  The library
+ * allocates and owns it; the figure is reported for capacity planning.
+ */
+size_t kda_forward_workspace_bytes(int32_t B, int64_t T, int32_t H, int32_t d_k,
+                                   int32_t d_v, int32_t chunk);
+
+/* Text of the last CUDA error seen by this thread's calls ("" if none). */
+const char* kda_last_error(void);
+
+/*
+ * Name of the kernel kda_forward would launch for these arguments, or NULL if
+ * it would reject them: "chunk_tc_bf16" (tcgen05 tensor-core kernel) or
+ * "chunk_simt_f32" (fp32 CUDA-core kernel).  Host-only, launches nothing.
+ */
+const char* kda_forward_kernel_name(int32_t d_k, int32_t d_v, int32_t chunk,
+                                    kda_dtype_t in_dtype, kda_dtype_t out_dtype);
+
+/*
+ * Number of kernels this library has launched in this process (all entry
+ * points, all threads).  A host-side counter, for accounting in benchmarks.
+ */
+uint64_t kda_launch_count(void);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* KDA_H_ */

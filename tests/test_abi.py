@@ -1,0 +1,89 @@
+"""The C-ABI library loads without a GPU, exports every entry point the header
+declares, and rejects bad arguments before launching anything."""
+import ctypes
+import os
+import re
+
+import pytest
+
+import gated_delta_rule_138_b200 as kda
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def _declared_symbols():
+    names = set()
+    for fn in os.listdir(os.path.join(ROOT, "include")):
+        if fn.endswith(".h"):
+            src = open(os.path.join(ROOT, "include", fn)).read()
+            src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+            names |= set(re.findall(r"\b(kda_\w+)\s*\(", src))
+    return names
+
+
+def test_header_declares_the_entry_points():
+    names = _declared_symbols()
+    for want in ("kda_forward", "kda_decode_step", "kda_status_string",
+                 "kda_forward_workspace_bytes", "kda_last_error"):
+        assert want in names
+
+
+def test_library_exports_every_declared_symbol():
+    lib = kda.load_library()
+    missing = [n for n in sorted(_declared_symbols()) if not hasattr(lib, n)]
+    assert not missing, missing
+
+
+def test_status_strings():
+    assert kda.kda_status_string(0) == "KDA_OK"
+    assert kda.kda_status_string(1) == "KDA_ERR_INVALID_ARG"
+    assert kda.kda_status_string(2) == "KDA_ERR_UNSUPPORTED"
+    assert kda.kda_status_string(3) == "KDA_ERR_CUDA"
+    assert kda.kda_status_string(4) == "KDA_ERR_DEVICE_TIMEOUT"
+    assert kda.kda_status_string(99) == "KDA_ERR_UNKNOWN"
+
+
+def _fwd_raw(**over):
+    """Call kda_forward with fake (never dereferenced) aligned pointers."""
+    lib = kda.load_library()
+    p = ctypes.c_void_p(0x10000)
+    args = dict(q=p, k=p, v=p, alpha=p, beta=p, S0=None, cu=None, nseq=0, out=p, Sf=None,
+                B=1, T=64, H=1, dk=64, dv=64, chunk=64, idt=0, odt=0)
+    args.update(over)
+    return lib.kda_forward(args["q"], args["k"], args["v"], args["alpha"], args["beta"],
+                           args["S0"], args["cu"], args["nseq"], args["out"], args["Sf"],
+                           args["B"], args["T"], args["H"], args["dk"], args["dv"],
+                           args["chunk"], args["idt"], args["odt"], None)
+
+
+@pytest.mark.parametrize("over,status", [
+    (dict(H=0), 1),                                  # no heads
+    (dict(B=-1), 1),
+    (dict(T=-5), 1),
+    (dict(idt=7), 1),                                # unknown dtype
+    (dict(q=None), 1),                               # missing input with tokens
+    (dict(q=ctypes.c_void_p(0x10002)), 1),           # misaligned
+    (dict(cu=ctypes.c_void_p(0x20000), B=2, nseq=1), 1),  # packed needs B == 1
+    (dict(dk=96), 2),                                # head dim without a kernel
+    (dict(dv=256), 2),
+    (dict(chunk=48), 2),
+    (dict(B=0), 0),                                  # nothing to do: OK, no launch
+])
+def test_forward_rejects_before_launch(over, status):
+    assert _fwd_raw(**over) == status
+
+
+def test_decode_rejects_before_launch():
+    lib = kda.load_library()
+    p = ctypes.c_void_p(0x10000)
+    call = lambda N=1, H=1, dk=128, dv=128, q=p, S=p: lib.kda_decode_step(
+        q, p, p, p, p, S, p, N, H, dk, dv, 1, 1, None)
+    assert call(H=0) == 1
+    assert call(q=None) == 1
+    assert call(S=ctypes.c_void_p(0x10008)) == 1
+    assert call(dk=32) == 2
+    assert call(N=0) == 0
+
+
+def test_workspace_query_is_host_only():
+    assert kda.kda_forward_workspace_bytes(8, 4096, 32, 128, 128, 64) >= 0
