@@ -31,6 +31,7 @@ kda_status_t cuda_status(cudaError_t e) {
 }
 
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+bool aligned_to(const void* p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p) & (a - 1)) == 0; }
 bool is_dtype(kda_dtype_t d) { return d == KDA_F32 || d == KDA_BF16; }
 bool head_dim_ok(int32_t d) { return d == 64 || d == 128; }
 
@@ -78,9 +79,11 @@ kda_status_t kda_forward(const void* q, const void* k, const void* v, const void
     const int64_t nseq = cu_seqlens ? (int64_t)num_seqs : (int64_t)B;
     const bool has_tokens = (int64_t)B * T > 0;
     if (has_tokens && (!q || !k || !v || !alpha || !beta || !out)) return KDA_ERR_INVALID_ARG;
-    const void* ptrs[] = {q, k, v, alpha, beta, S0, cu_seqlens, out, S_final};
+    const void* ptrs[] = {q, k, v, alpha, S0, out, S_final};
     for (const void* p : ptrs)
         if (p && !aligned16(p)) return KDA_ERR_INVALID_ARG;
+    if (!aligned_to(beta, in_dtype == KDA_BF16 ? 2 : 4) || !aligned_to(cu_seqlens, 4))
+        return KDA_ERR_INVALID_ARG;
     if (!head_dim_ok(d_k) || !head_dim_ok(d_v)) return KDA_ERR_UNSUPPORTED;
     if (chunk != 16 && chunk != 32 && chunk != 64) return KDA_ERR_UNSUPPORTED;
     if (nseq > 65535 || H > 65535) return KDA_ERR_UNSUPPORTED;  // grid y/z limits
@@ -101,9 +104,12 @@ kda_status_t kda_decode_step(const void* q, const void* k, const void* v, const 
     if (N < 0 || H <= 0 || !is_dtype(in_dtype) || !is_dtype(out_dtype))
         return KDA_ERR_INVALID_ARG;
     if (N > 0 && (!q || !k || !v || !alpha || !beta || !S || !out)) return KDA_ERR_INVALID_ARG;
-    const void* ptrs[] = {q, k, v, alpha, beta, S, out};
-    for (const void* p : ptrs)
-        if (p && !aligned16(p)) return KDA_ERR_INVALID_ARG;
+    // S is streamed with 16-byte accesses; the per-token vectors are read element-wise
+    const int es = in_dtype == KDA_BF16 ? 2 : 4;
+    if (S && !aligned16(S)) return KDA_ERR_INVALID_ARG;
+    if (!aligned_to(q, es) || !aligned_to(k, es) || !aligned_to(v, es) || !aligned_to(alpha, es) ||
+        !aligned_to(beta, es) || !aligned_to(out, out_dtype == KDA_BF16 ? 2 : 4))
+        return KDA_ERR_INVALID_ARG;
     if (!head_dim_ok(d_k) || !head_dim_ok(d_v)) return KDA_ERR_UNSUPPORTED;
     const int64_t NH = (int64_t)N * H;
     if (NH > 0x7fffffffLL) return KDA_ERR_UNSUPPORTED;

@@ -25,7 +25,9 @@
  *     entry point synchronises the device except where stated.
  *   - Arguments are validated before anything is launched; a rejected call has
  *     no side effects.  Nothing is thrown across the ABI.
- *   - Every pointer must be 16-byte aligned.
+ *   - Alignment: kda_forward's q, k, v, alpha, S0, out and S_final and
+ *     kda_decode_step's S must be 16-byte aligned; every other pointer must be
+ *     aligned to its element size.  A misaligned pointer is KDA_ERR_INVALID_ARG.
  */
 #ifndef KDA_H_
 #define KDA_H_

@@ -62,7 +62,8 @@ def _fwd_raw(**over):
     (dict(T=-5), 1),
     (dict(idt=7), 1),                                # unknown dtype
     (dict(q=None), 1),                               # missing input with tokens
-    (dict(q=ctypes.c_void_p(0x10002)), 1),           # misaligned
+    (dict(q=ctypes.c_void_p(0x10002)), 1),           # q misaligned (needs 16 bytes)
+    (dict(beta=ctypes.c_void_p(0x10001)), 1),        # beta not element-aligned
     (dict(cu=ctypes.c_void_p(0x20000), B=2, nseq=1), 1),  # packed needs B == 1
     (dict(dk=96), 2),                                # head dim without a kernel
     (dict(dv=256), 2),
@@ -80,7 +81,7 @@ def test_decode_rejects_before_launch():
         q, p, p, p, p, S, p, N, H, dk, dv, 1, 1, None)
     assert call(H=0) == 1
     assert call(q=None) == 1
-    assert call(S=ctypes.c_void_p(0x10008)) == 1
+    assert call(S=ctypes.c_void_p(0x10008)) == 1       # S needs 16 bytes
     assert call(dk=32) == 2
     assert call(N=0) == 0
 
