@@ -3,7 +3,9 @@
 // beyond the library-owned workspace, synchronises the device, or throws.
 #include <atomic>
 #include <cstdio>
+#include <cstdlib>
 #include <cstring>
+#include <mutex>
 
 #include "../../include/kda.h"
 #include "kda_common.cuh"
@@ -16,6 +18,10 @@ cudaError_t launch_chunk_simt(int in_bf16, int out_bf16, int chunk, const void* 
 cudaError_t launch_decode(int in_bf16, int out_bf16, const void* q, const void* k, const void* v,
                           const void* alpha, const void* beta, float* S, void* out, int64_t NH,
                           int DK, int DV, cudaStream_t s);
+cudaError_t launch_chunk_tc(const void* q, const void* k, const void* v, const void* alpha,
+                            const void* beta, const float* S0, const int32_t* cu, int nseq,
+                            void* out, float* S_final, int64_t rows, int64_t T, int H, int* status,
+                            cudaStream_t stream);
 }  // namespace kda
 
 namespace {
@@ -34,6 +40,38 @@ bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) ==
 bool aligned_to(const void* p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p) & (a - 1)) == 0; }
 bool is_dtype(kda_dtype_t d) { return d == KDA_F32 || d == KDA_BF16; }
 bool head_dim_ok(int32_t d) { return d == 64 || d == 128; }
+
+bool use_tc(int32_t d_k, int32_t d_v, int32_t chunk, kda_dtype_t in, kda_dtype_t out) {
+    return in == KDA_BF16 && out == KDA_BF16 && d_k == 128 && d_v == 128 && chunk == 64;
+}
+
+// One device status word per GPU: kernels set it when a bounded wait gives up.
+constexpr int kMaxDevices = 64;
+std::mutex g_status_mu;
+int* g_status[kMaxDevices] = {};
+
+cudaError_t device_status_word(int** out) {
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return e;
+    if (dev < 0 || dev >= kMaxDevices) return cudaErrorInvalidDevice;
+    std::lock_guard<std::mutex> lock(g_status_mu);
+    if (!g_status[dev]) {
+        int* p = nullptr;
+        e = cudaMalloc(&p, sizeof(int));
+        if (e != cudaSuccess) return e;
+        e = cudaMemset(p, 0, sizeof(int));
+        if (e != cudaSuccess) { cudaFree(p); return e; }
+        g_status[dev] = p;
+    }
+    *out = g_status[dev];
+    return cudaSuccess;
+}
+
+bool debug_sync() {
+    const char* v = std::getenv("KDA_DEBUG");
+    return v && v[0] && v[0] != '0';
+}
 
 }  // namespace
 
@@ -59,13 +97,30 @@ const char* kda_forward_kernel_name(int32_t d_k, int32_t d_v, int32_t chunk,
     if (!is_dtype(in_dtype) || !is_dtype(out_dtype)) return nullptr;
     if (!head_dim_ok(d_k) || !head_dim_ok(d_v)) return nullptr;
     if (chunk != 16 && chunk != 32 && chunk != 64) return nullptr;
-    return "chunk_simt_f32";
+    return use_tc(d_k, d_v, chunk, in_dtype, out_dtype) ? "chunk_tc_bf16" : "chunk_simt_f32";
+}
+
+kda_status_t kda_device_status(kda_stream_t stream) {
+    int* word = nullptr;
+    cudaError_t e = device_status_word(&word);
+    if (e != cudaSuccess) return cuda_status(e);
+    e = cudaStreamSynchronize(reinterpret_cast<cudaStream_t>(stream));
+    if (e != cudaSuccess) return cuda_status(e);
+    int v = 0;
+    e = cudaMemcpy(&v, word, sizeof(int), cudaMemcpyDeviceToHost);
+    if (e != cudaSuccess) return cuda_status(e);
+    if (v != 0) {
+        e = cudaMemset(word, 0, sizeof(int));
+        if (e != cudaSuccess) return cuda_status(e);
+        return KDA_ERR_DEVICE_TIMEOUT;
+    }
+    return KDA_OK;
 }
 
 size_t kda_forward_workspace_bytes(int32_t B, int64_t T, int32_t H, int32_t d_k, int32_t d_v,
                                    int32_t chunk) {
     (void)B; (void)T; (void)H; (void)d_k; (void)d_v; (void)chunk;
-    return 0;
+    return sizeof(int);  // the per-device status word, allocated once
 }
 
 kda_status_t kda_forward(const void* q, const void* k, const void* v, const void* alpha,
@@ -92,6 +147,17 @@ kda_status_t kda_forward(const void* q, const void* k, const void* v, const void
     const cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
     const int in_bf16 = in_dtype == KDA_BF16, out_bf16 = out_dtype == KDA_BF16;
     g_launches.fetch_add(1, std::memory_order_relaxed);
+    if (use_tc(d_k, d_v, chunk, in_dtype, out_dtype)) {
+        int* status = nullptr;
+        cudaError_t e = device_status_word(&status);
+        if (e != cudaSuccess) return cuda_status(e);
+        const int64_t rows = cu_seqlens ? T : (int64_t)B * T;
+        if (rows > 0x7fffffffLL) return KDA_ERR_UNSUPPORTED;  // TMA row coordinate is int32
+        e = kda::launch_chunk_tc(q, k, v, alpha, beta, S0, cu_seqlens, (int)nseq, out, S_final,
+                                 rows, T, H, status, s);
+        if (e != cudaSuccess) return cuda_status(e);
+        return debug_sync() ? kda_device_status(stream) : KDA_OK;
+    }
     return cuda_status(kda::launch_chunk_simt(in_bf16, out_bf16, chunk, q, k, v, alpha, beta, S0,
                                               cu_seqlens, (int)nseq, out, S_final, T, H, d_k, d_v,
                                               s));

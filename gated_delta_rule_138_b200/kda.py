@@ -74,6 +74,8 @@ def load_library(build_if_missing: bool = True) -> ctypes.CDLL:
     lib.kda_forward_kernel_name.argtypes = [i32, i32, i32, ctypes.c_int, ctypes.c_int]
     lib.kda_launch_count.restype = ctypes.c_uint64
     lib.kda_launch_count.argtypes = []
+    lib.kda_device_status.restype = ctypes.c_int
+    lib.kda_device_status.argtypes = [vp]
     _lib = lib
     return lib
 
@@ -117,6 +119,11 @@ def kda_forward_kernel_name(d_k: int, d_v: int, chunk: int, in_dtype: torch.dtyp
     r = load_library().kda_forward_kernel_name(d_k, d_v, chunk, code(in_dtype),
                                                 code(out_dtype or in_dtype))
     return None if r is None else r.decode()
+
+
+def kda_device_status(stream=None) -> None:
+    """Synchronise `stream` and raise KdaError if a kernel reported a device timeout."""
+    _check("kda_device_status", load_library().kda_device_status(_stream(stream)))
 
 
 def kda_launch_count() -> int:

@@ -116,8 +116,9 @@ kda_status_t kda_decode_step(const void* q, const void* k, const void* v,
 const char* kda_status_string(kda_status_t status);
 
 /*
- * Bytes of device workspace kda_forward uses for these sizes.  The library
- * allocates and owns it; the figure is reported for capacity planning.
+ * Bytes of device workspace kda_forward uses for these sizes: the per-device
+ * status word (4 bytes), allocated by the library on the first tensor-core call
+ * on a device and kept until exit.  No per-call workspace is allocated.
  */
 size_t kda_forward_workspace_bytes(int32_t B, int64_t T, int32_t H, int32_t d_k,
                                    int32_t d_v, int32_t chunk);
@@ -138,6 +139,17 @@ const char* kda_forward_kernel_name(int32_t d_k, int32_t d_v, int32_t chunk,
  * points, all threads).  A host-side counter, for accounting in benchmarks.
  */
 uint64_t kda_launch_count(void);
+
+/*
+ * Device-side error check.  Every wait inside the tensor-core kernel is
+ * bounded (2 s); a kernel whose wait gives up stops, frees its tensor memory
+ * and sets a per-device status word instead of hanging.  This call
+ * synchronises `stream`, reads and clears that word for the current device and
+ * returns KDA_ERR_DEVICE_TIMEOUT if it was set, else KDA_OK (or KDA_ERR_CUDA).
+ * With the environment variable KDA_DEBUG=1, kda_forward makes this check
+ * itself after every tensor-core launch (and therefore synchronises).
+ */
+kda_status_t kda_device_status(kda_stream_t stream);
 
 #ifdef __cplusplus
 }

@@ -208,3 +208,49 @@ def test_full_long_context_sampled():
         assert rel_l2(np32(out[:, :65536, h:h + 1]), ro) <= 2e-2
     _, rS = oracle_forward(inp, h=7)
     assert rel_l2(np32(Sf[:, 7:8]), rS) <= 2e-2
+
+
+# ------------------------------------------------ tensor-core path specifics
+
+def test_tc_kernel_selected_for_bf16_d128():
+    assert kda.kda_forward_kernel_name(128, 128, 64, torch.bfloat16) == "chunk_tc_bf16"
+    assert kda.kda_forward_kernel_name(128, 128, 64, torch.bfloat16, torch.float32) == "chunk_simt_f32"
+    assert kda.kda_forward_kernel_name(64, 64, 64, torch.float32) == "chunk_simt_f32"
+
+
+@pytest.mark.parametrize("T", [1, 63, 64, 65, 64 * 5 + 17])
+def test_tc_ragged_lengths(T):
+    inp = gen.draw_forward(2, T, 3, 128, 128, "bf16", 500 + T, device=DEV, s0=True)
+    out, Sf = kda.kda_forward(inp["q"], inp["k"], inp["v"], inp["alpha"], inp["beta"], inp["S0"])
+    torch.cuda.synchronize()
+    kda.kda_device_status()
+    ro, rS = oracle_forward(inp)
+    assert rel_l2(np32(out), ro) <= 2e-2
+    assert rel_l2(np32(Sf), rS) <= 2e-2
+
+
+def test_tc_extreme_gates():
+    """Whole channels at alpha = 1, below the clamp floor, and at the floor: the
+    sub-chunk factors reach e^-80 and 1/pi reaches e^80."""
+    inp = gen.draw_forward(1, 300, 2, 128, 128, "bf16", 600, device=DEV, s0=True)
+    al = inp["alpha"]
+    al[..., :40] = 1.0
+    al[..., 40:80] = 1e-4
+    al[..., 80:90] = gen.BF16_BELOW_EXP_M5
+    out, Sf = kda.kda_forward(inp["q"], inp["k"], inp["v"], al, inp["beta"], inp["S0"])
+    torch.cuda.synchronize()
+    ro, rS = oracle_forward(inp)
+    assert rel_l2(np32(out), ro) <= 2e-2
+    assert rel_l2(np32(Sf), rS) <= 2e-2
+
+
+def test_tc_matches_fp32_path():
+    """The tensor-core kernel and the fp32 CUDA-core kernel agree on the same
+    bf16 inputs (the latter selected by asking for an fp32 output)."""
+    inp = gen.draw_forward(2, 333, 4, 128, 128, "bf16", 700, device=DEV, s0=True)
+    o_tc, S_tc = kda.kda_forward(inp["q"], inp["k"], inp["v"], inp["alpha"], inp["beta"], inp["S0"])
+    o_f, S_f = kda.kda_forward(inp["q"], inp["k"], inp["v"], inp["alpha"], inp["beta"], inp["S0"],
+                               out_dtype=torch.float32)
+    torch.cuda.synchronize()
+    assert rel_l2(np32(o_tc), np32(o_f)) <= 2e-2
+    assert rel_l2(np32(S_tc), np32(S_f)) <= 2e-2
