@@ -32,6 +32,11 @@
 #include "kda_common.cuh"
 #include "kda_sm100.cuh"
 
+// Optional phase-boundary hook for profiling builds (no-op in the library).
+#ifndef KDA_TC_PHASE
+#define KDA_TC_PHASE(i)
+#endif
+
 namespace kda {
 using namespace sm100;
 
@@ -214,6 +219,7 @@ kda_chunk_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_consta
             sBeta[tid] = tid < Lc ? __bfloat162float(beta[(size_t)(row0 + tid) * H + h]) : 0.0f;
         if (ok && !mbar_wait_ns(barT, phT, kWaitNs)) ok = false;
         phT ^= 1u;
+        KDA_TC_PHASE(0);
 
         // ================= gate products and bf16 operands (all threads)
         {
@@ -314,6 +320,7 @@ kda_chunk_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_consta
         __syncthreads();
         tc_fence_after();
 
+        KDA_TC_PHASE(1);
         // ================= [A/beta | P] row blocks: four M=64, N=32 MMAs
         if (tid == 0) {
             const uint32_t r0 = smem_u32(sX + X_R), l0 = smem_u32(sX + X_L);
@@ -332,6 +339,7 @@ kda_chunk_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_consta
         }
         wait_mma();
 
+        KDA_TC_PHASE(2);
         // ================= A and P to fp32 shared memory (masked), P to the [I ; P] operand
         {
             float* Am = reinterpret_cast<float*>(sX + X_AM);
@@ -360,6 +368,7 @@ kda_chunk_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_consta
         tc_fence_before();
         __syncthreads();
 
+        KDA_TC_PHASE(3);
         // ================= Tinv = (I + A)^-1: diagonal 16x16 blocks by forward substitution
         {
             const float* Am = reinterpret_cast<const float*>(sX + X_AM);
@@ -423,6 +432,7 @@ kda_chunk_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_consta
         __syncthreads();
         tc_fence_after();
 
+        KDA_TC_PHASE(4);
         // ================= [Tb ; P Tb] = [I ; P] Tb   (M=128, N=64, K=64)
         if (tid == 0) {
             const uint32_t a0 = smem_u32(sIP), b0 = smem_u32(sX + X_TB);
@@ -453,6 +463,7 @@ kda_chunk_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_consta
         __syncthreads();
         tc_fence_after();
 
+        KDA_TC_PHASE(5);
         // ================= [W ; P W] = [Tb ; P Tb] (k*gamma)   (M=128, N=128, K=64)
         if (tid == 0) {
             const uint32_t a0 = smem_u32(sAl), b0 = smem_u32(sKT);
@@ -501,6 +512,7 @@ kda_chunk_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_consta
         __syncthreads();
         tc_fence_after();
 
+        KDA_TC_PHASE(6);
         // ================= [U ; O] = [-W ; Q'] S + [Tb ; P Tb] V   (two N=64 halves, K=128+64)
         if (tid == 0) {
             const uint32_t wq = smem_u32(sX + X_WQ), s0 = smem_u32(sS), tb = smem_u32(sAl),
@@ -567,6 +579,7 @@ kda_chunk_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_consta
         __syncthreads();
         tc_fence_after();
 
+        KDA_TC_PHASE(7);
         // ================= S += (k*eta)^T U   (M=128, two N=64 halves, K=64)
         if (tid == 0) {
             const uint32_t a0 = smem_u32(sKH), u0 = smem_u32(sX + X_U);
@@ -598,6 +611,7 @@ kda_chunk_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_consta
         tc_fence_before();
         const int any_timeout = __syncthreads_or(!ok);   // uniform: every thread leaves together
         tc_fence_after();
+        KDA_TC_PHASE(8);
         if (any_timeout) break;
     }
 
