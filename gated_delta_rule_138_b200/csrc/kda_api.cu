@@ -75,6 +75,14 @@ bool debug_sync() {
 
 }  // namespace
 
+namespace kda {
+// Shared with the other entry-point files of the library: the text returned by
+// kda_last_error for this thread.
+void set_last_error_text(const char* text) {
+    std::snprintf(g_last_error, sizeof(g_last_error), "%s", text ? text : "");
+}
+}  // namespace kda
+
 extern "C" {
 
 const char* kda_status_string(kda_status_t status) {

@@ -102,6 +102,9 @@ __device__ __forceinline__ void st_bf2(uint8_t* p, float a, float b) {
 // M=64 accumulator: row m lives in TMEM lane 32*(m/16) + m%16
 // M=128 accumulator: row m lives in lane m.
 
+// kCtaStatus = false: a timed-out wait sets the shared word *status to 1.
+// kCtaStatus = true:  every CTA writes its own word status[n * H + h] (0 or 1).
+template <bool kCtaStatus>
 __global__ void __launch_bounds__(NT, 1)
 kda_chunk_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                     const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmV,
@@ -617,8 +620,9 @@ kda_chunk_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_consta
 
     if (!ok) atomicExch(sFlag, 1);
     __syncthreads();
+    if (kCtaStatus && tid == 0) status[(size_t)n * H + h] = *sFlag;
     if (*sFlag) {
-        if (tid == 0) atomicExch(status, 1);
+        if (!kCtaStatus && tid == 0) atomicExch(status, 1);
     } else if (S_final) {
         const int c = 32 * q4 + lane;
         float* dst = S_final + (((size_t)n * H + h) * DK + c) * DV + 64 * hf;
@@ -672,23 +676,42 @@ static bool make_map(CUtensorMap* m, const void* base, int64_t rows, int H) {
 
 }  // namespace tc
 
-cudaError_t launch_chunk_tc(const void* q, const void* k, const void* v, const void* alpha,
-                            const void* beta, const float* S0, const int32_t* cu, int nseq,
-                            void* out, float* S_final, int64_t rows, int64_t T, int H, int* status,
-                            cudaStream_t stream) {
+template <bool kCtaStatus>
+static cudaError_t launch_tc_t(const void* q, const void* k, const void* v, const void* alpha,
+                               const void* beta, const float* S0, const int32_t* cu, int nseq,
+                               void* out, float* S_final, int64_t rows, int64_t T, int H,
+                               int* status, cudaStream_t stream) {
     CUtensorMap mq, mk, ma, mv;
     if (!tc::make_map(&mq, q, rows, H) || !tc::make_map(&mk, k, rows, H) ||
         !tc::make_map(&ma, alpha, rows, H) || !tc::make_map(&mv, v, rows, H))
         return cudaErrorInvalidValue;
-    cudaError_t e = cudaFuncSetAttribute(tc::kda_chunk_tc_kernel,
+    cudaError_t e = cudaFuncSetAttribute(tc::kda_chunk_tc_kernel<kCtaStatus>,
                                          cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          (int)tc::SMEM_BYTES);
     if (e != cudaSuccess) return e;
     dim3 grid(1, H, nseq);
-    tc::kda_chunk_tc_kernel<<<grid, tc::NT, tc::SMEM_BYTES, stream>>>(
+    tc::kda_chunk_tc_kernel<kCtaStatus><<<grid, tc::NT, tc::SMEM_BYTES, stream>>>(
         mq, mk, ma, mv, (const __nv_bfloat16*)beta, S0, cu, (__nv_bfloat16*)out, S_final, T, H,
         status);
     return cudaGetLastError();
+}
+
+cudaError_t launch_chunk_tc(const void* q, const void* k, const void* v, const void* alpha,
+                            const void* beta, const float* S0, const int32_t* cu, int nseq,
+                            void* out, float* S_final, int64_t rows, int64_t T, int H, int* status,
+                            cudaStream_t stream) {
+    return launch_tc_t<false>(q, k, v, alpha, beta, S0, cu, nseq, out, S_final, rows, T, H,
+                              status, stream);
+}
+
+// Same kernel, one status word per (sequence, head) CTA at status[n * H + h].
+cudaError_t launch_chunk_tc_cta_status(const void* q, const void* k, const void* v,
+                                       const void* alpha, const void* beta, const float* S0,
+                                       const int32_t* cu, int nseq, void* out, float* S_final,
+                                       int64_t rows, int64_t T, int H, int* status,
+                                       cudaStream_t stream) {
+    return launch_tc_t<true>(q, k, v, alpha, beta, S0, cu, nseq, out, S_final, rows, T, H,
+                             status, stream);
 }
 
 }  // namespace kda

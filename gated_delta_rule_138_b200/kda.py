@@ -76,6 +76,8 @@ def load_library(build_if_missing: bool = True) -> ctypes.CDLL:
     lib.kda_launch_count.argtypes = []
     lib.kda_device_status.restype = ctypes.c_int
     lib.kda_device_status.argtypes = [vp]
+    lib.kda_forward_noalloc.restype = ctypes.c_int
+    lib.kda_forward_noalloc.argtypes = lib.kda_forward.argtypes
     _lib = lib
     return lib
 
@@ -175,6 +177,32 @@ def kda_forward(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, alpha: torch.
                          int(B), int(T), int(H), int(dk), int(dv), int(chunk),
                          _dt(q), _dt(out), _stream(stream))
     _check("kda_forward", st)
+    return out, S_final
+
+
+def kda_forward_noalloc(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, alpha: torch.Tensor,
+                        beta: torch.Tensor, out: torch.Tensor, S_final: Optional[torch.Tensor],
+                        S0: Optional[torch.Tensor] = None,
+                        cu_seqlens: Optional[torch.Tensor] = None, chunk: int = 64,
+                        stream=None) -> Tuple[torch.Tensor, Optional[torch.Tensor]]:
+    """kda_forward without device allocation (bf16, d = 128, chunk 64 only).
+
+    The C entry point uses a fixed scratch array compiled into the library
+    instead of allocating; the caller passes the output buffers, so this
+    binding allocates nothing either.
+    """
+    lib = load_library()
+    B, T, H, dk = q.shape
+    dv = v.shape[-1]
+    nseq = B if cu_seqlens is None else cu_seqlens.numel() - 1
+    for name, t in (("q", q), ("k", k), ("v", v), ("alpha", alpha), ("beta", beta),
+                    ("S0", S0), ("cu_seqlens", cu_seqlens), ("out", out), ("S_final", S_final)):
+        _contig(name, t)
+    st = lib.kda_forward_noalloc(_ptr(q), _ptr(k), _ptr(v), _ptr(alpha), _ptr(beta), _ptr(S0),
+                                 _ptr(cu_seqlens), int(nseq), _ptr(out), _ptr(S_final),
+                                 int(B), int(T), int(H), int(dk), int(dv), int(chunk),
+                                 _dt(q), _dt(out), _stream(stream))
+    _check("kda_forward_noalloc", st)
     return out, S_final
 
 

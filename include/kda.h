@@ -151,6 +151,44 @@ uint64_t kda_launch_count(void);
  */
 kda_status_t kda_device_status(kda_stream_t stream);
 
+/*
+ * Capacity of kda_forward_noalloc's fixed scratch: (sequence, head) pairs per call.
+ */
+#define KDA_NOALLOC_MAX_SEQ_HEADS 16384
+
+/*
+ * kda_forward_noalloc -- kda_forward's tensor-core path without any device
+ * allocation.  The paper has no counterpart: this exists for callers that
+ * cannot call cudaMalloc (for example a server or training loop that has
+ * reserved the device memory for its own pool, or a latency-critical loop in
+ * which an allocation may synchronise the device).  kda_forward allocates one
+ * status word per GPU on its first tensor-core call; this entry point instead
+ * uses a fixed device array compiled into the library.
+ *
+ *   Arguments, layouts and results are those of kda_forward.  Only the
+ *   tensor-core configuration is accepted: in_dtype = out_dtype = KDA_BF16,
+ *   d_k = d_v = 128, chunk = 64 (anything else: KDA_ERR_UNSUPPORTED).
+ *   Scratch: one status word per (sequence, head), at most
+ *   KDA_NOALLOC_MAX_SEQ_HEADS (64 KiB per GPU, held by every GPU that loads
+ *   the library until the process exits).  More (sequence, head) pairs than
+ *   that: KDA_ERR_UNSUPPORTED, with the reason in kda_last_error().
+ *   Every call on a device shares the array, which keeps the last call's
+ *   contents (0 = finished, 1 = a bounded device wait gave up); each CTA
+ *   writes its own word, so nothing needs clearing first.  Calls whose
+ *   kernels overlap on the GPU race on the array.
+ *   The first call on a device looks up the array's device address
+ *   (cudaGetSymbolAddress) with that device current; make that first call
+ *   before any stream capture.  No cudaMalloc, cudaFree or other allocating
+ *   routine is called.
+ */
+kda_status_t kda_forward_noalloc(const void* q, const void* k, const void* v,
+                                 const void* alpha, const void* beta, const float* S0,
+                                 const int32_t* cu_seqlens, int32_t num_seqs,
+                                 void* out, float* S_final,
+                                 int32_t B, int64_t T, int32_t H, int32_t d_k, int32_t d_v,
+                                 int32_t chunk, kda_dtype_t in_dtype, kda_dtype_t out_dtype,
+                                 kda_stream_t stream);
+
 #ifdef __cplusplus
 }
 #endif
