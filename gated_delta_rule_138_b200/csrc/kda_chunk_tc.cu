@@ -68,20 +68,22 @@ constexpr uint32_t MISC_FLAG = 2836;     // int timeout seen
 constexpr uint32_t SMEM_BYTES = OFF_MISC + 2848 + 1024;  // + alignment slack
 
 // work region X, by phase
-constexpr uint32_t X_R = 0;              // R rows [160][128] sw128 (2 atoms of 160 rows)
-constexpr uint32_t X_L = 40960;          // L rows [128][128] sw128 (2 atoms of 128 rows)
-constexpr uint32_t X_AM = 0;             // float A [64][65]
-constexpr uint32_t X_PM = 16640;         // float P [64][65]
-constexpr uint32_t X_TM = 33280;         // float Tinv [64][65]
-constexpr uint32_t X_TB = 50176;         // Tb MN-major B [64 j][64 m]
-constexpr uint32_t X_SCR = 58368;        // float scratch 3 x [16][16]
+constexpr uint32_t X_R = 0;              // right operand rows [128][128] (2 atoms of 128 rows)
+constexpr uint32_t X_L = 32768;          // left operand rows  [128][128] (2 atoms of 128 rows)
+constexpr int AS = 68;                   // row stride (floats) of the fp32 A and Tinv tiles
+constexpr uint32_t X_AM = 0;             // float A    [64][68]
+constexpr uint32_t X_TM = 17408;         // float Tinv [64][68]
+constexpr uint32_t X_TB = 35840;         // Tb MN-major B [64 j][64 m] (1024-aligned)
+constexpr uint32_t X_XS = 44032;         // float scratch [32][36]
+// fp32 K-major 128B-swizzled tiles (32 floats per row) for the tf32 MMAs of the 32 -> 64 step
+constexpr uint32_t X_T0T = 49152;        // Tinv[0:32, 0:32]^T   [64 rows (32 used)][32]
+constexpr uint32_t X_T1 = 57344;         // Tinv[32:64, 32:64]   [64 rows (32 used)][32]
+constexpr uint32_t X_A10 = 65536;        // A[32:64, 0:32]       [32][32]
+constexpr uint32_t X_XT = 69632;         // (A10 T0)^T           [32][32]
 constexpr uint32_t X_WQ = 0;             // [-W ; Q'] K-major A [128][128] (2 atoms)
 constexpr uint32_t X_U = 32768;          // U MN-major B [64 j][128 n] (2 atoms of [64][64])
 
 constexpr uint32_t TM_S = 0, TM_UO = 128, TM_WK = 256;
-
-// row offsets of R^(I) in the R buffer; the M=64 window of R^(I) starts there
-__device__ __constant__ int kROff[4] = {0, 16, 48, 96};
 
 __device__ __forceinline__ uint32_t swz(uint32_t row, uint32_t chunk) {
     return row * 128u + (((chunk ^ row) & 7u) << 4);
@@ -91,12 +93,29 @@ __device__ __forceinline__ uint32_t swz(uint32_t row, uint32_t chunk) {
 __device__ __forceinline__ uint32_t pair_off(uint32_t row, uint32_t c, uint32_t rows) {
     return (c >> 6) * rows * 128u + swz(row, (c & 63u) >> 3) + ((c & 7u) << 1);
 }
+// byte offset of fp32 element (r, k) in a K-major 128B-swizzled tile with 32 floats per row
+__device__ __forceinline__ uint32_t f32_off(uint32_t r, uint32_t k) {
+    return r * 128u + ((((k >> 2) ^ r) & 7u) << 4) + ((k & 3u) << 2);
+}
 __device__ __forceinline__ float2 ld_bf2(const uint8_t* p) {
     const __nv_bfloat162 v = *reinterpret_cast<const __nv_bfloat162*>(p);
     return __bfloat1622float2(v);
 }
 __device__ __forceinline__ void st_bf2(uint8_t* p, float a, float b) {
     *reinterpret_cast<uint32_t*>(p) = pack_bf16x2(a, b);
+}
+
+// 64 consecutive fp32 columns of this thread's TMEM lane, one wait for all four loads
+__device__ __forceinline__ void tmem_ld64(uint32_t taddr, float (&v)[64]) {
+    tmem_ld16(taddr, *reinterpret_cast<float(*)[16]>(&v[0]));
+    tmem_ld16(taddr + 16, *reinterpret_cast<float(*)[16]>(&v[16]));
+    tmem_ld16(taddr + 32, *reinterpret_cast<float(*)[16]>(&v[32]));
+    tmem_ld16(taddr + 48, *reinterpret_cast<float(*)[16]>(&v[48]));
+    tmem_wait_ld();
+}
+__device__ __forceinline__ uint4 pack8(const float* v) {
+    return make_uint4(pack_bf16x2(v[0], v[1]), pack_bf16x2(v[2], v[3]), pack_bf16x2(v[4], v[5]),
+                      pack_bf16x2(v[6], v[7]));
 }
 
 // M=64 accumulator: row m lives in TMEM lane 32*(m/16) + m%16
@@ -156,6 +175,11 @@ kda_chunk_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_consta
         }
         *reinterpret_cast<uint4*>(sIP + swz(r, ch)) = make_uint4(w[0], w[1], w[2], w[3]);
     }
+    // P[r][j] = 0 for r < 32 <= j: never written by the per-chunk extraction
+    for (int i = tid; i < 32 * 4; i += NT) {
+        const int r = i >> 2, ch = 4 + (i & 3);
+        *reinterpret_cast<uint4*>(sIP + swz(64 + r, ch)) = make_uint4(0u, 0u, 0u, 0u);
+    }
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
@@ -207,6 +231,10 @@ kda_chunk_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_consta
     __syncthreads();
     tc_fence_after();
 
+    // beta of the next chunk is loaded one chunk ahead, into a register
+    float beta_next = 0.0f;
+    if (tid < C && tid < len) beta_next = __bfloat162float(beta[(size_t)(bos + tid) * H + h]);
+
     uint32_t phT = 0, phM = 0;
     bool ok = true;   // this thread has seen every wait complete
     auto wait_mma = [&]() {
@@ -218,22 +246,38 @@ kda_chunk_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_consta
     for (int chunk = 0; chunk < nchunks; ++chunk) {
         const int64_t row0 = bos + (int64_t)chunk * C;
         const int Lc = (int)((len - (int64_t)chunk * C) < C ? (len - (int64_t)chunk * C) : C);
-        if (tid < C)
-            sBeta[tid] = tid < Lc ? __bfloat162float(beta[(size_t)(row0 + tid) * H + h]) : 0.0f;
+        if (tid < C) sBeta[tid] = beta_next;
         if (ok && !mbar_wait_ns(barT, phT, kWaitNs)) ok = false;
         phT ^= 1u;
         KDA_TC_PHASE(0);
 
         // ================= gate products and bf16 operands (all threads)
         {
-            const int cp = tid & 63, I = tid >> 6, c0 = 2 * cp;
+            // thread = (channel pair c0, c0+1) x (16-token quarter Q).  Sub-chunk I = Q/2
+            // holds 32 tokens; its reference token is ref_I = 32I + 15.  With phi / psi the
+            // in-quarter forward (inclusive) / backward (exclusive) gate products and pi_Q
+            // the quarter product:
+            //   left  lam_t   = e^{g_t - g_ref}  = phi_t * (Q even ? 1/pi_Q : 1)
+            //   right rho^I_j = e^{g_ref - g_j}  = psi_j * c_I(Q(j))
+            //   c_0 = {1, 1/pi_1},  c_1 = {pi_1 pi_2, pi_2, 1, 1/pi_3}
+            // so that lam_r rho^I_j = prod_{s=j+1..r} a_s for j <= r, every factor within
+            // [e^-80, e^80] except right factors that underflow where the product is negligible.
+            // All tiles touched here have 8-row-aligned bases, so the swizzled offset of
+            // (row i of a 16-row group, this channel pair) is i*128 + xo[i & 7].
+            const int cp = tid & 63, Q = tid >> 6, c0 = 2 * cp, Isub = Q >> 1;
+            const uint32_t atom = (uint32_t)(c0 >> 6);
+            const uint32_t chk = (uint32_t)((c0 & 63) >> 3), inner = (uint32_t)((c0 & 7) << 1);
+            uint32_t xo[8];
+#pragma unroll
+            for (int k8 = 0; k8 < 8; ++k8) xo[k8] = (((chk ^ (uint32_t)k8) & 7u) << 4) | inner;
+            const uint32_t in_base = atom * 8192u + (uint32_t)(16 * Q) * 128u;   // 64-row input tiles
             float phi0[16], phi1[16], psi0[16], psi1[16];
             {
                 float a0[16], a1[16];
 #pragma unroll
                 for (int i = 0; i < 16; ++i) {
-                    const int r = 16 * I + i;
-                    float2 al = ld_bf2(sAl + pair_off(r, c0, 64));
+                    const int r = 16 * Q + i;
+                    const float2 al = ld_bf2(sAl + in_base + i * 128 + xo[i & 7]);
                     a0[i] = r < Lc ? clamp_gate(al.x) : 1.0f;
                     a1[i] = r < Lc ? clamp_gate(al.y) : 1.0f;
                 }
@@ -249,73 +293,67 @@ kda_chunk_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_consta
                     psi0[i] = s0; psi1[i] = s1;
                     s0 *= a0[i]; s1 *= a1[i];
                 }
-                sPi[I * DK + c0] = p0;
-                sPi[I * DK + c0 + 1] = p1;
+                *reinterpret_cast<float2*>(&sPi[Q * DK + c0]) = make_float2(p0, p1);
             }
             __syncthreads();
             float pi0[4], pi1[4];
 #pragma unroll
-            for (int M = 0; M < 4; ++M) { pi0[M] = sPi[M * DK + c0]; pi1[M] = sPi[M * DK + c0 + 1]; }
+            for (int M = 0; M < 4; ++M) {
+                const float2 pm = *reinterpret_cast<const float2*>(&sPi[M * DK + c0]);
+                pi0[M] = pm.x; pi1[M] = pm.y;
+            }
             float bef0 = 1.f, bef1 = 1.f, aft0 = 1.f, aft1 = 1.f;
 #pragma unroll
             for (int M = 0; M < 4; ++M) {
-                if (M < I) { bef0 *= pi0[M]; bef1 *= pi1[M]; }
-                if (M > I) { aft0 *= pi0[M]; aft1 *= pi1[M]; }
+                if (M < Q) { bef0 *= pi0[M]; bef1 *= pi1[M]; }
+                if (M > Q) { aft0 *= pi0[M]; aft1 *= pi1[M]; }
             }
-            if (I == 0) {
-                sGC[c0] = pi0[0] * pi0[1] * pi0[2] * pi0[3];
-                sGC[c0 + 1] = pi1[0] * pi1[1] * pi1[2] * pi1[3];
-            }
-            // Dp_{I', I} for I' >= I
-            float dp0[4], dp1[4];
-#pragma unroll
-            for (int Ip = 0; Ip < 4; ++Ip) {
-                float x0 = 1.f, x1 = 1.f;
-#pragma unroll
-                for (int M = 0; M < 4; ++M)
-                    if (M > I && M < Ip) { x0 *= pi0[M]; x1 *= pi1[M]; }
-                if (Ip == I) { x0 = 1.0f / pi0[I]; x1 = 1.0f / pi1[I]; }
-                dp0[Ip] = x0; dp1[Ip] = x1;
-            }
-            uint8_t* sR = sX + X_R;
-            uint8_t* sL = sX + X_L;
+            if (Q == 0)
+                *reinterpret_cast<float2*>(&sGC[c0]) =
+                    make_float2(pi0[0] * pi0[1] * pi0[2] * pi0[3], pi1[0] * pi1[1] * pi1[2] * pi1[3]);
+            // left scale d_Q and right scales c_0(Q) (Q < 2) and c_1(Q)
+            float dl0 = 1.f, dl1 = 1.f, r00 = 1.f, r01 = 1.f, r10 = 1.f, r11 = 1.f;
+            if ((Q & 1) == 0) { dl0 = __frcp_rn(pi0[Q]); dl1 = __frcp_rn(pi1[Q]); }
+            if (Q == 1) { r00 = __frcp_rn(pi0[1]); r01 = __frcp_rn(pi1[1]); }
+            if (Q == 0) { r10 = pi0[1] * pi0[2]; r11 = pi1[1] * pi1[2]; }
+            if (Q == 1) { r10 = pi0[2]; r11 = pi1[2]; }
+            if (Q == 3) { r10 = __frcp_rn(pi0[3]); r11 = __frcp_rn(pi1[3]); }
+            // left rows: sub-chunk I at rows 64I..64I+63 = [k-part 32 | q-part 32]
+            uint8_t* tLk = sX + X_L + atom * 16384u + (uint32_t)(64 * Isub + 16 * (Q & 1)) * 128u;
+            uint8_t* tLq = tLk + 32 * 128;
+            // right rows: rho^0 at rows 0..31, rho^1 at rows 64..127
+            uint8_t* tR0 = sX + X_R + atom * 16384u + (uint32_t)(16 * Q) * 128u;
+            uint8_t* tR1 = tR0 + 64 * 128;
+            uint8_t* tQ = sQ + in_base;
+            const uint8_t* tK = sK + in_base;
             float kt0[16], kt1[16], kh0[16], kh1[16];
 #pragma unroll
             for (int i = 0; i < 16; ++i) {
-                const int r = 16 * I + i;
-                float2 kk = ld_bf2(sK + pair_off(r, c0, 64));
-                float2 qq = ld_bf2(sQ + pair_off(r, c0, 64));
+                const int r = 16 * Q + i;
+                const uint32_t off = i * 128 + xo[i & 7];
+                float2 kk = ld_bf2(tK + off);
+                float2 qq = ld_bf2(tQ + off);
                 if (r >= Lc) { kk = make_float2(0.f, 0.f); qq = kk; }
                 const float kp0 = kk.x * phi0[i], kp1 = kk.y * phi1[i];
                 const float qp0 = qq.x * phi0[i], qp1 = qq.y * phi1[i];
                 const float ks0 = kk.x * psi0[i], ks1 = kk.y * psi1[i];
-                st_bf2(sL + pair_off(32 * I + i, c0, 128), kp0, kp1);
-                st_bf2(sL + pair_off(32 * I + 16 + i, c0, 128), qp0, qp1);
-#pragma unroll
-                for (int Ip = 0; Ip < 4; ++Ip)
-                    if (Ip >= I) st_bf2(sR + pair_off(kROff[Ip] + r, c0, 160), ks0 * dp0[Ip], ks1 * dp1[Ip]);
-                st_bf2(sQ + pair_off(r, c0, 64), qp0 * bef0, qp1 * bef1);   // q*gamma in place
-                kt0[i] = kp0 * bef0; kt1[i] = kp1 * bef1;                    // k*gamma
-                kh0[i] = ks0 * aft0; kh1[i] = ks1 * aft1;                    // k*eta
+                st_bf2(tLk + off, kp0 * dl0, kp1 * dl1);
+                st_bf2(tLq + off, qp0 * dl0, qp1 * dl1);
+                if (Q < 2) st_bf2(tR0 + off, ks0 * r00, ks1 * r01);
+                st_bf2(tR1 + off, ks0 * r10, ks1 * r11);
+                st_bf2(tQ + off, qp0 * bef0, qp1 * bef1);   // q*gamma in place
+                kt0[i] = kp0 * bef0; kt1[i] = kp1 * bef1;    // k*gamma
+                kh0[i] = ks0 * aft0; kh1[i] = ks1 * aft1;    // k*eta
             }
-            // transposed tiles [c][j]: tokens 16I..16I+15 are chunks 2I, 2I+1 of rows c0, c0+1
+            // transposed tiles [c][j]: tokens 16Q..16Q+15 are chunks 2Q, 2Q+1 of rows c0, c0+1
 #pragma unroll
             for (int half = 0; half < 2; ++half) {
-                const int ch = 2 * I + half;
+                const int ch = 2 * Q + half;
                 const int b = 8 * half;
-                uint4 w;
-                w = make_uint4(pack_bf16x2(kt0[b], kt0[b + 1]), pack_bf16x2(kt0[b + 2], kt0[b + 3]),
-                               pack_bf16x2(kt0[b + 4], kt0[b + 5]), pack_bf16x2(kt0[b + 6], kt0[b + 7]));
-                *reinterpret_cast<uint4*>(sKT + swz(c0, ch)) = w;
-                w = make_uint4(pack_bf16x2(kt1[b], kt1[b + 1]), pack_bf16x2(kt1[b + 2], kt1[b + 3]),
-                               pack_bf16x2(kt1[b + 4], kt1[b + 5]), pack_bf16x2(kt1[b + 6], kt1[b + 7]));
-                *reinterpret_cast<uint4*>(sKT + swz(c0 + 1, ch)) = w;
-                w = make_uint4(pack_bf16x2(kh0[b], kh0[b + 1]), pack_bf16x2(kh0[b + 2], kh0[b + 3]),
-                               pack_bf16x2(kh0[b + 4], kh0[b + 5]), pack_bf16x2(kh0[b + 6], kh0[b + 7]));
-                *reinterpret_cast<uint4*>(sKH + swz(c0, ch)) = w;
-                w = make_uint4(pack_bf16x2(kh1[b], kh1[b + 1]), pack_bf16x2(kh1[b + 2], kh1[b + 3]),
-                               pack_bf16x2(kh1[b + 4], kh1[b + 5]), pack_bf16x2(kh1[b + 6], kh1[b + 7]));
-                *reinterpret_cast<uint4*>(sKH + swz(c0 + 1, ch)) = w;
+                *reinterpret_cast<uint4*>(sKT + swz(c0, ch)) = pack8(&kt0[b]);
+                *reinterpret_cast<uint4*>(sKT + swz(c0 + 1, ch)) = pack8(&kt1[b]);
+                *reinterpret_cast<uint4*>(sKH + swz(c0, ch)) = pack8(&kh0[b]);
+                *reinterpret_cast<uint4*>(sKH + swz(c0 + 1, ch)) = pack8(&kh1[b]);
             }
         }
         fence_async_smem();
@@ -324,47 +362,44 @@ kda_chunk_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_consta
         tc_fence_after();
 
         KDA_TC_PHASE(1);
-        // ================= [A/beta | P] row blocks: four M=64, N=32 MMAs
+        // ================= [A/beta | P] by sub-chunk: one M=128, N=128, K=128 MMA group
+        //   D[j][n]:  rows 0..31  x cols 0..63   = sub-chunk 0 (j < 32; [A/beta | P] columns r)
+        //             rows 64..127 x cols 64..127 = sub-chunk 1 (j < 64; columns r - 32)
         if (tid == 0) {
             const uint32_t r0 = smem_u32(sX + X_R), l0 = smem_u32(sX + X_L);
-            constexpr uint32_t idesc = idesc_bf16(64, 32);
+            constexpr uint32_t idesc = idesc_bf16(128, 128);
 #pragma unroll
-            for (int I = 0; I < 4; ++I) {
-#pragma unroll
-                for (int ks = 0; ks < 8; ++ks) {
-                    const uint32_t atom = ks >> 2, within = (ks & 3) * 32;
-                    const uint32_t a = r0 + atom * (160 * 128) + kROff[I] * 128 + within;
-                    const uint32_t b = l0 + atom * (128 * 128) + (32 * I) * 128 + within;
-                    mma_bf16(tmem + TM_WK + 32 * I, sdesc_sw128(a), sdesc_sw128(b), idesc, ks > 0);
-                }
+            for (int ks = 0; ks < 8; ++ks) {
+                const uint32_t off = (ks >> 2) * 16384u + (ks & 3) * 32u;
+                mma_bf16(tmem + TM_WK, sdesc_sw128(r0 + off), sdesc_sw128(l0 + off), idesc, ks > 0);
             }
             mma_commit(barM);
         }
         wait_mma();
 
         KDA_TC_PHASE(2);
-        // ================= A and P to fp32 shared memory (masked), P to the [I ; P] operand
-        {
+        // ================= A to fp32 shared memory (masked), P to the [I ; P] operand
+        if (q4 != 1) {
             float* Am = reinterpret_cast<float*>(sX + X_AM);
-            float* Pm = reinterpret_cast<float*>(sX + X_PM);
-            const int j = 16 * q4 + (lane & 15);   // key token of this lane (lanes 0-15)
+            const int sub = q4 == 0 ? 0 : 1;                       // which sub-chunk's block row
+            const int j = q4 == 0 ? lane : 32 * (q4 - 2) + lane;   // key token of this lane
+            const uint32_t col = (uint32_t)(64 * sub + 32 * hf);   // A part (hf 0) or P part (hf 1)
+            float v[32];
+            tmem_ld16(tmem + tlane + TM_WK + col, *reinterpret_cast<float(*)[16]>(&v[0]));
+            tmem_ld16(tmem + tlane + TM_WK + col + 16, *reinterpret_cast<float(*)[16]>(&v[16]));
+            tmem_wait_ld();
+            if (hf == 0) {
 #pragma unroll
-            for (int t = 0; t < 2; ++t) {
-                const int I = 2 * hf + t;
-                float va[16], vp[16];
-                tmem_ld16(tmem + tlane + TM_WK + 32 * I, va);
-                tmem_ld16(tmem + tlane + TM_WK + 32 * I + 16, vp);
-                tmem_wait_ld();
-                if (lane < 16) {
+                for (int rr = 0; rr < 32; ++rr) {
+                    const int r = 32 * sub + rr;
+                    Am[r * AS + j] = (j < r) ? sBeta[r] * v[rr] : 0.0f;
+                }
+            } else {
 #pragma unroll
-                    for (int rr = 0; rr < 16; ++rr) {
-                        const int r = 16 * I + rr;
-                        Am[r * 65 + j] = (j < r) ? sBeta[r] * va[rr] : 0.0f;
-                        const float p = (j <= r) ? vp[rr] : 0.0f;
-                        Pm[r * 65 + j] = p;
-                        *reinterpret_cast<__nv_bfloat16*>(sIP + swz(64 + r, j >> 3) + ((j & 7) << 1)) =
-                            __float2bfloat16_rn(p);
-                    }
+                for (int rr = 0; rr < 32; ++rr) {
+                    const int r = 32 * sub + rr;
+                    *reinterpret_cast<__nv_bfloat16*>(sIP + swz(64 + r, j >> 3) + ((j & 7) << 1)) =
+                        __float2bfloat16_rn((j <= r) ? v[rr] : 0.0f);
                 }
             }
         }
@@ -372,63 +407,167 @@ kda_chunk_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_consta
         __syncthreads();
 
         KDA_TC_PHASE(3);
-        // ================= Tinv = (I + A)^-1: diagonal 16x16 blocks by forward substitution
+        // ================= Tinv = (I + A)^-1 by doubling: 16x16 blocks, then 32, then 64
+        //   inv([[X, 0], [Y, Z]]) = [[X^-1, 0], [-Z^-1 Y X^-1, Z^-1]]
         {
             const float* Am = reinterpret_cast<const float*>(sX + X_AM);
             float* Tm = reinterpret_cast<float*>(sX + X_TM);
-            if (tid < 64) {
-                const int I = tid >> 4, m = tid & 15, o = 16 * I;
+            float* Xs = reinterpret_cast<float*>(sX + X_XS);
+            if (warp < 4) {
+                // diagonal 16x16 blocks by forward substitution: warp I, lane m < 16 owns column m
+                const int I = warp, m = lane & 15, o = 16 * I;
                 float col[16];
 #pragma unroll
                 for (int r = 0; r < 16; ++r) {
-                    float s = 0.0f;
+                    float arow[16];
 #pragma unroll
-                    for (int jj = 0; jj < 16; ++jj)
-                        if (jj < r) s = fmaf(Am[(o + r) * 65 + o + jj], col[jj], s);
-                    col[r] = r < m ? 0.0f : (r == m ? 1.0f : -s);
-                    Tm[(o + r) * 65 + o + m] = col[r];
+                    for (int jj = 0; jj < 16; jj += 4)
+                        if (jj < r) *reinterpret_cast<float4*>(&arow[jj]) =
+                            *reinterpret_cast<const float4*>(&Am[(o + r) * AS + o + jj]);
+                    float s0 = 0.0f, s1 = 0.0f, s2 = 0.0f, s3 = 0.0f;
+#pragma unroll
+                    for (int jj = 0; jj < r; ++jj) {
+                        if ((jj & 3) == 0) s0 = fmaf(arow[jj], col[jj], s0);
+                        else if ((jj & 3) == 1) s1 = fmaf(arow[jj], col[jj], s1);
+                        else if ((jj & 3) == 2) s2 = fmaf(arow[jj], col[jj], s2);
+                        else s3 = fmaf(arow[jj], col[jj], s3);
+                    }
+                    col[r] = r < m ? 0.0f : (r == m ? 1.0f : -((s0 + s1) + (s2 + s3)));
                 }
+                if (lane < 16) {
+#pragma unroll
+                    for (int r = 0; r < 16; ++r) Tm[(o + r) * AS + o + m] = col[r];
+                }
+            } else {
+                // zeros above the diagonal blocks that the doubling steps read
+                const int t = tid - 128;                       // 0..127
+                const int r = t >> 2, cq = (t & 3) * 4;        // rows 0..31, 4 columns each
+                const int rb = r < 16 ? r : 16 + r;            // rows 0-15 and 32-47
+                const int cb = r < 16 ? 16 + cq : 48 + cq;     // columns 16-31 and 48-63
+                *reinterpret_cast<float4*>(&Tm[rb * AS + cb]) = make_float4(0.f, 0.f, 0.f, 0.f);
+                const int r2 = t >> 2;                         // rows 0..31, columns 32..63
+#pragma unroll
+                for (int c4 = 0; c4 < 2; ++c4)
+                    *reinterpret_cast<float4*>(&Tm[r2 * AS + 32 + 16 * c4 + cq]) =
+                        make_float4(0.f, 0.f, 0.f, 0.f);
             }
             __syncthreads();
-            // off-diagonal blocks, by distance d = I - J
-            float* scr = reinterpret_cast<float*>(sX + X_SCR);
-#pragma unroll 1
-            for (int d = 1; d < 4; ++d) {
-                const int nblk = 4 - d;
-                for (int e = tid; e < nblk * 256; e += NT) {
-                    const int J = e >> 8, I = J + d, r = (e >> 4) & 15, m = e & 15;
-                    float s = 0.0f;
-                    for (int M = J; M < I; ++M)
+            KDA_TC_PHASE(9);
+            // 16 -> 32: blocks (1,0) and (3,2).  thread: block b, row r, columns m2, m2+1
+            {
+                const int b = tid >> 7, r = (tid >> 3) & 15, m2 = (tid & 7) * 2;
+                const int o0 = 32 * b, o1 = o0 + 16;
+                float arow[16];
 #pragma unroll
-                        for (int jj = 0; jj < 16; ++jj)
-                            s = fmaf(Am[(16 * I + r) * 65 + 16 * M + jj], Tm[(16 * M + jj) * 65 + 16 * J + m], s);
-                    scr[e] = s;
-                }
-                __syncthreads();
-                for (int e = tid; e < nblk * 256; e += NT) {
-                    const int J = e >> 8, I = J + d, r = (e >> 4) & 15, m = e & 15;
-                    float s = 0.0f;
+                for (int j = 0; j < 16; j += 4)
+                    *reinterpret_cast<float4*>(&arow[j]) = *reinterpret_cast<const float4*>(&Am[(o1 + r) * AS + o0 + j]);
+                float x0 = 0.f, x1 = 0.f, x2 = 0.f, x3 = 0.f;
 #pragma unroll
-                    for (int jj = 0; jj < 16; ++jj)
-                        if (jj <= r) s = fmaf(Tm[(16 * I + r) * 65 + 16 * I + jj], scr[(J << 8) + jj * 16 + m], s);
-                    Tm[(16 * I + r) * 65 + 16 * J + m] = -s;
+                for (int j = 0; j < 16; j += 2) {
+                    const float2 t2 = *reinterpret_cast<const float2*>(&Tm[(o0 + j) * AS + o0 + m2]);
+                    const float2 t3 = *reinterpret_cast<const float2*>(&Tm[(o0 + j + 1) * AS + o0 + m2]);
+                    x0 = fmaf(arow[j], t2.x, x0); x1 = fmaf(arow[j], t2.y, x1);
+                    x2 = fmaf(arow[j + 1], t3.x, x2); x3 = fmaf(arow[j + 1], t3.y, x3);
                 }
+                x0 += x2; x1 += x3;
+                *reinterpret_cast<float2*>(&Xs[(16 * b + r) * 36 + m2]) = make_float2(x0, x1);
                 __syncthreads();
+                float y0 = 0.f, y1 = 0.f;
+#pragma unroll
+                for (int jj = 0; jj < 16; ++jj) {
+                    const float tz = Tm[(o1 + r) * AS + o1 + jj];
+                    const float2 xx = *reinterpret_cast<const float2*>(&Xs[(16 * b + jj) * 36 + m2]);
+                    y0 = fmaf(tz, xx.x, y0); y1 = fmaf(tz, xx.y, y1);
+                }
+                *reinterpret_cast<float2*>(&Tm[(o1 + r) * AS + o0 + m2]) = make_float2(-y0, -y1);
             }
+            __syncthreads();
+            KDA_TC_PHASE(10);
+            // 32 -> 64 on the tensor cores (tf32):  X^T = T0^T A10^T,  Y = T1 X,
+            // Tinv[32:64, 0:32] = -Y.  Operands: fp32 K-major tiles written here.
+            {
+                uint8_t* t0t = sX + X_T0T;
+                uint8_t* t1 = sX + X_T1;
+                const int rw = tid >> 3, k4 = (tid & 7) * 4;       // row 0..31, 4 columns
+                float4 c4;
+                c4.x = Tm[(k4 + 0) * AS + rw]; c4.y = Tm[(k4 + 1) * AS + rw];
+                c4.z = Tm[(k4 + 2) * AS + rw]; c4.w = Tm[(k4 + 3) * AS + rw];
+                *reinterpret_cast<float4*>(t0t + f32_off(rw, k4)) = c4;                 // T0^T[m][j]
+                *reinterpret_cast<float4*>(t1 + f32_off(rw, k4)) =
+                    *reinterpret_cast<const float4*>(&Tm[(32 + rw) * AS + 32 + k4]);  // T1[r][jj]
+                *reinterpret_cast<float4*>(sX + X_A10 + f32_off(rw, k4)) =
+                    *reinterpret_cast<const float4*>(&Am[(32 + rw) * AS + k4]);       // A10[r][j]
+            }
+            fence_async_smem();
+            tc_fence_before();
+            __syncthreads();
+            tc_fence_after();
+            if (tid == 0) {
+                constexpr uint32_t idesc = idesc_tf32(64, 32);
+                const uint32_t a0 = smem_u32(sX + X_T0T), b0 = smem_u32(sX + X_A10);
+#pragma unroll
+                for (int ks = 0; ks < 4; ++ks)
+                    mma_tf32(tmem + TM_WK, sdesc_sw128(a0 + ks * 32), sdesc_sw128(b0 + ks * 32), idesc, ks > 0);
+                mma_commit(barM);
+            }
+            wait_mma();
+            if (q4 < 2) {   // M=64 accumulator: rows m = 16*q4 + lane live in lanes 32*q4 + lane
+                float v[32];
+                tmem_ld16(tmem + tlane + TM_WK, *reinterpret_cast<float(*)[16]>(&v[0]));
+                tmem_ld16(tmem + tlane + TM_WK + 16, *reinterpret_cast<float(*)[16]>(&v[16]));
+                tmem_wait_ld();
+                if (hf == 0 && lane < 16) {
+                    const int m = 16 * q4 + lane;
+                    uint8_t* xt = sX + X_XT;
+#pragma unroll
+                    for (int c = 0; c < 32; c += 4)
+                        *reinterpret_cast<float4*>(xt + f32_off(m, c)) = make_float4(v[c], v[c + 1], v[c + 2], v[c + 3]);
+                }
+            }
+            fence_async_smem();
+            tc_fence_before();
+            __syncthreads();
+            tc_fence_after();
+            if (tid == 0) {
+                constexpr uint32_t idesc = idesc_tf32(64, 32);
+                const uint32_t a0 = smem_u32(sX + X_T1), b0 = smem_u32(sX + X_XT);
+#pragma unroll
+                for (int ks = 0; ks < 4; ++ks)
+                    mma_tf32(tmem + TM_WK + 32, sdesc_sw128(a0 + ks * 32), sdesc_sw128(b0 + ks * 32), idesc, ks > 0);
+                mma_commit(barM);
+            }
+            wait_mma();
+            if (q4 < 2) {
+                float v[32];
+                tmem_ld16(tmem + tlane + TM_WK + 32, *reinterpret_cast<float(*)[16]>(&v[0]));
+                tmem_ld16(tmem + tlane + TM_WK + 48, *reinterpret_cast<float(*)[16]>(&v[16]));
+                tmem_wait_ld();
+                if (hf == 0 && lane < 16) {
+                    const int r = 16 * q4 + lane;
+#pragma unroll
+                    for (int c = 0; c < 32; c += 4)
+                        *reinterpret_cast<float4*>(&Tm[(32 + r) * AS + c]) =
+                            make_float4(-v[c], -v[c + 1], -v[c + 2], -v[c + 3]);
+                }
+            }
+            tc_fence_before();
+            __syncthreads();
+            KDA_TC_PHASE(11);
             // Tb = Tinv diag(beta) as MN-major B: row j, column m; zero above the diagonal
             uint8_t* sTB = sX + X_TB;
-            for (int e = tid; e < 64 * 8; e += NT) {
-                const int jr = e >> 3, ch = e & 7;
+#pragma unroll
+            for (int rep = 0; rep < 2; ++rep) {
+                const int e = tid + NT * rep;
+                const int jr = e & 63, ch = e >> 6;
                 float v[8];
 #pragma unroll
                 for (int i = 0; i < 8; ++i) {
                     const int m = 8 * ch + i;
-                    v[i] = (jr >= m) ? Tm[jr * 65 + m] * sBeta[m] : 0.0f;
+                    v[i] = (jr >= m) ? Tm[jr * AS + m] * sBeta[m] : 0.0f;
                 }
-                *reinterpret_cast<uint4*>(sTB + swz(jr, ch)) =
-                    make_uint4(pack_bf16x2(v[0], v[1]), pack_bf16x2(v[2], v[3]),
-                               pack_bf16x2(v[4], v[5]), pack_bf16x2(v[6], v[7]));
+                *reinterpret_cast<uint4*>(sTB + swz(jr, ch)) = pack8(v);
             }
+            KDA_TC_PHASE(12);
         }
         fence_async_smem();
         tc_fence_before();
@@ -449,17 +588,13 @@ kda_chunk_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_consta
         wait_mma();
         {
             const int row = 32 * q4 + lane;
+            float v[32];
+            tmem_ld16(tmem + tlane + TM_WK + 32 * hf, *reinterpret_cast<float(*)[16]>(&v[0]));
+            tmem_ld16(tmem + tlane + TM_WK + 32 * hf + 16, *reinterpret_cast<float(*)[16]>(&v[16]));
+            tmem_wait_ld();
 #pragma unroll
-            for (int blk = 0; blk < 2; ++blk) {
-                float v[16];
-                tmem_ld16(tmem + tlane + TM_WK + 32 * hf + 16 * blk, v);
-                tmem_wait_ld();
-#pragma unroll
-                for (int ch = 0; ch < 2; ++ch)
-                    *reinterpret_cast<uint4*>(sAl + swz(row, 4 * hf + 2 * blk + ch)) =
-                        make_uint4(pack_bf16x2(v[8 * ch], v[8 * ch + 1]), pack_bf16x2(v[8 * ch + 2], v[8 * ch + 3]),
-                                   pack_bf16x2(v[8 * ch + 4], v[8 * ch + 5]), pack_bf16x2(v[8 * ch + 6], v[8 * ch + 7]));
-            }
+            for (int ch = 0; ch < 4; ++ch)
+                *reinterpret_cast<uint4*>(sAl + swz(row, 4 * hf + ch)) = pack8(&v[8 * ch]);
         }
         fence_async_smem();
         tc_fence_before();
@@ -481,32 +616,29 @@ kda_chunk_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_consta
             // [-W ; q*gamma - P W] as the K-major A operand of the state MMA
             const int row = 32 * q4 + lane;
             uint8_t* sWQ = sX + X_WQ;
+            float v[64];
+            tmem_ld64(tmem + tlane + TM_WK + 64 * hf, v);
+            if (row < 64) {
 #pragma unroll
-            for (int blk = 0; blk < 4; ++blk) {
-                float v[16];
-                tmem_ld16(tmem + tlane + TM_WK + 64 * hf + 16 * blk, v);
-                tmem_wait_ld();
-#pragma unroll
-                for (int ch = 0; ch < 2; ++ch) {
-                    const int chunk = 2 * blk + ch;           // 8-column chunk within the atom
+                for (int chunk = 0; chunk < 8; ++chunk) {
                     float w8[8];
-                    if (row < 64) {
 #pragma unroll
-                        for (int i = 0; i < 8; ++i) w8[i] = -v[8 * ch + i];
-                    } else {
-                        const uint4 qg = *reinterpret_cast<const uint4*>(
-                            sQ + hf * 8192 + swz(row - 64, chunk));
-                        const uint32_t qw[4] = {qg.x, qg.y, qg.z, qg.w};
+                    for (int i = 0; i < 8; ++i) w8[i] = -v[8 * chunk + i];
+                    *reinterpret_cast<uint4*>(sWQ + hf * 16384 + swz(row, chunk)) = pack8(w8);
+                }
+            } else {
 #pragma unroll
-                        for (int i = 0; i < 4; ++i) {
-                            const float2 f = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&qw[i]));
-                            w8[2 * i] = f.x - v[8 * ch + 2 * i];
-                            w8[2 * i + 1] = f.y - v[8 * ch + 2 * i + 1];
-                        }
+                for (int chunk = 0; chunk < 8; ++chunk) {
+                    const uint4 qg = *reinterpret_cast<const uint4*>(sQ + hf * 8192 + swz(row - 64, chunk));
+                    const uint32_t qw[4] = {qg.x, qg.y, qg.z, qg.w};
+                    float w8[8];
+#pragma unroll
+                    for (int i = 0; i < 4; ++i) {
+                        const float2 f = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&qw[i]));
+                        w8[2 * i] = f.x - v[8 * chunk + 2 * i];
+                        w8[2 * i + 1] = f.y - v[8 * chunk + 2 * i + 1];
                     }
-                    *reinterpret_cast<uint4*>(sWQ + hf * 16384 + swz(row, chunk)) =
-                        make_uint4(pack_bf16x2(w8[0], w8[1]), pack_bf16x2(w8[2], w8[3]),
-                                   pack_bf16x2(w8[4], w8[5]), pack_bf16x2(w8[6], w8[7]));
+                    *reinterpret_cast<uint4*>(sWQ + hf * 16384 + swz(row, chunk)) = pack8(w8);
                 }
             }
         }
@@ -520,61 +652,52 @@ kda_chunk_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_consta
         if (tid == 0) {
             const uint32_t wq = smem_u32(sX + X_WQ), s0 = smem_u32(sS), tb = smem_u32(sAl),
                            v0 = smem_u32(sV);
-            constexpr uint32_t idesc = idesc_bf16(128, 64, false, true);
+            // B operands are MN-major with two 64-column atoms: leading byte offset = atom stride
+            constexpr uint32_t idesc = idesc_bf16(128, 128, false, true);
+            const uint32_t d = tmem + TM_UO;
 #pragma unroll
-            for (int nh = 0; nh < 2; ++nh) {
-                const uint32_t d = tmem + TM_UO + 64 * nh;
+            for (int ks = 0; ks < 8; ++ks)
+                mma_bf16(d, sdesc_sw128(wq + (ks >> 2) * 16384 + (ks & 3) * 32),
+                         sdesc_sw128(s0 + ks * 2048, 1024, 16384), idesc, ks > 0);
 #pragma unroll
-                for (int ks = 0; ks < 8; ++ks)
-                    mma_bf16(d, sdesc_sw128(wq + (ks >> 2) * 16384 + (ks & 3) * 32),
-                             sdesc_sw128(s0 + nh * 16384 + ks * 2048), idesc, ks > 0);
-#pragma unroll
-                for (int ks = 0; ks < 4; ++ks)
-                    mma_bf16(d, sdesc_sw128(tb + ks * 32), sdesc_sw128(v0 + nh * 8192 + ks * 2048), idesc, 1);
-            }
+            for (int ks = 0; ks < 4; ++ks)
+                mma_bf16(d, sdesc_sw128(tb + ks * 32), sdesc_sw128(v0 + ks * 2048, 1024, 8192), idesc, 1);
             mma_commit(barM);
         }
         // meanwhile: S <- Diag(gamma_C) S in TMEM (the MMA reads the bf16 copy)
         {
             const int c = 32 * q4 + lane;
             const float g = sGC[c];
+            const uint32_t ta = tmem + tlane + TM_S + 64 * hf;
+            float v[64];
+            tmem_ld64(ta, v);
 #pragma unroll
-            for (int blk = 0; blk < 4; ++blk) {
-                float v[16];
-                const uint32_t ta = tmem + tlane + TM_S + 64 * hf + 16 * blk;
-                tmem_ld16(ta, v);
-                tmem_wait_ld();
+            for (int i = 0; i < 64; ++i) v[i] *= g;
 #pragma unroll
-                for (int i = 0; i < 16; ++i) v[i] *= g;
-                tmem_st16(ta, v);
-            }
+            for (int blk = 0; blk < 4; ++blk)
+                tmem_st16(ta + 16 * blk, *reinterpret_cast<float(*)[16]>(&v[16 * blk]));
             tmem_wait_st();
         }
         wait_mma();
         // all of q, k, alpha, v are consumed: prefetch the next chunk
         if (tid == 0 && chunk + 1 < nchunks) issue_tma(row0 + C);
+        if (tid < C) {
+            const int64_t nxt = (int64_t)(chunk + 1) * C + tid;   // token index in the sequence
+            beta_next = nxt < len ? __bfloat162float(beta[(size_t)(bos + nxt) * H + h]) : 0.0f;
+        }
         {
             const int row = 32 * q4 + lane;
             uint8_t* sU = sX + X_U;
+            float v[64];
+            tmem_ld64(tmem + tlane + TM_UO + 64 * hf, v);
+            if (row < 64) {
 #pragma unroll
-            for (int blk = 0; blk < 4; ++blk) {
-                float v[16];
-                tmem_ld16(tmem + tlane + TM_UO + 64 * hf + 16 * blk, v);
-                tmem_wait_ld();
-                uint4 w[2];
+                for (int chunk = 0; chunk < 8; ++chunk)
+                    *reinterpret_cast<uint4*>(sU + hf * 8192 + swz(row, chunk)) = pack8(&v[8 * chunk]);
+            } else if (row - 64 < Lc) {
+                uint4* dst = reinterpret_cast<uint4*>(out + ((size_t)(row0 + row - 64) * H + h) * DV + 64 * hf);
 #pragma unroll
-                for (int ch = 0; ch < 2; ++ch)
-                    w[ch] = make_uint4(pack_bf16x2(v[8 * ch], v[8 * ch + 1]), pack_bf16x2(v[8 * ch + 2], v[8 * ch + 3]),
-                                       pack_bf16x2(v[8 * ch + 4], v[8 * ch + 5]), pack_bf16x2(v[8 * ch + 6], v[8 * ch + 7]));
-                if (row < 64) {
-#pragma unroll
-                    for (int ch = 0; ch < 2; ++ch)
-                        *reinterpret_cast<uint4*>(sU + hf * 8192 + swz(row, 2 * blk + ch)) = w[ch];
-                } else if (row - 64 < Lc) {
-                    __nv_bfloat16* dst = out + ((size_t)(row0 + row - 64) * H + h) * DV + 64 * hf + 16 * blk;
-                    reinterpret_cast<uint4*>(dst)[0] = w[0];
-                    reinterpret_cast<uint4*>(dst)[1] = w[1];
-                }
+                for (int chunk = 0; chunk < 8; ++chunk) dst[chunk] = pack8(&v[8 * chunk]);
             }
         }
         fence_async_smem();
@@ -586,29 +709,21 @@ kda_chunk_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_consta
         // ================= S += (k*eta)^T U   (M=128, two N=64 halves, K=64)
         if (tid == 0) {
             const uint32_t a0 = smem_u32(sKH), u0 = smem_u32(sX + X_U);
-            constexpr uint32_t idesc = idesc_bf16(128, 64, false, true);
+            constexpr uint32_t idesc = idesc_bf16(128, 128, false, true);
 #pragma unroll
-            for (int nh = 0; nh < 2; ++nh)
-#pragma unroll
-                for (int ks = 0; ks < 4; ++ks)
-                    mma_bf16(tmem + TM_S + 64 * nh, sdesc_sw128(a0 + ks * 32),
-                             sdesc_sw128(u0 + nh * 8192 + ks * 2048), idesc, 1);
+            for (int ks = 0; ks < 4; ++ks)
+                mma_bf16(tmem + TM_S, sdesc_sw128(a0 + ks * 32), sdesc_sw128(u0 + ks * 2048, 1024, 8192),
+                         idesc, 1);
             mma_commit(barM);
         }
         wait_mma();
         {
             const int c = 32 * q4 + lane;
+            float v[64];
+            tmem_ld64(tmem + tlane + TM_S + 64 * hf, v);
 #pragma unroll
-            for (int blk = 0; blk < 4; ++blk) {
-                float v[16];
-                tmem_ld16(tmem + tlane + TM_S + 64 * hf + 16 * blk, v);
-                tmem_wait_ld();
-#pragma unroll
-                for (int ch = 0; ch < 2; ++ch)
-                    *reinterpret_cast<uint4*>(sS + hf * 16384 + swz(c, 2 * blk + ch)) =
-                        make_uint4(pack_bf16x2(v[8 * ch], v[8 * ch + 1]), pack_bf16x2(v[8 * ch + 2], v[8 * ch + 3]),
-                                   pack_bf16x2(v[8 * ch + 4], v[8 * ch + 5]), pack_bf16x2(v[8 * ch + 6], v[8 * ch + 7]));
-            }
+            for (int chunk = 0; chunk < 8; ++chunk)
+                *reinterpret_cast<uint4*>(sS + hf * 16384 + swz(c, chunk)) = pack8(&v[8 * chunk]);
         }
         fence_async_smem();
         tc_fence_before();

@@ -29,7 +29,14 @@ sub-chunk boundaries, where a product stays >= e^-80 > the fp32 minimum:
   I > J:  D(r, j) = (phi_r Delta_IJ) * psi_j
   I = J:  D(r, j) = (phi_r / pi_I) * psi_j      (j <= r)
 so A and P are products of a left operand x_r phi_r Delta'_IJ and one right
-operand k_j psi_j, with no factor above e^80.
+operand k_j psi_j, with no factor above e^80.  (fp32 CUDA-core kernel.)
+
+The tensor-core kernel uses 32-token sub-chunks with the reference at each
+sub-chunk's 16th token instead (one left operand per row, two right operands):
+  lam_r   = e^{g_r - g_ref(I(r))}  in [e^-80, e^75]
+  rho^I_j = e^{g_ref(I) - g_j}     in (0, e^80], for j < end(I)
+with D(r, j) = lam_r rho^{I(r)}_j; a right factor may underflow only where the
+true product is negligible.  Both factorizations are checked below.
 """
 import numpy as np
 import pytest
@@ -102,6 +109,44 @@ def chunk_forward_one(q, k, v, alpha, beta, S0, C):
         out[t0:t0 + L] = O1[:L]
         S = gamma[C - 1][:, None] * S + Kh.T @ U
     return out, S
+
+
+def mid_reference_factors(a):
+    """lam [C, dk], rho0 [32, dk], rho1 [64, dk] for one 64-token chunk of gates a."""
+    C, dk = a.shape
+    assert C == 64
+    phi = np.empty_like(a); psi = np.empty_like(a); pi = np.empty((4, dk))
+    for Q in range(4):
+        blk = a[16 * Q:16 * Q + 16]
+        phi[16 * Q:16 * Q + 16] = np.cumprod(blk, axis=0)
+        for i in range(16):
+            psi[16 * Q + i] = np.prod(blk[i + 1:], axis=0)
+        pi[Q] = phi[16 * Q + 15]
+    dq = [1 / pi[0], np.ones(dk), 1 / pi[2], np.ones(dk)]
+    c0 = [np.ones(dk), 1 / pi[1]]
+    c1 = [pi[1] * pi[2], pi[2], np.ones(dk), 1 / pi[3]]
+    lam = np.array([phi[r] * dq[r // 16] for r in range(64)])
+    rho0 = np.array([psi[j] * c0[j // 16] for j in range(32)])
+    rho1 = np.array([psi[j] * c1[j // 16] for j in range(64)])
+    return lam, rho0, rho1
+
+
+@pytest.mark.parametrize("extreme", [False, True])
+def test_mid_reference_factorization(extreme):
+    rng = np.random.default_rng(77 + extreme)
+    a = np.exp(-np.log1p(np.exp(rng.standard_normal((64, 16)))))
+    if extreme:
+        a[:, :4] = np.exp(-5.0)
+        a[:, 4:8] = 1.0
+    lam, rho0, rho1 = mid_reference_factors(a)
+    for r in range(64):
+        for j in range(r + 1):
+            D = np.prod(a[j + 1:r + 1], axis=0)
+            rho = rho0[j] if r < 32 else rho1[j]
+            np.testing.assert_allclose(lam[r] * rho, D, rtol=1e-12, atol=0)
+    lo = np.log(np.float64(np.float32(np.exp(-5.0))))
+    assert np.log(lam).min() >= 16 * lo - 1e-9 and np.log(lam).max() <= -15 * lo + 1e-9
+    assert np.log(rho0).max() <= -16 * lo + 1e-9 and np.log(rho1).max() <= -16 * lo + 1e-9
 
 
 def _case(seed, T, dk, dv, extreme=False):
