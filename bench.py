@@ -435,7 +435,8 @@ def run_ours(args, w):
     ms_per_step = elapsed_ms / args.steps
 
     # end to end: pinned host inputs -> device -> kda_forward -> host results
-    e2e = run_e2e(args, w, inp, dev, stream, world) if w.kind != "decode" else None
+    e2e = run_e2e(args, w, inp, dev, stream, world) if w.kind != "decode" and args.e2e_steps > 0 \
+        else None
 
     if rank == 0:
         achieved = algo_bytes / (kern_ms * 1e-3) / 1e9
@@ -504,7 +505,7 @@ def run_e2e(args, w, inp, dev, stream, world):
         out_h.copy_(out, non_blocking=True)
         Sf_h.copy_(Sf, non_blocking=True)
 
-    n = max(2, min(args.steps, 10))
+    n = max(1, min(args.steps, args.e2e_steps))
     for _ in range(2):
         step()
     torch.cuda.synchronize()
@@ -533,6 +534,8 @@ def main():
     ap.add_argument("--cpu-budget", type=float, default=15.0,
                     help="seconds of oracle time for the cpu_baseline sample")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--e2e-steps", type=int, default=10,
+                    help="steps of the end-to-end (host buffers) measurement; 0 skips it")
     args = ap.parse_args()
     from gated_delta_rule_138_b200 import inputs as gen
     w = gen.WORKLOADS[args.workload]

@@ -153,7 +153,14 @@ kda_chunk_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_consta
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int q4 = warp & 3;            // TMEM lane quarter this warp may touch
     const int hf = warp >> 2;           // which half of the columns this warp handles
-    const int h = blockIdx.y, n = blockIdx.z;
+    const int h = blockIdx.y;
+    __shared__ int s_seq;
+    if (threadIdx.x < 32) {
+        const int sq = longest_first_seq(cu_seqlens, (int)gridDim.z, (int)blockIdx.z, T);
+        if (threadIdx.x == 0) s_seq = sq;
+    }
+    __syncthreads();
+    const int n = s_seq;
     int64_t bos, len;
     seq_range(cu_seqlens, n, T, bos, len);
     const int nchunks = (int)((len + C - 1) / C);

@@ -48,4 +48,35 @@ __device__ __forceinline__ void seq_range(const int32_t* __restrict__ cu_seqlens
     len = b - a;
 }
 
+// Longest-first schedule for packed batches: CTAs are launched in blockIdx.z
+// order, so z-th CTA column takes the sequence of rank z in decreasing length
+// (ties by index).  Each CTA ranks the lengths itself from cu_seqlens: no
+// workspace, O(num_seqs^2) work, used only up to kMaxRankedSeqs sequences.
+constexpr int kMaxRankedSeqs = 1024;
+__device__ __forceinline__ int64_t seq_len_at(const int32_t* __restrict__ cu, int i, int64_t T) {
+    int64_t a = cu[i], b = cu[i + 1];
+    a = a < 0 ? 0 : (a > T ? T : a);
+    b = b < a ? a : (b > T ? T : b);
+    return b - a;
+}
+// Warp-collective (call from one full warp): the sequence of rank z.
+__device__ __forceinline__ int longest_first_seq(const int32_t* __restrict__ cu, int nseq, int z,
+                                                 int64_t T) {
+    if (cu == nullptr || nseq > kMaxRankedSeqs) return z;
+    const int lane = threadIdx.x & 31;
+    int found = -1;
+    for (int i = lane; i < nseq; i += 32) {
+        const int64_t li = seq_len_at(cu, i, T);
+        int rank = 0;
+        for (int j = 0; j < nseq; ++j) {
+            const int64_t lj = seq_len_at(cu, j, T);
+            rank += (lj > li) || (lj == li && j < i);
+        }
+        if (rank == z) found = i;
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) found = max(found, __shfl_xor_sync(0xffffffffu, found, o));
+    return found < 0 ? z : found;
+}
+
 }  // namespace kda
