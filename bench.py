@@ -74,10 +74,13 @@ def load_peaks():
         return dict(FALLBACK_PEAKS), "fallback"
 
 
-def kernel_source_digest(name: str) -> str:
-    path = os.path.join(ROOT, "gated_delta_rule_138_b200", "csrc", name)
-    with open(path, "rb") as fh:
-        return hashlib.sha256(fh.read()).hexdigest()[:16]
+def kernel_source_digest(names: str) -> str:
+    """sha256 (16 hex digits) of the concatenated csrc files, comma-separated."""
+    h = hashlib.sha256()
+    for name in names.split(","):
+        with open(os.path.join(ROOT, "gated_delta_rule_138_b200", "csrc", name), "rb") as fh:
+            h.update(fh.read())
+    return h.hexdigest()[:16]
 
 
 def recorded_traffic(kernel: str, workload: str):
