@@ -196,29 +196,18 @@ def dist_setup(n_gpus: int):
 
 
 def barrier(world):
-    if world > 1:
-        import torch.distributed as dist
-        dist.barrier()
+    from gated_delta_rule_138_b200 import ranks
+    ranks.barrier(world)
 
 
 def max_over_ranks(x: float, world: int) -> float:
-    if world == 1:
-        return x
-    import torch
-    import torch.distributed as dist
-    t = torch.tensor([x], dtype=torch.float64, device="cuda")
-    dist.all_reduce(t, op=dist.ReduceOp.MAX)
-    return float(t.item())
+    from gated_delta_rule_138_b200 import ranks
+    return ranks.reduce_max(x, world, device="cuda")
 
 
 def sum_over_ranks(x: float, world: int) -> float:
-    if world == 1:
-        return x
-    import torch
-    import torch.distributed as dist
-    t = torch.tensor([x], dtype=torch.float64, device="cuda")
-    dist.all_reduce(t, op=dist.ReduceOp.SUM)
-    return float(t.item())
+    from gated_delta_rule_138_b200 import ranks
+    return ranks.reduce_sum(x, world, device="cuda")
 
 
 def make_inputs(w, device, seed_offset: int):
@@ -368,7 +357,8 @@ def run_ours(args, w):
 
     rank, world, local = dist_setup(args.gpus)
     dev = torch.device("cuda", local)
-    inp = make_inputs(w, dev, 1000 * rank)
+    from gated_delta_rule_138_b200 import ranks
+    inp = make_inputs(w, dev, ranks.rank_seed_offset(rank))
     tokens, n_th, n_sh = counts(w, inp)
     peaks, peak_src = load_peaks()
     stream = torch.cuda.current_stream()
@@ -434,7 +424,7 @@ def run_ours(args, w):
     kern_ms = statistics.mean(a.elapsed_time(b) for a, b in ev)
     kern_ms = max_over_ranks(kern_ms, world)
     total_tokens = sum_over_ranks(tokens * args.steps, world)
-    value = total_tokens / (elapsed_ms * 1e-3)
+    value = ranks.weak_scaling_throughput(total_tokens, elapsed_ms)
     ms_per_step = elapsed_ms / args.steps
 
     # end to end: pinned host inputs -> device -> kda_forward -> host results

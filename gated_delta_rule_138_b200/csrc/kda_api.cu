@@ -9,6 +9,7 @@
 
 #include "../../include/kda.h"
 #include "kda_common.cuh"
+#include "kda_sm100.cuh"
 
 namespace kda {
 cudaError_t launch_chunk_simt(int in_bf16, int out_bf16, int chunk, const void* q, const void* k,
@@ -73,6 +74,20 @@ bool debug_sync() {
     return v && v[0] && v[0] != '0';
 }
 
+// Waits, bounded by limit_ns, on an mbarrier that nothing ever arrives on, and
+// records the timeout in the device status word exactly as the forward kernel
+// does.  No fault, no hang: the wait gives up and the kernel returns.
+__global__ void kda_selftest_wait_kernel(int* status, uint64_t limit_ns) {
+    __shared__ uint64_t bar;
+    if (threadIdx.x == 0) {
+        kda::sm100::mbar_init(&bar, 1);
+        kda::sm100::mbar_fence_init();
+    }
+    __syncthreads();
+    const bool done = kda::sm100::mbar_wait_ns(&bar, 0, limit_ns);
+    if (!done && threadIdx.x == 0) atomicExch(status, 1);
+}
+
 }  // namespace
 
 namespace kda {
@@ -129,6 +144,16 @@ size_t kda_forward_workspace_bytes(int32_t B, int64_t T, int32_t H, int32_t d_k,
                                    int32_t chunk) {
     (void)B; (void)T; (void)H; (void)d_k; (void)d_v; (void)chunk;
     return sizeof(int);  // the per-device status word, allocated once
+}
+
+kda_status_t kda_selftest_timeout(uint64_t limit_ns, kda_stream_t stream) {
+    if (limit_ns == 0 || limit_ns > 10000000000ull) return KDA_ERR_INVALID_ARG;
+    int* status = nullptr;
+    cudaError_t e = device_status_word(&status);
+    if (e != cudaSuccess) return cuda_status(e);
+    g_launches.fetch_add(1, std::memory_order_relaxed);
+    kda_selftest_wait_kernel<<<1, 32, 0, reinterpret_cast<cudaStream_t>(stream)>>>(status, limit_ns);
+    return cuda_status(cudaGetLastError());
 }
 
 kda_status_t kda_forward(const void* q, const void* k, const void* v, const void* alpha,

@@ -244,8 +244,15 @@ kda_chunk_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_consta
 
     uint32_t phT = 0, phM = 0;
     bool ok = true;   // this thread has seen every wait complete
+    // asynchronous work that a timed-out wait may leave in flight, drained before exit
+    bool tma_pending = nchunks > 0, mma_pending = false;
+    uint32_t tma_pending_phase = 0, mma_pending_phase = 0;
     auto wait_mma = [&]() {
-        if (ok && !mbar_wait_ns(barM, phM, kWaitNs)) ok = false;
+        if (ok && !mbar_wait_ns(barM, phM, kWaitNs)) {
+            ok = false;
+            mma_pending = true;
+            mma_pending_phase = phM;
+        }
         phM ^= 1u;
         tc_fence_after();
     };
@@ -254,7 +261,10 @@ kda_chunk_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_consta
         const int64_t row0 = bos + (int64_t)chunk * C;
         const int Lc = (int)((len - (int64_t)chunk * C) < C ? (len - (int64_t)chunk * C) : C);
         if (tid < C) sBeta[tid] = beta_next;
-        if (ok && !mbar_wait_ns(barT, phT, kWaitNs)) ok = false;
+        if (ok) {
+            if (mbar_wait_ns(barT, phT, kWaitNs)) tma_pending = false;
+            else ok = false;
+        }
         phT ^= 1u;
         KDA_TC_PHASE(0);
 
@@ -372,7 +382,7 @@ kda_chunk_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_consta
         // ================= [A/beta | P] by sub-chunk: one M=128, N=128, K=128 MMA group
         //   D[j][n]:  rows 0..31  x cols 0..63   = sub-chunk 0 (j < 32; [A/beta | P] columns r)
         //             rows 64..127 x cols 64..127 = sub-chunk 1 (j < 64; columns r - 32)
-        if (tid == 0) {
+        if (tid == 0 && ok) {   // nothing new is issued after a wait gave up
             const uint32_t r0 = smem_u32(sX + X_R), l0 = smem_u32(sX + X_L);
             constexpr uint32_t idesc = idesc_bf16(128, 128);
 #pragma unroll
@@ -509,7 +519,7 @@ kda_chunk_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_consta
             tc_fence_before();
             __syncthreads();
             tc_fence_after();
-            if (tid == 0) {
+            if (tid == 0 && ok) {
                 constexpr uint32_t idesc = idesc_tf32(64, 32);
                 const uint32_t a0 = smem_u32(sX + X_T0T), b0 = smem_u32(sX + X_A10);
 #pragma unroll
@@ -535,7 +545,7 @@ kda_chunk_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_consta
             tc_fence_before();
             __syncthreads();
             tc_fence_after();
-            if (tid == 0) {
+            if (tid == 0 && ok) {
                 constexpr uint32_t idesc = idesc_tf32(64, 32);
                 const uint32_t a0 = smem_u32(sX + X_T1), b0 = smem_u32(sX + X_XT);
 #pragma unroll
@@ -583,7 +593,7 @@ kda_chunk_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_consta
 
         KDA_TC_PHASE(4);
         // ================= [Tb ; P Tb] = [I ; P] Tb   (M=128, N=64, K=64)
-        if (tid == 0) {
+        if (tid == 0 && ok) {
             const uint32_t a0 = smem_u32(sIP), b0 = smem_u32(sX + X_TB);
             constexpr uint32_t idesc = idesc_bf16(128, 64, false, true);
 #pragma unroll
@@ -610,7 +620,7 @@ kda_chunk_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_consta
 
         KDA_TC_PHASE(5);
         // ================= [W ; P W] = [Tb ; P Tb] (k*gamma)   (M=128, N=128, K=64)
-        if (tid == 0) {
+        if (tid == 0 && ok) {
             const uint32_t a0 = smem_u32(sAl), b0 = smem_u32(sKT);
             constexpr uint32_t idesc = idesc_bf16(128, 128);
 #pragma unroll
@@ -656,7 +666,7 @@ kda_chunk_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_consta
 
         KDA_TC_PHASE(6);
         // ================= [U ; O] = [-W ; Q'] S + [Tb ; P Tb] V   (two N=64 halves, K=128+64)
-        if (tid == 0) {
+        if (tid == 0 && ok) {
             const uint32_t wq = smem_u32(sX + X_WQ), s0 = smem_u32(sS), tb = smem_u32(sAl),
                            v0 = smem_u32(sV);
             // B operands are MN-major with two 64-column atoms: leading byte offset = atom stride
@@ -687,7 +697,11 @@ kda_chunk_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_consta
         }
         wait_mma();
         // all of q, k, alpha, v are consumed: prefetch the next chunk
-        if (tid == 0 && chunk + 1 < nchunks) issue_tma(row0 + C);
+        if (chunk + 1 < nchunks && ok) {
+            if (tid == 0) issue_tma(row0 + C);
+            tma_pending = true;
+            tma_pending_phase = phT;
+        }
         if (tid < C) {
             const int64_t nxt = (int64_t)(chunk + 1) * C + tid;   // token index in the sequence
             beta_next = nxt < len ? __bfloat162float(beta[(size_t)(bos + nxt) * H + h]) : 0.0f;
@@ -714,7 +728,7 @@ kda_chunk_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_consta
 
         KDA_TC_PHASE(7);
         // ================= S += (k*eta)^T U   (M=128, two N=64 halves, K=64)
-        if (tid == 0) {
+        if (tid == 0 && ok) {
             const uint32_t a0 = smem_u32(sKH), u0 = smem_u32(sX + X_U);
             constexpr uint32_t idesc = idesc_bf16(128, 128, false, true);
 #pragma unroll
@@ -741,6 +755,15 @@ kda_chunk_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_consta
     }
 
     if (!ok) atomicExch(sFlag, 1);
+    __syncthreads();
+    if (*sFlag && tid == 0) {
+        // a wait gave up: let this CTA's own copies and MMAs in flight finish (bounded)
+        // before its shared and tensor memory are released.  Thread 0 issues every
+        // copy and MMA and stops issuing once one of its own waits gives up, so at
+        // most one of each is outstanding here.
+        if (tma_pending) mbar_wait_ns(barT, tma_pending_phase, kWaitNs);
+        if (mma_pending) mbar_wait_ns(barM, mma_pending_phase, kWaitNs);
+    }
     __syncthreads();
     if (kCtaStatus && tid == 0) status[(size_t)n * H + h] = *sFlag;
     if (*sFlag) {

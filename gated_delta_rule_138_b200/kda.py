@@ -76,6 +76,8 @@ def load_library(build_if_missing: bool = True) -> ctypes.CDLL:
     lib.kda_launch_count.argtypes = []
     lib.kda_device_status.restype = ctypes.c_int
     lib.kda_device_status.argtypes = [vp]
+    lib.kda_selftest_timeout.restype = ctypes.c_int
+    lib.kda_selftest_timeout.argtypes = [ctypes.c_uint64, vp]
     lib.kda_forward_noalloc.restype = ctypes.c_int
     lib.kda_forward_noalloc.argtypes = lib.kda_forward.argtypes
     _lib = lib
@@ -126,6 +128,12 @@ def kda_forward_kernel_name(d_k: int, d_v: int, chunk: int, in_dtype: torch.dtyp
 def kda_device_status(stream=None) -> None:
     """Synchronise `stream` and raise KdaError if a kernel reported a device timeout."""
     _check("kda_device_status", load_library().kda_device_status(_stream(stream)))
+
+
+def kda_selftest_timeout(limit_ns: int = 1_000_000, stream=None) -> None:
+    """Launch a wait that must time out (nothing arrives) and record it; check
+    it with kda_device_status()."""
+    _check("kda_selftest_timeout", load_library().kda_selftest_timeout(int(limit_ns), _stream(stream)))
 
 
 def kda_launch_count() -> int:

@@ -152,6 +152,16 @@ uint64_t kda_launch_count(void);
 kda_status_t kda_device_status(kda_stream_t stream);
 
 /*
+ * Self-test of the device-timeout path (no counterpart on the pages).  Launches
+ * one warp that waits, bounded by limit_ns nanoseconds (1 ns .. 10 s), on an
+ * mbarrier that nothing ever arrives on, using the same bounded wait as the
+ * tensor-core kernel; when the wait gives up the kernel sets the device status
+ * word and returns.  A following kda_device_status reports
+ * KDA_ERR_DEVICE_TIMEOUT (and clears the word).  Nothing faults or hangs.
+ */
+kda_status_t kda_selftest_timeout(uint64_t limit_ns, kda_stream_t stream);
+
+/*
  * Capacity of kda_forward_noalloc's fixed scratch: (sequence, head) pairs per call.
  */
 #define KDA_NOALLOC_MAX_SEQ_HEADS 16384

@@ -88,3 +88,9 @@ def test_decode_rejects_before_launch():
 
 def test_workspace_query_is_host_only():
     assert kda.kda_forward_workspace_bytes(8, 4096, 32, 128, 128, 64) >= 0
+
+
+def test_selftest_rejects_bad_limit():
+    lib = kda.load_library()
+    assert lib.kda_selftest_timeout(0, None) == 1
+    assert lib.kda_selftest_timeout(20_000_000_000, None) == 1

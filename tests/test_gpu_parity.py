@@ -254,3 +254,19 @@ def test_tc_matches_fp32_path():
     torch.cuda.synchronize()
     assert rel_l2(np32(o_tc), np32(o_f)) <= 2e-2
     assert rel_l2(np32(S_tc), np32(S_f)) <= 2e-2
+
+
+# ------------------------------------------------ failure detection (no fault, no hang)
+
+def test_bounded_wait_reports_timeout_and_context_survives():
+    """A wait on a barrier that nothing arrives on gives up after its limit and
+    reports KDA_ERR_DEVICE_TIMEOUT through the status word; the context stays
+    usable and a later forward is still correct."""
+    kda.kda_device_status()                       # clean slate
+    kda.kda_selftest_timeout(2_000_000)           # 2 ms limit
+    with pytest.raises(kda.KdaError) as ei:
+        kda.kda_device_status()
+    assert ei.value.status == 4                   # KDA_ERR_DEVICE_TIMEOUT
+    kda.kda_device_status()                       # cleared by the read
+    _, out, Sf, ro, rS = _forward_case(1, 100, 2, 128, 128, "bf16", 64, True, 808)
+    assert rel_l2(np32(out), ro) <= 2e-2 and rel_l2(np32(Sf), rS) <= 2e-2
