@@ -375,6 +375,7 @@ def run_ours(args, w):
             kda.kda_decode_step(inp["q"][i], inp["k"][i], inp["v"][i], inp["alpha"][i],
                                 inp["beta"][i], S, out=out)
         kname = "decode_f32state"
+        segments = None
         algo_bytes = decode_bytes(w, n_sh)
         algo_flops = decode_flops(w, n_sh)
         src_file = "kda_decode.cu"
@@ -390,6 +391,10 @@ def run_ours(args, w):
             kda.kda_forward(inp["q"], inp["k"], inp["v"], inp["alpha"], inp["beta"], inp["S0"],
                             cu_seqlens=cu, out=out, S_final=Sf, chunk=w.chunk)
         kname = kda.kda_forward_kernel_name(w.dk, w.dv, w.chunk, inp["q"].dtype, out.dtype)
+        # time segments per sequence of the tensor-core path (1: unsplit); with g > 1 a
+        # step is three launches (segment maps, scan, forward) timed together
+        segments = (kda.kda_forward_segments(nseq, -(-B * T // nseq), w.H)
+                    if kname == "chunk_tc_bf16" else 1)
         algo_bytes = forward_bytes(w, n_th, n_sh, inp["S0"] is not None)
         algo_flops = forward_flops(w, n_th)
         src_file = "kda_chunk_tc.cu" if kname == "chunk_tc_bf16" else "kda_chunk_simt.cu"
@@ -447,7 +452,8 @@ def run_ours(args, w):
             "roofline": {"bound": "hbm", "achieved": achieved, "peak": peaks["hbm_gbs"],
                          "unit": "GB/s", "frac": achieved / peaks["hbm_gbs"],
                          "traffic": recorded_traffic(kname, w.name),
-                         "kernel": kname, "algorithmic_bytes": algo_bytes,
+                         "kernel": kname, "time_segments": segments,
+                         "algorithmic_bytes": algo_bytes,
                          "kernel_ms": kern_ms, "peak_source": peak_src},
             "tensor": {"achieved_tflops": tflops, "peak": peaks["bf16_tflops"],
                        "frac": tflops / peaks["bf16_tflops"], "flops_per_step": algo_flops},

@@ -2,6 +2,7 @@
 // dispatch to the kernels.  No entry point allocates on the caller's behalf
 // beyond the library-owned workspace, synchronises the device, or throws.
 #include <atomic>
+#include <cmath>
 #include <cstdio>
 #include <cstdlib>
 #include <cstring>
@@ -23,6 +24,12 @@ cudaError_t launch_chunk_tc(const void* q, const void* k, const void* v, const v
                             const void* beta, const float* S0, const int32_t* cu, int nseq,
                             void* out, float* S_final, int64_t rows, int64_t T, int H, int* status,
                             cudaStream_t stream);
+size_t chunk_tc_segmented_workspace_floats(int64_t nseq, int H, int nseg);
+cudaError_t launch_chunk_tc_segmented(const void* q, const void* k, const void* v,
+                                      const void* alpha, const void* beta, const float* S0,
+                                      const int32_t* cu, int nseq, void* out, float* S_final,
+                                      int64_t rows, int64_t T, int H, int nseg, float* workspace,
+                                      int* status, cudaStream_t stream);
 }  // namespace kda
 
 namespace {
@@ -67,6 +74,40 @@ cudaError_t device_status_word(int** out) {
     }
     *out = g_status[dev];
     return cudaSuccess;
+}
+
+// Time segments per sequence for the tensor-core forward.  One CTA runs one
+// (sequence, head) segment on one SM and a segment costs in proportion to its
+// chunks; a split adds a summary pass (about 0.7 of a forward chunk) over all
+// but the last segment.  The cost, in units of the unsplit CTA's time, of g
+// segments is (waves of the forward + 0.7 waves of the summaries) / g, with
+// waves = ceil(CTAs / SMs); g = 1 costs ceil(units / SMs).  A small charge per
+// segment stands for the scan and launch overheads.  Segments keep >= 16 chunks.
+int segments_for(int64_t nseq, int64_t tokens_per_seq, int64_t H, int sms) {
+    const int64_t units = nseq * H;
+    if (units <= 0 || sms <= 0) return 1;
+    const int64_t chunks = (tokens_per_seq + 63) / 64;
+    const auto waves = [&](int64_t ctas) { return (double)((ctas + sms - 1) / sms); };
+    double best = waves(units);
+    int best_g = 1;
+    for (int g = 2; g <= 64 && chunks >= (int64_t)g * 16 && nseq * g <= 65535; ++g) {
+        const double cost = (waves(units * g) + 0.7 * waves(units * (g - 1))) / g + 0.002 * g;
+        if (cost < best) {
+            best = cost;
+            best_g = g;
+        }
+    }
+    return best_g;
+}
+
+int current_sms() {
+    int dev = 0, sms = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess ||
+        cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) {
+        cudaGetLastError();
+        return 148;   // no device visible: assume a B200
+    }
+    return sms;
 }
 
 bool debug_sync() {
@@ -142,8 +183,17 @@ kda_status_t kda_device_status(kda_stream_t stream) {
 
 size_t kda_forward_workspace_bytes(int32_t B, int64_t T, int32_t H, int32_t d_k, int32_t d_v,
                                    int32_t chunk) {
-    (void)B; (void)T; (void)H; (void)d_k; (void)d_v; (void)chunk;
-    return sizeof(int);  // the per-device status word, allocated once
+    size_t bytes = sizeof(int);  // the per-device status word, allocated once
+    if (B > 0 && T > 0 && H > 0 && use_tc(d_k, d_v, chunk, KDA_BF16, KDA_BF16)) {
+        const int nseg = segments_for(B, T, H, current_sms());
+        bytes += sizeof(float) * kda::chunk_tc_segmented_workspace_floats(B, H, nseg);
+    }
+    return bytes;
+}
+
+int32_t kda_forward_segments(int32_t num_seqs, int64_t tokens_per_seq, int32_t H, int32_t num_sms) {
+    if (num_seqs <= 0 || tokens_per_seq <= 0 || H <= 0) return 1;
+    return segments_for(num_seqs, tokens_per_seq, H, num_sms > 0 ? num_sms : current_sms());
 }
 
 kda_status_t kda_selftest_timeout(uint64_t limit_ns, kda_stream_t stream) {
@@ -186,8 +236,28 @@ kda_status_t kda_forward(const void* q, const void* k, const void* v, const void
         if (e != cudaSuccess) return cuda_status(e);
         const int64_t rows = cu_seqlens ? T : (int64_t)B * T;
         if (rows > 0x7fffffffLL) return KDA_ERR_UNSUPPORTED;  // TMA row coordinate is int32
-        e = kda::launch_chunk_tc(q, k, v, alpha, beta, S0, cu_seqlens, (int)nseq, out, S_final,
-                                 rows, T, H, status, s);
+        const int64_t per_seq = cu_seqlens ? (T + nseq - 1) / nseq : T;
+        const int nseg = segments_for(nseq, per_seq, H, current_sms());
+        float* ws = nullptr;
+        if (nseg > 1) {
+            // stream-ordered workspace for the segment maps and start states; if it
+            // cannot be had, the unsplit kernel computes the same result
+            const size_t bytes = sizeof(float) * kda::chunk_tc_segmented_workspace_floats(nseq, H, nseg);
+            if (cudaMallocAsync(reinterpret_cast<void**>(&ws), bytes, s) != cudaSuccess) {
+                cudaGetLastError();
+                ws = nullptr;
+            }
+        }
+        if (ws) {
+            g_launches.fetch_add(2, std::memory_order_relaxed);   // three kernels in all
+            e = kda::launch_chunk_tc_segmented(q, k, v, alpha, beta, S0, cu_seqlens, (int)nseq,
+                                               out, S_final, rows, T, H, nseg, ws, status, s);
+            const cudaError_t ef = cudaFreeAsync(ws, s);
+            if (e == cudaSuccess) e = ef;
+        } else {
+            e = kda::launch_chunk_tc(q, k, v, alpha, beta, S0, cu_seqlens, (int)nseq, out, S_final,
+                                     rows, T, H, status, s);
+        }
         if (e != cudaSuccess) return cuda_status(e);
         return debug_sync() ? kda_device_status(stream) : KDA_OK;
     }

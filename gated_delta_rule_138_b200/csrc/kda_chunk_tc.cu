@@ -23,10 +23,19 @@
 // so the 16-row block I of [A/beta | P] is  [k phi ; q phi]_I  times  R^(I)^T with
 // R^(I)_j = k_j psi_j Dp_{I,J(j)} for j < end(I): one M=64 tcgen05 MMA per I.
 //
-// One CTA (256 threads) owns one (sequence, head) and walks its chunks in
-// order.  Thread 0 issues the TMA loads and the MMAs; all eight warps do the
-// element-wise work.  TMEM (512 columns): S fp32 [0,128), U|O accumulator
-// [128,256), scratch accumulators [256,384).
+// One CTA (256 threads) owns one (sequence, head) -- or one segment of it --
+// and walks its chunks in order.  Thread 0 issues the TMA loads and the MMAs;
+// all eight warps do the element-wise work.  TMEM (512 columns): S fp32
+// [0,128), U|O accumulator [128,256), scratch accumulators [256,512).
+//
+// Long sequences with few (sequence, head) pairs are also split along time
+// into segments (the prefix scan of paragraph 3, within one GPU).  Over a
+// segment the state map is affine, S_end = M S_start + N with M (d_k x d_k) and
+// N (d_k x d_v); per chunk M_c = Diag(gamma_C) - (k*eta)^T W and
+// N_c = (k*eta)^T Tb V.  The same kernel in "summary" mode runs the chunk
+// recurrence on [M | N] from [I | 0] (no outputs); a small scan kernel chains
+// S_{g+1} = M_g S_g + N_g in fp32; the forward kernel then runs every segment
+// from its own start state.
 #include <cuda.h>
 
 #include "kda_common.cuh"
@@ -121,27 +130,41 @@ __device__ __forceinline__ uint4 pack8(const float* v) {
 // M=64 accumulator: row m lives in TMEM lane 32*(m/16) + m%16
 // M=128 accumulator: row m lives in lane m.
 
+// Time segments.  Sequence n's chunks are cut into `nseg` runs of
+// ceil(chunks / nseg) chunks (the last ones may be shorter or empty); CTA z of
+// a launch takes segment z % per_seq of the sequence of rank z / per_seq.
+struct Segments {
+    int nseg;             // segments per sequence (1: whole sequences)
+    int per_seq;          // segment CTAs per sequence in this launch
+    const float* start;   // forward with nseg > 1: start states [nseq * nseg, H, DK, DV]
+    float* maps;          // summary: [M | N] fp32 [nseq * (nseg - 1), H, DK, DK + DV]
+};
+
 // kCtaStatus = false: a timed-out wait sets the shared word *status to 1.
 // kCtaStatus = true:  every CTA writes its own word status[n * H + h] (0 or 1).
-template <bool kCtaStatus>
+// kSummary = true: the segment-map mode described at the top (q and out unused).
+template <bool kCtaStatus, bool kSummary>
 __global__ void __launch_bounds__(NT, 1)
 kda_chunk_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                     const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmV,
                     const __nv_bfloat16* __restrict__ beta, const float* S0,
                     const int32_t* __restrict__ cu_seqlens, __nv_bfloat16* __restrict__ out,
-                    float* S_final, int64_t T, int H, int* status) {
+                    float* S_final, int64_t T, int H, int* status, const Segments seg) {
     extern __shared__ uint8_t smem_raw[];
     uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~static_cast<uintptr_t>(1023));
+    // A summary loads no q tile: everything after it moves down 16 KB, and the
+    // bf16 copy of [M | N] (four 64-column atoms, 64 KB) ends where MISC starts.
+    constexpr uint32_t kSh = kSummary ? 16384u : 0u;
     uint8_t* sQ = sm + OFF_Q;
-    uint8_t* sK = sm + OFF_K;
-    uint8_t* sAl = sm + OFF_AL;
-    uint8_t* sV = sm + OFF_V;
-    uint8_t* sX = sm + OFF_X;
-    uint8_t* sKT = sm + OFF_KT;
-    uint8_t* sKH = sm + OFF_KH;
+    uint8_t* sK = sm + OFF_K - kSh;
+    uint8_t* sAl = sm + OFF_AL - kSh;
+    uint8_t* sV = sm + OFF_V - kSh;
+    uint8_t* sX = sm + OFF_X - kSh;
+    uint8_t* sKT = sm + OFF_KT - kSh;
+    uint8_t* sKH = sm + OFF_KH - kSh;
     uint8_t* sIP = sm + OFF_IP;
-    uint8_t* sS = sm + OFF_S;
+    uint8_t* sS = kSummary ? sm + OFF_KH : sm + OFF_S;
     float* sPi = reinterpret_cast<float*>(sm + OFF_MISC + MISC_PI);
     float* sGC = reinterpret_cast<float*>(sm + OFF_MISC + MISC_GC);
     float* sBeta = reinterpret_cast<float*>(sm + OFF_MISC + MISC_BETA);
@@ -154,16 +177,26 @@ kda_chunk_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_consta
     const int q4 = warp & 3;            // TMEM lane quarter this warp may touch
     const int hf = warp >> 2;           // which half of the columns this warp handles
     const int h = blockIdx.y;
+    const int per_seq = seg.per_seq, gseg = (int)blockIdx.z % per_seq;
     __shared__ int s_seq;
     if (threadIdx.x < 32) {
-        const int sq = longest_first_seq(cu_seqlens, (int)gridDim.z, (int)blockIdx.z, T);
+        const int sq = longest_first_seq(cu_seqlens, (int)gridDim.z / per_seq,
+                                         (int)blockIdx.z / per_seq, T);
         if (threadIdx.x == 0) s_seq = sq;
     }
     __syncthreads();
     const int n = s_seq;
     int64_t bos, len;
     seq_range(cu_seqlens, n, T, bos, len);
+    if (seg.nseg > 1) {   // this CTA's segment of the sequence
+        const int64_t nch = (len + C - 1) / C, cps = (nch + seg.nseg - 1) / seg.nseg;
+        const int64_t c0 = min((int64_t)gseg * cps, nch), c1 = min((int64_t)(gseg + 1) * cps, nch);
+        const int64_t t0 = min(c0 * C, len), t1 = min(c1 * C, len);
+        bos += t0;
+        len = t1 - t0;
+    }
     const int nchunks = (int)((len + C - 1) / C);
+    const bool last_seg = gseg == seg.nseg - 1;
 
     if (tid == 0) {
         mbar_init(barT, 1);
@@ -173,6 +206,7 @@ kda_chunk_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_consta
     }
     if (warp == 0) tmem_alloc(sTmem, 512);
     // identity rows of [I ; P]
+    if (!kSummary)
     for (int i = tid; i < 64 * 8; i += NT) {
         const int r = i >> 3, ch = i & 7;
         uint32_t w[4] = {0, 0, 0, 0};
@@ -183,6 +217,7 @@ kda_chunk_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_consta
         *reinterpret_cast<uint4*>(sIP + swz(r, ch)) = make_uint4(w[0], w[1], w[2], w[3]);
     }
     // P[r][j] = 0 for r < 32 <= j: never written by the per-chunk extraction
+    if (!kSummary)
     for (int i = tid; i < 32 * 4; i += NT) {
         const int r = i >> 2, ch = 4 + (i & 3);
         *reinterpret_cast<uint4*>(sIP + swz(64 + r, ch)) = make_uint4(0u, 0u, 0u, 0u);
@@ -194,9 +229,27 @@ kda_chunk_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_consta
     const uint32_t tlane = (uint32_t)(32 * q4) << 16;
 
     // ---- initial state: TMEM S (fp32) and its bf16 copy (MN-major B operand)
-    {
+    if constexpr (kSummary) {
+        // [M | N] = [I | 0]; this warp writes row c, columns 128 hf .. 128 hf + 127
         const int c = 32 * q4 + lane;
-        const float* src = S0 ? S0 + (((size_t)n * H + h) * DK + c) * DV + 64 * hf : nullptr;
+#pragma unroll
+        for (int blk = 0; blk < 8; ++blk) {
+            float v[16];
+#pragma unroll
+            for (int i = 0; i < 16; ++i) v[i] = (128 * hf + 16 * blk + i == c) ? 1.0f : 0.0f;
+            tmem_st16(tmem + tlane + TM_S + 128 * hf + 16 * blk, v);
+#pragma unroll
+            for (int ch = 0; ch < 2; ++ch)
+                *reinterpret_cast<uint4*>(sS + (2 * hf + (blk >> 2)) * 16384 +
+                                          swz(c, 2 * (blk & 3) + ch)) = pack8(&v[8 * ch]);
+        }
+        tmem_wait_st();
+    } else {
+        const int c = 32 * q4 + lane;
+        const float* base = seg.nseg > 1
+                                ? seg.start + (((size_t)n * seg.nseg + gseg) * H + h) * DK * DV
+                                : (S0 ? S0 + ((size_t)n * H + h) * DK * DV : nullptr);
+        const float* src = base ? base + (size_t)c * DV + 64 * hf : nullptr;
 #pragma unroll
         for (int blk = 0; blk < 4; ++blk) {
             float v[16];
@@ -221,12 +274,12 @@ kda_chunk_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_consta
     }
 
     auto issue_tma = [&](int64_t row0) {
-        mbar_arrive_expect_tx(barT, 4 * 16384);
+        mbar_arrive_expect_tx(barT, (kSummary ? 3 : 4) * 16384);
         const int y = (int)row0;
 #pragma unroll
         for (int a = 0; a < 2; ++a) {
             const int x = h * DK + 64 * a;
-            tma_load_2d(sQ + a * 8192, &tmQ, barT, x, y);
+            if (!kSummary) tma_load_2d(sQ + a * 8192, &tmQ, barT, x, y);
             tma_load_2d(sK + a * 8192, &tmK, barT, x, y);
             tma_load_2d(sAl + a * 8192, &tmA, barT, x, y);
             tma_load_2d(sV + a * 8192, &tmV, barT, h * DV + 64 * a, y);
@@ -255,6 +308,19 @@ kda_chunk_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_consta
         }
         phM ^= 1u;
         tc_fence_after();
+    };
+
+    // all of k, alpha, v (and q) of this chunk are consumed: load the next one
+    auto prefetch_next = [&](int chunk, int64_t row0) {
+        if (chunk + 1 < nchunks && ok) {
+            if (tid == 0) issue_tma(row0 + C);
+            tma_pending = true;
+            tma_pending_phase = phT;
+        }
+        if (tid < C) {
+            const int64_t nxt = (int64_t)(chunk + 1) * C + tid;   // token index in the segment
+            beta_next = nxt < len ? __bfloat162float(beta[(size_t)(bos + nxt) * H + h]) : 0.0f;
+        }
     };
 
     for (int chunk = 0; chunk < nchunks; ++chunk) {
@@ -349,16 +415,16 @@ kda_chunk_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_consta
                 const int r = 16 * Q + i;
                 const uint32_t off = i * 128 + xo[i & 7];
                 float2 kk = ld_bf2(tK + off);
-                float2 qq = ld_bf2(tQ + off);
+                float2 qq = kSummary ? make_float2(0.f, 0.f) : ld_bf2(tQ + off);
                 if (r >= Lc) { kk = make_float2(0.f, 0.f); qq = kk; }
                 const float kp0 = kk.x * phi0[i], kp1 = kk.y * phi1[i];
                 const float qp0 = qq.x * phi0[i], qp1 = qq.y * phi1[i];
                 const float ks0 = kk.x * psi0[i], ks1 = kk.y * psi1[i];
                 st_bf2(tLk + off, kp0 * dl0, kp1 * dl1);
-                st_bf2(tLq + off, qp0 * dl0, qp1 * dl1);
+                if (!kSummary) st_bf2(tLq + off, qp0 * dl0, qp1 * dl1);
                 if (Q < 2) st_bf2(tR0 + off, ks0 * r00, ks1 * r01);
                 st_bf2(tR1 + off, ks0 * r10, ks1 * r11);
-                st_bf2(tQ + off, qp0 * bef0, qp1 * bef1);   // q*gamma in place
+                if (!kSummary) st_bf2(tQ + off, qp0 * bef0, qp1 * bef1);   // q*gamma in place
                 kt0[i] = kp0 * bef0; kt1[i] = kp1 * bef1;    // k*gamma
                 kh0[i] = ks0 * aft0; kh1[i] = ks1 * aft1;    // k*eta
             }
@@ -411,7 +477,7 @@ kda_chunk_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_consta
                     const int r = 32 * sub + rr;
                     Am[r * AS + j] = (j < r) ? sBeta[r] * v[rr] : 0.0f;
                 }
-            } else {
+            } else if (!kSummary) {
 #pragma unroll
                 for (int rr = 0; rr < 32; ++rr) {
                     const int r = 32 * sub + rr;
@@ -570,8 +636,10 @@ kda_chunk_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_consta
             tc_fence_before();
             __syncthreads();
             KDA_TC_PHASE(11);
-            // Tb = Tinv diag(beta) as MN-major B: row j, column m; zero above the diagonal
-            uint8_t* sTB = sX + X_TB;
+            // Tb = Tinv diag(beta) as MN-major B: row j, column m; zero above the diagonal.
+            // The same bytes are Tb as a K-major A operand (row j, k = m): a summary
+            // needs no P Tb and writes it straight to where [Tb ; P Tb] goes.
+            uint8_t* sTB = kSummary ? sAl : sX + X_TB;
 #pragma unroll
             for (int rep = 0; rep < 2; ++rep) {
                 const int e = tid + NT * rep;
@@ -593,6 +661,7 @@ kda_chunk_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_consta
 
         KDA_TC_PHASE(4);
         // ================= [Tb ; P Tb] = [I ; P] Tb   (M=128, N=64, K=64)
+        if (!kSummary) {
         if (tid == 0 && ok) {
             const uint32_t a0 = smem_u32(sIP), b0 = smem_u32(sX + X_TB);
             constexpr uint32_t idesc = idesc_bf16(128, 64, false, true);
@@ -617,6 +686,7 @@ kda_chunk_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_consta
         tc_fence_before();
         __syncthreads();
         tc_fence_after();
+        }
 
         KDA_TC_PHASE(5);
         // ================= [W ; P W] = [Tb ; P Tb] (k*gamma)   (M=128, N=128, K=64)
@@ -643,7 +713,7 @@ kda_chunk_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_consta
                     for (int i = 0; i < 8; ++i) w8[i] = -v[8 * chunk + i];
                     *reinterpret_cast<uint4*>(sWQ + hf * 16384 + swz(row, chunk)) = pack8(w8);
                 }
-            } else {
+            } else if (!kSummary) {
 #pragma unroll
                 for (int chunk = 0; chunk < 8; ++chunk) {
                     const uint4 qg = *reinterpret_cast<const uint4*>(sQ + hf * 8192 + swz(row - 64, chunk));
@@ -665,6 +735,83 @@ kda_chunk_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_consta
         tc_fence_after();
 
         KDA_TC_PHASE(6);
+        if constexpr (kSummary) {
+        // ================= [U_M | U_N] = -W [M | N] + [0 | Tb V]   (M=128 of which rows
+        // 0..63 are used, N=256, K=128 (+64 for the N half))
+        if (tid == 0 && ok) {
+            const uint32_t wq = smem_u32(sX + X_WQ), s0 = smem_u32(sS), tb = smem_u32(sAl),
+                           v0 = smem_u32(sV);
+            const uint32_t d = tmem + TM_WK;
+            constexpr uint32_t idesc256 = idesc_bf16(128, 256, false, true);
+            constexpr uint32_t idesc128 = idesc_bf16(128, 128, false, true);
+#pragma unroll
+            for (int ks = 0; ks < 8; ++ks)
+                mma_bf16(d, sdesc_sw128(wq + (ks >> 2) * 16384 + (ks & 3) * 32),
+                         sdesc_sw128(s0 + ks * 2048, 1024, 16384), idesc256, ks > 0);
+#pragma unroll
+            for (int ks = 0; ks < 4; ++ks)
+                mma_bf16(d + 128, sdesc_sw128(tb + ks * 32), sdesc_sw128(v0 + ks * 2048, 1024, 8192),
+                         idesc128, 1);
+            mma_commit(barM);
+        }
+        // meanwhile: [M | N] <- Diag(gamma_C) [M | N] in TMEM
+        {
+            const int c = 32 * q4 + lane;
+            const float g = sGC[c];
+#pragma unroll
+            for (int p = 0; p < 2; ++p) {
+                const uint32_t ta = tmem + tlane + TM_S + 128 * hf + 64 * p;
+                float v[64];
+                tmem_ld64(ta, v);
+#pragma unroll
+                for (int i = 0; i < 64; ++i) v[i] *= g;
+#pragma unroll
+                for (int blk = 0; blk < 4; ++blk)
+                    tmem_st16(ta + 16 * blk, *reinterpret_cast<float(*)[16]>(&v[16 * blk]));
+            }
+            tmem_wait_st();
+        }
+        wait_mma();
+        prefetch_next(chunk, row0);
+        if (q4 < 2) {   // U rows (tokens) 0..63: MN-major B [64 j][256 n], four 8 KB atoms
+            const int row = 32 * q4 + lane;
+#pragma unroll
+            for (int p = 0; p < 2; ++p) {
+                float v[64];
+                tmem_ld64(tmem + tlane + TM_WK + 128 * hf + 64 * p, v);
+#pragma unroll
+                for (int ch = 0; ch < 8; ++ch)
+                    *reinterpret_cast<uint4*>(sX + X_U + (2 * hf + p) * 8192 + swz(row, ch)) =
+                        pack8(&v[8 * ch]);
+            }
+        }
+        fence_async_smem();
+        tc_fence_before();
+        __syncthreads();
+        tc_fence_after();
+        // ================= [M | N] += (k*eta)^T [U_M | U_N]   (M=128, N=256, K=64)
+        if (tid == 0 && ok) {
+            const uint32_t a0 = smem_u32(sKH), u0 = smem_u32(sX + X_U);
+            constexpr uint32_t idesc = idesc_bf16(128, 256, false, true);
+#pragma unroll
+            for (int ks = 0; ks < 4; ++ks)
+                mma_bf16(tmem + TM_S, sdesc_sw128(a0 + ks * 32), sdesc_sw128(u0 + ks * 2048, 1024, 8192),
+                         idesc, 1);
+            mma_commit(barM);
+        }
+        wait_mma();
+        {
+            const int c = 32 * q4 + lane;
+#pragma unroll
+            for (int p = 0; p < 2; ++p) {
+                float v[64];
+                tmem_ld64(tmem + tlane + TM_S + 128 * hf + 64 * p, v);
+#pragma unroll
+                for (int ch = 0; ch < 8; ++ch)
+                    *reinterpret_cast<uint4*>(sS + (2 * hf + p) * 16384 + swz(c, ch)) = pack8(&v[8 * ch]);
+            }
+        }
+        } else {
         // ================= [U ; O] = [-W ; Q'] S + [Tb ; P Tb] V   (two N=64 halves, K=128+64)
         if (tid == 0 && ok) {
             const uint32_t wq = smem_u32(sX + X_WQ), s0 = smem_u32(sS), tb = smem_u32(sAl),
@@ -696,16 +843,7 @@ kda_chunk_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_consta
             tmem_wait_st();
         }
         wait_mma();
-        // all of q, k, alpha, v are consumed: prefetch the next chunk
-        if (chunk + 1 < nchunks && ok) {
-            if (tid == 0) issue_tma(row0 + C);
-            tma_pending = true;
-            tma_pending_phase = phT;
-        }
-        if (tid < C) {
-            const int64_t nxt = (int64_t)(chunk + 1) * C + tid;   // token index in the sequence
-            beta_next = nxt < len ? __bfloat162float(beta[(size_t)(bos + nxt) * H + h]) : 0.0f;
-        }
+        prefetch_next(chunk, row0);
         {
             const int row = 32 * q4 + lane;
             uint8_t* sU = sX + X_U;
@@ -746,6 +884,7 @@ kda_chunk_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_consta
             for (int chunk = 0; chunk < 8; ++chunk)
                 *reinterpret_cast<uint4*>(sS + hf * 16384 + swz(c, chunk)) = pack8(&v[8 * chunk]);
         }
+        }
         fence_async_smem();
         tc_fence_before();
         const int any_timeout = __syncthreads_or(!ok);   // uniform: every thread leaves together
@@ -768,7 +907,20 @@ kda_chunk_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_consta
     if (kCtaStatus && tid == 0) status[(size_t)n * H + h] = *sFlag;
     if (*sFlag) {
         if (!kCtaStatus && tid == 0) atomicExch(status, 1);
-    } else if (S_final) {
+    } else if (kSummary) {
+        const int c = 32 * q4 + lane;
+        float* dst = seg.maps + ((((size_t)n * (seg.nseg - 1) + gseg) * H + h) * DK + c) * (DK + DV) +
+                     128 * hf;
+#pragma unroll
+        for (int blk = 0; blk < 8; ++blk) {
+            float v[16];
+            tmem_ld16(tmem + tlane + TM_S + 128 * hf + 16 * blk, v);
+            tmem_wait_ld();
+#pragma unroll
+            for (int i = 0; i < 16; i += 4)
+                *reinterpret_cast<float4*>(dst + 16 * blk + i) = make_float4(v[i], v[i + 1], v[i + 2], v[i + 3]);
+        }
+    } else if (S_final && last_seg) {
         const int c = 32 * q4 + lane;
         float* dst = S_final + (((size_t)n * H + h) * DK + c) * DV + 64 * hf;
 #pragma unroll
@@ -785,6 +937,55 @@ kda_chunk_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_consta
     __syncthreads();
     tc_fence_after();
     if (warp == 0) tmem_dealloc(tmem, 512);
+}
+
+// S_{g+1} = M_g S_g + N_g over the segments of one sequence, in fp32: one CTA
+// per (16 value columns, head, sequence), thread i owns row i of the state.
+// start[g = 0] receives S0 (or zeros), so the forward kernel never reads S0
+// itself and S_final may alias S0.
+constexpr int SCAN_COLS = 16;
+__global__ void __launch_bounds__(DK)
+kda_segment_scan_kernel(const float* S0, const float* __restrict__ maps, float* __restrict__ start,
+                        int nseg, int H) {
+    __shared__ __align__(16) float sS[DK][SCAN_COLS];
+    const int cb = blockIdx.x, h = blockIdx.y, n = blockIdx.z, i = threadIdx.x;
+    const size_t col = (size_t)SCAN_COLS * cb;
+    float cur[SCAN_COLS];
+    const float* src = S0 ? S0 + (((size_t)n * H + h) * DK + i) * DV + col : nullptr;
+#pragma unroll
+    for (int c = 0; c < SCAN_COLS; c += 4) {
+        const float4 f = src ? *reinterpret_cast<const float4*>(src + c) : make_float4(0.f, 0.f, 0.f, 0.f);
+        cur[c] = f.x; cur[c + 1] = f.y; cur[c + 2] = f.z; cur[c + 3] = f.w;
+    }
+    for (int g = 0;; ++g) {
+        float* dst = start + ((((size_t)n * nseg + g) * H + h) * DK + i) * DV + col;
+#pragma unroll
+        for (int c = 0; c < SCAN_COLS; c += 4)
+            *reinterpret_cast<float4*>(dst + c) = make_float4(cur[c], cur[c + 1], cur[c + 2], cur[c + 3]);
+        if (g == nseg - 1) break;
+        __syncthreads();   // the previous step's reads of sS are done
+#pragma unroll
+        for (int c = 0; c < SCAN_COLS; ++c) sS[i][c] = cur[c];
+        __syncthreads();
+        const float* Mrow = maps + ((((size_t)n * (nseg - 1) + g) * H + h) * DK + i) * (DK + DV);
+#pragma unroll
+        for (int c = 0; c < SCAN_COLS; ++c) cur[c] = Mrow[DK + col + c];   // N_g
+        for (int j = 0; j < DK; j += 4) {
+            const float4 m = *reinterpret_cast<const float4*>(Mrow + j);
+            const float mj[4] = {m.x, m.y, m.z, m.w};
+#pragma unroll
+            for (int jj = 0; jj < 4; ++jj) {
+#pragma unroll
+                for (int c = 0; c < SCAN_COLS; c += 4) {
+                    const float4 sv = *reinterpret_cast<const float4*>(&sS[j + jj][c]);
+                    cur[c] = fmaf(mj[jj], sv.x, cur[c]);
+                    cur[c + 1] = fmaf(mj[jj], sv.y, cur[c + 1]);
+                    cur[c + 2] = fmaf(mj[jj], sv.z, cur[c + 2]);
+                    cur[c + 3] = fmaf(mj[jj], sv.w, cur[c + 3]);
+                }
+            }
+        }
+    }
 }
 
 // ---------------------------------------------------------------- host side
@@ -821,23 +1022,28 @@ static bool make_map(CUtensorMap* m, const void* base, int64_t rows, int H) {
 
 }  // namespace tc
 
-template <bool kCtaStatus>
-static cudaError_t launch_tc_t(const void* q, const void* k, const void* v, const void* alpha,
-                               const void* beta, const float* S0, const int32_t* cu, int nseq,
-                               void* out, float* S_final, int64_t rows, int64_t T, int H,
-                               int* status, cudaStream_t stream) {
-    CUtensorMap mq, mk, ma, mv;
-    if (!tc::make_map(&mq, q, rows, H) || !tc::make_map(&mk, k, rows, H) ||
-        !tc::make_map(&ma, alpha, rows, H) || !tc::make_map(&mv, v, rows, H))
-        return cudaErrorInvalidValue;
-    cudaError_t e = cudaFuncSetAttribute(tc::kda_chunk_tc_kernel<kCtaStatus>,
+struct TcMaps {
+    CUtensorMap q, k, a, v;
+};
+
+static bool make_maps(TcMaps* m, const void* q, const void* k, const void* v, const void* alpha,
+                      int64_t rows, int H) {
+    return tc::make_map(&m->q, q, rows, H) && tc::make_map(&m->k, k, rows, H) &&
+           tc::make_map(&m->a, alpha, rows, H) && tc::make_map(&m->v, v, rows, H);
+}
+
+template <bool kCtaStatus, bool kSummary>
+static cudaError_t launch_tc_t(const TcMaps& m, const void* beta, const float* S0, const int32_t* cu,
+                               int nseq, void* out, float* S_final, int64_t T, int H, int* status,
+                               const tc::Segments& seg, cudaStream_t stream) {
+    cudaError_t e = cudaFuncSetAttribute(tc::kda_chunk_tc_kernel<kCtaStatus, kSummary>,
                                          cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          (int)tc::SMEM_BYTES);
     if (e != cudaSuccess) return e;
-    dim3 grid(1, H, nseq);
-    tc::kda_chunk_tc_kernel<kCtaStatus><<<grid, tc::NT, tc::SMEM_BYTES, stream>>>(
-        mq, mk, ma, mv, (const __nv_bfloat16*)beta, S0, cu, (__nv_bfloat16*)out, S_final, T, H,
-        status);
+    dim3 grid(1, H, nseq * seg.per_seq);
+    tc::kda_chunk_tc_kernel<kCtaStatus, kSummary><<<grid, tc::NT, tc::SMEM_BYTES, stream>>>(
+        m.q, m.k, m.a, m.v, (const __nv_bfloat16*)beta, S0, cu, (__nv_bfloat16*)out, S_final, T, H,
+        status, seg);
     return cudaGetLastError();
 }
 
@@ -845,8 +1051,44 @@ cudaError_t launch_chunk_tc(const void* q, const void* k, const void* v, const v
                             const void* beta, const float* S0, const int32_t* cu, int nseq,
                             void* out, float* S_final, int64_t rows, int64_t T, int H, int* status,
                             cudaStream_t stream) {
-    return launch_tc_t<false>(q, k, v, alpha, beta, S0, cu, nseq, out, S_final, rows, T, H,
-                              status, stream);
+    TcMaps m;
+    if (!make_maps(&m, q, k, v, alpha, rows, H)) return cudaErrorInvalidValue;
+    const tc::Segments whole{1, 1, nullptr, nullptr};
+    return launch_tc_t<false, false>(m, beta, S0, cu, nseq, out, S_final, T, H, status, whole,
+                                     stream);
+}
+
+// Floats of workspace the split forward uses: the segment maps [M | N] and the
+// segment start states.
+size_t chunk_tc_segmented_workspace_floats(int64_t nseq, int H, int nseg) {
+    if (nseg < 2) return 0;
+    return (size_t)nseq * H * ((size_t)(nseg - 1) * tc::DK * (tc::DK + tc::DV) +
+                               (size_t)nseg * tc::DK * tc::DV);
+}
+
+// The forward split along time into nseg segments per sequence: three launches
+// (segment maps, scan of the start states, forward of every segment).
+cudaError_t launch_chunk_tc_segmented(const void* q, const void* k, const void* v,
+                                      const void* alpha, const void* beta, const float* S0,
+                                      const int32_t* cu, int nseq, void* out, float* S_final,
+                                      int64_t rows, int64_t T, int H, int nseg, float* workspace,
+                                      int* status, cudaStream_t stream) {
+    if (nseg < 2 || nseq * (int64_t)nseg > 65535) return cudaErrorInvalidValue;
+    TcMaps m;
+    if (!make_maps(&m, q, k, v, alpha, rows, H)) return cudaErrorInvalidValue;
+    float* maps = workspace;
+    float* start = workspace + (size_t)nseq * H * (nseg - 1) * tc::DK * (tc::DK + tc::DV);
+    const tc::Segments summary{nseg, nseg - 1, nullptr, maps};
+    cudaError_t e = launch_tc_t<false, true>(m, beta, nullptr, cu, nseq, nullptr, nullptr, T, H,
+                                             status, summary, stream);
+    if (e != cudaSuccess) return e;
+    tc::kda_segment_scan_kernel<<<dim3(tc::DV / tc::SCAN_COLS, H, nseq), tc::DK, 0, stream>>>(
+        S0, maps, start, nseg, H);
+    e = cudaGetLastError();
+    if (e != cudaSuccess) return e;
+    const tc::Segments fwd{nseg, nseg, start, nullptr};
+    return launch_tc_t<false, false>(m, beta, nullptr, cu, nseq, out, S_final, T, H, status, fwd,
+                                     stream);
 }
 
 // Same kernel, one status word per (sequence, head) CTA at status[n * H + h].
@@ -855,8 +1097,11 @@ cudaError_t launch_chunk_tc_cta_status(const void* q, const void* k, const void*
                                        const int32_t* cu, int nseq, void* out, float* S_final,
                                        int64_t rows, int64_t T, int H, int* status,
                                        cudaStream_t stream) {
-    return launch_tc_t<true>(q, k, v, alpha, beta, S0, cu, nseq, out, S_final, rows, T, H,
-                             status, stream);
+    TcMaps m;
+    if (!make_maps(&m, q, k, v, alpha, rows, H)) return cudaErrorInvalidValue;
+    const tc::Segments whole{1, 1, nullptr, nullptr};
+    return launch_tc_t<true, false>(m, beta, S0, cu, nseq, out, S_final, T, H, status, whole,
+                                    stream);
 }
 
 }  // namespace kda

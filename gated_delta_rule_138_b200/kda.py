@@ -76,6 +76,8 @@ def load_library(build_if_missing: bool = True) -> ctypes.CDLL:
     lib.kda_launch_count.argtypes = []
     lib.kda_device_status.restype = ctypes.c_int
     lib.kda_device_status.argtypes = [vp]
+    lib.kda_forward_segments.restype = i32
+    lib.kda_forward_segments.argtypes = [i32, i64, i32, i32]
     lib.kda_selftest_timeout.restype = ctypes.c_int
     lib.kda_selftest_timeout.argtypes = [ctypes.c_uint64, vp]
     lib.kda_forward_noalloc.restype = ctypes.c_int
@@ -128,6 +130,11 @@ def kda_forward_kernel_name(d_k: int, d_v: int, chunk: int, in_dtype: torch.dtyp
 def kda_device_status(stream=None) -> None:
     """Synchronise `stream` and raise KdaError if a kernel reported a device timeout."""
     _check("kda_device_status", load_library().kda_device_status(_stream(stream)))
+
+
+def kda_forward_segments(num_seqs: int, tokens_per_seq: int, H: int, num_sms: int = 0) -> int:
+    """Time segments per sequence the tensor-core forward uses (1 = unsplit)."""
+    return int(load_library().kda_forward_segments(num_seqs, tokens_per_seq, H, num_sms))
 
 
 def kda_selftest_timeout(limit_ns: int = 1_000_000, stream=None) -> None:

@@ -116,12 +116,31 @@ kda_status_t kda_decode_step(const void* q, const void* k, const void* v,
 const char* kda_status_string(kda_status_t status);
 
 /*
- * Bytes of device workspace kda_forward uses for these sizes: the per-device
- * status word (4 bytes), allocated by the library on the first tensor-core call
- * on a device and kept until exit.  No per-call workspace is allocated.
+ * Bytes of device workspace kda_forward uses for a dense batch of these sizes:
+ * the per-device status word (4 bytes, allocated on the first tensor-core call
+ * on a device and kept until exit) plus, when the tensor-core path splits the
+ * sequences along time (see kda_forward_segments), the segment maps and start
+ * states: B * H * ((g - 1) * d_k * (d_k + d_v) + g * d_k * d_v) fp32 values for
+ * g segments.  That part is allocated stream-ordered (cudaMallocAsync) on the
+ * call's stream and freed (cudaFreeAsync) behind the call's kernels; if it
+ * cannot be allocated the call runs unsplit.  Host-only.
  */
 size_t kda_forward_workspace_bytes(int32_t B, int64_t T, int32_t H, int32_t d_k,
                                    int32_t d_v, int32_t chunk);
+
+/*
+ * Time segments per sequence that kda_forward's tensor-core path uses for
+ * num_seqs sequences of tokens_per_seq tokens (a packed batch uses its mean
+ * length) and H heads on a GPU with num_sms SMs (0: the current device's, 148
+ * if none is visible).  1 = each (sequence, head) runs whole on one CTA.  With
+ * g > 1, every sequence's chunks are cut into g runs; a first kernel computes
+ * each run's affine state map S_end = M S_start + N, a scan kernel chains the
+ * start states in fp32, and the forward kernel runs all runs in parallel (the
+ * article's paragraph 3: states reconstructed across chunks by a prefix scan).
+ * The choice only balances the SMs: every g gives the same result up to
+ * rounding.  Host-only.
+ */
+int32_t kda_forward_segments(int32_t num_seqs, int64_t tokens_per_seq, int32_t H, int32_t num_sms);
 
 /* Text of the last CUDA error seen by this thread's calls ("" if none). */
 const char* kda_last_error(void);

@@ -94,3 +94,19 @@ def test_selftest_rejects_bad_limit():
     lib = kda.load_library()
     assert lib.kda_selftest_timeout(0, None) == 1
     assert lib.kda_selftest_timeout(20_000_000_000, None) == 1
+
+
+def test_time_segment_choice():
+    """Host logic of the sequence split: only when few (sequence, head) pairs
+    would leave SMs idle and the sequences are long enough."""
+    seg = kda.kda_forward_segments
+    assert seg(8, 4096, 32, 148) == 1            # 256 CTAs already fill 148 SMs
+    assert seg(64, 5000, 16, 148) == 1           # packed batch of 1024 CTAs
+    assert seg(1, 64 * 31, 1, 148) == 1          # too short for two 16-chunk segments
+    assert seg(1, 64 * 32, 1, 148) == 2
+    g = seg(1, 1 << 20, 32, 148)                 # 32 CTAs on 148 SMs, 16384 chunks each
+    assert 4 <= g <= 64
+    assert (32 * g) % 148 > 100 or (32 * g) <= 148  # the last wave is mostly full
+    assert seg(0, 100, 4, 148) == 1 and seg(1, 0, 4, 148) == 1
+    for units_h in (1, 2, 4, 8, 16, 32, 64):
+        assert 1 <= seg(1, 1 << 22, units_h, 148) <= 64

@@ -186,3 +186,63 @@ def test_subchunk_factors_stay_in_fp32_range():
     assert 1.0 / phi_min < np.finfo(np.float32).max
     # one token more per sub-chunk would still fit, two sub-chunks would not
     assert lo ** (2 * SUB) < np.finfo(np.float32).tiny
+
+
+def chunk_maps_one(k, alpha, beta, v, C):
+    """The affine state map of a run of tokens, S_end = M S_start + N, built the
+    way the tensor-core kernel's summary mode builds it: per chunk
+    M_c = Diag(gamma_C) - (k*eta)^T W and N_c = (k*eta)^T Tb V, composed in order."""
+    T, dk = k.shape
+    dv = v.shape[1]
+    a_all = _clamp(alpha)
+    M = np.eye(dk)
+    N = np.zeros((dk, dv))
+    for t0 in range(0, T, C):
+        L = min(C, T - t0)
+        K = np.zeros((C, dk)); V = np.zeros((C, dv)); a = np.ones((C, dk)); b = np.zeros(C)
+        K[:L], V[:L], a[:L], b[:L] = k[t0:t0 + L], v[t0:t0 + L], a_all[t0:t0 + L], beta[t0:t0 + L]
+        A = np.zeros((C, C))
+        for r in range(C):
+            for j in range(r):
+                A[r, j] = b[r] * np.sum(K[r] * K[j] * np.prod(a[j + 1:r + 1], axis=0))
+        Tb = np.linalg.inv(np.eye(C) + A) * b[None, :]
+        gamma = np.cumprod(a, axis=0)
+        eta = np.array([np.prod(a[j + 1:], axis=0) for j in range(C)])
+        W = Tb @ (K * gamma)
+        Mc = np.diag(gamma[C - 1]) - (K * eta).T @ W
+        Nc = (K * eta).T @ (Tb @ V)
+        M, N = Mc @ M, Mc @ N + Nc
+    return M, N
+
+
+@pytest.mark.parametrize("T,nseg,extreme", [(300, 3, False), (256, 4, True), (130, 5, False), (40, 5, False)])
+def test_time_segments_scan_equals_oracle(T, nseg, extreme):
+    """Cutting a sequence into runs of whole chunks, chaining the runs' affine
+    maps S_{g+1} = M_g S_g + N_g and re-running every run from its own start
+    state gives the token recurrence's outputs and final state (the prefix
+    scan of the article's paragraph 3, here over segments of one sequence)."""
+    C, dk, dv = 16, 16, 8
+    q, k, v, al, be, S0 = (x.astype(np.float64) for x in _case(2000 + T, T, dk, dv, extreme))
+    ref_o, ref_S = oracle.forward(*(x[None, :, None].astype(np.float32) for x in (q, k, v, al, be)),
+                                  S0[None, None].astype(np.float32))
+    nch = -(-T // C)
+    cps = -(-nch // nseg)
+    bounds = [(min(g * cps * C, T), min((g + 1) * cps * C, T)) for g in range(nseg)]
+    assert bounds[-1][1] == T
+    starts = [S0]
+    for g in range(nseg - 1):
+        t0, t1 = bounds[g]
+        M, N = chunk_maps_one(k[t0:t1], al[t0:t1], be[t0:t1], v[t0:t1], C)
+        # the map agrees with running the recurrence from two start states
+        o_a, S_a = chunk_forward_one(q[t0:t1], k[t0:t1], v[t0:t1], al[t0:t1], be[t0:t1], starts[-1], C) \
+            if t1 > t0 else (None, starts[-1])
+        np.testing.assert_allclose(M @ starts[-1] + N, S_a, rtol=1e-10, atol=1e-12)
+        starts.append(M @ starts[-1] + N)
+    outs = []
+    for g, (t0, t1) in enumerate(bounds):
+        if t1 == t0:
+            continue
+        o, S_end = chunk_forward_one(q[t0:t1], k[t0:t1], v[t0:t1], al[t0:t1], be[t0:t1], starts[g], C)
+        outs.append(o)
+    np.testing.assert_allclose(np.concatenate(outs), ref_o[0, :, 0], rtol=1e-10, atol=1e-12)
+    np.testing.assert_allclose(S_end, ref_S[0, 0], rtol=1e-10, atol=1e-12)

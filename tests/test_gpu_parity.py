@@ -256,6 +256,63 @@ def test_tc_matches_fp32_path():
     assert rel_l2(np32(S_tc), np32(S_f)) <= 2e-2
 
 
+# ------------------------------------------------ time segments (sequence split + scan)
+
+@pytest.mark.parametrize("B,T,H", [(1, 64 * 65 + 37, 2), (2, 64 * 40, 1)])
+def test_tc_time_segments(B, T, H):
+    """Few (sequence, head) pairs and long sequences: the forward is split along
+    time (segment maps, fp32 scan of start states, forward of every segment).
+    Parity with the oracle, and with the unsplit kernel on the same inputs."""
+    nseg = kda.kda_forward_segments(B, T, H)
+    assert nseg > 1
+    inp = gen.draw_forward(B, T, H, 128, 128, "bf16", 900 + T, device=DEV, s0=True)
+    out, Sf = kda.kda_forward(inp["q"], inp["k"], inp["v"], inp["alpha"], inp["beta"], inp["S0"])
+    o1 = torch.empty_like(out)
+    S1 = torch.empty_like(Sf)
+    kda.kda_forward_noalloc(inp["q"], inp["k"], inp["v"], inp["alpha"], inp["beta"], o1, S1,
+                            inp["S0"])
+    torch.cuda.synchronize()
+    kda.kda_device_status()
+    ro, rS = oracle_forward(inp)
+    assert rel_l2(np32(out), ro) <= 2e-2
+    assert rel_l2(np32(Sf), rS) <= 2e-2
+    assert rel_l2(np32(out), np32(o1)) <= 1e-2
+    assert rel_l2(np32(Sf), np32(S1)) <= 1e-2
+
+
+def test_tc_time_segments_varlen_with_empty_segments():
+    """A packed batch whose short sequences leave some segments empty (one
+    chunk, zero tokens) next to a long one that is cut into several."""
+    lengths = [20000, 40, 0, 3000]
+    total = sum(lengths)
+    assert kda.kda_forward_segments(len(lengths), -(-total // len(lengths)), 1) >= 4
+    inp = gen.draw_varlen(lengths, 1, 128, 128, "bf16", 910, device=DEV, s0=True)
+    out, Sf = kda.kda_forward(inp["q"], inp["k"], inp["v"], inp["alpha"], inp["beta"],
+                              inp["S0"], cu_seqlens=inp["cu_seqlens"])
+    torch.cuda.synchronize()
+    kda.kda_device_status()
+    ro, rS = oracle_forward(inp, cu=np32(inp["cu_seqlens"]).astype(np.int32))
+    assert rel_l2(np32(out), ro) <= 2e-2
+    for n in range(len(lengths)):
+        assert rel_l2(np32(Sf[n:n + 1]), rS[n:n + 1]) <= 2e-2
+    # the empty sequence keeps its start state exactly
+    assert torch.equal(Sf[2], inp["S0"][2])
+
+
+def test_tc_time_segments_state_in_place():
+    """S_final aliasing S0 under the split: the start states are taken by the
+    scan before any segment writes S_final."""
+    B, T, H = 1, 64 * 48 + 5, 2
+    assert kda.kda_forward_segments(B, T, H) > 1
+    inp = gen.draw_forward(B, T, H, 128, 128, "bf16", 920, device=DEV, s0=True)
+    ro, rS = oracle_forward(inp)
+    S = inp["S0"].clone()
+    out, _ = kda.kda_forward(inp["q"], inp["k"], inp["v"], inp["alpha"], inp["beta"], S, S_final=S)
+    torch.cuda.synchronize()
+    assert rel_l2(np32(out), ro) <= 2e-2
+    assert rel_l2(np32(S), rS) <= 2e-2
+
+
 # ------------------------------------------------ failure detection (no fault, no hang)
 
 def test_bounded_wait_reports_timeout_and_context_survives():
