@@ -10,23 +10,27 @@
 //
 //   A[r,j] = beta_r sum_c k_rc k_jc D(r,j)_c  (j < r),  P[r,j] = sum_c q_rc k_jc D(r,j)_c  (j <= r)
 //   D(r,j) = prod_{s=j+1..r} a_s,   Tinv = (I + A)^-1,   Tb = Tinv diag(beta)
-//   [-W ; Q'] = [0 ; q*gamma] - [Tb ; P Tb] (k*gamma)          (gamma_r = prod_{s<=r} a_s)
-//   [ U ; O ] = [-W ; Q'] S + [Tb ; P Tb] V
-//   S        <- Diag(gamma_C) S + (k*eta)^T U                   (eta_j = prod_{s>j} a_s)
+//   W = Tb (k*gamma)                                   (gamma_r = prod_{s<=r} a_s)
+//   U = -W S + Tb V
+//   O = (q*gamma) S + P U
+//   S <- Diag(gamma_C) S + (k*eta)^T U                  (eta_j = prod_{s>j} a_s)
 //
-// D(r,j) is split at 16-token sub-chunk boundaries so that every factor stays
-// inside the fp32/bf16 exponent range (a product of 64 gates >= e^-5 can reach
-// e^-320, but a 16-token product stays >= e^-80):
-//   phi_r = prod_{s=start(I)..r} a_s,  psi_j = prod_{s=j+1..end(J)} a_s,
-//   pi_I = prod over sub-chunk I,      Dp_{I,J} = prod_{J<M<I} pi_M (I > J), 1/pi_I (I = J)
-//   D(r, j) = (phi_r) (psi_j Dp_{I(r),J(j)})
-// so the 16-row block I of [A/beta | P] is  [k phi ; q phi]_I  times  R^(I)^T with
-// R^(I)_j = k_j psi_j Dp_{I,J(j)} for j < end(I): one M=64 tcgen05 MMA per I.
+// Only U and the state update are sequential from chunk to chunk; O is issued
+// beside the state update.  D(r,j) never appears as a ratio of long products
+// (64 gates >= e^-5 reach e^-320, outside fp32/bf16): with 32-token
+// sub-chunks I and the reference token ref_I = 32 I + 15,
+//   D(r, j) = lam_r * rho^{I(r)}_j,  lam_r = e^{g_r - g_ref(I(r))},  rho^I_j = e^{g_ref(I) - g_j}
+// (g the running log-gate), every factor within [e^-80, e^80] except right
+// factors that underflow where the product itself is negligible.  All factors
+// are running products of the clamped gates; nothing evaluates exp or log.
+// So [A/beta ; P] = [k*lam ; q*lam] (k*rho^I)^T: two tcgen05 MMAs, one per I.
 //
 // One CTA (256 threads) owns one (sequence, head) -- or one segment of it --
 // and walks its chunks in order.  Thread 0 issues the TMA loads and the MMAs;
-// all eight warps do the element-wise work.  TMEM (512 columns): S fp32
-// [0,128), U|O accumulator [128,256), scratch accumulators [256,512).
+// all eight warps do the element-wise work.  Loads run one chunk ahead: q
+// (double buffered) at the start of a chunk, k and alpha once the gate phase
+// has consumed them, v once U has.  TMEM (512 columns): S fp32 [0,128), O
+// [128,256), scratch accumulators [256,384), U [384,512).
 //
 // Long sequences with few (sequence, head) pairs are also split along time
 // into segments (the prefix scan of paragraph 3, within one GPU).  Over a
@@ -58,49 +62,48 @@ constexpr int NT = 256;       // threads
 constexpr uint64_t kWaitNs = 2000000000ull;  // 2 s per wait, then report a timeout
 
 // shared-memory map (bytes from the 1024-aligned base)
-constexpr uint32_t OFF_Q = 0;            // q tile [64][128] sw128, becomes q*gamma in place
-constexpr uint32_t OFF_K = 16384;        // k tile
-constexpr uint32_t OFF_AL = 32768;       // alpha tile, becomes [Tb ; P Tb] (K-major [128][64])
-constexpr uint32_t OFF_V = 49152;        // v tile: MN-major B, two 64-column atoms of [64][64]
-constexpr uint32_t OFF_X = 65536;        // 72 KB work region, see below
+constexpr uint32_t OFF_S = 0;            // S bf16 MN-major B [128 c][128 n], two atoms 16 KB apart;
+                                         // a summary's [M | N] takes four atoms (64 KB, over the q tiles)
+constexpr uint32_t OFF_Q = 32768;        // q tiles, two buffers of [64][128] (two [64][64] atoms each),
+                                         // each becomes q*gamma in place (K-major A of the O MMA)
+constexpr uint32_t OFF_K = 65536;        // k tile
+constexpr uint32_t OFF_AL = 81920;       // alpha tile
+constexpr uint32_t OFF_V = 98304;        // v tile: MN-major B, two 64-column atoms of [64][64]
+constexpr uint32_t OFF_X = 114688;       // 72 KB work region, see below
 constexpr uint32_t OFF_KT = OFF_X + 73728;   // (k*gamma)^T  K-major B [128 c][64 j]
 constexpr uint32_t OFF_KH = OFF_KT + 16384;  // (k*eta)^T    K-major A [128 c][64 j]
-constexpr uint32_t OFF_IP = OFF_KH + 16384;  // [I ; P]      K-major A [128][64]
-constexpr uint32_t OFF_S = OFF_IP + 16384;   // S bf16       MN-major B [128 c][128 n], two atoms
-constexpr uint32_t OFF_MISC = OFF_S + 32768;
+constexpr uint32_t OFF_MISC = OFF_KH + 16384;
 constexpr uint32_t MISC_PI = 0;          // float [4][128]
 constexpr uint32_t MISC_GC = 2048;       // float [128] gamma_C
 constexpr uint32_t MISC_BETA = 2560;     // float [64]
-constexpr uint32_t MISC_BAR = 2816;      // 2 x uint64 mbarriers
-constexpr uint32_t MISC_TMEM = 2832;     // uint32 TMEM base
-constexpr uint32_t MISC_FLAG = 2836;     // int timeout seen
-constexpr uint32_t SMEM_BYTES = OFF_MISC + 2848 + 1024;  // + alignment slack
+constexpr uint32_t MISC_BAR = 2816;      // 4 x uint64 mbarriers: q, k+alpha, v, MMA
+constexpr uint32_t MISC_TMEM = 2848;     // uint32 TMEM base
+constexpr uint32_t MISC_FLAG = 2852;     // int timeout seen
+constexpr uint32_t SMEM_BYTES = OFF_MISC + 2880 + 1024;  // + alignment slack
 
 // work region X, by phase
-constexpr uint32_t X_R = 0;              // right operand rows [128][128] (2 atoms of 128 rows)
-constexpr uint32_t X_L = 32768;          // left operand rows  [128][128] (2 atoms of 128 rows)
+constexpr uint32_t X_L = 0;              // left rows [128][128]: k*lam rows 0..63, q*lam rows 64..127
+constexpr uint32_t X_R = 32768;          // right rows [96][128]: k*rho^0 rows 0..31 (tokens 0..31),
+                                         // k*rho^1 rows 32..95 (tokens 0..63); two 12 KB atoms
+constexpr uint32_t X_P = 57344;          // P, K-major A [64 r][64 j]; lives until the O MMA
 constexpr int AS = 68;                   // row stride (floats) of the fp32 A and Tinv tiles
 constexpr uint32_t X_AM = 0;             // float A    [64][68]
 constexpr uint32_t X_TM = 17408;         // float Tinv [64][68]
-constexpr uint32_t X_TB = 35840;         // Tb MN-major B [64 j][64 m] (1024-aligned)
-constexpr uint32_t X_XS = 44032;         // float scratch [32][36]
+constexpr uint32_t X_XS = 34816;         // float scratch [32][36]
 // fp32 K-major 128B-swizzled tiles (32 floats per row) for the tf32 MMAs of the 32 -> 64 step
-constexpr uint32_t X_T0T = 49152;        // Tinv[0:32, 0:32]^T   [64 rows (32 used)][32]
-constexpr uint32_t X_T1 = 57344;         // Tinv[32:64, 32:64]   [64 rows (32 used)][32]
+constexpr uint32_t X_T0T = 40960;        // Tinv[0:32, 0:32]^T   [64 rows (32 used)][32]
+constexpr uint32_t X_T1 = 49152;         // Tinv[32:64, 32:64]   [64 rows (32 used)][32]
 constexpr uint32_t X_A10 = 65536;        // A[32:64, 0:32]       [32][32]
 constexpr uint32_t X_XT = 69632;         // (A10 T0)^T           [32][32]
-constexpr uint32_t X_WQ = 0;             // [-W ; Q'] K-major A [128][128] (2 atoms)
-constexpr uint32_t X_U = 32768;          // U MN-major B [64 j][128 n] (2 atoms of [64][64])
+constexpr uint32_t X_TB = 40960;         // Tb, K-major A [64 r][64 m] (after the solve)
+constexpr uint32_t X_WQ = 0;             // -W, K-major A [64][128] (two [64][64] atoms 8 KB apart)
+constexpr uint32_t X_U = 16384;          // U, MN-major B [64 j][128 n] (two [64][64] atoms);
+                                         // a summary's [U_M | U_N] takes four atoms
 
-constexpr uint32_t TM_S = 0, TM_UO = 128, TM_WK = 256;
+constexpr uint32_t TM_S = 0, TM_O = 128, TM_WK = 256, TM_U = 384;
 
 __device__ __forceinline__ uint32_t swz(uint32_t row, uint32_t chunk) {
     return row * 128u + (((chunk ^ row) & 7u) << 4);
-}
-// byte offset of the bf16 pair (row, c..c+1), c even, in a tile with `rows`
-// rows per 64-column atom
-__device__ __forceinline__ uint32_t pair_off(uint32_t row, uint32_t c, uint32_t rows) {
-    return (c >> 6) * rows * 128u + swz(row, (c & 63u) >> 3) + ((c & 7u) << 1);
 }
 // byte offset of fp32 element (r, k) in a K-major 128B-swizzled tile with 32 floats per row
 __device__ __forceinline__ uint32_t f32_off(uint32_t r, uint32_t k) {
@@ -140,6 +143,13 @@ struct Segments {
     float* maps;          // summary: [M | N] fp32 [nseq * (nseg - 1), H, DK, DK + DV]
 };
 
+// One TMA stream's bookkeeping: the parity its next wait expects, and the load
+// (if any) issued but not yet waited for.
+struct LoadTrack {
+    uint32_t ph = 0, pend_ph = 0;
+    bool pend = false;
+};
+
 // kCtaStatus = false: a timed-out wait sets the shared word *status to 1.
 // kCtaStatus = true:  every CTA writes its own word status[n * H + h] (0 or 1).
 // kSummary = true: the segment-map mode described at the top (q and out unused).
@@ -153,23 +163,21 @@ kda_chunk_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_consta
     extern __shared__ uint8_t smem_raw[];
     uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~static_cast<uintptr_t>(1023));
-    // A summary loads no q tile: everything after it moves down 16 KB, and the
-    // bf16 copy of [M | N] (four 64-column atoms, 64 KB) ends where MISC starts.
-    constexpr uint32_t kSh = kSummary ? 16384u : 0u;
+    uint8_t* sS = sm + OFF_S;
     uint8_t* sQ = sm + OFF_Q;
-    uint8_t* sK = sm + OFF_K - kSh;
-    uint8_t* sAl = sm + OFF_AL - kSh;
-    uint8_t* sV = sm + OFF_V - kSh;
-    uint8_t* sX = sm + OFF_X - kSh;
-    uint8_t* sKT = sm + OFF_KT - kSh;
-    uint8_t* sKH = sm + OFF_KH - kSh;
-    uint8_t* sIP = sm + OFF_IP;
-    uint8_t* sS = kSummary ? sm + OFF_KH : sm + OFF_S;
+    uint8_t* sK = sm + OFF_K;
+    uint8_t* sAl = sm + OFF_AL;
+    uint8_t* sV = sm + OFF_V;
+    uint8_t* sX = sm + OFF_X;
+    uint8_t* sKT = sm + OFF_KT;
+    uint8_t* sKH = sm + OFF_KH;
     float* sPi = reinterpret_cast<float*>(sm + OFF_MISC + MISC_PI);
     float* sGC = reinterpret_cast<float*>(sm + OFF_MISC + MISC_GC);
     float* sBeta = reinterpret_cast<float*>(sm + OFF_MISC + MISC_BETA);
-    uint64_t* barT = reinterpret_cast<uint64_t*>(sm + OFF_MISC + MISC_BAR);
-    uint64_t* barM = barT + 1;
+    uint64_t* barQ = reinterpret_cast<uint64_t*>(sm + OFF_MISC + MISC_BAR);
+    uint64_t* barKA = barQ + 1;
+    uint64_t* barV = barQ + 2;
+    uint64_t* barM = barQ + 3;
     uint32_t* sTmem = reinterpret_cast<uint32_t*>(sm + OFF_MISC + MISC_TMEM);
     int* sFlag = reinterpret_cast<int*>(sm + OFF_MISC + MISC_FLAG);
 
@@ -199,29 +207,14 @@ kda_chunk_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_consta
     const bool last_seg = gseg == seg.nseg - 1;
 
     if (tid == 0) {
-        mbar_init(barT, 1);
+        mbar_init(barQ, 1);
+        mbar_init(barKA, 1);
+        mbar_init(barV, 1);
         mbar_init(barM, 1);
         mbar_fence_init();
         *sFlag = 0;
     }
     if (warp == 0) tmem_alloc(sTmem, 512);
-    // identity rows of [I ; P]
-    if (!kSummary)
-    for (int i = tid; i < 64 * 8; i += NT) {
-        const int r = i >> 3, ch = i & 7;
-        uint32_t w[4] = {0, 0, 0, 0};
-        if ((r >> 3) == ch) {
-            const int e = r & 7;  // element within the 8-wide chunk
-            w[e >> 1] = (e & 1) ? 0x3F800000u : 0x00003F80u;  // bf16 1.0 in the hi/lo half
-        }
-        *reinterpret_cast<uint4*>(sIP + swz(r, ch)) = make_uint4(w[0], w[1], w[2], w[3]);
-    }
-    // P[r][j] = 0 for r < 32 <= j: never written by the per-chunk extraction
-    if (!kSummary)
-    for (int i = tid; i < 32 * 4; i += NT) {
-        const int r = i >> 2, ch = 4 + (i & 3);
-        *reinterpret_cast<uint4*>(sIP + swz(64 + r, ch)) = make_uint4(0u, 0u, 0u, 0u);
-    }
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
@@ -261,31 +254,104 @@ kda_chunk_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_consta
             }
             tmem_st16(tmem + tlane + TM_S + 64 * hf + 16 * blk, v);
 #pragma unroll
-            for (int ch = 0; ch < 2; ++ch) {
-                uint4 w;
-                w.x = pack_bf16x2(v[8 * ch + 0], v[8 * ch + 1]);
-                w.y = pack_bf16x2(v[8 * ch + 2], v[8 * ch + 3]);
-                w.z = pack_bf16x2(v[8 * ch + 4], v[8 * ch + 5]);
-                w.w = pack_bf16x2(v[8 * ch + 6], v[8 * ch + 7]);
-                *reinterpret_cast<uint4*>(sS + hf * 16384 + swz(c, 2 * blk + ch)) = w;
-            }
+            for (int ch = 0; ch < 2; ++ch)
+                *reinterpret_cast<uint4*>(sS + hf * 16384 + swz(c, 2 * blk + ch)) = pack8(&v[8 * ch]);
         }
         tmem_wait_st();
     }
 
-    auto issue_tma = [&](int64_t row0) {
-        mbar_arrive_expect_tx(barT, (kSummary ? 3 : 4) * 16384);
-        const int y = (int)row0;
+    auto issue_q = [&](int64_t row0, int buf) {
+        mbar_arrive_expect_tx(barQ, 16384);
+#pragma unroll
+        for (int a = 0; a < 2; ++a)
+            tma_load_2d(sQ + buf * 16384 + a * 8192, &tmQ, barQ, h * DK + 64 * a, (int)row0);
+    };
+    auto issue_ka = [&](int64_t row0) {
+        mbar_arrive_expect_tx(barKA, 2 * 16384);
 #pragma unroll
         for (int a = 0; a < 2; ++a) {
-            const int x = h * DK + 64 * a;
-            if (!kSummary) tma_load_2d(sQ + a * 8192, &tmQ, barT, x, y);
-            tma_load_2d(sK + a * 8192, &tmK, barT, x, y);
-            tma_load_2d(sAl + a * 8192, &tmA, barT, x, y);
-            tma_load_2d(sV + a * 8192, &tmV, barT, h * DV + 64 * a, y);
+            tma_load_2d(sK + a * 8192, &tmK, barKA, h * DK + 64 * a, (int)row0);
+            tma_load_2d(sAl + a * 8192, &tmA, barKA, h * DK + 64 * a, (int)row0);
         }
     };
-    if (tid == 0 && nchunks > 0) issue_tma(bos);
+    auto issue_v = [&](int64_t row0) {
+        mbar_arrive_expect_tx(barV, 16384);
+#pragma unroll
+        for (int a = 0; a < 2; ++a)
+            tma_load_2d(sV + a * 8192, &tmV, barV, h * DV + 64 * a, (int)row0);
+    };
+
+    bool ok = true;   // this thread has seen every wait complete
+    // asynchronous work that a timed-out wait may leave in flight, drained before exit
+    LoadTrack tq, tka, tv;
+    uint32_t phM = 0, mma_out_ph = 0;
+    bool mma_out = false;   // (thread 0) an MMA group committed and not yet waited for
+    auto wait_load = [&](uint64_t* bar, LoadTrack& t) {
+        if (ok) {
+            if (mbar_wait_ns(bar, t.ph, kWaitNs)) t.pend = false;
+            else ok = false;
+        }
+        t.ph ^= 1u;
+    };
+    auto issued = [&](LoadTrack& t) {
+        t.pend = true;
+        t.pend_ph = t.ph;
+    };
+    auto commit_mma = [&]() {   // thread 0, after issuing an MMA group
+        mma_commit(barM);
+        mma_out = true;
+        mma_out_ph = phM;
+    };
+    auto wait_mma = [&]() {
+        if (ok) {
+            if (mbar_wait_ns(barM, phM, kWaitNs)) mma_out = false;
+            else ok = false;
+        }
+        phM ^= 1u;
+        tc_fence_after();
+    };
+
+    // The state update (and O) of a chunk is waited for, and its results taken out
+    // of TMEM, only inside the next chunk's gate phase: nothing before the next
+    // chunk's U MMA needs them.  S goes to its bf16 copy, O to the output rows.
+    auto finish_prev = [&](int64_t prow0, int pLc) {
+        wait_mma();
+        const int c = 32 * q4 + lane;
+        if constexpr (kSummary) {
+#pragma unroll
+            for (int p = 0; p < 2; ++p) {
+                float v[64];
+                tmem_ld64(tmem + tlane + TM_S + 128 * hf + 64 * p, v);
+#pragma unroll
+                for (int ch = 0; ch < 8; ++ch)
+                    *reinterpret_cast<uint4*>(sS + (2 * hf + p) * 16384 + swz(c, ch)) = pack8(&v[8 * ch]);
+            }
+        } else {
+            float v[64];
+            tmem_ld64(tmem + tlane + TM_S + 64 * hf, v);
+#pragma unroll
+            for (int ch = 0; ch < 8; ++ch)
+                *reinterpret_cast<uint4*>(sS + hf * 16384 + swz(c, ch)) = pack8(&v[8 * ch]);
+            tmem_ld64(tmem + tlane + TM_O + 64 * hf, v);
+            const int r = 16 * q4 + lane;
+            if (lane < 16 && r < pLc) {
+                uint4* dst = reinterpret_cast<uint4*>(out + ((size_t)(prow0 + r) * H + h) * DV + 64 * hf);
+#pragma unroll
+                for (int ch = 0; ch < 8; ++ch) dst[ch] = pack8(&v[8 * ch]);
+            }
+        }
+    };
+
+    if (nchunks > 0) {
+        if (tid == 0) {
+            if (!kSummary) issue_q(bos, 0);
+            issue_ka(bos);
+            issue_v(bos);
+        }
+        if (!kSummary) issued(tq);
+        issued(tka);
+        issued(tv);
+    }
     fence_async_smem();
     tc_fence_before();
     __syncthreads();
@@ -295,43 +361,14 @@ kda_chunk_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_consta
     float beta_next = 0.0f;
     if (tid < C && tid < len) beta_next = __bfloat162float(beta[(size_t)(bos + tid) * H + h]);
 
-    uint32_t phT = 0, phM = 0;
-    bool ok = true;   // this thread has seen every wait complete
-    // asynchronous work that a timed-out wait may leave in flight, drained before exit
-    bool tma_pending = nchunks > 0, mma_pending = false;
-    uint32_t tma_pending_phase = 0, mma_pending_phase = 0;
-    auto wait_mma = [&]() {
-        if (ok && !mbar_wait_ns(barM, phM, kWaitNs)) {
-            ok = false;
-            mma_pending = true;
-            mma_pending_phase = phM;
-        }
-        phM ^= 1u;
-        tc_fence_after();
-    };
-
-    // all of k, alpha, v (and q) of this chunk are consumed: load the next one
-    auto prefetch_next = [&](int chunk, int64_t row0) {
-        if (chunk + 1 < nchunks && ok) {
-            if (tid == 0) issue_tma(row0 + C);
-            tma_pending = true;
-            tma_pending_phase = phT;
-        }
-        if (tid < C) {
-            const int64_t nxt = (int64_t)(chunk + 1) * C + tid;   // token index in the segment
-            beta_next = nxt < len ? __bfloat162float(beta[(size_t)(bos + nxt) * H + h]) : 0.0f;
-        }
-    };
-
+    bool broke = false;
     for (int chunk = 0; chunk < nchunks; ++chunk) {
         const int64_t row0 = bos + (int64_t)chunk * C;
         const int Lc = (int)((len - (int64_t)chunk * C) < C ? (len - (int64_t)chunk * C) : C);
+        uint8_t* sQc = sQ + (chunk & 1) * 16384;
         if (tid < C) sBeta[tid] = beta_next;
-        if (ok) {
-            if (mbar_wait_ns(barT, phT, kWaitNs)) tma_pending = false;
-            else ok = false;
-        }
-        phT ^= 1u;
+        wait_load(barKA, tka);
+        if (!kSummary) wait_load(barQ, tq);
         KDA_TC_PHASE(0);
 
         // ================= gate products and bf16 operands (all threads)
@@ -347,7 +384,7 @@ kda_chunk_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_consta
             // [e^-80, e^80] except right factors that underflow where the product is negligible.
             // All tiles touched here have 8-row-aligned bases, so the swizzled offset of
             // (row i of a 16-row group, this channel pair) is i*128 + xo[i & 7].
-            const int cp = tid & 63, Q = tid >> 6, c0 = 2 * cp, Isub = Q >> 1;
+            const int cp = tid & 63, Q = tid >> 6, c0 = 2 * cp;
             const uint32_t atom = (uint32_t)(c0 >> 6);
             const uint32_t chk = (uint32_t)((c0 & 63) >> 3), inner = (uint32_t)((c0 & 7) << 1);
             uint32_t xo[8];
@@ -379,6 +416,13 @@ kda_chunk_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_consta
                 *reinterpret_cast<float2*>(&sPi[Q * DK + c0]) = make_float2(p0, p1);
             }
             __syncthreads();
+            // the previous chunk's state update and O (their operands KH, U, P and the
+            // q buffer are overwritten from here on)
+            if (chunk > 0) finish_prev(row0 - C, C);
+            if (!kSummary && chunk + 1 < nchunks && ok) {
+                if (tid == 0) issue_q(row0 + C, (chunk + 1) & 1);
+                issued(tq);
+            }
             float pi0[4], pi1[4];
 #pragma unroll
             for (int M = 0; M < 4; ++M) {
@@ -401,13 +445,13 @@ kda_chunk_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_consta
             if (Q == 0) { r10 = pi0[1] * pi0[2]; r11 = pi1[1] * pi1[2]; }
             if (Q == 1) { r10 = pi0[2]; r11 = pi1[2]; }
             if (Q == 3) { r10 = __frcp_rn(pi0[3]); r11 = __frcp_rn(pi1[3]); }
-            // left rows: sub-chunk I at rows 64I..64I+63 = [k-part 32 | q-part 32]
-            uint8_t* tLk = sX + X_L + atom * 16384u + (uint32_t)(64 * Isub + 16 * (Q & 1)) * 128u;
-            uint8_t* tLq = tLk + 32 * 128;
-            // right rows: rho^0 at rows 0..31, rho^1 at rows 64..127
-            uint8_t* tR0 = sX + X_R + atom * 16384u + (uint32_t)(16 * Q) * 128u;
-            uint8_t* tR1 = tR0 + 64 * 128;
-            uint8_t* tQ = sQ + in_base;
+            // left rows: k*lam at row t, q*lam at row 64 + t (atoms of 128 rows)
+            uint8_t* tLk = sX + X_L + atom * 16384u + (uint32_t)(16 * Q) * 128u;
+            uint8_t* tLq = tLk + 64 * 128;
+            // right rows: rho^0 of token t < 32 at row t, rho^1 of token t at row 32 + t
+            uint8_t* tR0 = sX + X_R + atom * 12288u + (uint32_t)(16 * Q) * 128u;
+            uint8_t* tR1 = tR0 + 32 * 128;
+            uint8_t* tQ = sQc + in_base;
             const uint8_t* tK = sK + in_base;
             float kt0[16], kt1[16], kh0[16], kh1[16];
 #pragma unroll
@@ -443,52 +487,71 @@ kda_chunk_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_consta
         tc_fence_before();
         __syncthreads();
         tc_fence_after();
+        // k and alpha are consumed: load the next chunk's
+        if (chunk + 1 < nchunks && ok) {
+            if (tid == 0) issue_ka(row0 + C);
+            issued(tka);
+        }
 
         KDA_TC_PHASE(1);
-        // ================= [A/beta | P] by sub-chunk: one M=128, N=128, K=128 MMA group
-        //   D[j][n]:  rows 0..31  x cols 0..63   = sub-chunk 0 (j < 32; [A/beta | P] columns r)
-        //             rows 64..127 x cols 64..127 = sub-chunk 1 (j < 64; columns r - 32)
+        // ================= [A/beta ; P] = [k*lam ; q*lam] [k*rho^0 ; k*rho^1]^T   (M=128, N=96, K=128)
+        //   rows 0..63 are A/beta rows r, rows 64..127 are P rows r.  Columns [0, 32) hold
+        //   rho^0 (j < 32, valid for r < 32), columns [32, 96) hold rho^1 (j < 64, valid for r >= 32).
         if (tid == 0 && ok) {   // nothing new is issued after a wait gave up
-            const uint32_t r0 = smem_u32(sX + X_R), l0 = smem_u32(sX + X_L);
-            constexpr uint32_t idesc = idesc_bf16(128, 128);
+            const uint32_t l0 = smem_u32(sX + X_L), r0 = smem_u32(sX + X_R);
+            constexpr uint32_t idesc = idesc_bf16(128, 96);
 #pragma unroll
-            for (int ks = 0; ks < 8; ++ks) {
-                const uint32_t off = (ks >> 2) * 16384u + (ks & 3) * 32u;
-                mma_bf16(tmem + TM_WK, sdesc_sw128(r0 + off), sdesc_sw128(l0 + off), idesc, ks > 0);
-            }
-            mma_commit(barM);
+            for (int ks = 0; ks < 8; ++ks)
+                mma_bf16(tmem + TM_WK, sdesc_sw128(l0 + (ks >> 2) * 16384u + (ks & 3) * 32u),
+                         sdesc_sw128(r0 + (ks >> 2) * 12288u + (ks & 3) * 32u), idesc, ks > 0);
+            commit_mma();
         }
         wait_mma();
 
         KDA_TC_PHASE(2);
-        // ================= A to fp32 shared memory (masked), P to the [I ; P] operand
-        if (q4 != 1) {
-            float* Am = reinterpret_cast<float*>(sX + X_AM);
-            const int sub = q4 == 0 ? 0 : 1;                       // which sub-chunk's block row
-            const int j = q4 == 0 ? lane : 32 * (q4 - 2) + lane;   // key token of this lane
-            const uint32_t col = (uint32_t)(64 * sub + 32 * hf);   // A part (hf 0) or P part (hf 1)
+        // ================= A (fp32, times beta_r, j < r) and P (bf16 K-major A operand, j <= r)
+        {
+            // lane = row R of the accumulator: R < 64 is A row r = R, R >= 64 is P row r = R - 64;
+            // this warp's column half covers j in [32 hf, 32 hf + 32)
+            const int R = 32 * q4 + lane, r = R & 63, j0 = 32 * hf;
+            const bool lower = (q4 & 1) == 0;          // r < 32: group 1 columns
+            const bool zero = lower && hf == 1;        // j >= 32 > r: all zero
             float v[32];
-            tmem_ld16(tmem + tlane + TM_WK + col, *reinterpret_cast<float(*)[16]>(&v[0]));
-            tmem_ld16(tmem + tlane + TM_WK + col + 16, *reinterpret_cast<float(*)[16]>(&v[16]));
-            tmem_wait_ld();
-            if (hf == 0) {
+            if (!zero && (q4 < 2 || !kSummary)) {
+                const uint32_t col = lower ? 0u : 32u + 32u * hf;
+                tmem_ld16(tmem + tlane + TM_WK + col, *reinterpret_cast<float(*)[16]>(&v[0]));
+                tmem_ld16(tmem + tlane + TM_WK + col + 16, *reinterpret_cast<float(*)[16]>(&v[16]));
+                tmem_wait_ld();
+            } else {
 #pragma unroll
-                for (int rr = 0; rr < 32; ++rr) {
-                    const int r = 32 * sub + rr;
-                    Am[r * AS + j] = (j < r) ? sBeta[r] * v[rr] : 0.0f;
+                for (int i = 0; i < 32; ++i) v[i] = 0.0f;
+            }
+            if (q4 < 2) {
+                float* Am = reinterpret_cast<float*>(sX + X_AM);
+                const float b = sBeta[r];
+#pragma unroll
+                for (int i = 0; i < 32; i += 4) {
+                    float4 f;
+                    f.x = (j0 + i + 0 < r) ? b * v[i + 0] : 0.0f;
+                    f.y = (j0 + i + 1 < r) ? b * v[i + 1] : 0.0f;
+                    f.z = (j0 + i + 2 < r) ? b * v[i + 2] : 0.0f;
+                    f.w = (j0 + i + 3 < r) ? b * v[i + 3] : 0.0f;
+                    *reinterpret_cast<float4*>(&Am[r * AS + j0 + i]) = f;
                 }
             } else if (!kSummary) {
+                uint8_t* sP = sX + X_P;
 #pragma unroll
-                for (int rr = 0; rr < 32; ++rr) {
-                    const int r = 32 * sub + rr;
-                    *reinterpret_cast<__nv_bfloat16*>(sIP + swz(64 + r, j >> 3) + ((j & 7) << 1)) =
-                        __float2bfloat16_rn((j <= r) ? v[rr] : 0.0f);
+                for (int c8 = 0; c8 < 4; ++c8) {
+                    float w[8];
+#pragma unroll
+                    for (int i = 0; i < 8; ++i) w[i] = (j0 + 8 * c8 + i <= r) ? v[8 * c8 + i] : 0.0f;
+                    *reinterpret_cast<uint4*>(sP + swz(r, (j0 >> 3) + c8)) = pack8(w);
                 }
             }
         }
+        fence_async_smem();
         tc_fence_before();
         __syncthreads();
-
         KDA_TC_PHASE(3);
         // ================= Tinv = (I + A)^-1 by doubling: 16x16 blocks, then 32, then 64
         //   inv([[X, 0], [Y, Z]]) = [[X^-1, 0], [-Z^-1 Y X^-1, Z^-1]]
@@ -591,7 +654,7 @@ kda_chunk_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_consta
 #pragma unroll
                 for (int ks = 0; ks < 4; ++ks)
                     mma_tf32(tmem + TM_WK, sdesc_sw128(a0 + ks * 32), sdesc_sw128(b0 + ks * 32), idesc, ks > 0);
-                mma_commit(barM);
+                commit_mma();
             }
             wait_mma();
             if (q4 < 2) {   // M=64 accumulator: rows m = 16*q4 + lane live in lanes 32*q4 + lane
@@ -617,7 +680,7 @@ kda_chunk_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_consta
 #pragma unroll
                 for (int ks = 0; ks < 4; ++ks)
                     mma_tf32(tmem + TM_WK + 32, sdesc_sw128(a0 + ks * 32), sdesc_sw128(b0 + ks * 32), idesc, ks > 0);
-                mma_commit(barM);
+                commit_mma();
             }
             wait_mma();
             if (q4 < 2) {
@@ -636,10 +699,8 @@ kda_chunk_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_consta
             tc_fence_before();
             __syncthreads();
             KDA_TC_PHASE(11);
-            // Tb = Tinv diag(beta) as MN-major B: row j, column m; zero above the diagonal.
-            // The same bytes are Tb as a K-major A operand (row j, k = m): a summary
-            // needs no P Tb and writes it straight to where [Tb ; P Tb] goes.
-            uint8_t* sTB = kSummary ? sAl : sX + X_TB;
+            // Tb = Tinv diag(beta) as the K-major A operand [64 r][64 m]; zero above the diagonal
+            uint8_t* sTB = sX + X_TB;
 #pragma unroll
             for (int rep = 0; rep < 2; ++rep) {
                 const int e = tid + NT * rep;
@@ -660,72 +721,28 @@ kda_chunk_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_consta
         tc_fence_after();
 
         KDA_TC_PHASE(4);
-        // ================= [Tb ; P Tb] = [I ; P] Tb   (M=128, N=64, K=64)
-        if (!kSummary) {
+        // ================= W = Tb (k*gamma)   (M=64, N=128, K=64)
         if (tid == 0 && ok) {
-            const uint32_t a0 = smem_u32(sIP), b0 = smem_u32(sX + X_TB);
-            constexpr uint32_t idesc = idesc_bf16(128, 64, false, true);
-#pragma unroll
-            for (int ks = 0; ks < 4; ++ks)
-                mma_bf16(tmem + TM_WK, sdesc_sw128(a0 + ks * 32), sdesc_sw128(b0 + ks * 2048), idesc,
-                         ks > 0);
-            mma_commit(barM);
-        }
-        wait_mma();
-        {
-            const int row = 32 * q4 + lane;
-            float v[32];
-            tmem_ld16(tmem + tlane + TM_WK + 32 * hf, *reinterpret_cast<float(*)[16]>(&v[0]));
-            tmem_ld16(tmem + tlane + TM_WK + 32 * hf + 16, *reinterpret_cast<float(*)[16]>(&v[16]));
-            tmem_wait_ld();
-#pragma unroll
-            for (int ch = 0; ch < 4; ++ch)
-                *reinterpret_cast<uint4*>(sAl + swz(row, 4 * hf + ch)) = pack8(&v[8 * ch]);
-        }
-        fence_async_smem();
-        tc_fence_before();
-        __syncthreads();
-        tc_fence_after();
-        }
-
-        KDA_TC_PHASE(5);
-        // ================= [W ; P W] = [Tb ; P Tb] (k*gamma)   (M=128, N=128, K=64)
-        if (tid == 0 && ok) {
-            const uint32_t a0 = smem_u32(sAl), b0 = smem_u32(sKT);
-            constexpr uint32_t idesc = idesc_bf16(128, 128);
+            const uint32_t a0 = smem_u32(sX + X_TB), b0 = smem_u32(sKT);
+            constexpr uint32_t idesc = idesc_bf16(64, 128);
 #pragma unroll
             for (int ks = 0; ks < 4; ++ks)
                 mma_bf16(tmem + TM_WK, sdesc_sw128(a0 + ks * 32), sdesc_sw128(b0 + ks * 32), idesc, ks > 0);
-            mma_commit(barM);
+            commit_mma();
         }
         wait_mma();
         {
-            // [-W ; q*gamma - P W] as the K-major A operand of the state MMA
-            const int row = 32 * q4 + lane;
-            uint8_t* sWQ = sX + X_WQ;
+            // -W as the K-major A operand of the U MMA; M=64 rows m = 16 q4 + lane (lane < 16)
             float v[64];
             tmem_ld64(tmem + tlane + TM_WK + 64 * hf, v);
-            if (row < 64) {
+            if (lane < 16) {
+                const int m = 16 * q4 + lane;
 #pragma unroll
-                for (int chunk = 0; chunk < 8; ++chunk) {
+                for (int ch = 0; ch < 8; ++ch) {
                     float w8[8];
 #pragma unroll
-                    for (int i = 0; i < 8; ++i) w8[i] = -v[8 * chunk + i];
-                    *reinterpret_cast<uint4*>(sWQ + hf * 16384 + swz(row, chunk)) = pack8(w8);
-                }
-            } else if (!kSummary) {
-#pragma unroll
-                for (int chunk = 0; chunk < 8; ++chunk) {
-                    const uint4 qg = *reinterpret_cast<const uint4*>(sQ + hf * 8192 + swz(row - 64, chunk));
-                    const uint32_t qw[4] = {qg.x, qg.y, qg.z, qg.w};
-                    float w8[8];
-#pragma unroll
-                    for (int i = 0; i < 4; ++i) {
-                        const float2 f = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&qw[i]));
-                        w8[2 * i] = f.x - v[8 * chunk + 2 * i];
-                        w8[2 * i + 1] = f.y - v[8 * chunk + 2 * i + 1];
-                    }
-                    *reinterpret_cast<uint4*>(sWQ + hf * 16384 + swz(row, chunk)) = pack8(w8);
+                    for (int i = 0; i < 8; ++i) w8[i] = -v[8 * ch + i];
+                    *reinterpret_cast<uint4*>(sX + X_WQ + hf * 8192 + swz(m, ch)) = pack8(w8);
                 }
             }
         }
@@ -733,26 +750,26 @@ kda_chunk_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_consta
         tc_fence_before();
         __syncthreads();
         tc_fence_after();
+        wait_load(barV, tv);
 
-        KDA_TC_PHASE(6);
+        KDA_TC_PHASE(5);
         if constexpr (kSummary) {
-        // ================= [U_M | U_N] = -W [M | N] + [0 | Tb V]   (M=128 of which rows
-        // 0..63 are used, N=256, K=128 (+64 for the N half))
+        // ================= [U_M | U_N] = -W [M | N] + [0 | Tb V]   (M=64, N=256, K=128 (+64))
         if (tid == 0 && ok) {
-            const uint32_t wq = smem_u32(sX + X_WQ), s0 = smem_u32(sS), tb = smem_u32(sAl),
+            const uint32_t wq = smem_u32(sX + X_WQ), s0 = smem_u32(sS), tb = smem_u32(sX + X_TB),
                            v0 = smem_u32(sV);
             const uint32_t d = tmem + TM_WK;
-            constexpr uint32_t idesc256 = idesc_bf16(128, 256, false, true);
-            constexpr uint32_t idesc128 = idesc_bf16(128, 128, false, true);
+            constexpr uint32_t id256 = idesc_bf16(64, 256, false, true);
+            constexpr uint32_t id128 = idesc_bf16(64, 128, false, true);
 #pragma unroll
             for (int ks = 0; ks < 8; ++ks)
-                mma_bf16(d, sdesc_sw128(wq + (ks >> 2) * 16384 + (ks & 3) * 32),
-                         sdesc_sw128(s0 + ks * 2048, 1024, 16384), idesc256, ks > 0);
+                mma_bf16(d, sdesc_sw128(wq + (ks >> 2) * 8192 + (ks & 3) * 32),
+                         sdesc_sw128(s0 + ks * 2048, 1024, 16384), id256, ks > 0);
 #pragma unroll
             for (int ks = 0; ks < 4; ++ks)
                 mma_bf16(d + 128, sdesc_sw128(tb + ks * 32), sdesc_sw128(v0 + ks * 2048, 1024, 8192),
-                         idesc128, 1);
-            mma_commit(barM);
+                         id128, 1);
+            commit_mma();
         }
         // meanwhile: [M | N] <- Diag(gamma_C) [M | N] in TMEM
         {
@@ -772,23 +789,33 @@ kda_chunk_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_consta
             tmem_wait_st();
         }
         wait_mma();
-        prefetch_next(chunk, row0);
-        if (q4 < 2) {   // U rows (tokens) 0..63: MN-major B [64 j][256 n], four 8 KB atoms
-            const int row = 32 * q4 + lane;
+        if (chunk + 1 < nchunks && ok) {   // v is consumed
+            if (tid == 0) issue_v(row0 + C);
+            issued(tv);
+        }
+        if (tid < C) {
+            const int64_t nxt = (int64_t)(chunk + 1) * C + tid;   // token index in the segment
+            beta_next = nxt < len ? __bfloat162float(beta[(size_t)(bos + nxt) * H + h]) : 0.0f;
+        }
+        {   // U rows j = 16 q4 + lane: MN-major B [64 j][256 n], four 8 KB atoms
 #pragma unroll
             for (int p = 0; p < 2; ++p) {
                 float v[64];
                 tmem_ld64(tmem + tlane + TM_WK + 128 * hf + 64 * p, v);
+                if (lane < 16) {
+                    const int j = 16 * q4 + lane;
 #pragma unroll
-                for (int ch = 0; ch < 8; ++ch)
-                    *reinterpret_cast<uint4*>(sX + X_U + (2 * hf + p) * 8192 + swz(row, ch)) =
-                        pack8(&v[8 * ch]);
+                    for (int ch = 0; ch < 8; ++ch)
+                        *reinterpret_cast<uint4*>(sX + X_U + (2 * hf + p) * 8192 + swz(j, ch)) =
+                            pack8(&v[8 * ch]);
+                }
             }
         }
         fence_async_smem();
         tc_fence_before();
         __syncthreads();
         tc_fence_after();
+        KDA_TC_PHASE(6);
         // ================= [M | N] += (k*eta)^T [U_M | U_N]   (M=128, N=256, K=64)
         if (tid == 0 && ok) {
             const uint32_t a0 = smem_u32(sKH), u0 = smem_u32(sX + X_U);
@@ -797,38 +824,27 @@ kda_chunk_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_consta
             for (int ks = 0; ks < 4; ++ks)
                 mma_bf16(tmem + TM_S, sdesc_sw128(a0 + ks * 32), sdesc_sw128(u0 + ks * 2048, 1024, 8192),
                          idesc, 1);
-            mma_commit(barM);
+            commit_mma();
         }
-        wait_mma();
-        {
-            const int c = 32 * q4 + lane;
-#pragma unroll
-            for (int p = 0; p < 2; ++p) {
-                float v[64];
-                tmem_ld64(tmem + tlane + TM_S + 128 * hf + 64 * p, v);
-#pragma unroll
-                for (int ch = 0; ch < 8; ++ch)
-                    *reinterpret_cast<uint4*>(sS + (2 * hf + p) * 16384 + swz(c, ch)) = pack8(&v[8 * ch]);
-            }
-        }
+        KDA_TC_PHASE(7);
         } else {
-        // ================= [U ; O] = [-W ; Q'] S + [Tb ; P Tb] V   (two N=64 halves, K=128+64)
+        // ================= U = -W S + Tb V   (M=64, N=128, K=128+64)
         if (tid == 0 && ok) {
-            const uint32_t wq = smem_u32(sX + X_WQ), s0 = smem_u32(sS), tb = smem_u32(sAl),
+            const uint32_t wq = smem_u32(sX + X_WQ), s0 = smem_u32(sS), tb = smem_u32(sX + X_TB),
                            v0 = smem_u32(sV);
             // B operands are MN-major with two 64-column atoms: leading byte offset = atom stride
-            constexpr uint32_t idesc = idesc_bf16(128, 128, false, true);
-            const uint32_t d = tmem + TM_UO;
+            constexpr uint32_t idesc = idesc_bf16(64, 128, false, true);
+            const uint32_t d = tmem + TM_U;
 #pragma unroll
             for (int ks = 0; ks < 8; ++ks)
-                mma_bf16(d, sdesc_sw128(wq + (ks >> 2) * 16384 + (ks & 3) * 32),
+                mma_bf16(d, sdesc_sw128(wq + (ks >> 2) * 8192 + (ks & 3) * 32),
                          sdesc_sw128(s0 + ks * 2048, 1024, 16384), idesc, ks > 0);
 #pragma unroll
             for (int ks = 0; ks < 4; ++ks)
                 mma_bf16(d, sdesc_sw128(tb + ks * 32), sdesc_sw128(v0 + ks * 2048, 1024, 8192), idesc, 1);
-            mma_commit(barM);
+            commit_mma();
         }
-        // meanwhile: S <- Diag(gamma_C) S in TMEM (the MMA reads the bf16 copy)
+        // meanwhile: S <- Diag(gamma_C) S in TMEM (the MMAs read the bf16 copy)
         {
             const int c = 32 * q4 + lane;
             const float g = sGC[c];
@@ -843,20 +859,22 @@ kda_chunk_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_consta
             tmem_wait_st();
         }
         wait_mma();
-        prefetch_next(chunk, row0);
-        {
-            const int row = 32 * q4 + lane;
-            uint8_t* sU = sX + X_U;
+        if (chunk + 1 < nchunks && ok) {   // v is consumed
+            if (tid == 0) issue_v(row0 + C);
+            issued(tv);
+        }
+        if (tid < C) {
+            const int64_t nxt = (int64_t)(chunk + 1) * C + tid;   // token index in the segment
+            beta_next = nxt < len ? __bfloat162float(beta[(size_t)(bos + nxt) * H + h]) : 0.0f;
+        }
+        {   // U as the MN-major B operand [64 j][128 n]: rows j = 16 q4 + lane (lane < 16)
             float v[64];
-            tmem_ld64(tmem + tlane + TM_UO + 64 * hf, v);
-            if (row < 64) {
+            tmem_ld64(tmem + tlane + TM_U + 64 * hf, v);
+            if (lane < 16) {
+                const int j = 16 * q4 + lane;
 #pragma unroll
-                for (int chunk = 0; chunk < 8; ++chunk)
-                    *reinterpret_cast<uint4*>(sU + hf * 8192 + swz(row, chunk)) = pack8(&v[8 * chunk]);
-            } else if (row - 64 < Lc) {
-                uint4* dst = reinterpret_cast<uint4*>(out + ((size_t)(row0 + row - 64) * H + h) * DV + 64 * hf);
-#pragma unroll
-                for (int chunk = 0; chunk < 8; ++chunk) dst[chunk] = pack8(&v[8 * chunk]);
+                for (int ch = 0; ch < 8; ++ch)
+                    *reinterpret_cast<uint4*>(sX + X_U + hf * 8192 + swz(j, ch)) = pack8(&v[8 * ch]);
             }
         }
         fence_async_smem();
@@ -864,34 +882,42 @@ kda_chunk_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_consta
         __syncthreads();
         tc_fence_after();
 
-        KDA_TC_PHASE(7);
-        // ================= S += (k*eta)^T U   (M=128, two N=64 halves, K=64)
+        KDA_TC_PHASE(6);
+        // ================= S += (k*eta)^T U   (M=128, N=128, K=64)
+        //                   O  = (q*gamma) S_start + P U   (M=64, N=128, K=128+64)
         if (tid == 0 && ok) {
-            const uint32_t a0 = smem_u32(sKH), u0 = smem_u32(sX + X_U);
-            constexpr uint32_t idesc = idesc_bf16(128, 128, false, true);
+            const uint32_t kh = smem_u32(sKH), u0 = smem_u32(sX + X_U), s0 = smem_u32(sS),
+                           qg = smem_u32(sQc), p0 = smem_u32(sX + X_P);
+            constexpr uint32_t id_s = idesc_bf16(128, 128, false, true);
+            constexpr uint32_t id_o = idesc_bf16(64, 128, false, true);
 #pragma unroll
             for (int ks = 0; ks < 4; ++ks)
-                mma_bf16(tmem + TM_S, sdesc_sw128(a0 + ks * 32), sdesc_sw128(u0 + ks * 2048, 1024, 8192),
-                         idesc, 1);
-            mma_commit(barM);
-        }
-        wait_mma();
-        {
-            const int c = 32 * q4 + lane;
-            float v[64];
-            tmem_ld64(tmem + tlane + TM_S + 64 * hf, v);
+                mma_bf16(tmem + TM_S, sdesc_sw128(kh + ks * 32), sdesc_sw128(u0 + ks * 2048, 1024, 8192),
+                         id_s, 1);
 #pragma unroll
-            for (int chunk = 0; chunk < 8; ++chunk)
-                *reinterpret_cast<uint4*>(sS + hf * 16384 + swz(c, chunk)) = pack8(&v[8 * chunk]);
+            for (int ks = 0; ks < 8; ++ks)
+                mma_bf16(tmem + TM_O, sdesc_sw128(qg + (ks >> 2) * 8192 + (ks & 3) * 32),
+                         sdesc_sw128(s0 + ks * 2048, 1024, 16384), id_o, ks > 0);
+#pragma unroll
+            for (int ks = 0; ks < 4; ++ks)
+                mma_bf16(tmem + TM_O, sdesc_sw128(p0 + ks * 32), sdesc_sw128(u0 + ks * 2048, 1024, 8192),
+                         id_o, 1);
+            commit_mma();
         }
+        KDA_TC_PHASE(7);
         }
         fence_async_smem();
         tc_fence_before();
         const int any_timeout = __syncthreads_or(!ok);   // uniform: every thread leaves together
         tc_fence_after();
         KDA_TC_PHASE(8);
-        if (any_timeout) break;
+        if (any_timeout) {
+            broke = true;
+            break;
+        }
     }
+    // the last chunk's state update and outputs
+    if (nchunks > 0 && !broke) finish_prev(bos + (int64_t)(nchunks - 1) * C, (int)(len - (int64_t)(nchunks - 1) * C));
 
     if (!ok) atomicExch(sFlag, 1);
     __syncthreads();
@@ -899,9 +925,11 @@ kda_chunk_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_consta
         // a wait gave up: let this CTA's own copies and MMAs in flight finish (bounded)
         // before its shared and tensor memory are released.  Thread 0 issues every
         // copy and MMA and stops issuing once one of its own waits gives up, so at
-        // most one of each is outstanding here.
-        if (tma_pending) mbar_wait_ns(barT, tma_pending_phase, kWaitNs);
-        if (mma_pending) mbar_wait_ns(barM, mma_pending_phase, kWaitNs);
+        // most one of each stream is outstanding here.
+        if (tq.pend) mbar_wait_ns(barQ, tq.pend_ph, kWaitNs);
+        if (tka.pend) mbar_wait_ns(barKA, tka.pend_ph, kWaitNs);
+        if (tv.pend) mbar_wait_ns(barV, tv.pend_ph, kWaitNs);
+        if (mma_out) mbar_wait_ns(barM, mma_out_ph, kWaitNs);
     }
     __syncthreads();
     if (kCtaStatus && tid == 0) status[(size_t)n * H + h] = *sFlag;
