@@ -70,16 +70,16 @@ constexpr uint32_t OFF_K = 65536;        // k tile
 constexpr uint32_t OFF_AL = 81920;       // alpha tile
 constexpr uint32_t OFF_V = 98304;        // v tile: MN-major B, two 64-column atoms of [64][64]
 constexpr uint32_t OFF_X = 114688;       // 72 KB work region, see below
-constexpr uint32_t OFF_KT = OFF_X + 73728;   // (k*gamma)^T  K-major B [128 c][64 j]
-constexpr uint32_t OFF_KH = OFF_KT + 16384;  // (k*eta)^T    K-major A [128 c][64 j]
+constexpr uint32_t OFF_KT = OFF_X + 73728;   // k*gamma  MN-major B [64 j][128 c] (two [64][64] atoms)
+constexpr uint32_t OFF_KH = OFF_KT + 16384;  // k*eta    MN-major A [64 j][128 c] (two [64][64] atoms)
 constexpr uint32_t OFF_MISC = OFF_KH + 16384;
-constexpr uint32_t MISC_PI = 0;          // float [4][128]
-constexpr uint32_t MISC_GC = 2048;       // float [128] gamma_C
-constexpr uint32_t MISC_BETA = 2560;     // float [64]
-constexpr uint32_t MISC_BAR = 2816;      // 4 x uint64 mbarriers: q, k+alpha, v, MMA
-constexpr uint32_t MISC_TMEM = 2848;     // uint32 TMEM base
-constexpr uint32_t MISC_FLAG = 2852;     // int timeout seen
-constexpr uint32_t SMEM_BYTES = OFF_MISC + 2880 + 1024;  // + alignment slack
+constexpr uint32_t MISC_PI = 0;          // float [8][128] octant gate products
+constexpr uint32_t MISC_GC = 4096;       // float [128] gamma_C
+constexpr uint32_t MISC_BETA = 4608;     // float [64]
+constexpr uint32_t MISC_BAR = 4864;      // 4 x uint64 mbarriers: q, k+alpha, v, MMA
+constexpr uint32_t MISC_TMEM = 4896;     // uint32 TMEM base
+constexpr uint32_t MISC_FLAG = 4900;     // int timeout seen
+constexpr uint32_t SMEM_BYTES = OFF_MISC + 4928 + 1024;  // + alignment slack
 
 // work region X, by phase
 constexpr uint32_t X_L = 0;              // left rows [128][128]: k*lam rows 0..63, q*lam rows 64..127
@@ -109,12 +109,13 @@ __device__ __forceinline__ uint32_t swz(uint32_t row, uint32_t chunk) {
 __device__ __forceinline__ uint32_t f32_off(uint32_t r, uint32_t k) {
     return r * 128u + ((((k >> 2) ^ r) & 7u) << 4) + ((k & 3u) << 2);
 }
-__device__ __forceinline__ float2 ld_bf2(const uint8_t* p) {
-    const __nv_bfloat162 v = *reinterpret_cast<const __nv_bfloat162*>(p);
-    return __bfloat1622float2(v);
+__device__ __forceinline__ void unpack4_bf16(uint2 raw, float (&v)[4]) {
+    const float2 lo = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&raw.x));
+    const float2 hi = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&raw.y));
+    v[0] = lo.x; v[1] = lo.y; v[2] = hi.x; v[3] = hi.y;
 }
-__device__ __forceinline__ void st_bf2(uint8_t* p, float a, float b) {
-    *reinterpret_cast<uint32_t*>(p) = pack_bf16x2(a, b);
+__device__ __forceinline__ void st4_bf16(uint8_t* p, const float (&v)[4]) {
+    *reinterpret_cast<uint2*>(p) = make_uint2(pack_bf16x2(v[0], v[1]), pack_bf16x2(v[2], v[3]));
 }
 
 // 64 consecutive fp32 columns of this thread's TMEM lane, one wait for all four loads
@@ -157,7 +158,7 @@ template <bool kCtaStatus, bool kSummary>
 __global__ void __launch_bounds__(NT, 1)
 kda_chunk_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                     const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmV,
-                    const __nv_bfloat16* __restrict__ beta, const float* S0,
+                    const __grid_constant__ CUtensorMap tmO, const __nv_bfloat16* __restrict__ beta, const float* S0,
                     const int32_t* __restrict__ cu_seqlens, __nv_bfloat16* __restrict__ out,
                     float* S_final, int64_t T, int H, int* status, const Segments seg) {
     extern __shared__ uint8_t smem_raw[];
@@ -314,7 +315,10 @@ kda_chunk_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_consta
     // The state update (and O) of a chunk is waited for, and its results taken out
     // of TMEM, only inside the next chunk's gate phase: nothing before the next
     // chunk's U MMA needs them.  S goes to its bf16 copy, O to the output rows.
-    auto finish_prev = [&](int64_t prow0, int pLc) {
+    // A full chunk's O is staged in the q buffer the next q load will use (row-major,
+    // 128-byte swizzled, the TMA box layout) and written by one TMA store; a
+    // partial last chunk is stored row by row.
+    auto finish_prev = [&](int64_t prow0, int pLc, uint8_t* stage) {
         wait_mma();
         const int c = 32 * q4 + lane;
         if constexpr (kSummary) {
@@ -334,12 +338,23 @@ kda_chunk_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_consta
                 *reinterpret_cast<uint4*>(sS + hf * 16384 + swz(c, ch)) = pack8(&v[8 * ch]);
             tmem_ld64(tmem + tlane + TM_O + 64 * hf, v);
             const int r = 16 * q4 + lane;
-            if (lane < 16 && r < pLc) {
+            if (pLc == C) {
+                if (lane < 16) {
+#pragma unroll
+                    for (int ch = 0; ch < 8; ++ch)
+                        *reinterpret_cast<uint4*>(stage + hf * 8192 + swz(r, ch)) = pack8(&v[8 * ch]);
+                }
+            } else if (lane < 16 && r < pLc) {
                 uint4* dst = reinterpret_cast<uint4*>(out + ((size_t)(prow0 + r) * H + h) * DV + 64 * hf);
 #pragma unroll
                 for (int ch = 0; ch < 8; ++ch) dst[ch] = pack8(&v[8 * ch]);
             }
         }
+    };
+    auto store_o = [&](uint8_t* stage, int64_t prow0) {   // thread 0, after a barrier
+#pragma unroll
+        for (int a = 0; a < 2; ++a) tma_store_2d(&tmO, stage + a * 8192, h * DV + 64 * a, (int)prow0);
+        bulk_commit_group();
     };
 
     if (nchunks > 0) {
@@ -373,120 +388,143 @@ kda_chunk_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_consta
 
         // ================= gate products and bf16 operands (all threads)
         {
-            // thread = (channel pair c0, c0+1) x (16-token quarter Q).  Sub-chunk I = Q/2
-            // holds 32 tokens; its reference token is ref_I = 32I + 15.  With phi / psi the
-            // in-quarter forward (inclusive) / backward (exclusive) gate products and pi_Q
-            // the quarter product:
+            // thread = (channels c0..c0+3) x (8-token octant O).  Quarter Q = O/2 holds 16
+            // tokens, sub-chunk I = Q/2 holds 32; the reference token of I is ref_I = 32I + 15.
+            // With phi / psi the in-quarter forward (inclusive) / backward (exclusive) gate
+            // products and pi_Q the quarter product:
             //   left  lam_t   = e^{g_t - g_ref}  = phi_t * (Q even ? 1/pi_Q : 1)
             //   right rho^I_j = e^{g_ref - g_j}  = psi_j * c_I(Q(j))
             //   c_0 = {1, 1/pi_1},  c_1 = {pi_1 pi_2, pi_2, 1, 1/pi_3}
             // so that lam_r rho^I_j = prod_{s=j+1..r} a_s for j <= r, every factor within
             // [e^-80, e^80] except right factors that underflow where the product is negligible.
-            // All tiles touched here have 8-row-aligned bases, so the swizzled offset of
-            // (row i of a 16-row group, this channel pair) is i*128 + xo[i & 7].
-            const int cp = tid & 63, Q = tid >> 6, c0 = 2 * cp;
-            const uint32_t atom = (uint32_t)(c0 >> 6);
+            // In-quarter products come from in-octant ones phi8, psi8 and the octant products
+            // pi8: phi = phi8 * (O odd ? pi8_{O-1} : 1), psi = psi8 * (O even ? pi8_{O+1} : 1);
+            // those octant factors are folded into the per-thread scales below.
+            // Every tile touched here is row-major with 128-byte swizzled rows; a warp covers
+            // one token row of all 128 channels (8 bytes per thread).
+            const int cq = tid & 31, O = tid >> 5, Q = O >> 1, c0 = 4 * cq;
             const uint32_t chk = (uint32_t)((c0 & 63) >> 3), inner = (uint32_t)((c0 & 7) << 1);
-            uint32_t xo[8];
+            const uint32_t a64 = (uint32_t)(c0 >> 6);
+            float phi[8][4], psi[8][4];   // psi holds the clamped gates until the backward pass
 #pragma unroll
-            for (int k8 = 0; k8 < 8; ++k8) xo[k8] = (((chk ^ (uint32_t)k8) & 7u) << 4) | inner;
-            const uint32_t in_base = atom * 8192u + (uint32_t)(16 * Q) * 128u;   // 64-row input tiles
-            float phi0[16], phi1[16], psi0[16], psi1[16];
-            {
-                float a0[16], a1[16];
+            for (int i = 0; i < 8; ++i) {
+                const int r = 8 * O + i;
+                const uint32_t off = a64 * 8192u + (uint32_t)r * 128u + (((chk ^ (uint32_t)r) & 7u) << 4) + inner;
+                float a[4];
+                unpack4_bf16(*reinterpret_cast<const uint2*>(sAl + off), a);
 #pragma unroll
-                for (int i = 0; i < 16; ++i) {
-                    const int r = 16 * Q + i;
-                    const float2 al = ld_bf2(sAl + in_base + i * 128 + xo[i & 7]);
-                    a0[i] = r < Lc ? clamp_gate(al.x) : 1.0f;
-                    a1[i] = r < Lc ? clamp_gate(al.y) : 1.0f;
-                }
-                float p0 = 1.f, p1 = 1.f;
-#pragma unroll
-                for (int i = 0; i < 16; ++i) {
-                    p0 *= a0[i]; p1 *= a1[i];
-                    phi0[i] = p0; phi1[i] = p1;
-                }
-                float s0 = 1.f, s1 = 1.f;
-#pragma unroll
-                for (int i = 15; i >= 0; --i) {
-                    psi0[i] = s0; psi1[i] = s1;
-                    s0 *= a0[i]; s1 *= a1[i];
-                }
-                *reinterpret_cast<float2*>(&sPi[Q * DK + c0]) = make_float2(p0, p1);
+                for (int c = 0; c < 4; ++c) psi[i][c] = r < Lc ? clamp_gate(a[c]) : 1.0f;
             }
+            {
+                float p[4] = {1.f, 1.f, 1.f, 1.f}, b[4] = {1.f, 1.f, 1.f, 1.f};
+#pragma unroll
+                for (int i = 0; i < 8; ++i)
+#pragma unroll
+                    for (int c = 0; c < 4; ++c) { p[c] *= psi[i][c]; phi[i][c] = p[c]; }
+#pragma unroll
+                for (int i = 7; i >= 0; --i)
+#pragma unroll
+                    for (int c = 0; c < 4; ++c) { const float a = psi[i][c]; psi[i][c] = b[c]; b[c] *= a; }
+                *reinterpret_cast<float4*>(&sPi[O * DK + c0]) = make_float4(p[0], p[1], p[2], p[3]);
+            }
+            KDA_TC_PHASE(13);
             __syncthreads();
+            KDA_TC_PHASE(14);
             // the previous chunk's state update and O (their operands KH, U, P and the
             // q buffer are overwritten from here on)
-            if (chunk > 0) finish_prev(row0 - C, C);
-            if (!kSummary && chunk + 1 < nchunks && ok) {
-                if (tid == 0) issue_q(row0 + C, (chunk + 1) & 1);
-                issued(tq);
-            }
-            float pi0[4], pi1[4];
+            if (chunk > 0) finish_prev(row0 - C, C, sQ + ((chunk + 1) & 1) * 16384);
+            KDA_TC_PHASE(15);
+            // per-thread scales: quarter products, gamma before / eta after this quarter
+            float dlf[4], bf[4], r0g[4], r1g[4], ag[4];
+            {
+                float pq[4][4];   // [quarter][channel]
 #pragma unroll
-            for (int M = 0; M < 4; ++M) {
-                const float2 pm = *reinterpret_cast<const float2*>(&sPi[M * DK + c0]);
-                pi0[M] = pm.x; pi1[M] = pm.y;
-            }
-            float bef0 = 1.f, bef1 = 1.f, aft0 = 1.f, aft1 = 1.f;
+                for (int M = 0; M < 4; ++M) {
+                    const float4 u = *reinterpret_cast<const float4*>(&sPi[(2 * M) * DK + c0]);
+                    const float4 v = *reinterpret_cast<const float4*>(&sPi[(2 * M + 1) * DK + c0]);
+                    pq[M][0] = u.x * v.x; pq[M][1] = u.y * v.y; pq[M][2] = u.z * v.z; pq[M][3] = u.w * v.w;
+                }
+                // the partner octant of this quarter: phi8 -> phi (O odd), psi8 -> psi (O even)
+                const float4 po = *reinterpret_cast<const float4*>(&sPi[(O ^ 1) * DK + c0]);
+                const float pov[4] = {po.x, po.y, po.z, po.w};
 #pragma unroll
-            for (int M = 0; M < 4; ++M) {
-                if (M < Q) { bef0 *= pi0[M]; bef1 *= pi1[M]; }
-                if (M > Q) { aft0 *= pi0[M]; aft1 *= pi1[M]; }
-            }
-            if (Q == 0)
-                *reinterpret_cast<float2*>(&sGC[c0]) =
-                    make_float2(pi0[0] * pi0[1] * pi0[2] * pi0[3], pi1[0] * pi1[1] * pi1[2] * pi1[3]);
-            // left scale d_Q and right scales c_0(Q) (Q < 2) and c_1(Q)
-            float dl0 = 1.f, dl1 = 1.f, r00 = 1.f, r01 = 1.f, r10 = 1.f, r11 = 1.f;
-            if ((Q & 1) == 0) { dl0 = __frcp_rn(pi0[Q]); dl1 = __frcp_rn(pi1[Q]); }
-            if (Q == 1) { r00 = __frcp_rn(pi0[1]); r01 = __frcp_rn(pi1[1]); }
-            if (Q == 0) { r10 = pi0[1] * pi0[2]; r11 = pi1[1] * pi1[2]; }
-            if (Q == 1) { r10 = pi0[2]; r11 = pi1[2]; }
-            if (Q == 3) { r10 = __frcp_rn(pi0[3]); r11 = __frcp_rn(pi1[3]); }
-            // left rows: k*lam at row t, q*lam at row 64 + t (atoms of 128 rows)
-            uint8_t* tLk = sX + X_L + atom * 16384u + (uint32_t)(16 * Q) * 128u;
-            uint8_t* tLq = tLk + 64 * 128;
-            // right rows: rho^0 of token t < 32 at row t, rho^1 of token t at row 32 + t
-            uint8_t* tR0 = sX + X_R + atom * 12288u + (uint32_t)(16 * Q) * 128u;
-            uint8_t* tR1 = tR0 + 32 * 128;
-            uint8_t* tQ = sQc + in_base;
-            const uint8_t* tK = sK + in_base;
-            float kt0[16], kt1[16], kh0[16], kh1[16];
+                for (int c = 0; c < 4; ++c) {
+                    float bef = 1.f, aft = 1.f, own = 1.f;
 #pragma unroll
-            for (int i = 0; i < 16; ++i) {
-                const int r = 16 * Q + i;
-                const uint32_t off = i * 128 + xo[i & 7];
-                float2 kk = ld_bf2(tK + off);
-                float2 qq = kSummary ? make_float2(0.f, 0.f) : ld_bf2(tQ + off);
-                if (r >= Lc) { kk = make_float2(0.f, 0.f); qq = kk; }
-                const float kp0 = kk.x * phi0[i], kp1 = kk.y * phi1[i];
-                const float qp0 = qq.x * phi0[i], qp1 = qq.y * phi1[i];
-                const float ks0 = kk.x * psi0[i], ks1 = kk.y * psi1[i];
-                st_bf2(tLk + off, kp0 * dl0, kp1 * dl1);
-                if (!kSummary) st_bf2(tLq + off, qp0 * dl0, qp1 * dl1);
-                if (Q < 2) st_bf2(tR0 + off, ks0 * r00, ks1 * r01);
-                st_bf2(tR1 + off, ks0 * r10, ks1 * r11);
-                if (!kSummary) st_bf2(tQ + off, qp0 * bef0, qp1 * bef1);   // q*gamma in place
-                kt0[i] = kp0 * bef0; kt1[i] = kp1 * bef1;    // k*gamma
-                kh0[i] = ks0 * aft0; kh1[i] = ks1 * aft1;    // k*eta
+                    for (int M = 0; M < 4; ++M) {
+                        if (M < Q) bef *= pq[M][c];
+                        if (M > Q) aft *= pq[M][c];
+                        if (M == Q) own = pq[M][c];
+                    }
+                    if (O == 0) sGC[c0 + c] = pq[0][c] * pq[1][c] * pq[2][c] * pq[3][c];
+                    const float fO = (O & 1) ? pov[c] : 1.0f;
+                    const float gO = (O & 1) ? 1.0f : pov[c];
+                    const float dl = (Q & 1) ? 1.0f : __frcp_rn(own);
+                    const float r0 = Q == 1 ? __frcp_rn(own) : 1.0f;
+                    const float r1 = Q == 0 ? pq[1][c] * pq[2][c]
+                                            : (Q == 1 ? pq[2][c] : (Q == 2 ? 1.0f : __frcp_rn(own)));
+                    dlf[c] = dl * fO;
+                    bf[c] = bef * fO;
+                    r0g[c] = r0 * gO;
+                    r1g[c] = r1 * gO;
+                    ag[c] = aft * gO;
+                }
             }
-            // transposed tiles [c][j]: tokens 16Q..16Q+15 are chunks 2Q, 2Q+1 of rows c0, c0+1
 #pragma unroll
-            for (int half = 0; half < 2; ++half) {
-                const int ch = 2 * Q + half;
-                const int b = 8 * half;
-                *reinterpret_cast<uint4*>(sKT + swz(c0, ch)) = pack8(&kt0[b]);
-                *reinterpret_cast<uint4*>(sKT + swz(c0 + 1, ch)) = pack8(&kt1[b]);
-                *reinterpret_cast<uint4*>(sKH + swz(c0, ch)) = pack8(&kh0[b]);
-                *reinterpret_cast<uint4*>(sKH + swz(c0 + 1, ch)) = pack8(&kh1[b]);
+            for (int i = 0; i < 8; ++i) {
+                const int r = 8 * O + i;
+                const uint32_t sw = (uint32_t)r * 128u + (((chk ^ (uint32_t)r) & 7u) << 4) + inner;
+                const uint32_t in_off = a64 * 8192u + sw;    // 64-row tiles: q, k, KT, KH
+                float k[4], q[4] = {0.f, 0.f, 0.f, 0.f};
+                unpack4_bf16(*reinterpret_cast<const uint2*>(sK + in_off), k);
+                if (!kSummary) unpack4_bf16(*reinterpret_cast<const uint2*>(sQc + in_off), q);
+                if (r >= Lc) {
+#pragma unroll
+                    for (int c = 0; c < 4; ++c) { k[c] = 0.0f; q[c] = 0.0f; }
+                }
+                float kp[4], qp[4], ks[4], w[4];
+#pragma unroll
+                for (int c = 0; c < 4; ++c) {
+                    kp[c] = k[c] * phi[i][c];
+                    qp[c] = q[c] * phi[i][c];
+                    ks[c] = k[c] * psi[i][c];
+                }
+                uint8_t* lrow = sX + X_L + a64 * 16384u + sw;             // 128-row atoms
+                uint8_t* rrow = sX + X_R + a64 * 12288u + sw;             // 96-row atoms
+#pragma unroll
+                for (int c = 0; c < 4; ++c) w[c] = kp[c] * dlf[c];
+                st4_bf16(lrow, w);                                        // k*lam, row r
+                if (!kSummary) {
+#pragma unroll
+                    for (int c = 0; c < 4; ++c) w[c] = qp[c] * dlf[c];
+                    st4_bf16(lrow + 64 * 128, w);                         // q*lam, row 64 + r
+#pragma unroll
+                    for (int c = 0; c < 4; ++c) w[c] = qp[c] * bf[c];
+                    st4_bf16(sQc + in_off, w);                            // q*gamma in place
+                }
+                if (O < 4) {
+#pragma unroll
+                    for (int c = 0; c < 4; ++c) w[c] = ks[c] * r0g[c];
+                    st4_bf16(rrow, w);                                    // k*rho^0, row r < 32
+                }
+#pragma unroll
+                for (int c = 0; c < 4; ++c) w[c] = ks[c] * r1g[c];
+                st4_bf16(rrow + 32 * 128, w);                             // k*rho^1, row 32 + r
+#pragma unroll
+                for (int c = 0; c < 4; ++c) w[c] = kp[c] * bf[c];
+                st4_bf16(sKT + in_off, w);                                // k*gamma
+#pragma unroll
+                for (int c = 0; c < 4; ++c) w[c] = ks[c] * ag[c];
+                st4_bf16(sKH + in_off, w);                                // k*eta
             }
+            KDA_TC_PHASE(16);
         }
         fence_async_smem();
         tc_fence_before();
         __syncthreads();
         tc_fence_after();
+        // the previous chunk's O tile is staged: store it
+        if (!kSummary && chunk > 0 && tid == 0) store_o(sQ + ((chunk + 1) & 1) * 16384, row0 - C);
         // k and alpha are consumed: load the next chunk's
         if (chunk + 1 < nchunks && ok) {
             if (tid == 0) issue_ka(row0 + C);
@@ -507,6 +545,13 @@ kda_chunk_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_consta
             commit_mma();
         }
         wait_mma();
+        // the O store has read its staging buffer by now (checked, so that the buffer
+        // may be reused): load the next q there
+        if (!kSummary && tid == 0) bulk_wait_read_all();
+        if (!kSummary && chunk + 1 < nchunks && ok) {
+            if (tid == 0) issue_q(row0 + C, (chunk + 1) & 1);
+            issued(tq);
+        }
 
         KDA_TC_PHASE(2);
         // ================= A (fp32, times beta_r, j < r) and P (bf16 K-major A operand, j <= r)
@@ -724,10 +769,11 @@ kda_chunk_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_consta
         // ================= W = Tb (k*gamma)   (M=64, N=128, K=64)
         if (tid == 0 && ok) {
             const uint32_t a0 = smem_u32(sX + X_TB), b0 = smem_u32(sKT);
-            constexpr uint32_t idesc = idesc_bf16(64, 128);
+            constexpr uint32_t idesc = idesc_bf16(64, 128, false, true);
 #pragma unroll
             for (int ks = 0; ks < 4; ++ks)
-                mma_bf16(tmem + TM_WK, sdesc_sw128(a0 + ks * 32), sdesc_sw128(b0 + ks * 32), idesc, ks > 0);
+                mma_bf16(tmem + TM_WK, sdesc_sw128(a0 + ks * 32), sdesc_sw128(b0 + ks * 2048, 1024, 8192),
+                         idesc, ks > 0);
             commit_mma();
         }
         wait_mma();
@@ -819,11 +865,11 @@ kda_chunk_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_consta
         // ================= [M | N] += (k*eta)^T [U_M | U_N]   (M=128, N=256, K=64)
         if (tid == 0 && ok) {
             const uint32_t a0 = smem_u32(sKH), u0 = smem_u32(sX + X_U);
-            constexpr uint32_t idesc = idesc_bf16(128, 256, false, true);
+            constexpr uint32_t idesc = idesc_bf16(128, 256, true, true);
 #pragma unroll
             for (int ks = 0; ks < 4; ++ks)
-                mma_bf16(tmem + TM_S, sdesc_sw128(a0 + ks * 32), sdesc_sw128(u0 + ks * 2048, 1024, 8192),
-                         idesc, 1);
+                mma_bf16(tmem + TM_S, sdesc_sw128(a0 + ks * 2048, 1024, 8192),
+                         sdesc_sw128(u0 + ks * 2048, 1024, 8192), idesc, 1);
             commit_mma();
         }
         KDA_TC_PHASE(7);
@@ -888,12 +934,12 @@ kda_chunk_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_consta
         if (tid == 0 && ok) {
             const uint32_t kh = smem_u32(sKH), u0 = smem_u32(sX + X_U), s0 = smem_u32(sS),
                            qg = smem_u32(sQc), p0 = smem_u32(sX + X_P);
-            constexpr uint32_t id_s = idesc_bf16(128, 128, false, true);
+            constexpr uint32_t id_s = idesc_bf16(128, 128, true, true);
             constexpr uint32_t id_o = idesc_bf16(64, 128, false, true);
 #pragma unroll
             for (int ks = 0; ks < 4; ++ks)
-                mma_bf16(tmem + TM_S, sdesc_sw128(kh + ks * 32), sdesc_sw128(u0 + ks * 2048, 1024, 8192),
-                         id_s, 1);
+                mma_bf16(tmem + TM_S, sdesc_sw128(kh + ks * 2048, 1024, 8192),
+                         sdesc_sw128(u0 + ks * 2048, 1024, 8192), id_s, 1);
 #pragma unroll
             for (int ks = 0; ks < 8; ++ks)
                 mma_bf16(tmem + TM_O, sdesc_sw128(qg + (ks >> 2) * 8192 + (ks & 3) * 32),
@@ -916,11 +962,19 @@ kda_chunk_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_consta
             break;
         }
     }
-    // the last chunk's state update and outputs
-    if (nchunks > 0 && !broke) finish_prev(bos + (int64_t)(nchunks - 1) * C, (int)(len - (int64_t)(nchunks - 1) * C));
+    // the last chunk's state update and outputs (staged in the q buffer it did not use)
+    const int last_Lc = nchunks > 0 ? (int)(len - (int64_t)(nchunks - 1) * C) : 0;
+    uint8_t* last_stage = sQ + (nchunks & 1) * 16384;
+    if (nchunks > 0 && !broke) finish_prev(bos + (int64_t)(nchunks - 1) * C, last_Lc, last_stage);
+    fence_async_smem();
 
     if (!ok) atomicExch(sFlag, 1);
     __syncthreads();
+    if (!kSummary && tid == 0) {
+        if (nchunks > 0 && !broke && !*sFlag && last_Lc == C)
+            store_o(last_stage, bos + (int64_t)(nchunks - 1) * C);
+        bulk_wait_all();   // every O store has completed before shared memory is released
+    }
     if (*sFlag && tid == 0) {
         // a wait gave up: let this CTA's own copies and MMAs in flight finish (bounded)
         // before its shared and tensor memory are released.  Thread 0 issues every
@@ -1051,13 +1105,15 @@ static bool make_map(CUtensorMap* m, const void* base, int64_t rows, int H) {
 }  // namespace tc
 
 struct TcMaps {
-    CUtensorMap q, k, a, v;
+    CUtensorMap q, k, a, v, o;
 };
 
+// out may be null (segment summaries write no output): its map then reuses v's.
 static bool make_maps(TcMaps* m, const void* q, const void* k, const void* v, const void* alpha,
-                      int64_t rows, int H) {
+                      const void* out, int64_t rows, int H) {
     return tc::make_map(&m->q, q, rows, H) && tc::make_map(&m->k, k, rows, H) &&
-           tc::make_map(&m->a, alpha, rows, H) && tc::make_map(&m->v, v, rows, H);
+           tc::make_map(&m->a, alpha, rows, H) && tc::make_map(&m->v, v, rows, H) &&
+           tc::make_map(&m->o, out ? out : v, rows, H);
 }
 
 template <bool kCtaStatus, bool kSummary>
@@ -1070,7 +1126,7 @@ static cudaError_t launch_tc_t(const TcMaps& m, const void* beta, const float* S
     if (e != cudaSuccess) return e;
     dim3 grid(1, H, nseq * seg.per_seq);
     tc::kda_chunk_tc_kernel<kCtaStatus, kSummary><<<grid, tc::NT, tc::SMEM_BYTES, stream>>>(
-        m.q, m.k, m.a, m.v, (const __nv_bfloat16*)beta, S0, cu, (__nv_bfloat16*)out, S_final, T, H,
+        m.q, m.k, m.a, m.v, m.o, (const __nv_bfloat16*)beta, S0, cu, (__nv_bfloat16*)out, S_final, T, H,
         status, seg);
     return cudaGetLastError();
 }
@@ -1080,7 +1136,7 @@ cudaError_t launch_chunk_tc(const void* q, const void* k, const void* v, const v
                             void* out, float* S_final, int64_t rows, int64_t T, int H, int* status,
                             cudaStream_t stream) {
     TcMaps m;
-    if (!make_maps(&m, q, k, v, alpha, rows, H)) return cudaErrorInvalidValue;
+    if (!make_maps(&m, q, k, v, alpha, out, rows, H)) return cudaErrorInvalidValue;
     const tc::Segments whole{1, 1, nullptr, nullptr};
     return launch_tc_t<false, false>(m, beta, S0, cu, nseq, out, S_final, T, H, status, whole,
                                      stream);
@@ -1103,7 +1159,7 @@ cudaError_t launch_chunk_tc_segmented(const void* q, const void* k, const void* 
                                       int* status, cudaStream_t stream) {
     if (nseg < 2 || nseq * (int64_t)nseg > 65535) return cudaErrorInvalidValue;
     TcMaps m;
-    if (!make_maps(&m, q, k, v, alpha, rows, H)) return cudaErrorInvalidValue;
+    if (!make_maps(&m, q, k, v, alpha, out, rows, H)) return cudaErrorInvalidValue;
     float* maps = workspace;
     float* start = workspace + (size_t)nseq * H * (nseg - 1) * tc::DK * (tc::DK + tc::DV);
     const tc::Segments summary{nseg, nseg - 1, nullptr, maps};
@@ -1126,7 +1182,7 @@ cudaError_t launch_chunk_tc_cta_status(const void* q, const void* k, const void*
                                        int64_t rows, int64_t T, int H, int* status,
                                        cudaStream_t stream) {
     TcMaps m;
-    if (!make_maps(&m, q, k, v, alpha, rows, H)) return cudaErrorInvalidValue;
+    if (!make_maps(&m, q, k, v, alpha, out, rows, H)) return cudaErrorInvalidValue;
     const tc::Segments whole{1, 1, nullptr, nullptr};
     return launch_tc_t<true, false>(m, beta, S0, cu, nseq, out, S_final, T, H, status, whole,
                                     stream);
