@@ -58,7 +58,8 @@ namespace tc {
 constexpr int C = 64;         // tokens per chunk
 constexpr int DK = 128;       // key channels
 constexpr int DV = 128;       // value channels
-constexpr int NT = 256;       // threads
+constexpr int NT = 256;       // compute threads (8 warps)
+constexpr int NTHREADS = NT + 32;   // plus one control warp that issues every TMA copy and MMA
 constexpr uint64_t kWaitNs = 2000000000ull;  // 2 s per wait, then report a timeout
 
 // shared-memory map (bytes from the 1024-aligned base)
@@ -131,6 +132,9 @@ __device__ __forceinline__ uint4 pack8(const float* v) {
                       pack_bf16x2(v[6], v[7]));
 }
 
+// barrier among the eight compute warps only (the control warp is not held up)
+__device__ __forceinline__ void sync_compute() { asm volatile("bar.sync 1, 256;" ::: "memory"); }
+
 // M=64 accumulator: row m lives in TMEM lane 32*(m/16) + m%16
 // M=128 accumulator: row m lives in lane m.
 
@@ -144,18 +148,17 @@ struct Segments {
     float* maps;          // summary: [M | N] fp32 [nseq * (nseg - 1), H, DK, DK + DV]
 };
 
-// One TMA stream's bookkeeping: the parity its next wait expects, and the load
-// (if any) issued but not yet waited for.
+// One TMA stream's bookkeeping: the parity a thread's next wait on it expects,
+// and (control thread) how many loads were issued on it.
 struct LoadTrack {
-    uint32_t ph = 0, pend_ph = 0;
-    bool pend = false;
+    uint32_t ph = 0, issued = 0;
 };
 
 // kCtaStatus = false: a timed-out wait sets the shared word *status to 1.
 // kCtaStatus = true:  every CTA writes its own word status[n * H + h] (0 or 1).
 // kSummary = true: the segment-map mode described at the top (q and out unused).
 template <bool kCtaStatus, bool kSummary>
-__global__ void __launch_bounds__(NT, 1)
+__global__ void __launch_bounds__(NTHREADS, 1)
 kda_chunk_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                     const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmV,
                     const __grid_constant__ CUtensorMap tmO, const __nv_bfloat16* __restrict__ beta, const float* S0,
@@ -183,6 +186,8 @@ kda_chunk_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_consta
     int* sFlag = reinterpret_cast<int*>(sm + OFF_MISC + MISC_FLAG);
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const bool compute = warp < NT / 32;   // warps 0-7; warp 8 is the control warp
+    const bool ctl = warp == NT / 32 && lane == 0;   // the thread that issues copies and MMAs
     const int q4 = warp & 3;            // TMEM lane quarter this warp may touch
     const int hf = warp >> 2;           // which half of the columns this warp handles
     const int h = blockIdx.y;
@@ -223,7 +228,8 @@ kda_chunk_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_consta
     const uint32_t tlane = (uint32_t)(32 * q4) << 16;
 
     // ---- initial state: TMEM S (fp32) and its bf16 copy (MN-major B operand)
-    if constexpr (kSummary) {
+    if (!compute) {
+    } else if constexpr (kSummary) {
         // [M | N] = [I | 0]; this warp writes row c, columns 128 hf .. 128 hf + 127
         const int c = 32 * q4 + lane;
 #pragma unroll
@@ -286,19 +292,13 @@ kda_chunk_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_consta
     // asynchronous work that a timed-out wait may leave in flight, drained before exit
     LoadTrack tq, tka, tv;
     uint32_t phM = 0, mma_out_ph = 0;
-    bool mma_out = false;   // (thread 0) an MMA group committed and not yet waited for
+    bool mma_out = false;   // (control thread) an MMA group committed and not yet waited for
     auto wait_load = [&](uint64_t* bar, LoadTrack& t) {
-        if (ok) {
-            if (mbar_wait_ns(bar, t.ph, kWaitNs)) t.pend = false;
-            else ok = false;
-        }
+        if (ok && !mbar_wait_ns(bar, t.ph, kWaitNs)) ok = false;
         t.ph ^= 1u;
     };
-    auto issued = [&](LoadTrack& t) {
-        t.pend = true;
-        t.pend_ph = t.ph;
-    };
-    auto commit_mma = [&]() {   // thread 0, after issuing an MMA group
+    auto issued = [&](LoadTrack& t) { ++t.issued; };
+    auto commit_mma = [&]() {   // control thread, after issuing an MMA group
         mma_commit(barM);
         mma_out = true;
         mma_out_ph = phM;
@@ -351,20 +351,20 @@ kda_chunk_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_consta
             }
         }
     };
-    auto store_o = [&](uint8_t* stage, int64_t prow0) {   // thread 0, after a barrier
+    auto store_o = [&](uint8_t* stage, int64_t prow0) {   // control thread, after a barrier
 #pragma unroll
         for (int a = 0; a < 2; ++a) tma_store_2d(&tmO, stage + a * 8192, h * DV + 64 * a, (int)prow0);
         bulk_commit_group();
     };
 
-    if (nchunks > 0) {
-        if (tid == 0) {
-            if (!kSummary) issue_q(bos, 0);
-            issue_ka(bos);
-            issue_v(bos);
+    if (nchunks > 0 && ctl) {
+        if (!kSummary) {
+            issue_q(bos, 0);
+            issued(tq);
         }
-        if (!kSummary) issued(tq);
+        issue_ka(bos);
         issued(tka);
+        issue_v(bos);
         issued(tv);
     }
     fence_async_smem();
@@ -377,6 +377,7 @@ kda_chunk_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_consta
     if (tid < C && tid < len) beta_next = __bfloat162float(beta[(size_t)(bos + tid) * H + h]);
 
     bool broke = false;
+    if (compute)
     for (int chunk = 0; chunk < nchunks; ++chunk) {
         const int64_t row0 = bos + (int64_t)chunk * C;
         const int Lc = (int)((len - (int64_t)chunk * C) < C ? (len - (int64_t)chunk * C) : C);
@@ -428,7 +429,7 @@ kda_chunk_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_consta
                 *reinterpret_cast<float4*>(&sPi[O * DK + c0]) = make_float4(p[0], p[1], p[2], p[3]);
             }
             KDA_TC_PHASE(13);
-            __syncthreads();
+            sync_compute();
             KDA_TC_PHASE(14);
             // the previous chunk's state update and O (their operands KH, U, P and the
             // q buffer are overwritten from here on)
@@ -523,35 +524,12 @@ kda_chunk_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_consta
         tc_fence_before();
         __syncthreads();
         tc_fence_after();
-        // the previous chunk's O tile is staged: store it
-        if (!kSummary && chunk > 0 && tid == 0) store_o(sQ + ((chunk + 1) & 1) * 16384, row0 - C);
-        // k and alpha are consumed: load the next chunk's
-        if (chunk + 1 < nchunks && ok) {
-            if (tid == 0) issue_ka(row0 + C);
-            issued(tka);
-        }
 
         KDA_TC_PHASE(1);
         // ================= [A/beta ; P] = [k*lam ; q*lam] [k*rho^0 ; k*rho^1]^T   (M=128, N=96, K=128)
         //   rows 0..63 are A/beta rows r, rows 64..127 are P rows r.  Columns [0, 32) hold
         //   rho^0 (j < 32, valid for r < 32), columns [32, 96) hold rho^1 (j < 64, valid for r >= 32).
-        if (tid == 0 && ok) {   // nothing new is issued after a wait gave up
-            const uint32_t l0 = smem_u32(sX + X_L), r0 = smem_u32(sX + X_R);
-            constexpr uint32_t idesc = idesc_bf16(128, 96);
-#pragma unroll
-            for (int ks = 0; ks < 8; ++ks)
-                mma_bf16(tmem + TM_WK, sdesc_sw128(l0 + (ks >> 2) * 16384u + (ks & 3) * 32u),
-                         sdesc_sw128(r0 + (ks >> 2) * 12288u + (ks & 3) * 32u), idesc, ks > 0);
-            commit_mma();
-        }
         wait_mma();
-        // the O store has read its staging buffer by now (checked, so that the buffer
-        // may be reused): load the next q there
-        if (!kSummary && tid == 0) bulk_wait_read_all();
-        if (!kSummary && chunk + 1 < nchunks && ok) {
-            if (tid == 0) issue_q(row0 + C, (chunk + 1) & 1);
-            issued(tq);
-        }
 
         KDA_TC_PHASE(2);
         // ================= A (fp32, times beta_r, j < r) and P (bf16 K-major A operand, j <= r)
@@ -596,7 +574,7 @@ kda_chunk_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_consta
         }
         fence_async_smem();
         tc_fence_before();
-        __syncthreads();
+        sync_compute();
         KDA_TC_PHASE(3);
         // ================= Tinv = (I + A)^-1 by doubling: 16x16 blocks, then 32, then 64
         //   inv([[X, 0], [Y, Z]]) = [[X^-1, 0], [-Z^-1 Y X^-1, Z^-1]]
@@ -642,7 +620,7 @@ kda_chunk_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_consta
                     *reinterpret_cast<float4*>(&Tm[r2 * AS + 32 + 16 * c4 + cq]) =
                         make_float4(0.f, 0.f, 0.f, 0.f);
             }
-            __syncthreads();
+            sync_compute();
             KDA_TC_PHASE(9);
             // 16 -> 32: blocks (1,0) and (3,2).  thread: block b, row r, columns m2, m2+1
             {
@@ -662,7 +640,7 @@ kda_chunk_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_consta
                 }
                 x0 += x2; x1 += x3;
                 *reinterpret_cast<float2*>(&Xs[(16 * b + r) * 36 + m2]) = make_float2(x0, x1);
-                __syncthreads();
+                sync_compute();
                 float y0 = 0.f, y1 = 0.f;
 #pragma unroll
                 for (int jj = 0; jj < 16; ++jj) {
@@ -672,7 +650,7 @@ kda_chunk_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_consta
                 }
                 *reinterpret_cast<float2*>(&Tm[(o1 + r) * AS + o0 + m2]) = make_float2(-y0, -y1);
             }
-            __syncthreads();
+            sync_compute();
             KDA_TC_PHASE(10);
             // 32 -> 64 on the tensor cores (tf32):  X^T = T0^T A10^T,  Y = T1 X,
             // Tinv[32:64, 0:32] = -Y.  Operands: fp32 K-major tiles written here.
@@ -693,14 +671,6 @@ kda_chunk_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_consta
             tc_fence_before();
             __syncthreads();
             tc_fence_after();
-            if (tid == 0 && ok) {
-                constexpr uint32_t idesc = idesc_tf32(64, 32);
-                const uint32_t a0 = smem_u32(sX + X_T0T), b0 = smem_u32(sX + X_A10);
-#pragma unroll
-                for (int ks = 0; ks < 4; ++ks)
-                    mma_tf32(tmem + TM_WK, sdesc_sw128(a0 + ks * 32), sdesc_sw128(b0 + ks * 32), idesc, ks > 0);
-                commit_mma();
-            }
             wait_mma();
             if (q4 < 2) {   // M=64 accumulator: rows m = 16*q4 + lane live in lanes 32*q4 + lane
                 float v[32];
@@ -719,14 +689,6 @@ kda_chunk_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_consta
             tc_fence_before();
             __syncthreads();
             tc_fence_after();
-            if (tid == 0 && ok) {
-                constexpr uint32_t idesc = idesc_tf32(64, 32);
-                const uint32_t a0 = smem_u32(sX + X_T1), b0 = smem_u32(sX + X_XT);
-#pragma unroll
-                for (int ks = 0; ks < 4; ++ks)
-                    mma_tf32(tmem + TM_WK + 32, sdesc_sw128(a0 + ks * 32), sdesc_sw128(b0 + ks * 32), idesc, ks > 0);
-                commit_mma();
-            }
             wait_mma();
             if (q4 < 2) {
                 float v[32];
@@ -742,7 +704,7 @@ kda_chunk_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_consta
                 }
             }
             tc_fence_before();
-            __syncthreads();
+            sync_compute();
             KDA_TC_PHASE(11);
             // Tb = Tinv diag(beta) as the K-major A operand [64 r][64 m]; zero above the diagonal
             uint8_t* sTB = sX + X_TB;
@@ -767,15 +729,6 @@ kda_chunk_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_consta
 
         KDA_TC_PHASE(4);
         // ================= W = Tb (k*gamma)   (M=64, N=128, K=64)
-        if (tid == 0 && ok) {
-            const uint32_t a0 = smem_u32(sX + X_TB), b0 = smem_u32(sKT);
-            constexpr uint32_t idesc = idesc_bf16(64, 128, false, true);
-#pragma unroll
-            for (int ks = 0; ks < 4; ++ks)
-                mma_bf16(tmem + TM_WK, sdesc_sw128(a0 + ks * 32), sdesc_sw128(b0 + ks * 2048, 1024, 8192),
-                         idesc, ks > 0);
-            commit_mma();
-        }
         wait_mma();
         {
             // -W as the K-major A operand of the U MMA; M=64 rows m = 16 q4 + lane (lane < 16)
@@ -796,27 +749,10 @@ kda_chunk_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_consta
         tc_fence_before();
         __syncthreads();
         tc_fence_after();
-        wait_load(barV, tv);
 
         KDA_TC_PHASE(5);
         if constexpr (kSummary) {
         // ================= [U_M | U_N] = -W [M | N] + [0 | Tb V]   (M=64, N=256, K=128 (+64))
-        if (tid == 0 && ok) {
-            const uint32_t wq = smem_u32(sX + X_WQ), s0 = smem_u32(sS), tb = smem_u32(sX + X_TB),
-                           v0 = smem_u32(sV);
-            const uint32_t d = tmem + TM_WK;
-            constexpr uint32_t id256 = idesc_bf16(64, 256, false, true);
-            constexpr uint32_t id128 = idesc_bf16(64, 128, false, true);
-#pragma unroll
-            for (int ks = 0; ks < 8; ++ks)
-                mma_bf16(d, sdesc_sw128(wq + (ks >> 2) * 8192 + (ks & 3) * 32),
-                         sdesc_sw128(s0 + ks * 2048, 1024, 16384), id256, ks > 0);
-#pragma unroll
-            for (int ks = 0; ks < 4; ++ks)
-                mma_bf16(d + 128, sdesc_sw128(tb + ks * 32), sdesc_sw128(v0 + ks * 2048, 1024, 8192),
-                         id128, 1);
-            commit_mma();
-        }
         // meanwhile: [M | N] <- Diag(gamma_C) [M | N] in TMEM
         {
             const int c = 32 * q4 + lane;
@@ -835,10 +771,6 @@ kda_chunk_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_consta
             tmem_wait_st();
         }
         wait_mma();
-        if (chunk + 1 < nchunks && ok) {   // v is consumed
-            if (tid == 0) issue_v(row0 + C);
-            issued(tv);
-        }
         if (tid < C) {
             const int64_t nxt = (int64_t)(chunk + 1) * C + tid;   // token index in the segment
             beta_next = nxt < len ? __bfloat162float(beta[(size_t)(bos + nxt) * H + h]) : 0.0f;
@@ -857,39 +789,10 @@ kda_chunk_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_consta
                 }
             }
         }
-        fence_async_smem();
-        tc_fence_before();
-        __syncthreads();
-        tc_fence_after();
         KDA_TC_PHASE(6);
-        // ================= [M | N] += (k*eta)^T [U_M | U_N]   (M=128, N=256, K=64)
-        if (tid == 0 && ok) {
-            const uint32_t a0 = smem_u32(sKH), u0 = smem_u32(sX + X_U);
-            constexpr uint32_t idesc = idesc_bf16(128, 256, true, true);
-#pragma unroll
-            for (int ks = 0; ks < 4; ++ks)
-                mma_bf16(tmem + TM_S, sdesc_sw128(a0 + ks * 2048, 1024, 8192),
-                         sdesc_sw128(u0 + ks * 2048, 1024, 8192), idesc, 1);
-            commit_mma();
-        }
-        KDA_TC_PHASE(7);
+        // (the control warp then issues [M | N] += (k*eta)^T [U_M | U_N])
         } else {
-        // ================= U = -W S + Tb V   (M=64, N=128, K=128+64)
-        if (tid == 0 && ok) {
-            const uint32_t wq = smem_u32(sX + X_WQ), s0 = smem_u32(sS), tb = smem_u32(sX + X_TB),
-                           v0 = smem_u32(sV);
-            // B operands are MN-major with two 64-column atoms: leading byte offset = atom stride
-            constexpr uint32_t idesc = idesc_bf16(64, 128, false, true);
-            const uint32_t d = tmem + TM_U;
-#pragma unroll
-            for (int ks = 0; ks < 8; ++ks)
-                mma_bf16(d, sdesc_sw128(wq + (ks >> 2) * 8192 + (ks & 3) * 32),
-                         sdesc_sw128(s0 + ks * 2048, 1024, 16384), idesc, ks > 0);
-#pragma unroll
-            for (int ks = 0; ks < 4; ++ks)
-                mma_bf16(d, sdesc_sw128(tb + ks * 32), sdesc_sw128(v0 + ks * 2048, 1024, 8192), idesc, 1);
-            commit_mma();
-        }
+        // ================= U = Tb V - W S   (issued by the control warp)
         // meanwhile: S <- Diag(gamma_C) S in TMEM (the MMAs read the bf16 copy)
         {
             const int c = 32 * q4 + lane;
@@ -905,10 +808,6 @@ kda_chunk_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_consta
             tmem_wait_st();
         }
         wait_mma();
-        if (chunk + 1 < nchunks && ok) {   // v is consumed
-            if (tid == 0) issue_v(row0 + C);
-            issued(tv);
-        }
         if (tid < C) {
             const int64_t nxt = (int64_t)(chunk + 1) * C + tid;   // token index in the segment
             beta_next = nxt < len ? __bfloat162float(beta[(size_t)(bos + nxt) * H + h]) : 0.0f;
@@ -923,38 +822,13 @@ kda_chunk_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_consta
                     *reinterpret_cast<uint4*>(sX + X_U + hf * 8192 + swz(j, ch)) = pack8(&v[8 * ch]);
             }
         }
-        fence_async_smem();
-        tc_fence_before();
-        __syncthreads();
-        tc_fence_after();
-
         KDA_TC_PHASE(6);
-        // ================= S += (k*eta)^T U   (M=128, N=128, K=64)
-        //                   O  = (q*gamma) S_start + P U   (M=64, N=128, K=128+64)
-        if (tid == 0 && ok) {
-            const uint32_t kh = smem_u32(sKH), u0 = smem_u32(sX + X_U), s0 = smem_u32(sS),
-                           qg = smem_u32(sQc), p0 = smem_u32(sX + X_P);
-            constexpr uint32_t id_s = idesc_bf16(128, 128, true, true);
-            constexpr uint32_t id_o = idesc_bf16(64, 128, false, true);
-#pragma unroll
-            for (int ks = 0; ks < 4; ++ks)
-                mma_bf16(tmem + TM_S, sdesc_sw128(kh + ks * 2048, 1024, 8192),
-                         sdesc_sw128(u0 + ks * 2048, 1024, 8192), id_s, 1);
-#pragma unroll
-            for (int ks = 0; ks < 8; ++ks)
-                mma_bf16(tmem + TM_O, sdesc_sw128(qg + (ks >> 2) * 8192 + (ks & 3) * 32),
-                         sdesc_sw128(s0 + ks * 2048, 1024, 16384), id_o, ks > 0);
-#pragma unroll
-            for (int ks = 0; ks < 4; ++ks)
-                mma_bf16(tmem + TM_O, sdesc_sw128(p0 + ks * 32), sdesc_sw128(u0 + ks * 2048, 1024, 8192),
-                         id_o, 1);
-            commit_mma();
+        // (the control warp then issues S += (k*eta)^T U and O += P U)
         }
-        KDA_TC_PHASE(7);
-        }
+        // U is handed over; every thread leaves together on a timeout
         fence_async_smem();
         tc_fence_before();
-        const int any_timeout = __syncthreads_or(!ok);   // uniform: every thread leaves together
+        const int any_timeout = __syncthreads_or(!ok);
         tc_fence_after();
         KDA_TC_PHASE(8);
         if (any_timeout) {
@@ -962,33 +836,203 @@ kda_chunk_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_consta
             break;
         }
     }
+
+    // ---- the control warp: one thread issues every copy and MMA group at the barriers
+    // where the compute warps hand over their operands, and waits for each committed
+    // group in order.  Groups without a commit ride on the next group's commit (the
+    // tensor pipe runs one thread's MMAs in issue order).
+    //   barrier A (operands of [A/beta ; P]):  [A/beta ; P] (commit), then (q*gamma) S_start
+    //   barriers B, C (tf32 solve operands):     the two 32 -> 64 solve products (commit)
+    //   barrier D (Tb):                          W = Tb (k*gamma) (commit), then Tb V
+    //   barrier E (-W):                          U (or [U_M | U_N]) += -W S (commit)
+    //   barrier F (U):                           S += (k*eta)^T U and O += P U (commit)
+    const uint32_t idM64 = idesc_bf16(64, 128, false, true);   // M=64, N=128, B MN-major
+    auto mma_ap = [&]() {
+        const uint32_t l0 = smem_u32(sX + X_L), r0 = smem_u32(sX + X_R);
+        constexpr uint32_t idesc = idesc_bf16(128, 96);
+#pragma unroll
+        for (int ks = 0; ks < 8; ++ks)
+            mma_bf16(tmem + TM_WK, sdesc_sw128(l0 + (ks >> 2) * 16384u + (ks & 3) * 32u),
+                     sdesc_sw128(r0 + (ks >> 2) * 12288u + (ks & 3) * 32u), idesc, ks > 0);
+        commit_mma();
+    };
+    auto mma_qs = [&](uint8_t* sQc) {   // O = (q*gamma) S_start (no commit)
+        const uint32_t qg = smem_u32(sQc), s0 = smem_u32(sS);
+#pragma unroll
+        for (int ks = 0; ks < 8; ++ks)
+            mma_bf16(tmem + TM_O, sdesc_sw128(qg + (ks >> 2) * 8192 + (ks & 3) * 32),
+                     sdesc_sw128(s0 + ks * 2048, 1024, 16384), idM64, ks > 0);
+    };
+    auto mma_tf1 = [&]() {
+        constexpr uint32_t idesc = idesc_tf32(64, 32);
+        const uint32_t a0 = smem_u32(sX + X_T0T), b0 = smem_u32(sX + X_A10);
+#pragma unroll
+        for (int ks = 0; ks < 4; ++ks)
+            mma_tf32(tmem + TM_WK, sdesc_sw128(a0 + ks * 32), sdesc_sw128(b0 + ks * 32), idesc, ks > 0);
+        commit_mma();
+    };
+    auto mma_tf2 = [&]() {
+        constexpr uint32_t idesc = idesc_tf32(64, 32);
+        const uint32_t a0 = smem_u32(sX + X_T1), b0 = smem_u32(sX + X_XT);
+#pragma unroll
+        for (int ks = 0; ks < 4; ++ks)
+            mma_tf32(tmem + TM_WK + 32, sdesc_sw128(a0 + ks * 32), sdesc_sw128(b0 + ks * 32), idesc, ks > 0);
+        commit_mma();
+    };
+    auto mma_w = [&]() {
+        const uint32_t a0 = smem_u32(sX + X_TB), b0 = smem_u32(sKT);
+#pragma unroll
+        for (int ks = 0; ks < 4; ++ks)
+            mma_bf16(tmem + TM_WK, sdesc_sw128(a0 + ks * 32), sdesc_sw128(b0 + ks * 2048, 1024, 8192),
+                     idM64, ks > 0);
+        commit_mma();
+    };
+    auto mma_tbv = [&]() {   // Tb V into U (or U_N) (no commit)
+        const uint32_t tb = smem_u32(sX + X_TB), v0 = smem_u32(sV);
+        const uint32_t d = tmem + (kSummary ? TM_WK + 128 : TM_U);
+#pragma unroll
+        for (int ks = 0; ks < 4; ++ks)
+            mma_bf16(d, sdesc_sw128(tb + ks * 32), sdesc_sw128(v0 + ks * 2048, 1024, 8192), idM64, ks > 0);
+    };
+    auto mma_u = [&]() {
+        const uint32_t wq = smem_u32(sX + X_WQ), s0 = smem_u32(sS);
+        if constexpr (kSummary) {
+            // U_M = -W M (fresh, over W's accumulator) and U_N += -W N
+#pragma unroll
+            for (int ks = 0; ks < 8; ++ks)
+                mma_bf16(tmem + TM_WK, sdesc_sw128(wq + (ks >> 2) * 8192 + (ks & 3) * 32),
+                         sdesc_sw128(s0 + ks * 2048, 1024, 16384), idM64, ks > 0);
+#pragma unroll
+            for (int ks = 0; ks < 8; ++ks)
+                mma_bf16(tmem + TM_WK + 128, sdesc_sw128(wq + (ks >> 2) * 8192 + (ks & 3) * 32),
+                         sdesc_sw128(s0 + 32768 + ks * 2048, 1024, 16384), idM64, 1);
+        } else {
+#pragma unroll
+            for (int ks = 0; ks < 8; ++ks)
+                mma_bf16(tmem + TM_U, sdesc_sw128(wq + (ks >> 2) * 8192 + (ks & 3) * 32),
+                         sdesc_sw128(s0 + ks * 2048, 1024, 16384), idM64, 1);
+        }
+        commit_mma();
+    };
+    auto mma_s = [&]() {
+        const uint32_t kh = smem_u32(sKH), u0 = smem_u32(sX + X_U);
+        if constexpr (kSummary) {
+            constexpr uint32_t idesc = idesc_bf16(128, 256, true, true);
+#pragma unroll
+            for (int ks = 0; ks < 4; ++ks)
+                mma_bf16(tmem + TM_S, sdesc_sw128(kh + ks * 2048, 1024, 8192),
+                         sdesc_sw128(u0 + ks * 2048, 1024, 8192), idesc, 1);
+        } else {
+            constexpr uint32_t id_s = idesc_bf16(128, 128, true, true);
+            const uint32_t p0 = smem_u32(sX + X_P);
+#pragma unroll
+            for (int ks = 0; ks < 4; ++ks)
+                mma_bf16(tmem + TM_S, sdesc_sw128(kh + ks * 2048, 1024, 8192),
+                         sdesc_sw128(u0 + ks * 2048, 1024, 8192), id_s, 1);
+#pragma unroll
+            for (int ks = 0; ks < 4; ++ks)
+                mma_bf16(tmem + TM_O, sdesc_sw128(p0 + ks * 32), sdesc_sw128(u0 + ks * 2048, 1024, 8192),
+                         idM64, 1);
+        }
+        commit_mma();
+    };
+    auto handoff = [&]() {
+        tc_fence_before();
+        __syncthreads();
+        tc_fence_after();
+    };
+    if (!compute)
+    for (int chunk = 0; chunk < nchunks; ++chunk) {
+        const int64_t row0 = bos + (int64_t)chunk * C;
+        uint8_t* sQc = sQ + (chunk & 1) * 16384;
+        if (ctl && chunk > 0) wait_mma();   // the previous chunk's state update (and O)
+        handoff();   // A
+        if (ctl) {
+            if (ok) {
+                mma_ap();
+                if (!kSummary) mma_qs(sQc);
+            }
+            if (!kSummary && chunk > 0) store_o(sQ + ((chunk + 1) & 1) * 16384, row0 - C);
+            if (chunk + 1 < nchunks && ok) {   // k and alpha are consumed
+                issue_ka(row0 + C);
+                issued(tka);
+            }
+            wait_mma();
+            if (!kSummary) {
+                // the O store has read its staging buffer: load the next q there
+                bulk_wait_read_all();
+                if (chunk + 1 < nchunks && ok) {
+                    issue_q(row0 + C, (chunk + 1) & 1);
+                    issued(tq);
+                }
+            }
+        }
+        handoff();   // B
+        if (ctl) {
+            if (ok) mma_tf1();
+            wait_mma();
+        }
+        handoff();   // C
+        if (ctl) {
+            if (ok) mma_tf2();
+            wait_mma();
+        }
+        handoff();   // D
+        if (ctl) {
+            if (ok) mma_w();
+            wait_load(barV, tv);
+            if (ok) mma_tbv();
+            wait_mma();
+        }
+        handoff();   // E
+        if (ctl) {
+            if (ok) mma_u();
+            wait_mma();
+            if (chunk + 1 < nchunks && ok) {   // v is consumed
+                issue_v(row0 + C);
+                issued(tv);
+            }
+        }
+        tc_fence_before();
+        const int any_timeout = __syncthreads_or(!ok);   // F, uniform: every thread leaves together
+        tc_fence_after();
+        if (any_timeout) {
+            broke = true;
+            break;
+        }
+        if (ctl && ok) mma_s();
+    }
+    if (ctl && nchunks > 0 && !broke) wait_mma();
+
     // the last chunk's state update and outputs (staged in the q buffer it did not use)
     const int last_Lc = nchunks > 0 ? (int)(len - (int64_t)(nchunks - 1) * C) : 0;
     uint8_t* last_stage = sQ + (nchunks & 1) * 16384;
-    if (nchunks > 0 && !broke) finish_prev(bos + (int64_t)(nchunks - 1) * C, last_Lc, last_stage);
+    if (compute && nchunks > 0 && !broke)
+        finish_prev(bos + (int64_t)(nchunks - 1) * C, last_Lc, last_stage);
     fence_async_smem();
 
     if (!ok) atomicExch(sFlag, 1);
     __syncthreads();
-    if (!kSummary && tid == 0) {
+    if (!kSummary && ctl) {
         if (nchunks > 0 && !broke && !*sFlag && last_Lc == C)
             store_o(last_stage, bos + (int64_t)(nchunks - 1) * C);
         bulk_wait_all();   // every O store has completed before shared memory is released
     }
-    if (*sFlag && tid == 0) {
+    if (*sFlag && ctl) {
         // a wait gave up: let this CTA's own copies and MMAs in flight finish (bounded)
-        // before its shared and tensor memory are released.  Thread 0 issues every
-        // copy and MMA and stops issuing once one of its own waits gives up, so at
-        // most one of each stream is outstanding here.
-        if (tq.pend) mbar_wait_ns(barQ, tq.pend_ph, kWaitNs);
-        if (tka.pend) mbar_wait_ns(barKA, tka.pend_ph, kWaitNs);
-        if (tv.pend) mbar_wait_ns(barV, tv.pend_ph, kWaitNs);
+        // before its shared and tensor memory are released.  The control thread issues
+        // every copy and MMA group and waits for each group in order; a load stream's
+        // last copy completes the phase of parity (issued - 1) & 1.
+        if (tq.issued) mbar_wait_ns(barQ, (tq.issued - 1) & 1u, kWaitNs);
+        if (tka.issued) mbar_wait_ns(barKA, (tka.issued - 1) & 1u, kWaitNs);
+        if (tv.issued) mbar_wait_ns(barV, (tv.issued - 1) & 1u, kWaitNs);
         if (mma_out) mbar_wait_ns(barM, mma_out_ph, kWaitNs);
     }
     __syncthreads();
     if (kCtaStatus && tid == 0) status[(size_t)n * H + h] = *sFlag;
     if (*sFlag) {
         if (!kCtaStatus && tid == 0) atomicExch(status, 1);
+    } else if (!compute) {
     } else if (kSummary) {
         const int c = 32 * q4 + lane;
         float* dst = seg.maps + ((((size_t)n * (seg.nseg - 1) + gseg) * H + h) * DK + c) * (DK + DV) +
@@ -1125,7 +1169,7 @@ static cudaError_t launch_tc_t(const TcMaps& m, const void* beta, const float* S
                                          (int)tc::SMEM_BYTES);
     if (e != cudaSuccess) return e;
     dim3 grid(1, H, nseq * seg.per_seq);
-    tc::kda_chunk_tc_kernel<kCtaStatus, kSummary><<<grid, tc::NT, tc::SMEM_BYTES, stream>>>(
+    tc::kda_chunk_tc_kernel<kCtaStatus, kSummary><<<grid, tc::NTHREADS, tc::SMEM_BYTES, stream>>>(
         m.q, m.k, m.a, m.v, m.o, (const __nv_bfloat16*)beta, S0, cu, (__nv_bfloat16*)out, S_final, T, H,
         status, seg);
     return cudaGetLastError();
