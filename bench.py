@@ -10,6 +10,11 @@ rank runs its own batch (independent sequences, no data-path collective:
 weak scaling); the time is the max over ranks and `value` counts all ranks'
 tokens.  Rank 0 prints ONE JSON line.
 
+--seqpar (forward workloads with one sequence per batch row) instead splits
+time across the ranks: rank r runs the r-th contiguous segment of every
+sequence; segment state maps are all-gathered (NCCL) and scanned to each rank's
+start state (strong scaling, the same total tokens at every N).
+
 --impl reference times the CPU oracle (fp64, token by token) as it stands on
 the host cores, on a bounded sample of the same workload.
 """
@@ -390,6 +395,17 @@ def run_ours(args, w):
         def step():
             kda.kda_forward(inp["q"], inp["k"], inp["v"], inp["alpha"], inp["beta"], inp["S0"],
                             cu_seqlens=cu, out=out, S_final=Sf, chunk=w.chunk)
+        if args.seqpar and w.kind == "forward":
+            # this rank's time segment; maps exchanged through the process group
+            from gated_delta_rule_138_b200.seqpar import kda_forward_sequence_parallel, split_time
+            part = {n: split_time(inp[n], world, rank) for n in ("q", "k", "v", "alpha", "beta")}
+            S0 = inp["S0"]
+            del inp
+            inp = dict(part, S0=S0)
+
+            def step():
+                kda_forward_sequence_parallel(part["q"], part["k"], part["v"], part["alpha"],
+                                              part["beta"], S0)
         kname = kda.kda_forward_kernel_name(w.dk, w.dv, w.chunk, inp["q"].dtype, out.dtype)
         # time segments per sequence of the tensor-core path (1: unsplit); with g > 1 a
         # step is three launches (segment maps, scan, forward) timed together
@@ -428,24 +444,33 @@ def run_ours(args, w):
     elapsed_ms = max_over_ranks(e0.elapsed_time(e1), world)
     kern_ms = statistics.mean(a.elapsed_time(b) for a, b in ev)
     kern_ms = max_over_ranks(kern_ms, world)
-    total_tokens = sum_over_ranks(tokens * args.steps, world)
+    seqpar = bool(args.seqpar and w.kind == "forward")
+    # replicas: every rank's own tokens; sequence-parallel: one job split over the ranks
+    total_tokens = tokens * args.steps if seqpar else sum_over_ranks(tokens * args.steps, world)
     value = ranks.weak_scaling_throughput(total_tokens, elapsed_ms)
     ms_per_step = elapsed_ms / args.steps
 
     # end to end: pinned host inputs -> device -> kda_forward -> host results
-    e2e = run_e2e(args, w, inp, dev, stream, world) if w.kind != "decode" and args.e2e_steps > 0 \
+    e2e = run_e2e(args, w, inp, dev, stream, world) \
+        if w.kind != "decode" and args.e2e_steps > 0 and not seqpar \
         else None
 
     if rank == 0:
-        achieved = algo_bytes / (kern_ms * 1e-3) / 1e9
-        tflops = algo_flops / (kern_ms * 1e-3) / 1e12
+        # per GPU: a sequence-parallel step moves 1/world of the job's bytes on each GPU
+        share = world if seqpar else 1
+        achieved = algo_bytes / share / (kern_ms * 1e-3) / 1e9
+        tflops = algo_flops / share / (kern_ms * 1e-3) / 1e12
+        cfg = config_of(w, world)
+        if seqpar:
+            cfg["parallelism"] = "sequence x%d (time segments per rank, maps all-gathered)" % world
         line = {
             "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world,
             "steps": args.steps, "warmup": warm, "ms_per_step": ms_per_step,
-            "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+            "higher_is_better": True, "scaling": "strong" if seqpar else "weak",
+            "vs_baseline": None,
             "dtype": "bf16" if kname == "chunk_tc_bf16" else "f32",
             "data": "synthetic (seeded generators, the workload's shapes and distributions)",
-            "config": dict(config_of(w, world),
+            "config": dict(cfg,
                            l2="no flush: inputs %.2f GB per step > 126 MB L2"
                               % (algo_bytes / 1e9)),
             "tflops": tflops,
@@ -533,6 +558,8 @@ def main():
     ap.add_argument("--cpu-budget", type=float, default=15.0,
                     help="seconds of oracle time for the cpu_baseline sample")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--seqpar", action="store_true",
+                    help="split every sequence's time axis across the ranks (strong scaling)")
     ap.add_argument("--e2e-steps", type=int, default=10,
                     help="steps of the end-to-end (host buffers) measurement; 0 skips it")
     args = ap.parse_args()

@@ -9,11 +9,11 @@ call does, and it raises if the library is missing.
 from .kda import (KdaError, kda_forward, kda_decode_step, kda_status_string,  # noqa: F401
                   kda_forward_workspace_bytes, kda_forward_kernel_name, kda_launch_count,
                   kda_device_status, kda_forward_noalloc, kda_selftest_timeout,
-                  kda_forward_segments,
+                  kda_forward_segments, kda_segment_maps, kda_segment_scan,
                   library_path, load_library)
 
 __all__ = ["KdaError", "kda_forward", "kda_decode_step", "kda_status_string",
            "kda_forward_workspace_bytes", "kda_forward_kernel_name", "kda_launch_count",
            "kda_device_status", "kda_forward_noalloc", "kda_selftest_timeout",
-           "kda_forward_segments",
+           "kda_forward_segments", "kda_segment_maps", "kda_segment_scan",
            "library_path", "load_library"]

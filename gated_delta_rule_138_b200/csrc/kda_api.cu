@@ -25,6 +25,11 @@ cudaError_t launch_chunk_tc(const void* q, const void* k, const void* v, const v
                             void* out, float* S_final, int64_t rows, int64_t T, int H, int* status,
                             cudaStream_t stream);
 size_t chunk_tc_segmented_workspace_floats(int64_t nseq, int H, int nseg);
+cudaError_t launch_segment_maps(const void* k, const void* v, const void* alpha, const void* beta,
+                                const int32_t* cu, int nseq, float* maps, int64_t rows, int64_t T,
+                                int H, int* status, cudaStream_t stream);
+cudaError_t launch_apply_maps(const float* S0, const float* maps, int G, int nseq, int H, float* out,
+                              cudaStream_t stream);
 cudaError_t launch_chunk_tc_segmented(const void* q, const void* k, const void* v,
                                       const void* alpha, const void* beta, const float* S0,
                                       const int32_t* cu, int nseq, void* out, float* S_final,
@@ -264,6 +269,54 @@ kda_status_t kda_forward(const void* q, const void* k, const void* v, const void
     return cuda_status(kda::launch_chunk_simt(in_bf16, out_bf16, chunk, q, k, v, alpha, beta, S0,
                                               cu_seqlens, (int)nseq, out, S_final, T, H, d_k, d_v,
                                               s));
+}
+
+kda_status_t kda_segment_maps(const void* k, const void* v, const void* alpha, const void* beta,
+                              const int32_t* cu_seqlens, int32_t num_seqs, float* maps, int32_t B,
+                              int64_t T, int32_t H, int32_t d_k, int32_t d_v, int32_t chunk,
+                              kda_dtype_t in_dtype, kda_stream_t stream) {
+    if (B < 0 || T < 0 || H <= 0 || !is_dtype(in_dtype)) return KDA_ERR_INVALID_ARG;
+    if (cu_seqlens != nullptr && (B != 1 || num_seqs < 0)) return KDA_ERR_INVALID_ARG;
+    const int64_t nseq = cu_seqlens ? (int64_t)num_seqs : (int64_t)B;
+    if (nseq > 0 && !maps) return KDA_ERR_INVALID_ARG;
+    if ((int64_t)B * T > 0 && (!k || !v || !alpha || !beta)) return KDA_ERR_INVALID_ARG;
+    const void* p16[] = {k, v, alpha, maps};
+    for (const void* p : p16)
+        if (p && !aligned16(p)) return KDA_ERR_INVALID_ARG;
+    if (!aligned_to(beta, 2) || !aligned_to(cu_seqlens, 4)) return KDA_ERR_INVALID_ARG;
+    if (!use_tc(d_k, d_v, chunk, in_dtype, KDA_BF16)) {
+        std::snprintf(g_last_error, sizeof(g_last_error),
+                      "kda_segment_maps: only bf16 inputs, d_k = d_v = 128, chunk 64");
+        return KDA_ERR_UNSUPPORTED;
+    }
+    if (nseq > 65535 || H > 65535) return KDA_ERR_UNSUPPORTED;
+    const int64_t rows = cu_seqlens ? T : (int64_t)B * T;
+    if (rows > 0x7fffffffLL) return KDA_ERR_UNSUPPORTED;
+    if (nseq == 0) return KDA_OK;
+    g_last_error[0] = '\0';
+    int* status = nullptr;
+    cudaError_t e = device_status_word(&status);
+    if (e != cudaSuccess) return cuda_status(e);
+    g_launches.fetch_add(1, std::memory_order_relaxed);
+    e = kda::launch_segment_maps(k, v, alpha, beta, cu_seqlens, (int)nseq, maps, rows, T, H, status,
+                                 reinterpret_cast<cudaStream_t>(stream));
+    if (e != cudaSuccess) return cuda_status(e);
+    return debug_sync() ? kda_device_status(stream) : KDA_OK;
+}
+
+kda_status_t kda_segment_scan(const float* S0, const float* maps, int32_t num_maps, float* out,
+                              int32_t num_seqs, int32_t H, int32_t d_k, int32_t d_v,
+                              kda_stream_t stream) {
+    if (num_maps < 0 || num_seqs < 0 || H <= 0) return KDA_ERR_INVALID_ARG;
+    if (d_k != 128 || d_v != 128) return KDA_ERR_UNSUPPORTED;
+    if (num_seqs == 0) return KDA_OK;
+    if (!out || (num_maps > 0 && !maps)) return KDA_ERR_INVALID_ARG;
+    if (!aligned16(out) || (S0 && !aligned16(S0)) || (maps && !aligned16(maps))) return KDA_ERR_INVALID_ARG;
+    if (num_seqs > 65535 || H > 65535) return KDA_ERR_UNSUPPORTED;
+    g_last_error[0] = '\0';
+    g_launches.fetch_add(1, std::memory_order_relaxed);
+    return cuda_status(kda::launch_apply_maps(S0, maps, num_maps, num_seqs, H, out,
+                                              reinterpret_cast<cudaStream_t>(stream)));
 }
 
 kda_status_t kda_decode_step(const void* q, const void* k, const void* v, const void* alpha,

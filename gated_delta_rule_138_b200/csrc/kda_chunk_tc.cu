@@ -145,7 +145,7 @@ struct Segments {
     int nseg;             // segments per sequence (1: whole sequences)
     int per_seq;          // segment CTAs per sequence in this launch
     const float* start;   // forward with nseg > 1: start states [nseq * nseg, H, DK, DV]
-    float* maps;          // summary: [M | N] fp32 [nseq * (nseg - 1), H, DK, DK + DV]
+    float* maps;          // summary: [M | N] fp32 [nseq * per_seq, H, DK, DK + DV]
 };
 
 // One TMA stream's bookkeeping: the parity a thread's next wait on it expects,
@@ -1035,7 +1035,7 @@ kda_chunk_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_consta
     } else if (!compute) {
     } else if (kSummary) {
         const int c = 32 * q4 + lane;
-        float* dst = seg.maps + ((((size_t)n * (seg.nseg - 1) + gseg) * H + h) * DK + c) * (DK + DV) +
+        float* dst = seg.maps + ((((size_t)n * seg.per_seq + gseg) * H + h) * DK + c) * (DK + DV) +
                      128 * hf;
 #pragma unroll
         for (int blk = 0; blk < 8; ++blk) {
@@ -1112,6 +1112,53 @@ kda_segment_scan_kernel(const float* S0, const float* __restrict__ maps, float* 
             }
         }
     }
+}
+
+// out = the state after maps 0..G-1 applied in order to S0 (S <- M_g S + N_g), fp32.
+// maps: [G][nseq][H][DK][DK + DV] (one map per segment, e.g. one per rank); S0 and out:
+// [nseq][H][DK][DV] (S0 may be null = 0, out may alias S0: each CTA reads its own
+// 16 columns before it writes them).
+__global__ void __launch_bounds__(DK)
+kda_apply_maps_kernel(const float* S0, const float* __restrict__ maps, int G, int nseq, int H,
+                      float* out) {
+    __shared__ __align__(16) float sS[DK][SCAN_COLS];
+    const int cb = blockIdx.x, h = blockIdx.y, n = blockIdx.z, i = threadIdx.x;
+    const size_t col = (size_t)SCAN_COLS * cb;
+    float cur[SCAN_COLS];
+    const float* src = S0 ? S0 + (((size_t)n * H + h) * DK + i) * DV + col : nullptr;
+#pragma unroll
+    for (int c = 0; c < SCAN_COLS; c += 4) {
+        const float4 f = src ? *reinterpret_cast<const float4*>(src + c) : make_float4(0.f, 0.f, 0.f, 0.f);
+        cur[c] = f.x; cur[c + 1] = f.y; cur[c + 2] = f.z; cur[c + 3] = f.w;
+    }
+    for (int g = 0; g < G; ++g) {
+        __syncthreads();   // the previous step's reads of sS are done
+#pragma unroll
+        for (int c = 0; c < SCAN_COLS; ++c) sS[i][c] = cur[c];
+        __syncthreads();
+        const float* Mrow = maps + ((((size_t)g * nseq + n) * H + h) * DK + i) * (DK + DV);
+#pragma unroll
+        for (int c = 0; c < SCAN_COLS; ++c) cur[c] = Mrow[DK + col + c];   // N_g
+        for (int j = 0; j < DK; j += 4) {
+            const float4 m = *reinterpret_cast<const float4*>(Mrow + j);
+            const float mj[4] = {m.x, m.y, m.z, m.w};
+#pragma unroll
+            for (int jj = 0; jj < 4; ++jj) {
+#pragma unroll
+                for (int c = 0; c < SCAN_COLS; c += 4) {
+                    const float4 sv = *reinterpret_cast<const float4*>(&sS[j + jj][c]);
+                    cur[c] = fmaf(mj[jj], sv.x, cur[c]);
+                    cur[c + 1] = fmaf(mj[jj], sv.y, cur[c + 1]);
+                    cur[c + 2] = fmaf(mj[jj], sv.z, cur[c + 2]);
+                    cur[c + 3] = fmaf(mj[jj], sv.w, cur[c + 3]);
+                }
+            }
+        }
+    }
+    float* dst = out + (((size_t)n * H + h) * DK + i) * DV + col;
+#pragma unroll
+    for (int c = 0; c < SCAN_COLS; c += 4)
+        *reinterpret_cast<float4*>(dst + c) = make_float4(cur[c], cur[c + 1], cur[c + 2], cur[c + 3]);
 }
 
 // ---------------------------------------------------------------- host side
@@ -1217,6 +1264,25 @@ cudaError_t launch_chunk_tc_segmented(const void* q, const void* k, const void* 
     const tc::Segments fwd{nseg, nseg, start, nullptr};
     return launch_tc_t<false, false>(m, beta, nullptr, cu, nseq, out, S_final, T, H, status, fwd,
                                      stream);
+}
+
+// Segment maps of whole sequences: maps [nseq][H][DK][DK + DV] fp32 with
+// S_end = M S_start + N over each sequence's tokens (the summary mode, one segment).
+cudaError_t launch_segment_maps(const void* k, const void* v, const void* alpha, const void* beta,
+                                const int32_t* cu, int nseq, float* maps, int64_t rows, int64_t T,
+                                int H, int* status, cudaStream_t stream) {
+    TcMaps m;
+    if (!make_maps(&m, k, k, v, alpha, nullptr, rows, H)) return cudaErrorInvalidValue;
+    const tc::Segments one{1, 1, nullptr, maps};
+    return launch_tc_t<false, true>(m, beta, nullptr, cu, nseq, nullptr, nullptr, T, H, status, one,
+                                    stream);
+}
+
+cudaError_t launch_apply_maps(const float* S0, const float* maps, int G, int nseq, int H, float* out,
+                              cudaStream_t stream) {
+    tc::kda_apply_maps_kernel<<<dim3(tc::DV / tc::SCAN_COLS, H, nseq), tc::DK, 0, stream>>>(
+        S0, maps, G, nseq, H, out);
+    return cudaGetLastError();
 }
 
 // Same kernel, one status word per (sequence, head) CTA at status[n * H + h].

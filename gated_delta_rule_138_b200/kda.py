@@ -76,6 +76,11 @@ def load_library(build_if_missing: bool = True) -> ctypes.CDLL:
     lib.kda_launch_count.argtypes = []
     lib.kda_device_status.restype = ctypes.c_int
     lib.kda_device_status.argtypes = [vp]
+    lib.kda_segment_maps.restype = ctypes.c_int
+    lib.kda_segment_maps.argtypes = [vp, vp, vp, vp, vp, i32, vp, i32, i64, i32, i32, i32, i32,
+                                     ctypes.c_int, vp]
+    lib.kda_segment_scan.restype = ctypes.c_int
+    lib.kda_segment_scan.argtypes = [vp, vp, i32, vp, i32, i32, i32, i32, vp]
     lib.kda_forward_segments.restype = i32
     lib.kda_forward_segments.argtypes = [i32, i64, i32, i32]
     lib.kda_selftest_timeout.restype = ctypes.c_int
@@ -193,6 +198,43 @@ def kda_forward(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, alpha: torch.
                          _dt(q), _dt(out), _stream(stream))
     _check("kda_forward", st)
     return out, S_final
+
+
+def kda_segment_maps(k: torch.Tensor, v: torch.Tensor, alpha: torch.Tensor, beta: torch.Tensor,
+                     cu_seqlens: Optional[torch.Tensor] = None, maps: Optional[torch.Tensor] = None,
+                     chunk: int = 64, stream=None) -> torch.Tensor:
+    """Affine state map [M | N] (fp32 [N, H, d_k, d_k + d_v]) of every sequence's
+    tokens: S_end = M S_start + N."""
+    lib = load_library()
+    B, T, H, dk = k.shape
+    dv = v.shape[-1]
+    for name, t in (("k", k), ("v", v), ("alpha", alpha), ("beta", beta),
+                    ("cu_seqlens", cu_seqlens), ("maps", maps)):
+        _contig(name, t)
+    nseq = B if cu_seqlens is None else cu_seqlens.numel() - 1
+    if maps is None:
+        maps = torch.empty(nseq, H, dk, dk + dv, dtype=torch.float32, device=k.device)
+    st = lib.kda_segment_maps(_ptr(k), _ptr(v), _ptr(alpha), _ptr(beta), _ptr(cu_seqlens),
+                              int(nseq), _ptr(maps), int(B), int(T), int(H), int(dk), int(dv),
+                              int(chunk), _dt(k), _stream(stream))
+    _check("kda_segment_maps", st)
+    return maps
+
+
+def kda_segment_scan(maps: torch.Tensor, S0: Optional[torch.Tensor] = None,
+                     out: Optional[torch.Tensor] = None, stream=None) -> torch.Tensor:
+    """Apply stacked segment maps [G, N, H, d_k, d_k + d_v] in order to S0 (or 0)."""
+    lib = load_library()
+    G, N, H, dk, w = maps.shape
+    dv = w - dk
+    for name, t in (("maps", maps), ("S0", S0), ("out", out)):
+        _contig(name, t)
+    if out is None:
+        out = torch.empty(N, H, dk, dv, dtype=torch.float32, device=maps.device)
+    st = lib.kda_segment_scan(_ptr(S0), _ptr(maps), int(G), _ptr(out), int(N), int(H), int(dk),
+                              int(dv), _stream(stream))
+    _check("kda_segment_scan", st)
+    return out
 
 
 def kda_forward_noalloc(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, alpha: torch.Tensor,

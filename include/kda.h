@@ -112,6 +112,47 @@ kda_status_t kda_decode_step(const void* q, const void* k, const void* v,
                              kda_dtype_t in_dtype, kda_dtype_t out_dtype,
                              kda_stream_t stream);
 
+/*
+ * kda_segment_maps -- the affine state map of every sequence's token range:
+ * S_end = M S_start + N, with M (d_k x d_k) and N (d_k x d_v), for the
+ * sequence-parallel forward.  The article's paragraph 3 reconstructs the
+ * sequential states across GPUs with a prefix scan; the pages give no algebra
+ * for it.  Here each rank holds one contiguous time segment of the sequences,
+ * computes these maps for it, exchanges them (an all-gather) and applies the
+ * maps of the earlier segments to S0 with kda_segment_scan to get its own start
+ * state, then runs kda_forward from that state.  Per chunk of C tokens the map is
+ * M_c = Diag(gamma_C) - (k*eta)^T Tb (k*gamma) and N_c = (k*eta)^T Tb V
+ * (notation of kda_forward's chunk form), composed in order.
+ *
+ *   k, alpha : [B, T, H, d_k]   in_dtype;  v : [B, T, H, d_v];  beta : [B, T, H]
+ *   cu_seqlens, num_seqs : as kda_forward (packed batch when non-NULL)
+ *   maps     : fp32 [N, H, d_k, d_k + d_v], row c = [M[c, :] | N[c, :]] (written)
+ *
+ * Supported: bf16 inputs, d_k = d_v = 128, chunk 64 (the tensor-core kernel in
+ * its map mode).  A sequence with no tokens gets [I | 0].  16-byte alignment for
+ * k, v, alpha and maps.  Returns as kda_forward.
+ */
+kda_status_t kda_segment_maps(const void* k, const void* v, const void* alpha, const void* beta,
+                              const int32_t* cu_seqlens, int32_t num_seqs, float* maps,
+                              int32_t B, int64_t T, int32_t H, int32_t d_k, int32_t d_v,
+                              int32_t chunk, kda_dtype_t in_dtype, kda_stream_t stream);
+
+/*
+ * kda_segment_scan -- applies num_maps segment maps in order to S0:
+ * S <- M_g S + N_g for g = 0 .. num_maps-1, in fp32, and writes the result.
+ *
+ *   S0   : NULL (zero state) or fp32 [N, H, d_k, d_v]
+ *   maps : fp32 [num_maps, N, H, d_k, d_k + d_v] (kda_segment_maps outputs, stacked
+ *          in segment order)
+ *   out  : fp32 [N, H, d_k, d_v]; may alias S0 exactly
+ *
+ * Supported: d_k = d_v = 128; num_maps >= 0 (0 copies S0, or zeros).  16-byte
+ * alignment for every pointer.  Returns as kda_forward.
+ */
+kda_status_t kda_segment_scan(const float* S0, const float* maps, int32_t num_maps, float* out,
+                              int32_t num_seqs, int32_t H, int32_t d_k, int32_t d_v,
+                              kda_stream_t stream);
+
 /* A static, human-readable name for a status code (never NULL). */
 const char* kda_status_string(kda_status_t status);
 

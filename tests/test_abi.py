@@ -110,3 +110,41 @@ def test_time_segment_choice():
     assert seg(0, 100, 4, 148) == 1 and seg(1, 0, 4, 148) == 1
     for units_h in (1, 2, 4, 8, 16, 32, 64):
         assert 1 <= seg(1, 1 << 22, units_h, 148) <= 64
+
+
+def test_segment_calls_reject_before_launch():
+    lib = kda.load_library()
+    # unsupported shape or dtype: no launch, no device touched
+    assert lib.kda_segment_maps(None, None, None, None, None, 0, None, 0, 0, 1, 128, 128, 64,
+                                0, None) == 2          # fp32 inputs
+    assert lib.kda_segment_maps(None, None, None, None, None, 0, None, 0, 0, 1, 64, 64, 64,
+                                1, None) == 2          # d = 64
+    assert lib.kda_segment_maps(None, None, None, None, None, 0, None, 1, 64, 1, 128, 128, 64,
+                                1, None) == 1          # tokens but no pointers
+    assert lib.kda_segment_scan(None, None, -1, None, 1, 1, 128, 128, None) == 1
+    assert lib.kda_segment_scan(None, None, 0, None, 1, 1, 64, 128, None) == 2
+    assert lib.kda_segment_scan(None, None, 1, None, 1, 1, 128, 128, None) == 1   # no out / maps
+    assert lib.kda_segment_scan(None, None, 0, None, 0, 1, 128, 128, None) == 0   # nothing to do
+
+
+def test_split_time_slices():
+    import torch
+    from gated_delta_rule_138_b200.seqpar import split_time
+    x = torch.arange(2 * 12 * 3).reshape(2, 12, 3)
+    parts = [split_time(x, 4, r) for r in range(4)]
+    assert all(p.shape == (2, 3, 3) for p in parts)
+    assert torch.equal(torch.cat(parts, dim=1), x)
+    with pytest.raises(ValueError):
+        split_time(x, 5, 0)
+
+
+def test_sequence_parallel_without_process_group_is_one_rank(monkeypatch):
+    """No process group: one rank, no maps, no exchange -- just the forward."""
+    from gated_delta_rule_138_b200 import seqpar
+    calls = []
+    monkeypatch.setattr(seqpar.kda, "kda_forward", lambda *a, **k: calls.append("fwd") or ("o", "s"))
+    monkeypatch.setattr(seqpar.kda, "kda_segment_maps", lambda *a, **k: calls.append("maps"))
+    import torch
+    x = torch.zeros(1, 4, 1, 8)
+    assert seqpar.kda_forward_sequence_parallel(x, x, x, x, x[..., 0]) == ("o", "s")
+    assert calls == ["fwd"]
