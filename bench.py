@@ -273,7 +273,7 @@ def time_oracle(w, inp, budget_s: float, cores: int):
         lens = np.full(w.B, w.T)
     Tmax = int(lens.max()) if len(lens) else 0
     flat = {n: inp[n].reshape(-1, *inp[n].shape[2:]) for n in ("q", "k", "v", "alpha", "beta")}
-    S0 = inp.get("S0")
+    S0 = inp["S_pool"][inp["slots"].long()] if w.kind == "pooled" else inp.get("S0")
     pairs = [(s, h) for s in range(len(lens)) for h in range(w.H)]
     P, Ts = min(len(pairs), 2 * cores), min(Tmax, 1024)
     while True:
@@ -351,6 +351,8 @@ def config_of(w, n_gpus):
         c.update({"B": w.B, "T": w.T, "global_batch": w.B * n_gpus, "seq_len": w.T})
     elif w.kind == "varlen":
         c.update({"num_seqs": w.nseq, "len_range": [w.min_len, w.max_len]})
+    elif w.kind == "pooled":
+        c.update({"N": w.B, "tokens_per_seq": w.T, "pool_slots": w.nseq})
     else:
         c.update({"N": w.B, "steps_per_run": w.steps})
     return c
@@ -384,6 +386,19 @@ def run_ours(args, w):
         algo_bytes = decode_bytes(w, n_sh)
         algo_flops = decode_flops(w, n_sh)
         src_file = "kda_decode.cu"
+    elif w.kind == "pooled":
+        # a serving step: T tokens per sequence from and into pooled state slots
+        out = torch.empty(w.B, w.T, w.H, w.dv, dtype=torch.bfloat16, device=dev)
+        pool = inp["S_pool"]
+
+        def step():
+            kda.kda_forward_indexed(inp["q"], inp["k"], inp["v"], inp["alpha"], inp["beta"], pool,
+                                    inp["slots"], out=out, chunk=w.chunk)
+        kname = kda.kda_forward_kernel_name(w.dk, w.dv, w.chunk, inp["q"].dtype, out.dtype)
+        segments = 1
+        algo_bytes = forward_bytes(w, n_th, n_sh, True)   # state read and written once
+        algo_flops = forward_flops(w, n_th)
+        src_file = "kda_chunk_tc.cu"
     else:
         cu = inp.get("cu_seqlens")
         B, T = inp["q"].shape[0], inp["q"].shape[1]
@@ -452,7 +467,7 @@ def run_ours(args, w):
 
     # end to end: pinned host inputs -> device -> kda_forward -> host results
     e2e = run_e2e(args, w, inp, dev, stream, world) \
-        if w.kind != "decode" and args.e2e_steps > 0 and not seqpar \
+        if w.kind in ("forward", "varlen") and args.e2e_steps > 0 and not seqpar \
         else None
 
     if rank == 0:

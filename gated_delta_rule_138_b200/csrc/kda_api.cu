@@ -16,14 +16,16 @@ namespace kda {
 cudaError_t launch_chunk_simt(int in_bf16, int out_bf16, int chunk, const void* q, const void* k,
                               const void* v, const void* alpha, const void* beta, const float* S0,
                               const int32_t* cu, int nseq, void* out, float* S_final, int64_t T,
-                              int H, int DK, int DV, cudaStream_t s);
+                              int H, int DK, int DV, cudaStream_t s, const int32_t* slots = nullptr,
+                              int num_slots = 0);
 cudaError_t launch_decode(int in_bf16, int out_bf16, const void* q, const void* k, const void* v,
                           const void* alpha, const void* beta, float* S, void* out, int64_t NH,
-                          int DK, int DV, cudaStream_t s);
+                          int DK, int DV, cudaStream_t s, const int32_t* slots, int num_slots,
+                          int H, int T = 1);
 cudaError_t launch_chunk_tc(const void* q, const void* k, const void* v, const void* alpha,
                             const void* beta, const float* S0, const int32_t* cu, int nseq,
                             void* out, float* S_final, int64_t rows, int64_t T, int H, int* status,
-                            cudaStream_t stream);
+                            cudaStream_t stream, const int32_t* slots = nullptr, int num_slots = 0);
 size_t chunk_tc_segmented_workspace_floats(int64_t nseq, int H, int nseg);
 cudaError_t launch_segment_maps(const void* k, const void* v, const void* alpha, const void* beta,
                                 const int32_t* cu, int nseq, float* maps, int64_t rows, int64_t T,
@@ -114,6 +116,10 @@ int current_sms() {
     }
     return sms;
 }
+
+// Dense multi-token steps of at most this many tokens per sequence take the
+// token-sequential kernel (state in registers) instead of the chunk kernels.
+constexpr int64_t kMaxStepTokens = 16;
 
 bool debug_sync() {
     const char* v = std::getenv("KDA_DEBUG");
@@ -271,6 +277,82 @@ kda_status_t kda_forward(const void* q, const void* k, const void* v, const void
                                               s));
 }
 
+kda_status_t kda_forward_indexed(const void* q, const void* k, const void* v, const void* alpha,
+                                 const void* beta, float* S_pool, int32_t num_slots,
+                                 const int32_t* slots, const int32_t* cu_seqlens, int32_t num_seqs,
+                                 void* out, int32_t B, int64_t T, int32_t H, int32_t d_k,
+                                 int32_t d_v, int32_t chunk, kda_dtype_t in_dtype,
+                                 kda_dtype_t out_dtype, kda_stream_t stream) {
+    if (B < 0 || T < 0 || H <= 0 || num_slots < 0 || !is_dtype(in_dtype) || !is_dtype(out_dtype))
+        return KDA_ERR_INVALID_ARG;
+    if (cu_seqlens != nullptr && (B != 1 || num_seqs < 0)) return KDA_ERR_INVALID_ARG;
+    const int64_t nseq = cu_seqlens ? (int64_t)num_seqs : (int64_t)B;
+    if (nseq > 0 && (!S_pool || !slots)) return KDA_ERR_INVALID_ARG;
+    if ((int64_t)B * T > 0 && (!q || !k || !v || !alpha || !beta || !out)) return KDA_ERR_INVALID_ARG;
+    const void* p16[] = {q, k, v, alpha, S_pool, out};
+    for (const void* p : p16)
+        if (p && !aligned16(p)) return KDA_ERR_INVALID_ARG;
+    if (!aligned_to(beta, in_dtype == KDA_BF16 ? 2 : 4) || !aligned_to(cu_seqlens, 4) ||
+        !aligned_to(slots, 4))
+        return KDA_ERR_INVALID_ARG;
+    if (!head_dim_ok(d_k) || !head_dim_ok(d_v)) return KDA_ERR_UNSUPPORTED;
+    if (chunk != 16 && chunk != 32 && chunk != 64) return KDA_ERR_UNSUPPORTED;
+    if (nseq > 65535 || H > 65535) return KDA_ERR_UNSUPPORTED;
+    if (nseq == 0) return KDA_OK;
+    g_last_error[0] = '\0';
+    const cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    g_launches.fetch_add(1, std::memory_order_relaxed);
+    if (cu_seqlens == nullptr && T <= kMaxStepTokens) {
+        // a short multi-token step: the state stays in registers across the T tokens
+        if (T == 0) return KDA_OK;   // nothing advances; every state unchanged
+        if ((int64_t)B * H > 0x7fffffffLL) return KDA_ERR_UNSUPPORTED;
+        return cuda_status(kda::launch_decode(in_dtype == KDA_BF16, out_dtype == KDA_BF16, q, k, v,
+                                              alpha, beta, S_pool, out, (int64_t)B * H, d_k, d_v,
+                                              s, slots, num_slots, H, (int)T));
+    }
+    if (use_tc(d_k, d_v, chunk, in_dtype, out_dtype)) {
+        int* status = nullptr;
+        cudaError_t e = device_status_word(&status);
+        if (e != cudaSuccess) return cuda_status(e);
+        const int64_t rows = cu_seqlens ? T : (int64_t)B * T;
+        if (rows > 0x7fffffffLL) return KDA_ERR_UNSUPPORTED;
+        e = kda::launch_chunk_tc(q, k, v, alpha, beta, S_pool, cu_seqlens, (int)nseq, out, S_pool,
+                                 rows, T, H, status, s, slots, num_slots);
+        if (e != cudaSuccess) return cuda_status(e);
+        return debug_sync() ? kda_device_status(stream) : KDA_OK;
+    }
+    return cuda_status(kda::launch_chunk_simt(in_dtype == KDA_BF16, out_dtype == KDA_BF16, chunk, q,
+                                              k, v, alpha, beta, S_pool, cu_seqlens, (int)nseq, out,
+                                              S_pool, T, H, d_k, d_v, s, slots, num_slots));
+}
+
+kda_status_t kda_decode_step_indexed(const void* q, const void* k, const void* v,
+                                     const void* alpha, const void* beta, float* S_pool,
+                                     int32_t num_slots, const int32_t* slots, void* out, int32_t N,
+                                     int32_t H, int32_t d_k, int32_t d_v, kda_dtype_t in_dtype,
+                                     kda_dtype_t out_dtype, kda_stream_t stream) {
+    if (N < 0 || H <= 0 || num_slots < 0 || !is_dtype(in_dtype) || !is_dtype(out_dtype))
+        return KDA_ERR_INVALID_ARG;
+    if (N > 0 && (!q || !k || !v || !alpha || !beta || !S_pool || !slots || !out))
+        return KDA_ERR_INVALID_ARG;
+    const int es = in_dtype == KDA_BF16 ? 2 : 4;
+    if (S_pool && !aligned16(S_pool)) return KDA_ERR_INVALID_ARG;
+    if (!aligned_to(q, es) || !aligned_to(k, es) || !aligned_to(v, es) || !aligned_to(alpha, es) ||
+        !aligned_to(beta, es) || !aligned_to(out, out_dtype == KDA_BF16 ? 2 : 4) ||
+        !aligned_to(slots, 4))
+        return KDA_ERR_INVALID_ARG;
+    if (!head_dim_ok(d_k) || !head_dim_ok(d_v)) return KDA_ERR_UNSUPPORTED;
+    const int64_t NH = (int64_t)N * H;
+    if (NH > 0x7fffffffLL) return KDA_ERR_UNSUPPORTED;
+    if (NH == 0) return KDA_OK;
+    g_last_error[0] = '\0';
+    g_launches.fetch_add(1, std::memory_order_relaxed);
+    return cuda_status(kda::launch_decode(in_dtype == KDA_BF16, out_dtype == KDA_BF16, q, k, v,
+                                          alpha, beta, S_pool, out, NH, d_k, d_v,
+                                          reinterpret_cast<cudaStream_t>(stream), slots, num_slots,
+                                          H));
+}
+
 kda_status_t kda_segment_maps(const void* k, const void* v, const void* alpha, const void* beta,
                               const int32_t* cu_seqlens, int32_t num_seqs, float* maps, int32_t B,
                               int64_t T, int32_t H, int32_t d_k, int32_t d_v, int32_t chunk,
@@ -340,7 +422,7 @@ kda_status_t kda_decode_step(const void* q, const void* k, const void* v, const 
     const cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
     g_launches.fetch_add(1, std::memory_order_relaxed);
     return cuda_status(kda::launch_decode(in_dtype == KDA_BF16, out_dtype == KDA_BF16, q, k, v,
-                                          alpha, beta, S, out, NH, d_k, d_v, s));
+                                          alpha, beta, S, out, NH, d_k, d_v, s, nullptr, 0, H));
 }
 
 }  // extern "C"

@@ -51,7 +51,8 @@ kda_chunk_simt_kernel(const Tin* __restrict__ q, const Tin* __restrict__ k,
                       const Tin* __restrict__ v, const Tin* __restrict__ alpha,
                       const Tin* __restrict__ beta, const float* S0,
                       const int32_t* __restrict__ cu_seqlens, Tout* __restrict__ out,
-                      float* S_final, int64_t T, int H, int DV) {
+                      float* S_final, int64_t T, int H, int DV, const int32_t* slots,
+                      int num_slots) {
     using L = SimtSmem<DK, NV, C>;
     constexpr int NSUB = L::NSUB, DKP = L::DKP, CP = L::CP, NVP = L::NVP;
     extern __shared__ float smem[];
@@ -75,11 +76,15 @@ kda_chunk_simt_kernel(const Tin* __restrict__ q, const Tin* __restrict__ k,
     const int j0 = blockIdx.x * NV, h = blockIdx.y, n = blockIdx.z;
     int64_t bos, len;
     seq_range(cu_seqlens, n, T, bos, len);
-    const size_t sbase = ((size_t)n * H + h) * (size_t)DK * DV + j0;
+    // state slot of this sequence (slots null: n); an invalid slot starts from zero
+    // and writes no state
+    const int slot = slots ? slots[n] : n;
+    const bool slot_ok = !slots || (slot >= 0 && slot < num_slots);
+    const size_t sbase = ((size_t)(slot_ok ? slot : 0) * H + h) * (size_t)DK * DV + j0;
 
     for (int i = tid; i < DK * NV; i += kSimtThreads) {
         const int c = i / NV, jj = i % NV;
-        Ss[c * NVP + jj] = S0 ? S0[sbase + (size_t)c * DV + jj] : 0.0f;
+        Ss[c * NVP + jj] = S0 && slot_ok ? S0[sbase + (size_t)c * DV + jj] : 0.0f;
     }
     __syncthreads();
 
@@ -265,7 +270,7 @@ kda_chunk_simt_kernel(const Tin* __restrict__ q, const Tin* __restrict__ k,
         __syncthreads();
     }
 
-    if (S_final) {
+    if (S_final && slot_ok) {
         for (int i = tid; i < DK * NV; i += kSimtThreads) {
             const int c = i / NV, jj = i % NV;
             S_final[sbase + (size_t)c * DV + jj] = Ss[c * NVP + jj];
@@ -279,7 +284,7 @@ template <typename Tin, typename Tout, int DK, int NV, int C>
 static cudaError_t launch_simt_t(const void* q, const void* k, const void* v, const void* alpha,
                                  const void* beta, const float* S0, const int32_t* cu_seqlens,
                                  int nseq, void* out, float* S_final, int64_t T, int H, int DV,
-                                 cudaStream_t stream) {
+                                 cudaStream_t stream, const int32_t* slots, int num_slots) {
     using L = SimtSmem<DK, NV, C>;
     auto kern = kda_chunk_simt_kernel<Tin, Tout, DK, NV, C>;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
@@ -288,7 +293,7 @@ static cudaError_t launch_simt_t(const void* q, const void* k, const void* v, co
     dim3 grid(DV / NV, H, nseq);
     kern<<<grid, kSimtThreads, L::bytes, stream>>>(
         (const Tin*)q, (const Tin*)k, (const Tin*)v, (const Tin*)alpha, (const Tin*)beta, S0,
-        cu_seqlens, (Tout*)out, S_final, T, H, DV);
+        cu_seqlens, (Tout*)out, S_final, T, H, DV, slots, num_slots);
     return cudaGetLastError();
 }
 
@@ -296,11 +301,12 @@ template <typename Tin, typename Tout, int DK>
 static cudaError_t launch_simt_dk(int chunk, const void* q, const void* k, const void* v,
                                   const void* alpha, const void* beta, const float* S0,
                                   const int32_t* cu, int nseq, void* out, float* S_final,
-                                  int64_t T, int H, int DV, cudaStream_t s) {
+                                  int64_t T, int H, int DV, cudaStream_t s, const int32_t* slots,
+                                  int num_slots) {
     switch (chunk) {
-        case 16: return launch_simt_t<Tin, Tout, DK, 32, 16>(q, k, v, alpha, beta, S0, cu, nseq, out, S_final, T, H, DV, s);
-        case 32: return launch_simt_t<Tin, Tout, DK, 32, 32>(q, k, v, alpha, beta, S0, cu, nseq, out, S_final, T, H, DV, s);
-        default: return launch_simt_t<Tin, Tout, DK, 32, 64>(q, k, v, alpha, beta, S0, cu, nseq, out, S_final, T, H, DV, s);
+        case 16: return launch_simt_t<Tin, Tout, DK, 32, 16>(q, k, v, alpha, beta, S0, cu, nseq, out, S_final, T, H, DV, s, slots, num_slots);
+        case 32: return launch_simt_t<Tin, Tout, DK, 32, 32>(q, k, v, alpha, beta, S0, cu, nseq, out, S_final, T, H, DV, s, slots, num_slots);
+        default: return launch_simt_t<Tin, Tout, DK, 32, 64>(q, k, v, alpha, beta, S0, cu, nseq, out, S_final, T, H, DV, s, slots, num_slots);
     }
 }
 
@@ -308,12 +314,13 @@ static cudaError_t launch_simt_dk(int chunk, const void* q, const void* k, const
 cudaError_t launch_chunk_simt(int in_bf16, int out_bf16, int chunk, const void* q, const void* k,
                               const void* v, const void* alpha, const void* beta, const float* S0,
                               const int32_t* cu, int nseq, void* out, float* S_final, int64_t T,
-                              int H, int DK, int DV, cudaStream_t s) {
+                              int H, int DK, int DV, cudaStream_t s, const int32_t* slots,
+                              int num_slots) {
 #define KDA_SIMT_CASE(TI, TO)                                                                  \
     return DK == 64 ? launch_simt_dk<TI, TO, 64>(chunk, q, k, v, alpha, beta, S0, cu, nseq, out, \
-                                                 S_final, T, H, DV, s)                       \
+                                                 S_final, T, H, DV, s, slots, num_slots)     \
                     : launch_simt_dk<TI, TO, 128>(chunk, q, k, v, alpha, beta, S0, cu, nseq,   \
-                                                  out, S_final, T, H, DV, s);
+                                                  out, S_final, T, H, DV, s, slots, num_slots);
     if (!in_bf16 && !out_bf16) { KDA_SIMT_CASE(float, float) }
     if (!in_bf16 && out_bf16) { KDA_SIMT_CASE(float, __nv_bfloat16) }
     if (in_bf16 && !out_bf16) { KDA_SIMT_CASE(__nv_bfloat16, float) }

@@ -146,6 +146,11 @@ struct Segments {
     int per_seq;          // segment CTAs per sequence in this launch
     const float* start;   // forward with nseg > 1: start states [nseq * nseg, H, DK, DV]
     float* maps;          // summary: [M | N] fp32 [nseq * per_seq, H, DK, DK + DV]
+    // state slots (whole sequences only): sequence n reads S0 and writes S_final at
+    // slot slots[n] of a pool of num_slots states; a slot outside [0, num_slots)
+    // starts from zero and writes no state.  Null: slot n.
+    const int32_t* slots;
+    int num_slots;
 };
 
 // One TMA stream's bookkeeping: the parity a thread's next wait on it expects,
@@ -211,6 +216,8 @@ kda_chunk_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_consta
     }
     const int nchunks = (int)((len + C - 1) / C);
     const bool last_seg = gseg == seg.nseg - 1;
+    const int slot = seg.slots ? seg.slots[n] : n;
+    const bool slot_ok = !seg.slots || (slot >= 0 && slot < seg.num_slots);
 
     if (tid == 0) {
         mbar_init(barQ, 1);
@@ -248,7 +255,7 @@ kda_chunk_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_consta
         const int c = 32 * q4 + lane;
         const float* base = seg.nseg > 1
                                 ? seg.start + (((size_t)n * seg.nseg + gseg) * H + h) * DK * DV
-                                : (S0 ? S0 + ((size_t)n * H + h) * DK * DV : nullptr);
+                                : (S0 && slot_ok ? S0 + ((size_t)slot * H + h) * DK * DV : nullptr);
         const float* src = base ? base + (size_t)c * DV + 64 * hf : nullptr;
 #pragma unroll
         for (int blk = 0; blk < 4; ++blk) {
@@ -1046,9 +1053,9 @@ kda_chunk_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_consta
             for (int i = 0; i < 16; i += 4)
                 *reinterpret_cast<float4*>(dst + 16 * blk + i) = make_float4(v[i], v[i + 1], v[i + 2], v[i + 3]);
         }
-    } else if (S_final && last_seg) {
+    } else if (S_final && last_seg && slot_ok) {
         const int c = 32 * q4 + lane;
-        float* dst = S_final + (((size_t)n * H + h) * DK + c) * DV + 64 * hf;
+        float* dst = S_final + (((size_t)slot * H + h) * DK + c) * DV + 64 * hf;
 #pragma unroll
         for (int blk = 0; blk < 4; ++blk) {
             float v[16];
@@ -1225,10 +1232,10 @@ static cudaError_t launch_tc_t(const TcMaps& m, const void* beta, const float* S
 cudaError_t launch_chunk_tc(const void* q, const void* k, const void* v, const void* alpha,
                             const void* beta, const float* S0, const int32_t* cu, int nseq,
                             void* out, float* S_final, int64_t rows, int64_t T, int H, int* status,
-                            cudaStream_t stream) {
+                            cudaStream_t stream, const int32_t* slots, int num_slots) {
     TcMaps m;
     if (!make_maps(&m, q, k, v, alpha, out, rows, H)) return cudaErrorInvalidValue;
-    const tc::Segments whole{1, 1, nullptr, nullptr};
+    const tc::Segments whole{1, 1, nullptr, nullptr, slots, num_slots};
     return launch_tc_t<false, false>(m, beta, S0, cu, nseq, out, S_final, T, H, status, whole,
                                      stream);
 }

@@ -14,7 +14,9 @@
 //
 // The state is fp32 and HBM-bound: one CTA per (sequence, head) streams its
 // d_k x d_v slab with 16-byte loads and stores, keeping it in registers between
-// the reduction and the update.
+// the reduction and the update.  A multi-token step (T tokens per sequence,
+// inputs [N, T, H, d]) keeps the state in registers across its T tokens: the
+// state is read and written once per step, not once per token.
 #include "kda_common.cuh"
 
 namespace kda {
@@ -23,7 +25,8 @@ template <typename Tin, typename Tout, int DK, int DV>
 __global__ void __launch_bounds__(256)
 kda_decode_kernel(const Tin* __restrict__ q, const Tin* __restrict__ k,
                   const Tin* __restrict__ v, const Tin* __restrict__ alpha,
-                  const Tin* __restrict__ beta, float* __restrict__ S, Tout* __restrict__ out) {
+                  const Tin* __restrict__ beta, float* __restrict__ S, Tout* __restrict__ out,
+                  const int32_t* __restrict__ slots, int num_slots, int H, int T) {
     constexpr int NT = 256;
     constexpr int TX = DV / 4;       // threads across a row (float4 each)
     constexpr int TY = NT / TX;      // rows per pass
@@ -36,14 +39,23 @@ kda_decode_kernel(const Tin* __restrict__ q, const Tin* __restrict__ k,
 
     const int tid = threadIdx.x, tx = tid % TX, ty = tid / TX;
     const size_t nh = blockIdx.x;                 // (sequence, head) flattened
-    const size_t kb = nh * DK, vb = nh * DV;
-    float4* Sv = reinterpret_cast<float4*>(S + nh * (size_t)DK * DV);
+    // state slot (slots null: the sequence's own index); an invalid slot decodes
+    // from a zero state and writes no state
+    const int64_t n = (int64_t)(nh / H), hh = (int64_t)(nh % H);
+    const int64_t slot = slots ? (int64_t)slots[n] : n;
+    const bool slot_ok = !slots || (slot >= 0 && slot < num_slots);
+    float4* Sv = reinterpret_cast<float4*>(S + ((size_t)(slot_ok ? slot : 0) * H + hh) * (size_t)DK * DV);
 
     // issue the state loads first: they are the HBM traffic
     float4 s[RPT];
 #pragma unroll
-    for (int i = 0; i < RPT; ++i) s[i] = Sv[(size_t)(ty + TY * i) * TX + tx];
+    for (int i = 0; i < RPT; ++i)
+        s[i] = slot_ok ? Sv[(size_t)(ty + TY * i) * TX + tx] : make_float4(0.f, 0.f, 0.f, 0.f);
 
+    for (int t = 0; t < T; ++t) {
+    const size_t tok = ((size_t)n * T + t) * H + hh;   // (sequence, token, head)
+    const size_t kb = tok * DK, vb = tok * DV;
+    if (t > 0) __syncthreads();   // the previous token's update has read ga, kk and us
     float kqp = 0.0f;
     if (tid < DK) {
         const float a = clamp_gate(to_f32(alpha[kb + tid]));
@@ -80,7 +92,7 @@ kda_decode_kernel(const Tin* __restrict__ q, const Tin* __restrict__ k,
         float kq = 0.0f;
 #pragma unroll
         for (int i = 0; i < NT / 32; ++i) kq += kq_part[i];
-        const float b = to_f32(beta[nh]);
+        const float b = to_f32(beta[tok]);
         const float u = b * (to_f32(v[vb + tid]) - x);
         us[tid] = u;
         out[vb + tid] = from_f32<Tout>(fmaf(u, kq, y));
@@ -98,37 +110,45 @@ kda_decode_kernel(const Tin* __restrict__ q, const Tin* __restrict__ k,
         r.y = fmaf(a, s[i].y, kc * u4.y);
         r.z = fmaf(a, s[i].z, kc * u4.z);
         r.w = fmaf(a, s[i].w, kc * u4.w);
-        Sv[(size_t)c * TX + tx] = r;
+        s[i] = r;
+    }
+    }
+    if (slot_ok) {
+#pragma unroll
+        for (int i = 0; i < RPT; ++i) Sv[(size_t)(ty + TY * i) * TX + tx] = s[i];
     }
 }
 
 template <typename Tin, typename Tout, int DK, int DV>
 static cudaError_t launch_decode_t(const void* q, const void* k, const void* v, const void* alpha,
                                    const void* beta, float* S, void* out, int64_t NH,
-                                   cudaStream_t stream) {
+                                   cudaStream_t stream, const int32_t* slots, int num_slots, int H,
+                                   int T) {
     kda_decode_kernel<Tin, Tout, DK, DV><<<(unsigned)NH, 256, 0, stream>>>(
         (const Tin*)q, (const Tin*)k, (const Tin*)v, (const Tin*)alpha, (const Tin*)beta, S,
-        (Tout*)out);
+        (Tout*)out, slots, num_slots, H, T);
     return cudaGetLastError();
 }
 
 template <typename Tin, typename Tout>
 static cudaError_t launch_decode_d(int DK, int DV, const void* q, const void* k, const void* v,
                                    const void* alpha, const void* beta, float* S, void* out,
-                                   int64_t NH, cudaStream_t s) {
-    if (DK == 64 && DV == 64) return launch_decode_t<Tin, Tout, 64, 64>(q, k, v, alpha, beta, S, out, NH, s);
-    if (DK == 64 && DV == 128) return launch_decode_t<Tin, Tout, 64, 128>(q, k, v, alpha, beta, S, out, NH, s);
-    if (DK == 128 && DV == 64) return launch_decode_t<Tin, Tout, 128, 64>(q, k, v, alpha, beta, S, out, NH, s);
-    return launch_decode_t<Tin, Tout, 128, 128>(q, k, v, alpha, beta, S, out, NH, s);
+                                   int64_t NH, cudaStream_t s, const int32_t* slots, int num_slots,
+                                   int H, int T) {
+    if (DK == 64 && DV == 64) return launch_decode_t<Tin, Tout, 64, 64>(q, k, v, alpha, beta, S, out, NH, s, slots, num_slots, H, T);
+    if (DK == 64 && DV == 128) return launch_decode_t<Tin, Tout, 64, 128>(q, k, v, alpha, beta, S, out, NH, s, slots, num_slots, H, T);
+    if (DK == 128 && DV == 64) return launch_decode_t<Tin, Tout, 128, 64>(q, k, v, alpha, beta, S, out, NH, s, slots, num_slots, H, T);
+    return launch_decode_t<Tin, Tout, 128, 128>(q, k, v, alpha, beta, S, out, NH, s, slots, num_slots, H, T);
 }
 
 cudaError_t launch_decode(int in_bf16, int out_bf16, const void* q, const void* k, const void* v,
                           const void* alpha, const void* beta, float* S, void* out, int64_t NH,
-                          int DK, int DV, cudaStream_t s) {
-    if (!in_bf16 && !out_bf16) return launch_decode_d<float, float>(DK, DV, q, k, v, alpha, beta, S, out, NH, s);
-    if (!in_bf16 && out_bf16) return launch_decode_d<float, __nv_bfloat16>(DK, DV, q, k, v, alpha, beta, S, out, NH, s);
-    if (in_bf16 && !out_bf16) return launch_decode_d<__nv_bfloat16, float>(DK, DV, q, k, v, alpha, beta, S, out, NH, s);
-    return launch_decode_d<__nv_bfloat16, __nv_bfloat16>(DK, DV, q, k, v, alpha, beta, S, out, NH, s);
+                          int DK, int DV, cudaStream_t s, const int32_t* slots, int num_slots,
+                          int H, int T) {
+    if (!in_bf16 && !out_bf16) return launch_decode_d<float, float>(DK, DV, q, k, v, alpha, beta, S, out, NH, s, slots, num_slots, H, T);
+    if (!in_bf16 && out_bf16) return launch_decode_d<float, __nv_bfloat16>(DK, DV, q, k, v, alpha, beta, S, out, NH, s, slots, num_slots, H, T);
+    if (in_bf16 && !out_bf16) return launch_decode_d<__nv_bfloat16, float>(DK, DV, q, k, v, alpha, beta, S, out, NH, s, slots, num_slots, H, T);
+    return launch_decode_d<__nv_bfloat16, __nv_bfloat16>(DK, DV, q, k, v, alpha, beta, S, out, NH, s, slots, num_slots, H, T);
 }
 
 }  // namespace kda

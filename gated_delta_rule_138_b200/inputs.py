@@ -34,7 +34,7 @@ BF16_BELOW_EXP_M5 = 0.0067138671875  # largest bf16 value below e^-5
 @dataclass(frozen=True)
 class Workload:
     name: str
-    kind: str                 # "forward" | "decode" | "varlen"
+    kind: str                 # "forward" | "decode" | "varlen" | "pooled"
     dtype: str                # input dtype: "f32" | "bf16"
     H: int
     dk: int
@@ -45,7 +45,7 @@ class Workload:
     s0: bool = False
     special_alpha: bool = False
     steps: int = 0            # decode only
-    nseq: int = 0             # varlen only
+    nseq: int = 0             # varlen only; pooled: slots in the state pool
     min_len: int = 0
     max_len: int = 0
     seed: int = 0
@@ -72,6 +72,10 @@ WORKLOADS = {
     "decode_N256_H32_d128": Workload("decode_N256_H32_d128", "decode", "bf16", H=32,
                                      dk=128, dv=128, B=256, steps=128, s0=True, seed=1003),
     # packed variable-length batch: 64 sequences, log-uniform lengths
+    # serving step: 4 tokens for each of 256 sequences whose states live in a pool of
+    # 512 slots (a seeded choice of slots)
+    "pooled_N256_T4_H32_d128": Workload("pooled_N256_T4_H32_d128", "pooled", "bf16", H=32,
+                                        dk=128, dv=128, B=256, T=4, nseq=512, seed=5000),
     "varlen_64seq_H16_d128": Workload("varlen_64seq_H16_d128", "varlen", "bf16", H=16,
                                       dk=128, dv=128, nseq=64, min_len=128, max_len=32768,
                                       s0=True, seed=4000),
@@ -196,4 +200,10 @@ def draw_workload(w: Workload, device="cpu", **over) -> dict:
     if w.kind == "decode":
         return draw_decode(over.get("B", w.B), w.H, w.dk, w.dv, over.get("steps", w.steps),
                            w.dtype, w.seed, device=device)
+    if w.kind == "pooled":
+        out = draw_forward(w.B, w.T, w.H, w.dk, w.dv, w.dtype, w.seed, device=device, s0=False)
+        g = _gen(w.seed + 1, "cpu")
+        out["S_pool"] = (0.1 * torch.randn(w.nseq, w.H, w.dk, w.dv, generator=g)).to(device)
+        out["slots"] = torch.randperm(w.nseq, generator=g)[:w.B].to(torch.int32).to(device)
+        return out
     raise ValueError(w.kind)

@@ -87,6 +87,12 @@ def load_library(build_if_missing: bool = True) -> ctypes.CDLL:
     lib.kda_selftest_timeout.argtypes = [ctypes.c_uint64, vp]
     lib.kda_forward_noalloc.restype = ctypes.c_int
     lib.kda_forward_noalloc.argtypes = lib.kda_forward.argtypes
+    lib.kda_forward_indexed.restype = ctypes.c_int
+    lib.kda_forward_indexed.argtypes = [vp, vp, vp, vp, vp, vp, i32, vp, vp, i32, vp,
+                                        i32, i64, i32, i32, i32, i32, ctypes.c_int, ctypes.c_int, vp]
+    lib.kda_decode_step_indexed.restype = ctypes.c_int
+    lib.kda_decode_step_indexed.argtypes = [vp, vp, vp, vp, vp, vp, i32, vp, vp, i32, i32, i32, i32,
+                                            ctypes.c_int, ctypes.c_int, vp]
     _lib = lib
     return lib
 
@@ -283,4 +289,58 @@ def kda_decode_step(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, alpha: to
                              _ptr(out), int(N), int(H), int(dk), int(dv), _dt(q), _dt(out),
                              _stream(stream))
     _check("kda_decode_step", st)
+    return out
+
+
+def kda_forward_indexed(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, alpha: torch.Tensor,
+                        beta: torch.Tensor, S_pool: torch.Tensor, slots: torch.Tensor,
+                        cu_seqlens: Optional[torch.Tensor] = None,
+                        out: Optional[torch.Tensor] = None, chunk: int = 64,
+                        out_dtype: Optional[torch.dtype] = None, stream=None) -> torch.Tensor:
+    """kda_forward from and into pooled states: sequence n starts from, and
+    leaves its final state in, S_pool[slots[n]] (fp32 [P, H, d_k, d_v]; int32
+    slots, a slot outside [0, P) = padding).  Returns out [B, T, H, d_v]."""
+    lib = load_library()
+    B, T, H, dk = q.shape
+    dv = v.shape[-1]
+    for name, t in (("q", q), ("k", k), ("v", v), ("alpha", alpha), ("beta", beta),
+                    ("S_pool", S_pool), ("slots", slots), ("cu_seqlens", cu_seqlens)):
+        _contig(name, t)
+    nseq = B if cu_seqlens is None else cu_seqlens.numel() - 1
+    if slots.dtype != torch.int32 or slots.numel() != nseq:
+        raise ValueError("slots must be int32 [N]")
+    if S_pool.dtype != torch.float32 or tuple(S_pool.shape[1:]) != (H, dk, dv):
+        raise ValueError("S_pool must be fp32 [P, H, d_k, d_v]")
+    if out is None:
+        out = torch.empty(B, T, H, dv, dtype=out_dtype or q.dtype, device=q.device)
+    st = lib.kda_forward_indexed(_ptr(q), _ptr(k), _ptr(v), _ptr(alpha), _ptr(beta), _ptr(S_pool),
+                                 int(S_pool.shape[0]), _ptr(slots), _ptr(cu_seqlens), int(nseq),
+                                 _ptr(out), int(B), int(T), int(H), int(dk), int(dv), int(chunk),
+                                 _dt(q), _dt(out), _stream(stream))
+    _check("kda_forward_indexed", st)
+    return out
+
+
+def kda_decode_step_indexed(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor,
+                            alpha: torch.Tensor, beta: torch.Tensor, S_pool: torch.Tensor,
+                            slots: torch.Tensor, out: Optional[torch.Tensor] = None,
+                            out_dtype: Optional[torch.dtype] = None, stream=None) -> torch.Tensor:
+    """One decode step with the state of sequence n at S_pool[slots[n]] (in place)."""
+    lib = load_library()
+    N, H, dk = q.shape
+    dv = v.shape[-1]
+    for name, t in (("q", q), ("k", k), ("v", v), ("alpha", alpha), ("beta", beta),
+                    ("S_pool", S_pool), ("slots", slots)):
+        _contig(name, t)
+    if slots.dtype != torch.int32 or slots.numel() != N:
+        raise ValueError("slots must be int32 [N]")
+    if S_pool.dtype != torch.float32 or tuple(S_pool.shape[1:]) != (H, dk, dv):
+        raise ValueError("S_pool must be fp32 [P, H, d_k, d_v]")
+    if out is None:
+        out = torch.empty(N, H, dv, dtype=out_dtype or q.dtype, device=q.device)
+    st = lib.kda_decode_step_indexed(_ptr(q), _ptr(k), _ptr(v), _ptr(alpha), _ptr(beta),
+                                     _ptr(S_pool), int(S_pool.shape[0]), _ptr(slots), _ptr(out),
+                                     int(N), int(H), int(dk), int(dv), _dt(q), _dt(out),
+                                     _stream(stream))
+    _check("kda_decode_step_indexed", st)
     return out

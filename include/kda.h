@@ -153,6 +153,42 @@ kda_status_t kda_segment_scan(const float* S0, const float* maps, int32_t num_ma
                               int32_t num_seqs, int32_t H, int32_t d_k, int32_t d_v,
                               kda_stream_t stream);
 
+/*
+ * State slots for serving (no counterpart on the pages beyond paragraph 2's
+ * fixed-size state that replaces the KV cache): the states of many sequences
+ * live in one pool S_pool, fp32 [num_slots, H, d_k, d_v], and each call names
+ * the slot of every sequence it advances, int32 slots[N] (device memory).  A
+ * slot outside [0, num_slots) marks a padding sequence: it is computed from a
+ * zero state and no state is written.  Two sequences of one call must not name
+ * the same slot (undefined result).  Every slot not named is left untouched.
+ *
+ * kda_forward_indexed -- kda_forward over N sequences of any length (e.g. 2-16
+ * draft tokens per sequence in a multi-token decode step), starting from and
+ * updating S_pool[slots[n]] in place.  Arguments otherwise as kda_forward; it
+ * never splits sequences along time.  A dense batch of at most 16 tokens per
+ * sequence runs token by token in fp32 with the state held on chip for the
+ * whole step (read and written once); longer or packed batches run on the
+ * chunk kernels.
+ *
+ * kda_decode_step_indexed -- kda_decode_step with the state of sequence n at
+ * S_pool[slots[n]], updated in place.
+ *
+ * Returns as kda_forward.
+ */
+kda_status_t kda_forward_indexed(const void* q, const void* k, const void* v,
+                                 const void* alpha, const void* beta, float* S_pool,
+                                 int32_t num_slots, const int32_t* slots,
+                                 const int32_t* cu_seqlens, int32_t num_seqs, void* out,
+                                 int32_t B, int64_t T, int32_t H, int32_t d_k, int32_t d_v,
+                                 int32_t chunk, kda_dtype_t in_dtype, kda_dtype_t out_dtype,
+                                 kda_stream_t stream);
+kda_status_t kda_decode_step_indexed(const void* q, const void* k, const void* v,
+                                     const void* alpha, const void* beta, float* S_pool,
+                                     int32_t num_slots, const int32_t* slots, void* out,
+                                     int32_t N, int32_t H, int32_t d_k, int32_t d_v,
+                                     kda_dtype_t in_dtype, kda_dtype_t out_dtype,
+                                     kda_stream_t stream);
+
 /* A static, human-readable name for a status code (never NULL). */
 const char* kda_status_string(kda_status_t status);
 

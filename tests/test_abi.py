@@ -148,3 +148,16 @@ def test_sequence_parallel_without_process_group_is_one_rank(monkeypatch):
     x = torch.zeros(1, 4, 1, 8)
     assert seqpar.kda_forward_sequence_parallel(x, x, x, x, x[..., 0]) == ("o", "s")
     assert calls == ["fwd"]
+
+
+def test_indexed_calls_reject_before_launch():
+    lib = kda.load_library()
+    # negative pool size, missing slots, unsupported head dim: no launch
+    assert lib.kda_decode_step_indexed(None, None, None, None, None, None, -1, None, None, 0, 1,
+                                       128, 128, 1, 1, None) == 1
+    assert lib.kda_decode_step_indexed(None, None, None, None, None, None, 4, None, None, 2, 1,
+                                       128, 128, 1, 1, None) == 1
+    assert lib.kda_forward_indexed(None, None, None, None, None, None, 4, None, None, 0, None,
+                                   1, 4, 1, 96, 128, 64, 1, 1, None) == 1   # no pool / slots
+    assert lib.kda_forward_indexed(None, None, None, None, None, None, 4, None, None, 0, None,
+                                   0, 4, 1, 96, 128, 64, 1, 1, None) == 2   # d_k = 96
