@@ -410,6 +410,11 @@ def run_ours(args, w):
         def step():
             kda.kda_forward(inp["q"], inp["k"], inp["v"], inp["alpha"], inp["beta"], inp["S0"],
                             cu_seqlens=cu, out=out, S_final=Sf, chunk=w.chunk)
+        if args.fused:
+            # the same tensors read as raw inputs: alpha and beta as logits, q and k unnormalised
+            def step():
+                kda.kda_forward_fused(inp["q"], inp["k"], inp["v"], inp["alpha"], inp["beta"],
+                                      inp["S0"], cu_seqlens=cu, out=out, S_final=Sf, chunk=w.chunk)
         if args.seqpar and w.kind == "forward":
             # this rank's time segment; maps exchanged through the process group
             from gated_delta_rule_138_b200.seqpar import kda_forward_sequence_parallel, split_time
@@ -476,6 +481,8 @@ def run_ours(args, w):
         achieved = algo_bytes / share / (kern_ms * 1e-3) / 1e9
         tflops = algo_flops / share / (kern_ms * 1e-3) / 1e12
         cfg = config_of(w, world)
+        if args.fused:
+            cfg["inputs"] = "raw: gate logits, unnormalised q and k (kda_forward_fused)"
         if seqpar:
             cfg["parallelism"] = "sequence x%d (time segments per rank, maps all-gathered)" % world
         line = {
@@ -573,6 +580,9 @@ def main():
     ap.add_argument("--cpu-budget", type=float, default=15.0,
                     help="seconds of oracle time for the cpu_baseline sample")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--fused", action="store_true",
+                    help="forward workloads through kda_forward_fused (gates as logits, q and k "
+                         "normalised inside the kernel)")
     ap.add_argument("--seqpar", action="store_true",
                     help="split every sequence's time axis across the ranks (strong scaling)")
     ap.add_argument("--e2e-steps", type=int, default=10,

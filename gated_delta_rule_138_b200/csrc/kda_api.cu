@@ -21,11 +21,12 @@ cudaError_t launch_chunk_simt(int in_bf16, int out_bf16, int chunk, const void* 
 cudaError_t launch_decode(int in_bf16, int out_bf16, const void* q, const void* k, const void* v,
                           const void* alpha, const void* beta, float* S, void* out, int64_t NH,
                           int DK, int DV, cudaStream_t s, const int32_t* slots, int num_slots,
-                          int H, int T = 1);
+                          int H, int T = 1, int fused = 0);
 cudaError_t launch_chunk_tc(const void* q, const void* k, const void* v, const void* alpha,
                             const void* beta, const float* S0, const int32_t* cu, int nseq,
                             void* out, float* S_final, int64_t rows, int64_t T, int H, int* status,
-                            cudaStream_t stream, const int32_t* slots = nullptr, int num_slots = 0);
+                            cudaStream_t stream, const int32_t* slots = nullptr, int num_slots = 0,
+                            int fused = 0);
 size_t chunk_tc_segmented_workspace_floats(int64_t nseq, int H, int nseg);
 cudaError_t launch_segment_maps(const void* k, const void* v, const void* alpha, const void* beta,
                                 const int32_t* cu, int nseq, float* maps, int64_t rows, int64_t T,
@@ -36,7 +37,7 @@ cudaError_t launch_chunk_tc_segmented(const void* q, const void* k, const void* 
                                       const void* alpha, const void* beta, const float* S0,
                                       const int32_t* cu, int nseq, void* out, float* S_final,
                                       int64_t rows, int64_t T, int H, int nseg, float* workspace,
-                                      int* status, cudaStream_t stream);
+                                      int* status, cudaStream_t stream, int fused = 0);
 }  // namespace kda
 
 namespace {
@@ -217,11 +218,18 @@ kda_status_t kda_selftest_timeout(uint64_t limit_ns, kda_stream_t stream) {
     return cuda_status(cudaGetLastError());
 }
 
-kda_status_t kda_forward(const void* q, const void* k, const void* v, const void* alpha,
-                         const void* beta, const float* S0, const int32_t* cu_seqlens,
-                         int32_t num_seqs, void* out, float* S_final, int32_t B, int64_t T,
-                         int32_t H, int32_t d_k, int32_t d_v, int32_t chunk,
-                         kda_dtype_t in_dtype, kda_dtype_t out_dtype, kda_stream_t stream) {
+}  // extern "C"
+
+namespace {
+
+// kda_forward and kda_forward_fused; `fused`: logits for alpha and beta, q and k
+// unnormalised (tensor-core kernel only).
+kda_status_t forward_impl(const void* q, const void* k, const void* v, const void* alpha,
+                          const void* beta, const float* S0, const int32_t* cu_seqlens,
+                          int32_t num_seqs, void* out, float* S_final, int32_t B, int64_t T,
+                          int32_t H, int32_t d_k, int32_t d_v, int32_t chunk,
+                          kda_dtype_t in_dtype, kda_dtype_t out_dtype, kda_stream_t stream,
+                          int fused) {
     if (B < 0 || T < 0 || H <= 0 || !is_dtype(in_dtype) || !is_dtype(out_dtype))
         return KDA_ERR_INVALID_ARG;
     if (cu_seqlens != nullptr && (B != 1 || num_seqs < 0)) return KDA_ERR_INVALID_ARG;
@@ -236,6 +244,11 @@ kda_status_t kda_forward(const void* q, const void* k, const void* v, const void
     if (!head_dim_ok(d_k) || !head_dim_ok(d_v)) return KDA_ERR_UNSUPPORTED;
     if (chunk != 16 && chunk != 32 && chunk != 64) return KDA_ERR_UNSUPPORTED;
     if (nseq > 65535 || H > 65535) return KDA_ERR_UNSUPPORTED;  // grid y/z limits
+    if (fused && !use_tc(d_k, d_v, chunk, in_dtype, out_dtype)) {
+        std::snprintf(g_last_error, sizeof(g_last_error),
+                      "kda_forward_fused: only bf16 in/out, d_k = d_v = 128, chunk 64");
+        return KDA_ERR_UNSUPPORTED;
+    }
     if (nseq == 0) return KDA_OK;
     g_last_error[0] = '\0';
     const cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
@@ -262,12 +275,13 @@ kda_status_t kda_forward(const void* q, const void* k, const void* v, const void
         if (ws) {
             g_launches.fetch_add(2, std::memory_order_relaxed);   // three kernels in all
             e = kda::launch_chunk_tc_segmented(q, k, v, alpha, beta, S0, cu_seqlens, (int)nseq,
-                                               out, S_final, rows, T, H, nseg, ws, status, s);
+                                               out, S_final, rows, T, H, nseg, ws, status, s,
+                                               fused);
             const cudaError_t ef = cudaFreeAsync(ws, s);
             if (e == cudaSuccess) e = ef;
         } else {
             e = kda::launch_chunk_tc(q, k, v, alpha, beta, S0, cu_seqlens, (int)nseq, out, S_final,
-                                     rows, T, H, status, s);
+                                     rows, T, H, status, s, nullptr, 0, fused);
         }
         if (e != cudaSuccess) return cuda_status(e);
         return debug_sync() ? kda_device_status(stream) : KDA_OK;
@@ -275,6 +289,29 @@ kda_status_t kda_forward(const void* q, const void* k, const void* v, const void
     return cuda_status(kda::launch_chunk_simt(in_bf16, out_bf16, chunk, q, k, v, alpha, beta, S0,
                                               cu_seqlens, (int)nseq, out, S_final, T, H, d_k, d_v,
                                               s));
+}
+
+}  // namespace
+
+extern "C" {
+
+kda_status_t kda_forward(const void* q, const void* k, const void* v, const void* alpha,
+                         const void* beta, const float* S0, const int32_t* cu_seqlens,
+                         int32_t num_seqs, void* out, float* S_final, int32_t B, int64_t T,
+                         int32_t H, int32_t d_k, int32_t d_v, int32_t chunk,
+                         kda_dtype_t in_dtype, kda_dtype_t out_dtype, kda_stream_t stream) {
+    return forward_impl(q, k, v, alpha, beta, S0, cu_seqlens, num_seqs, out, S_final, B, T, H, d_k,
+                        d_v, chunk, in_dtype, out_dtype, stream, 0);
+}
+
+kda_status_t kda_forward_fused(const void* q, const void* k, const void* v,
+                               const void* alpha_logits, const void* beta_logits, const float* S0,
+                               const int32_t* cu_seqlens, int32_t num_seqs, void* out,
+                               float* S_final, int32_t B, int64_t T, int32_t H, int32_t d_k,
+                               int32_t d_v, int32_t chunk, kda_dtype_t in_dtype,
+                               kda_dtype_t out_dtype, kda_stream_t stream) {
+    return forward_impl(q, k, v, alpha_logits, beta_logits, S0, cu_seqlens, num_seqs, out, S_final,
+                        B, T, H, d_k, d_v, chunk, in_dtype, out_dtype, stream, 1);
 }
 
 kda_status_t kda_forward_indexed(const void* q, const void* k, const void* v, const void* alpha,
@@ -401,10 +438,10 @@ kda_status_t kda_segment_scan(const float* S0, const float* maps, int32_t num_ma
                                               reinterpret_cast<cudaStream_t>(stream)));
 }
 
-kda_status_t kda_decode_step(const void* q, const void* k, const void* v, const void* alpha,
+static kda_status_t decode_impl(const void* q, const void* k, const void* v, const void* alpha,
                              const void* beta, float* S, void* out, int32_t N, int32_t H,
                              int32_t d_k, int32_t d_v, kda_dtype_t in_dtype,
-                             kda_dtype_t out_dtype, kda_stream_t stream) {
+                             kda_dtype_t out_dtype, kda_stream_t stream, int fused) {
     if (N < 0 || H <= 0 || !is_dtype(in_dtype) || !is_dtype(out_dtype))
         return KDA_ERR_INVALID_ARG;
     if (N > 0 && (!q || !k || !v || !alpha || !beta || !S || !out)) return KDA_ERR_INVALID_ARG;
@@ -422,7 +459,24 @@ kda_status_t kda_decode_step(const void* q, const void* k, const void* v, const 
     const cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
     g_launches.fetch_add(1, std::memory_order_relaxed);
     return cuda_status(kda::launch_decode(in_dtype == KDA_BF16, out_dtype == KDA_BF16, q, k, v,
-                                          alpha, beta, S, out, NH, d_k, d_v, s, nullptr, 0, H));
+                                          alpha, beta, S, out, NH, d_k, d_v, s, nullptr, 0, H, 1,
+                                          fused));
+}
+
+kda_status_t kda_decode_step(const void* q, const void* k, const void* v, const void* alpha,
+                             const void* beta, float* S, void* out, int32_t N, int32_t H,
+                             int32_t d_k, int32_t d_v, kda_dtype_t in_dtype,
+                             kda_dtype_t out_dtype, kda_stream_t stream) {
+    return decode_impl(q, k, v, alpha, beta, S, out, N, H, d_k, d_v, in_dtype, out_dtype, stream, 0);
+}
+
+kda_status_t kda_decode_step_fused(const void* q, const void* k, const void* v,
+                                   const void* alpha_logits, const void* beta_logits, float* S,
+                                   void* out, int32_t N, int32_t H, int32_t d_k, int32_t d_v,
+                                   kda_dtype_t in_dtype, kda_dtype_t out_dtype,
+                                   kda_stream_t stream) {
+    return decode_impl(q, k, v, alpha_logits, beta_logits, S, out, N, H, d_k, d_v, in_dtype,
+                       out_dtype, stream, 1);
 }
 
 }  // extern "C"

@@ -162,7 +162,9 @@ struct LoadTrack {
 // kCtaStatus = false: a timed-out wait sets the shared word *status to 1.
 // kCtaStatus = true:  every CTA writes its own word status[n * H + h] (0 or 1).
 // kSummary = true: the segment-map mode described at the top (q and out unused).
-template <bool kCtaStatus, bool kSummary>
+// kFused = true: alpha and beta arrive as logits (alpha = 1/(1+e^x), beta =
+// sigmoid(x)) and q, k unnormalised (L2-normalised per token and head here).
+template <bool kCtaStatus, bool kSummary, bool kFused>
 __global__ void __launch_bounds__(NTHREADS, 1)
 kda_chunk_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                     const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmV,
@@ -380,8 +382,13 @@ kda_chunk_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_consta
     tc_fence_after();
 
     // beta of the next chunk is loaded one chunk ahead, into a register
+    constexpr bool fused = kFused;
+    auto load_beta = [&](int64_t token) {   // token index in the segment, < len
+        const float x = __bfloat162float(beta[(size_t)(bos + token) * H + h]);
+        return fused ? sigmoid_f(x) : x;
+    };
     float beta_next = 0.0f;
-    if (tid < C && tid < len) beta_next = __bfloat162float(beta[(size_t)(bos + tid) * H + h]);
+    if (tid < C && tid < len) beta_next = load_beta(tid);
 
     bool broke = false;
     if (compute)
@@ -421,7 +428,8 @@ kda_chunk_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_consta
                 float a[4];
                 unpack4_bf16(*reinterpret_cast<const uint2*>(sAl + off), a);
 #pragma unroll
-                for (int c = 0; c < 4; ++c) psi[i][c] = r < Lc ? clamp_gate(a[c]) : 1.0f;
+                for (int c = 0; c < 4; ++c)
+                    psi[i][c] = r < Lc ? clamp_gate(fused ? gate_from_logit(a[c]) : a[c]) : 1.0f;
             }
             {
                 float p[4] = {1.f, 1.f, 1.f, 1.f}, b[4] = {1.f, 1.f, 1.f, 1.f};
@@ -478,6 +486,31 @@ kda_chunk_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_consta
                     ag[c] = aft * gO;
                 }
             }
+            // fused inputs: k and q rows L2-normalised in place (bf16), before any
+            // operand is formed.  A warp holds all 128 channels of its eight rows, four
+            // per lane, and each thread rewrites only the elements it reads again below.
+            if constexpr (kFused) {
+#pragma unroll
+                for (int i = 0; i < 8; ++i) {
+                    const int r = 8 * O + i;
+                    const uint32_t in_off = a64 * 8192u + (uint32_t)r * 128u + (((chk ^ (uint32_t)r) & 7u) << 4) + inner;
+                    float k[4], q[4] = {0.f, 0.f, 0.f, 0.f};
+                    unpack4_bf16(*reinterpret_cast<const uint2*>(sK + in_off), k);
+                    if (!kSummary) unpack4_bf16(*reinterpret_cast<const uint2*>(sQc + in_off), q);
+                    float sk = k[0] * k[0] + k[1] * k[1] + k[2] * k[2] + k[3] * k[3];
+                    float sq = q[0] * q[0] + q[1] * q[1] + q[2] * q[2] + q[3] * q[3];
+#pragma unroll
+                    for (int o = 16; o > 0; o >>= 1) {
+                        sk += __shfl_xor_sync(0xffffffffu, sk, o);
+                        sq += __shfl_xor_sync(0xffffffffu, sq, o);
+                    }
+                    const float ik = rsqrtf(fmaxf(sk, 1e-12f)), iq = rsqrtf(fmaxf(sq, 1e-12f));
+#pragma unroll
+                    for (int c = 0; c < 4; ++c) { k[c] *= ik; q[c] *= iq; }
+                    st4_bf16(sK + in_off, k);
+                    if (!kSummary) st4_bf16(sQc + in_off, q);
+                }
+            }
 #pragma unroll
             for (int i = 0; i < 8; ++i) {
                 const int r = 8 * O + i;
@@ -486,6 +519,7 @@ kda_chunk_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_consta
                 float k[4], q[4] = {0.f, 0.f, 0.f, 0.f};
                 unpack4_bf16(*reinterpret_cast<const uint2*>(sK + in_off), k);
                 if (!kSummary) unpack4_bf16(*reinterpret_cast<const uint2*>(sQc + in_off), q);
+
                 if (r >= Lc) {
 #pragma unroll
                     for (int c = 0; c < 4; ++c) { k[c] = 0.0f; q[c] = 0.0f; }
@@ -780,7 +814,7 @@ kda_chunk_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_consta
         wait_mma();
         if (tid < C) {
             const int64_t nxt = (int64_t)(chunk + 1) * C + tid;   // token index in the segment
-            beta_next = nxt < len ? __bfloat162float(beta[(size_t)(bos + nxt) * H + h]) : 0.0f;
+            beta_next = nxt < len ? load_beta(nxt) : 0.0f;
         }
         {   // U rows j = 16 q4 + lane: MN-major B [64 j][256 n], four 8 KB atoms
 #pragma unroll
@@ -817,7 +851,7 @@ kda_chunk_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_consta
         wait_mma();
         if (tid < C) {
             const int64_t nxt = (int64_t)(chunk + 1) * C + tid;   // token index in the segment
-            beta_next = nxt < len ? __bfloat162float(beta[(size_t)(bos + nxt) * H + h]) : 0.0f;
+            beta_next = nxt < len ? load_beta(nxt) : 0.0f;
         }
         {   // U as the MN-major B operand [64 j][128 n]: rows j = 16 q4 + lane (lane < 16)
             float v[64];
@@ -1214,16 +1248,16 @@ static bool make_maps(TcMaps* m, const void* q, const void* k, const void* v, co
            tc::make_map(&m->o, out ? out : v, rows, H);
 }
 
-template <bool kCtaStatus, bool kSummary>
+template <bool kCtaStatus, bool kSummary, bool kFused = false>
 static cudaError_t launch_tc_t(const TcMaps& m, const void* beta, const float* S0, const int32_t* cu,
                                int nseq, void* out, float* S_final, int64_t T, int H, int* status,
                                const tc::Segments& seg, cudaStream_t stream) {
-    cudaError_t e = cudaFuncSetAttribute(tc::kda_chunk_tc_kernel<kCtaStatus, kSummary>,
+    cudaError_t e = cudaFuncSetAttribute(tc::kda_chunk_tc_kernel<kCtaStatus, kSummary, kFused>,
                                          cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          (int)tc::SMEM_BYTES);
     if (e != cudaSuccess) return e;
     dim3 grid(1, H, nseq * seg.per_seq);
-    tc::kda_chunk_tc_kernel<kCtaStatus, kSummary><<<grid, tc::NTHREADS, tc::SMEM_BYTES, stream>>>(
+    tc::kda_chunk_tc_kernel<kCtaStatus, kSummary, kFused><<<grid, tc::NTHREADS, tc::SMEM_BYTES, stream>>>(
         m.q, m.k, m.a, m.v, m.o, (const __nv_bfloat16*)beta, S0, cu, (__nv_bfloat16*)out, S_final, T, H,
         status, seg);
     return cudaGetLastError();
@@ -1232,12 +1266,14 @@ static cudaError_t launch_tc_t(const TcMaps& m, const void* beta, const float* S
 cudaError_t launch_chunk_tc(const void* q, const void* k, const void* v, const void* alpha,
                             const void* beta, const float* S0, const int32_t* cu, int nseq,
                             void* out, float* S_final, int64_t rows, int64_t T, int H, int* status,
-                            cudaStream_t stream, const int32_t* slots, int num_slots) {
+                            cudaStream_t stream, const int32_t* slots, int num_slots, int fused) {
     TcMaps m;
     if (!make_maps(&m, q, k, v, alpha, out, rows, H)) return cudaErrorInvalidValue;
     const tc::Segments whole{1, 1, nullptr, nullptr, slots, num_slots};
-    return launch_tc_t<false, false>(m, beta, S0, cu, nseq, out, S_final, T, H, status, whole,
-                                     stream);
+    return fused ? launch_tc_t<false, false, true>(m, beta, S0, cu, nseq, out, S_final, T, H, status,
+                                                   whole, stream)
+                 : launch_tc_t<false, false>(m, beta, S0, cu, nseq, out, S_final, T, H, status,
+                                             whole, stream);
 }
 
 // Floats of workspace the split forward uses: the segment maps [M | N] and the
@@ -1254,23 +1290,27 @@ cudaError_t launch_chunk_tc_segmented(const void* q, const void* k, const void* 
                                       const void* alpha, const void* beta, const float* S0,
                                       const int32_t* cu, int nseq, void* out, float* S_final,
                                       int64_t rows, int64_t T, int H, int nseg, float* workspace,
-                                      int* status, cudaStream_t stream) {
+                                      int* status, cudaStream_t stream, int fused) {
     if (nseg < 2 || nseq * (int64_t)nseg > 65535) return cudaErrorInvalidValue;
     TcMaps m;
     if (!make_maps(&m, q, k, v, alpha, out, rows, H)) return cudaErrorInvalidValue;
     float* maps = workspace;
     float* start = workspace + (size_t)nseq * H * (nseg - 1) * tc::DK * (tc::DK + tc::DV);
     const tc::Segments summary{nseg, nseg - 1, nullptr, maps};
-    cudaError_t e = launch_tc_t<false, true>(m, beta, nullptr, cu, nseq, nullptr, nullptr, T, H,
-                                             status, summary, stream);
+    cudaError_t e = fused ? launch_tc_t<false, true, true>(m, beta, nullptr, cu, nseq, nullptr,
+                                                           nullptr, T, H, status, summary, stream)
+                          : launch_tc_t<false, true>(m, beta, nullptr, cu, nseq, nullptr, nullptr, T,
+                                                     H, status, summary, stream);
     if (e != cudaSuccess) return e;
     tc::kda_segment_scan_kernel<<<dim3(tc::DV / tc::SCAN_COLS, H, nseq), tc::DK, 0, stream>>>(
         S0, maps, start, nseg, H);
     e = cudaGetLastError();
     if (e != cudaSuccess) return e;
     const tc::Segments fwd{nseg, nseg, start, nullptr};
-    return launch_tc_t<false, false>(m, beta, nullptr, cu, nseq, out, S_final, T, H, status, fwd,
-                                     stream);
+    return fused ? launch_tc_t<false, false, true>(m, beta, nullptr, cu, nseq, out, S_final, T, H,
+                                                   status, fwd, stream)
+                 : launch_tc_t<false, false>(m, beta, nullptr, cu, nseq, out, S_final, T, H, status,
+                                             fwd, stream);
 }
 
 // Segment maps of whole sequences: maps [nseq][H][DK][DK + DV] fp32 with

@@ -26,7 +26,7 @@ __global__ void __launch_bounds__(256)
 kda_decode_kernel(const Tin* __restrict__ q, const Tin* __restrict__ k,
                   const Tin* __restrict__ v, const Tin* __restrict__ alpha,
                   const Tin* __restrict__ beta, float* __restrict__ S, Tout* __restrict__ out,
-                  const int32_t* __restrict__ slots, int num_slots, int H, int T) {
+                  const int32_t* __restrict__ slots, int num_slots, int H, int T, int fused) {
     constexpr int NT = 256;
     constexpr int TX = DV / 4;       // threads across a row (float4 each)
     constexpr int TY = NT / TX;      // rows per pass
@@ -35,7 +35,7 @@ kda_decode_kernel(const Tin* __restrict__ q, const Tin* __restrict__ k,
     __shared__ float ka[DK], qa[DK], kk[DK], ga[DK];
     __shared__ float red_x[TY][DV], red_y[TY][DV];
     __shared__ float us[DV];
-    __shared__ float kq_part[NT / 32];
+    __shared__ float kq_part[NT / 32], nk_part[NT / 32], nq_part[NT / 32];
 
     const int tid = threadIdx.x, tx = tid % TX, ty = tid / TX;
     const size_t nh = blockIdx.x;                 // (sequence, head) flattened
@@ -56,10 +56,33 @@ kda_decode_kernel(const Tin* __restrict__ q, const Tin* __restrict__ k,
     const size_t tok = ((size_t)n * T + t) * H + hh;   // (sequence, token, head)
     const size_t kb = tok * DK, vb = tok * DV;
     if (t > 0) __syncthreads();   // the previous token's update has read ga, kk and us
+    // fused inputs: alpha and beta are logits, q and k are L2-normalised here
+    float ikn = 1.0f, iqn = 1.0f;
+    if (fused) {
+        float pk = 0.0f, pq = 0.0f;
+        if (tid < DK) {
+            const float kv = to_f32(k[kb + tid]), qv = to_f32(q[kb + tid]);
+            pk = kv * kv;
+            pq = qv * qv;
+        }
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) {
+            pk += __shfl_xor_sync(0xffffffffu, pk, o);
+            pq += __shfl_xor_sync(0xffffffffu, pq, o);
+        }
+        if ((tid & 31) == 0) { nk_part[tid >> 5] = pk; nq_part[tid >> 5] = pq; }
+        __syncthreads();
+        float sk = 0.0f, sq = 0.0f;
+#pragma unroll
+        for (int i = 0; i < NT / 32; ++i) { sk += nk_part[i]; sq += nq_part[i]; }
+        ikn = rsqrtf(fmaxf(sk, 1e-12f));
+        iqn = rsqrtf(fmaxf(sq, 1e-12f));
+    }
     float kqp = 0.0f;
     if (tid < DK) {
-        const float a = clamp_gate(to_f32(alpha[kb + tid]));
-        const float kv = to_f32(k[kb + tid]), qv = to_f32(q[kb + tid]);
+        const float ax = to_f32(alpha[kb + tid]);
+        const float a = clamp_gate(fused ? gate_from_logit(ax) : ax);
+        const float kv = to_f32(k[kb + tid]) * ikn, qv = to_f32(q[kb + tid]) * iqn;
         ga[tid] = a;
         ka[tid] = a * kv;
         qa[tid] = a * qv;
@@ -92,7 +115,8 @@ kda_decode_kernel(const Tin* __restrict__ q, const Tin* __restrict__ k,
         float kq = 0.0f;
 #pragma unroll
         for (int i = 0; i < NT / 32; ++i) kq += kq_part[i];
-        const float b = to_f32(beta[tok]);
+        const float bx = to_f32(beta[tok]);
+        const float b = fused ? sigmoid_f(bx) : bx;
         const float u = b * (to_f32(v[vb + tid]) - x);
         us[tid] = u;
         out[vb + tid] = from_f32<Tout>(fmaf(u, kq, y));
@@ -123,10 +147,10 @@ template <typename Tin, typename Tout, int DK, int DV>
 static cudaError_t launch_decode_t(const void* q, const void* k, const void* v, const void* alpha,
                                    const void* beta, float* S, void* out, int64_t NH,
                                    cudaStream_t stream, const int32_t* slots, int num_slots, int H,
-                                   int T) {
+                                   int T, int fused) {
     kda_decode_kernel<Tin, Tout, DK, DV><<<(unsigned)NH, 256, 0, stream>>>(
         (const Tin*)q, (const Tin*)k, (const Tin*)v, (const Tin*)alpha, (const Tin*)beta, S,
-        (Tout*)out, slots, num_slots, H, T);
+        (Tout*)out, slots, num_slots, H, T, fused);
     return cudaGetLastError();
 }
 
@@ -134,21 +158,21 @@ template <typename Tin, typename Tout>
 static cudaError_t launch_decode_d(int DK, int DV, const void* q, const void* k, const void* v,
                                    const void* alpha, const void* beta, float* S, void* out,
                                    int64_t NH, cudaStream_t s, const int32_t* slots, int num_slots,
-                                   int H, int T) {
-    if (DK == 64 && DV == 64) return launch_decode_t<Tin, Tout, 64, 64>(q, k, v, alpha, beta, S, out, NH, s, slots, num_slots, H, T);
-    if (DK == 64 && DV == 128) return launch_decode_t<Tin, Tout, 64, 128>(q, k, v, alpha, beta, S, out, NH, s, slots, num_slots, H, T);
-    if (DK == 128 && DV == 64) return launch_decode_t<Tin, Tout, 128, 64>(q, k, v, alpha, beta, S, out, NH, s, slots, num_slots, H, T);
-    return launch_decode_t<Tin, Tout, 128, 128>(q, k, v, alpha, beta, S, out, NH, s, slots, num_slots, H, T);
+                                   int H, int T, int fused) {
+    if (DK == 64 && DV == 64) return launch_decode_t<Tin, Tout, 64, 64>(q, k, v, alpha, beta, S, out, NH, s, slots, num_slots, H, T, fused);
+    if (DK == 64 && DV == 128) return launch_decode_t<Tin, Tout, 64, 128>(q, k, v, alpha, beta, S, out, NH, s, slots, num_slots, H, T, fused);
+    if (DK == 128 && DV == 64) return launch_decode_t<Tin, Tout, 128, 64>(q, k, v, alpha, beta, S, out, NH, s, slots, num_slots, H, T, fused);
+    return launch_decode_t<Tin, Tout, 128, 128>(q, k, v, alpha, beta, S, out, NH, s, slots, num_slots, H, T, fused);
 }
 
 cudaError_t launch_decode(int in_bf16, int out_bf16, const void* q, const void* k, const void* v,
                           const void* alpha, const void* beta, float* S, void* out, int64_t NH,
                           int DK, int DV, cudaStream_t s, const int32_t* slots, int num_slots,
-                          int H, int T) {
-    if (!in_bf16 && !out_bf16) return launch_decode_d<float, float>(DK, DV, q, k, v, alpha, beta, S, out, NH, s, slots, num_slots, H, T);
-    if (!in_bf16 && out_bf16) return launch_decode_d<float, __nv_bfloat16>(DK, DV, q, k, v, alpha, beta, S, out, NH, s, slots, num_slots, H, T);
-    if (in_bf16 && !out_bf16) return launch_decode_d<__nv_bfloat16, float>(DK, DV, q, k, v, alpha, beta, S, out, NH, s, slots, num_slots, H, T);
-    return launch_decode_d<__nv_bfloat16, __nv_bfloat16>(DK, DV, q, k, v, alpha, beta, S, out, NH, s, slots, num_slots, H, T);
+                          int H, int T, int fused) {
+    if (!in_bf16 && !out_bf16) return launch_decode_d<float, float>(DK, DV, q, k, v, alpha, beta, S, out, NH, s, slots, num_slots, H, T, fused);
+    if (!in_bf16 && out_bf16) return launch_decode_d<float, __nv_bfloat16>(DK, DV, q, k, v, alpha, beta, S, out, NH, s, slots, num_slots, H, T, fused);
+    if (in_bf16 && !out_bf16) return launch_decode_d<__nv_bfloat16, float>(DK, DV, q, k, v, alpha, beta, S, out, NH, s, slots, num_slots, H, T, fused);
+    return launch_decode_d<__nv_bfloat16, __nv_bfloat16>(DK, DV, q, k, v, alpha, beta, S, out, NH, s, slots, num_slots, H, T, fused);
 }
 
 }  // namespace kda

@@ -87,6 +87,10 @@ def load_library(build_if_missing: bool = True) -> ctypes.CDLL:
     lib.kda_selftest_timeout.argtypes = [ctypes.c_uint64, vp]
     lib.kda_forward_noalloc.restype = ctypes.c_int
     lib.kda_forward_noalloc.argtypes = lib.kda_forward.argtypes
+    lib.kda_forward_fused.restype = ctypes.c_int
+    lib.kda_forward_fused.argtypes = lib.kda_forward.argtypes
+    lib.kda_decode_step_fused.restype = ctypes.c_int
+    lib.kda_decode_step_fused.argtypes = lib.kda_decode_step.argtypes
     lib.kda_forward_indexed.restype = ctypes.c_int
     lib.kda_forward_indexed.argtypes = [vp, vp, vp, vp, vp, vp, i32, vp, vp, i32, vp,
                                         i32, i64, i32, i32, i32, i32, ctypes.c_int, ctypes.c_int, vp]
@@ -343,4 +347,50 @@ def kda_decode_step_indexed(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor,
                                      int(N), int(H), int(dk), int(dv), _dt(q), _dt(out),
                                      _stream(stream))
     _check("kda_decode_step_indexed", st)
+    return out
+
+
+def kda_forward_fused(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor,
+                      alpha_logits: torch.Tensor, beta_logits: torch.Tensor,
+                      S0: Optional[torch.Tensor] = None, cu_seqlens: Optional[torch.Tensor] = None,
+                      out: Optional[torch.Tensor] = None, S_final: Optional[torch.Tensor] = None,
+                      chunk: int = 64, stream=None) -> Tuple[torch.Tensor, Optional[torch.Tensor]]:
+    """kda_forward from raw inputs: alpha = 1/(1 + e^x), beta = sigmoid(y), q and k
+    L2-normalised per (token, head) inside the kernel (bf16, d = 128)."""
+    lib = load_library()
+    B, T, H, dk = q.shape
+    dv = v.shape[-1]
+    for name, t in (("q", q), ("k", k), ("v", v), ("alpha_logits", alpha_logits),
+                    ("beta_logits", beta_logits), ("S0", S0), ("cu_seqlens", cu_seqlens)):
+        _contig(name, t)
+    nseq = B if cu_seqlens is None else cu_seqlens.numel() - 1
+    if out is None:
+        out = torch.empty(B, T, H, dv, dtype=q.dtype, device=q.device)
+    if S_final is None:
+        S_final = torch.empty(nseq, H, dk, dv, dtype=torch.float32, device=q.device)
+    st = lib.kda_forward_fused(_ptr(q), _ptr(k), _ptr(v), _ptr(alpha_logits), _ptr(beta_logits),
+                               _ptr(S0), _ptr(cu_seqlens), int(nseq), _ptr(out), _ptr(S_final),
+                               int(B), int(T), int(H), int(dk), int(dv), int(chunk), _dt(q),
+                               _dt(out), _stream(stream))
+    _check("kda_forward_fused", st)
+    return out, S_final
+
+
+def kda_decode_step_fused(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor,
+                          alpha_logits: torch.Tensor, beta_logits: torch.Tensor, S: torch.Tensor,
+                          out: Optional[torch.Tensor] = None,
+                          out_dtype: Optional[torch.dtype] = None, stream=None) -> torch.Tensor:
+    """kda_decode_step from raw inputs (see kda_forward_fused); S updated in place."""
+    lib = load_library()
+    N, H, dk = q.shape
+    dv = v.shape[-1]
+    for name, t in (("q", q), ("k", k), ("v", v), ("alpha_logits", alpha_logits),
+                    ("beta_logits", beta_logits), ("S", S)):
+        _contig(name, t)
+    if out is None:
+        out = torch.empty(N, H, dv, dtype=out_dtype or q.dtype, device=q.device)
+    st = lib.kda_decode_step_fused(_ptr(q), _ptr(k), _ptr(v), _ptr(alpha_logits),
+                                   _ptr(beta_logits), _ptr(S), _ptr(out), int(N), int(H), int(dk),
+                                   int(dv), _dt(q), _dt(out), _stream(stream))
+    _check("kda_decode_step_fused", st)
     return out

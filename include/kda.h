@@ -154,6 +154,33 @@ kda_status_t kda_segment_scan(const float* S0, const float* maps, int32_t num_ma
                               kda_stream_t stream);
 
 /*
+ * Fused input-side transforms (no counterpart on the pages: the forms that the
+ * gates and keys take before the update).  Same arguments and layouts as
+ * kda_forward / kda_decode_step, but:
+ *   alpha_logits x : the gate is alpha = exp(-softplus(x)) = 1 / (1 + e^x), then
+ *                    clamped to [e^-5, 1] as usual;
+ *   beta_logits  y : beta = sigmoid(y) = 1 / (1 + e^-y);
+ *   q, k           : raw; each (token, head) vector is L2-normalised inside
+ *                    (q / sqrt(max(||q||^2, 1e-12))), in fp32.
+ * The transforms run inside the kernels that consume the inputs, so no extra
+ * pass over the inputs is made.  kda_forward_fused supports the tensor-core
+ * configuration only (bf16 in and out, d_k = d_v = 128, chunk 64; time
+ * segments as kda_forward); kda_decode_step_fused every configuration of
+ * kda_decode_step.  Returns as kda_forward.
+ */
+kda_status_t kda_forward_fused(const void* q, const void* k, const void* v,
+                               const void* alpha_logits, const void* beta_logits,
+                               const float* S0, const int32_t* cu_seqlens, int32_t num_seqs,
+                               void* out, float* S_final, int32_t B, int64_t T, int32_t H,
+                               int32_t d_k, int32_t d_v, int32_t chunk, kda_dtype_t in_dtype,
+                               kda_dtype_t out_dtype, kda_stream_t stream);
+kda_status_t kda_decode_step_fused(const void* q, const void* k, const void* v,
+                                   const void* alpha_logits, const void* beta_logits, float* S,
+                                   void* out, int32_t N, int32_t H, int32_t d_k, int32_t d_v,
+                                   kda_dtype_t in_dtype, kda_dtype_t out_dtype,
+                                   kda_stream_t stream);
+
+/*
  * State slots for serving (no counterpart on the pages beyond paragraph 2's
  * fixed-size state that replaces the KV cache): the states of many sequences
  * live in one pool S_pool, fp32 [num_slots, H, d_k, d_v], and each call names

@@ -112,3 +112,23 @@ def available_cores() -> int:
         return len(os.sched_getaffinity(0))
     except AttributeError:  # pragma: no cover
         return os.cpu_count() or 1
+
+
+def fused_inputs(q, k, alpha_logits, beta_logits):
+    """Input-side transforms of the fused entry points, written from their plain
+    definitions in fp64 (the pages name none of them; the workload generators draw
+    the gates this way):
+        alpha = exp(-softplus(x)) = exp(-log(1 + e^x)),   beta = 1 / (1 + e^-y),
+        q_hat = q / sqrt(max(||q||^2, 1e-12)) over the last axis (per token and head),
+        k_hat likewise.
+    Returns (q_hat, k_hat, alpha, beta) as fp64 arrays."""
+    q = np.asarray(q, dtype=np.float64)
+    k = np.asarray(k, dtype=np.float64)
+    x = np.asarray(alpha_logits, dtype=np.float64)
+    y = np.asarray(beta_logits, dtype=np.float64)
+    with np.errstate(over="ignore"):
+        alpha = np.exp(-np.log1p(np.exp(x)))
+        beta = 1.0 / (1.0 + np.exp(-y))
+    nq = np.sqrt(np.maximum((q * q).sum(-1, keepdims=True), 1e-12))
+    nk = np.sqrt(np.maximum((k * k).sum(-1, keepdims=True), 1e-12))
+    return q / nq, k / nk, alpha, beta

@@ -362,3 +362,17 @@ def test_brute_force_matrix_product(T):
             St = St + R @ (beta[s] * np.outer(k[s], v[s]))
         np.testing.assert_allclose(out[0, t, 0], St.T @ q[t], rtol=1e-13, atol=1e-14)
     np.testing.assert_allclose(Sf[0, 0], St, rtol=1e-13, atol=1e-14)
+
+
+def test_fused_input_transforms():
+    """The fused entry points' transforms against closed forms and limits."""
+    x = np.array([-30.0, -2.0, 0.0, 0.5, 3.0, 50.0, 800.0])
+    q = np.array([[3.0, 4.0], [0.0, 0.0], [1e-9, 0.0]])
+    qh, kh, a, b = oracle.fused_inputs(q, 2 * q, x, x)
+    np.testing.assert_allclose(a[:-1], 1.0 / (1.0 + np.exp(x[:-1])), rtol=1e-12, atol=0)
+    assert a[2] == 0.5 and b[2] == 0.5 and a[-1] == 0.0 and b[-1] == 1.0
+    np.testing.assert_allclose(a + b, 1.0, rtol=0, atol=1e-15)      # sigma(-x) + sigma(x) = 1
+    np.testing.assert_allclose(qh[0], [0.6, 0.8], rtol=1e-15)
+    np.testing.assert_allclose(kh[0], [0.6, 0.8], rtol=1e-15)       # scale-free
+    assert np.all(qh[1] == 0.0)                                      # zero stays zero
+    np.testing.assert_allclose(qh[2], [1e-9 / 1e-6, 0.0], rtol=1e-12)   # floored norm
