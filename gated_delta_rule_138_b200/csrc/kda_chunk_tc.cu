@@ -22,15 +22,20 @@
 //   D(r, j) = lam_r * rho^{I(r)}_j,  lam_r = e^{g_r - g_ref(I(r))},  rho^I_j = e^{g_ref(I) - g_j}
 // (g the running log-gate), every factor within [e^-80, e^80] except right
 // factors that underflow where the product itself is negligible.  All factors
-// are running products of the clamped gates; nothing evaluates exp or log.
-// So [A/beta ; P] = [k*lam ; q*lam] (k*rho^I)^T: two tcgen05 MMAs, one per I.
+// are running products of the clamped gates; nothing evaluates exp or log
+// (except the optional transforms of the fused variant).  So
+// [A/beta ; P] = [k*lam ; q*lam] [k*rho^0 ; k*rho^1]^T is one tcgen05 MMA group
+// whose columns hold both sub-chunks' right operands.
 //
-// One CTA (256 threads) owns one (sequence, head) -- or one segment of it --
-// and walks its chunks in order.  Thread 0 issues the TMA loads and the MMAs;
-// all eight warps do the element-wise work.  Loads run one chunk ahead: q
-// (double buffered) at the start of a chunk, k and alpha once the gate phase
-// has consumed them, v once U has.  TMEM (512 columns): S fp32 [0,128), O
-// [128,256), scratch accumulators [256,384), U [384,512).
+// One CTA owns one (sequence, head) -- or one segment of it -- and walks its
+// chunks in order: eight compute warps do the element-wise work, and one thread
+// of a ninth (control) warp issues every TMA copy and MMA group at the barriers
+// where the compute warps hand their operands over, so that MMA issue never
+// stalls the compute warps.  Loads run about a chunk ahead: k and alpha once the
+// gate phase has consumed them, q (double buffered) after the [A/beta ; P] MMA,
+// v once U has consumed it.  O leaves through TMA stores from a staging tile.
+// TMEM (512 columns): S fp32 [0,128), O [128,256), scratch accumulators
+// [256,384), U [384,512).
 //
 // Long sequences with few (sequence, head) pairs are also split along time
 // into segments (the prefix scan of paragraph 3, within one GPU).  Over a
