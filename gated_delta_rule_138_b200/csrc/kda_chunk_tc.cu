@@ -100,7 +100,6 @@ constexpr uint32_t X_XS = 34816;         // float scratch [32][36]
 constexpr uint32_t X_T0T = 40960;        // Tinv[0:32, 0:32]^T   [64 rows (32 used)][32]
 constexpr uint32_t X_T1 = 49152;         // Tinv[32:64, 32:64]   [64 rows (32 used)][32]
 constexpr uint32_t X_A10 = 65536;        // A[32:64, 0:32]       [32][32]
-constexpr uint32_t X_XT = 69632;         // (A10 T0)^T           [32][32]
 constexpr uint32_t X_TB = 40960;         // Tb, K-major A [64 r][64 m] (after the solve)
 constexpr uint32_t X_WQ = 0;             // -W, K-major A [64][128] (two [64][64] atoms 8 KB apart)
 constexpr uint32_t X_U = 16384;          // U, MN-major B [64 j][128 n] (two [64][64] atoms);
@@ -698,8 +697,9 @@ kda_chunk_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_consta
             }
             sync_compute();
             KDA_TC_PHASE(10);
-            // 32 -> 64 on the tensor cores (tf32):  X^T = T0^T A10^T,  Y = T1 X,
-            // Tinv[32:64, 0:32] = -Y.  Operands: fp32 K-major tiles written here.
+            // 32 -> 64 on the tensor cores (tf32): X^T = T0^T A10^T, then Y^T = X^T T1^T with
+            // X^T read back from TMEM by the second MMA; Tinv[32:64, 0:32] = -Y.  Operands:
+            // fp32 K-major tiles written here (T1 serves as the second product's B).
             {
                 uint8_t* t0t = sX + X_T0T;
                 uint8_t* t1 = sX + X_T1;
@@ -718,35 +718,17 @@ kda_chunk_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_consta
             __syncthreads();
             tc_fence_after();
             wait_mma();
-            if (q4 < 2) {   // M=64 accumulator: rows m = 16*q4 + lane live in lanes 32*q4 + lane
-                float v[32];
-                tmem_ld16(tmem + tlane + TM_WK, *reinterpret_cast<float(*)[16]>(&v[0]));
-                tmem_ld16(tmem + tlane + TM_WK + 16, *reinterpret_cast<float(*)[16]>(&v[16]));
-                tmem_wait_ld();
-                if (hf == 0 && lane < 16) {
-                    const int m = 16 * q4 + lane;
-                    uint8_t* xt = sX + X_XT;
-#pragma unroll
-                    for (int c = 0; c < 32; c += 4)
-                        *reinterpret_cast<float4*>(xt + f32_off(m, c)) = make_float4(v[c], v[c + 1], v[c + 2], v[c + 3]);
-                }
-            }
-            fence_async_smem();
-            tc_fence_before();
-            __syncthreads();
-            tc_fence_after();
-            wait_mma();
+            // both products are done: Y^T = X^T T1^T is in TMEM (M=64 rows c = 16 q4 + lane,
+            // columns r'); Tinv[32 + r', c] = -Y[r', c]
             if (q4 < 2) {
                 float v[32];
                 tmem_ld16(tmem + tlane + TM_WK + 32, *reinterpret_cast<float(*)[16]>(&v[0]));
                 tmem_ld16(tmem + tlane + TM_WK + 48, *reinterpret_cast<float(*)[16]>(&v[16]));
                 tmem_wait_ld();
                 if (hf == 0 && lane < 16) {
-                    const int r = 16 * q4 + lane;
+                    const int c = 16 * q4 + lane;
 #pragma unroll
-                    for (int c = 0; c < 32; c += 4)
-                        *reinterpret_cast<float4*>(&Tm[(32 + r) * AS + c]) =
-                            make_float4(-v[c], -v[c + 1], -v[c + 2], -v[c + 3]);
+                    for (int r = 0; r < 32; ++r) Tm[(32 + r) * AS + c] = -v[r];
                 }
             }
             tc_fence_before();
@@ -888,7 +870,8 @@ kda_chunk_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_consta
     // group in order.  Groups without a commit ride on the next group's commit (the
     // tensor pipe runs one thread's MMAs in issue order).
     //   barrier A (operands of [A/beta ; P]):  [A/beta ; P] (commit), then (q*gamma) S_start
-    //   barriers B, C (tf32 solve operands):     the two 32 -> 64 solve products (commit)
+    //   barrier B (tf32 solve operands):          the two chained 32 -> 64 solve products
+    //                                            (the second reads the first from TMEM; commit)
     //   barrier D (Tb):                          W = Tb (k*gamma) (commit), then Tb V
     //   barrier E (-W):                          U (or [U_M | U_N]) += -W S (commit)
     //   barrier F (U):                           S += (k*eta)^T U and O += P U (commit)
@@ -909,20 +892,20 @@ kda_chunk_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_consta
             mma_bf16(tmem + TM_O, sdesc_sw128(qg + (ks >> 2) * 8192 + (ks & 3) * 32),
                      sdesc_sw128(s0 + ks * 2048, 1024, 16384), idM64, ks > 0);
     };
-    auto mma_tf1 = [&]() {
+    auto mma_tf1 = [&]() {   // X^T = T0^T A10^T (no commit: the second product's covers it)
         constexpr uint32_t idesc = idesc_tf32(64, 32);
         const uint32_t a0 = smem_u32(sX + X_T0T), b0 = smem_u32(sX + X_A10);
 #pragma unroll
         for (int ks = 0; ks < 4; ++ks)
             mma_tf32(tmem + TM_WK, sdesc_sw128(a0 + ks * 32), sdesc_sw128(b0 + ks * 32), idesc, ks > 0);
-        commit_mma();
     };
-    auto mma_tf2 = [&]() {
+    auto mma_tf2 = [&]() {   // Y^T = X^T T1^T with X^T taken from TMEM (the first product)
         constexpr uint32_t idesc = idesc_tf32(64, 32);
-        const uint32_t a0 = smem_u32(sX + X_T1), b0 = smem_u32(sX + X_XT);
+        const uint32_t b0 = smem_u32(sX + X_T1);
 #pragma unroll
         for (int ks = 0; ks < 4; ++ks)
-            mma_tf32(tmem + TM_WK + 32, sdesc_sw128(a0 + ks * 32), sdesc_sw128(b0 + ks * 32), idesc, ks > 0);
+            mma_tf32_ts(tmem + TM_WK + 32, tmem + TM_WK + 8 * ks, sdesc_sw128(b0 + ks * 32), idesc,
+                        ks > 0);
         commit_mma();
     };
     auto mma_w = [&]() {
@@ -1015,12 +998,10 @@ kda_chunk_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_consta
         }
         handoff();   // B
         if (ctl) {
-            if (ok) mma_tf1();
-            wait_mma();
-        }
-        handoff();   // C
-        if (ctl) {
-            if (ok) mma_tf2();
+            if (ok) {
+                mma_tf1();
+                mma_tf2();
+            }
             wait_mma();
         }
         handoff();   // D

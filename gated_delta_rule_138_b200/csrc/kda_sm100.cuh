@@ -46,6 +46,17 @@ __device__ __forceinline__ uint64_t sdesc_sw128(uint32_t saddr, uint32_t sbo_byt
     return d;
 }
 
+// D[tmem] (+)= A[tmem] * B[smem]^T with tf32 operands, A read from tensor memory
+// (one K = 8 step: 8 consecutive 32-bit columns of A), issued by one thread.
+__device__ __forceinline__ void mma_tf32_ts(uint32_t tmem_d, uint32_t tmem_a, uint64_t bdesc,
+                                            uint32_t idesc, uint32_t accumulate) {
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "setp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::1.kind::tf32 [%0], [%1], %2, %3, p;\n\t}\n"
+        :: "r"(tmem_d), "r"(tmem_a), "l"(bdesc), "r"(idesc), "r"(accumulate));
+}
+
 // Instruction descriptor, kind::f16: D fp32, A and B bf16, dense.
 //   bits 4-5 D format (1 = f32), 7-9 A format (1 = bf16), 10-12 B format,
 //   13/14 negate A/B, 15/16 A/B major (0 = K-major, 1 = MN-major),
