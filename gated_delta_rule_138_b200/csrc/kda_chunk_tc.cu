@@ -11,12 +11,15 @@
 //   A[r,j] = beta_r sum_c k_rc k_jc D(r,j)_c  (j < r),  P[r,j] = sum_c q_rc k_jc D(r,j)_c  (j <= r)
 //   D(r,j) = prod_{s=j+1..r} a_s,   Tinv = (I + A)^-1,   Tb = Tinv diag(beta)
 //   W = Tb (k*gamma)                                   (gamma_r = prod_{s<=r} a_s)
-//   U = -W S + Tb V
+//   U = -W S + Tb V = Tb (V - (k*gamma) S)
 //   O = (q*gamma) S + P U
 //   S <- Diag(gamma_C) S + (k*eta)^T U                  (eta_j = prod_{s>j} a_s)
 //
 // Only U and the state update are sequential from chunk to chunk; O is issued
-// beside the state update.  D(r,j) never appears as a ratio of long products
+// beside the state update.  The forward mode forms V - (k*gamma) S (its product
+// issued beside [A/beta ; P], the difference taken while the solve runs) so that
+// one M=64, K=64 MMA follows the solve; the summary mode, whose state is twice
+// as wide, keeps the W form.  D(r,j) never appears as a ratio of long products
 // (64 gates >= e^-5 reach e^-320, outside fp32/bf16): with 32-token
 // sub-chunks I and the reference token ref_I = 32 I + 15,
 //   D(r, j) = lam_r * rho^{I(r)}_j,  lam_r = e^{g_r - g_ref(I(r))},  rho^I_j = e^{g_ref(I) - g_j}
@@ -35,7 +38,7 @@
 // gate phase has consumed them, q (double buffered) after the [A/beta ; P] MMA,
 // v once U has consumed it.  O leaves through TMA stores from a staging tile.
 // TMEM (512 columns): S fp32 [0,128), O [128,256), scratch accumulators
-// [256,384), U [384,512).
+// [256,384), U [384,512) (first (k*gamma) S_start, then U).
 //
 // Long sequences with few (sequence, head) pairs are also split along time
 // into segments (the prefix scan of paragraph 3, within one GPU).  Over a
@@ -82,9 +85,9 @@ constexpr uint32_t OFF_MISC = OFF_KH + 16384;
 constexpr uint32_t MISC_PI = 0;          // float [8][128] octant gate products
 constexpr uint32_t MISC_GC = 4096;       // float [128] gamma_C
 constexpr uint32_t MISC_BETA = 4608;     // float [64]
-constexpr uint32_t MISC_BAR = 4864;      // 4 x uint64 mbarriers: q, k+alpha, v, MMA
-constexpr uint32_t MISC_TMEM = 4896;     // uint32 TMEM base
-constexpr uint32_t MISC_FLAG = 4900;     // int timeout seen
+constexpr uint32_t MISC_BAR = 4864;      // 5 x uint64 mbarriers: q, k+alpha, v, MMA, (k*gamma) S
+constexpr uint32_t MISC_TMEM = 4904;     // uint32 TMEM base
+constexpr uint32_t MISC_FLAG = 4908;     // int timeout seen
 constexpr uint32_t SMEM_BYTES = OFF_MISC + 4928 + 1024;  // + alignment slack
 
 // work region X, by phase
@@ -193,6 +196,7 @@ kda_chunk_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_consta
     uint64_t* barKA = barQ + 1;
     uint64_t* barV = barQ + 2;
     uint64_t* barM = barQ + 3;
+    uint64_t* barZ = barQ + 4;   // (k*gamma) S_start, forward mode
     uint32_t* sTmem = reinterpret_cast<uint32_t*>(sm + OFF_MISC + MISC_TMEM);
     int* sFlag = reinterpret_cast<int*>(sm + OFF_MISC + MISC_FLAG);
 
@@ -230,6 +234,7 @@ kda_chunk_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_consta
         mbar_init(barKA, 1);
         mbar_init(barV, 1);
         mbar_init(barM, 1);
+        mbar_init(barZ, 1);
         mbar_fence_init();
         *sFlag = 0;
     }
@@ -304,8 +309,9 @@ kda_chunk_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_consta
     bool ok = true;   // this thread has seen every wait complete
     // asynchronous work that a timed-out wait may leave in flight, drained before exit
     LoadTrack tq, tka, tv;
-    uint32_t phM = 0, mma_out_ph = 0;
+    uint32_t phM = 0, mma_out_ph = 0, phZ = 0, z_out_ph = 0;
     bool mma_out = false;   // (control thread) an MMA group committed and not yet waited for
+    bool z_out = false;     // (control thread) the same for the (k*gamma) S group
     auto wait_load = [&](uint64_t* bar, LoadTrack& t) {
         if (ok && !mbar_wait_ns(bar, t.ph, kWaitNs)) ok = false;
         t.ph ^= 1u;
@@ -322,6 +328,19 @@ kda_chunk_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_consta
             else ok = false;
         }
         phM ^= 1u;
+        tc_fence_after();
+    };
+    auto commit_z = [&]() {
+        mma_commit(barZ);
+        z_out = true;
+        z_out_ph = phZ;
+    };
+    auto wait_z = [&]() {
+        if (ok) {
+            if (mbar_wait_ns(barZ, phZ, kWaitNs)) z_out = false;
+            else ok = false;
+        }
+        phZ ^= 1u;
         tc_fence_after();
     };
 
@@ -515,15 +534,25 @@ kda_chunk_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_consta
                     if (!kSummary) st4_bf16(sQc + in_off, q);
                 }
             }
+            // each row's k (and q) is read before the previous row's stores: q*gamma is
+            // written in place, so a load placed after a store could not be moved above it
+            auto in_off_of = [&](int r) {
+                return a64 * 8192u + (uint32_t)r * 128u + (((chk ^ (uint32_t)r) & 7u) << 4) + inner;
+            };
+            uint2 kn = *reinterpret_cast<const uint2*>(sK + in_off_of(8 * O));
+            uint2 qn = kSummary ? make_uint2(0u, 0u) : *reinterpret_cast<const uint2*>(sQc + in_off_of(8 * O));
 #pragma unroll
             for (int i = 0; i < 8; ++i) {
                 const int r = 8 * O + i;
                 const uint32_t sw = (uint32_t)r * 128u + (((chk ^ (uint32_t)r) & 7u) << 4) + inner;
                 const uint32_t in_off = a64 * 8192u + sw;    // 64-row tiles: q, k, KT, KH
                 float k[4], q[4] = {0.f, 0.f, 0.f, 0.f};
-                unpack4_bf16(*reinterpret_cast<const uint2*>(sK + in_off), k);
-                if (!kSummary) unpack4_bf16(*reinterpret_cast<const uint2*>(sQc + in_off), q);
-
+                unpack4_bf16(kn, k);
+                if (!kSummary) unpack4_bf16(qn, q);
+                if (i < 7) {
+                    kn = *reinterpret_cast<const uint2*>(sK + in_off_of(r + 1));
+                    if (!kSummary) qn = *reinterpret_cast<const uint2*>(sQc + in_off_of(r + 1));
+                }
                 if (r >= Lc) {
 #pragma unroll
                     for (int c = 0; c < 4; ++c) { k[c] = 0.0f; q[c] = 0.0f; }
@@ -664,6 +693,37 @@ kda_chunk_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_consta
                 for (int c4 = 0; c4 < 2; ++c4)
                     *reinterpret_cast<float4*>(&Tm[r2 * AS + 32 + 16 * c4 + cq]) =
                         make_float4(0.f, 0.f, 0.f, 0.f);
+                if constexpr (!kSummary) {
+                    // V - (k*gamma) S_start, written over the v tile (the MN-major B operand of
+                    // the U MMA).  (k*gamma) S_start is an M=64 accumulator in U's columns:
+                    // row j = 16 q4 + lane for lane < 16.
+                    wait_z();
+                    KDA_TC_PHASE(17);
+                    wait_load(barV, tv);
+                    KDA_TC_PHASE(18);
+                    const int j = 16 * q4 + lane;
+#pragma unroll
+                    for (int a = 0; a < 2; ++a) {
+                        float z[64];
+                        tmem_ld64(tmem + tlane + TM_U + 64 * a, z);
+                        if (lane < 16) {
+                            // each 16-byte piece is read before the previous one is written back
+                            uint4 nxt = *reinterpret_cast<const uint4*>(sV + a * 8192 + swz(j, 0));
+#pragma unroll
+                            for (int ch = 0; ch < 8; ++ch) {
+                                const uint4 raw = nxt;
+                                if (ch < 7) nxt = *reinterpret_cast<const uint4*>(sV + a * 8192 + swz(j, ch + 1));
+                                float v8[8];
+                                unpack4_bf16(make_uint2(raw.x, raw.y), *reinterpret_cast<float(*)[4]>(&v8[0]));
+                                unpack4_bf16(make_uint2(raw.z, raw.w), *reinterpret_cast<float(*)[4]>(&v8[4]));
+#pragma unroll
+                                for (int i = 0; i < 8; ++i) v8[i] -= z[8 * ch + i];
+                                *reinterpret_cast<uint4*>(sV + a * 8192 + swz(j, ch)) = pack8(v8);
+                            }
+                        }
+                    }
+                    KDA_TC_PHASE(19);
+                }
             }
             sync_compute();
             KDA_TC_PHASE(9);
@@ -756,6 +816,7 @@ kda_chunk_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_consta
         tc_fence_after();
 
         KDA_TC_PHASE(4);
+        if constexpr (kSummary) {
         // ================= W = Tb (k*gamma)   (M=64, N=128, K=64)
         wait_mma();
         {
@@ -777,6 +838,7 @@ kda_chunk_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_consta
         tc_fence_before();
         __syncthreads();
         tc_fence_after();
+        }
 
         KDA_TC_PHASE(5);
         if constexpr (kSummary) {
@@ -820,7 +882,7 @@ kda_chunk_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_consta
         KDA_TC_PHASE(6);
         // (the control warp then issues [M | N] += (k*eta)^T [U_M | U_N])
         } else {
-        // ================= U = Tb V - W S   (issued by the control warp)
+        // ================= U = Tb (V - (k*gamma) S)   (issued by the control warp)
         // meanwhile: S <- Diag(gamma_C) S in TMEM (the MMAs read the bf16 copy)
         {
             const int c = 32 * q4 + lane;
@@ -869,11 +931,13 @@ kda_chunk_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_consta
     // where the compute warps hand over their operands, and waits for each committed
     // group in order.  Groups without a commit ride on the next group's commit (the
     // tensor pipe runs one thread's MMAs in issue order).
-    //   barrier A (operands of [A/beta ; P]):  [A/beta ; P] (commit), then (q*gamma) S_start
+    //   barrier A (operands of [A/beta ; P]):  [A/beta ; P] (commit); forward: (k*gamma) S_start
+    //                                            (own barrier), then (q*gamma) S_start
     //   barrier B (tf32 solve operands):          the two chained 32 -> 64 solve products
     //                                            (the second reads the first from TMEM; commit)
-    //   barrier D (Tb):                          W = Tb (k*gamma) (commit), then Tb V
-    //   barrier E (-W):                          U (or [U_M | U_N]) += -W S (commit)
+    //   barrier D (Tb):                          forward: U = Tb (V - (k*gamma) S) (commit);
+    //                                            summary: W = Tb (k*gamma) (commit), then Tb V
+    //   barrier E (-W, summary only):            [U_M | U_N] += -W [M | N] (commit)
     //   barrier F (U):                           S += (k*eta)^T U and O += P U (commit)
     const uint32_t idM64 = idesc_bf16(64, 128, false, true);   // M=64, N=128, B MN-major
     auto mma_ap = [&]() {
@@ -884,6 +948,14 @@ kda_chunk_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_consta
             mma_bf16(tmem + TM_WK, sdesc_sw128(l0 + (ks >> 2) * 16384u + (ks & 3) * 32u),
                      sdesc_sw128(r0 + (ks >> 2) * 12288u + (ks & 3) * 32u), idesc, ks > 0);
         commit_mma();
+    };
+    auto mma_z = [&]() {   // (k*gamma) S_start into U's columns (own barrier)
+        const uint32_t kg = smem_u32(sKT), s0 = smem_u32(sS);
+#pragma unroll
+        for (int ks = 0; ks < 8; ++ks)
+            mma_bf16(tmem + TM_U, sdesc_sw128(kg + (ks >> 2) * 8192 + (ks & 3) * 32),
+                     sdesc_sw128(s0 + ks * 2048, 1024, 16384), idM64, ks > 0);
+        commit_z();
     };
     auto mma_qs = [&](uint8_t* sQc) {   // O = (q*gamma) S_start (no commit)
         const uint32_t qg = smem_u32(sQc), s0 = smem_u32(sS);
@@ -923,24 +995,16 @@ kda_chunk_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_consta
         for (int ks = 0; ks < 4; ++ks)
             mma_bf16(d, sdesc_sw128(tb + ks * 32), sdesc_sw128(v0 + ks * 2048, 1024, 8192), idM64, ks > 0);
     };
-    auto mma_u = [&]() {
+    auto mma_u = [&]() {   // summary: U_M = -W M (fresh, over W's accumulator), U_N += -W N
         const uint32_t wq = smem_u32(sX + X_WQ), s0 = smem_u32(sS);
-        if constexpr (kSummary) {
-            // U_M = -W M (fresh, over W's accumulator) and U_N += -W N
 #pragma unroll
-            for (int ks = 0; ks < 8; ++ks)
-                mma_bf16(tmem + TM_WK, sdesc_sw128(wq + (ks >> 2) * 8192 + (ks & 3) * 32),
-                         sdesc_sw128(s0 + ks * 2048, 1024, 16384), idM64, ks > 0);
+        for (int ks = 0; ks < 8; ++ks)
+            mma_bf16(tmem + TM_WK, sdesc_sw128(wq + (ks >> 2) * 8192 + (ks & 3) * 32),
+                     sdesc_sw128(s0 + ks * 2048, 1024, 16384), idM64, ks > 0);
 #pragma unroll
-            for (int ks = 0; ks < 8; ++ks)
-                mma_bf16(tmem + TM_WK + 128, sdesc_sw128(wq + (ks >> 2) * 8192 + (ks & 3) * 32),
-                         sdesc_sw128(s0 + 32768 + ks * 2048, 1024, 16384), idM64, 1);
-        } else {
-#pragma unroll
-            for (int ks = 0; ks < 8; ++ks)
-                mma_bf16(tmem + TM_U, sdesc_sw128(wq + (ks >> 2) * 8192 + (ks & 3) * 32),
-                         sdesc_sw128(s0 + ks * 2048, 1024, 16384), idM64, 1);
-        }
+        for (int ks = 0; ks < 8; ++ks)
+            mma_bf16(tmem + TM_WK + 128, sdesc_sw128(wq + (ks >> 2) * 8192 + (ks & 3) * 32),
+                     sdesc_sw128(s0 + 32768 + ks * 2048, 1024, 16384), idM64, 1);
         commit_mma();
     };
     auto mma_s = [&]() {
@@ -977,9 +1041,13 @@ kda_chunk_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_consta
         if (ctl && chunk > 0) wait_mma();   // the previous chunk's state update (and O)
         handoff();   // A
         if (ctl) {
+            KDA_TC_PHASE(20);
             if (ok) {
                 mma_ap();
-                if (!kSummary) mma_qs(sQc);
+                if (!kSummary) {
+                    mma_z();
+                    mma_qs(sQc);
+                }
             }
             if (!kSummary && chunk > 0) store_o(sQ + ((chunk + 1) & 1) * 16384, row0 - C);
             if (chunk + 1 < nchunks && ok) {   // k and alpha are consumed
@@ -987,6 +1055,7 @@ kda_chunk_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_consta
                 issued(tka);
             }
             wait_mma();
+            KDA_TC_PHASE(21);
             if (!kSummary) {
                 // the O store has read its staging buffer: load the next q there
                 bulk_wait_read_all();
@@ -994,6 +1063,8 @@ kda_chunk_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_consta
                     issue_q(row0 + C, (chunk + 1) & 1);
                     issued(tq);
                 }
+                wait_z();
+                KDA_TC_PHASE(22);
             }
         }
         handoff();   // B
@@ -1006,19 +1077,28 @@ kda_chunk_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_consta
         }
         handoff();   // D
         if (ctl) {
-            if (ok) mma_w();
-            wait_load(barV, tv);
-            if (ok) mma_tbv();
-            wait_mma();
-        }
-        handoff();   // E
-        if (ctl) {
-            if (ok) mma_u();
-            wait_mma();
-            if (chunk + 1 < nchunks && ok) {   // v is consumed
-                issue_v(row0 + C);
-                issued(tv);
+            KDA_TC_PHASE(23);
+            if constexpr (kSummary) {
+                if (ok) mma_w();
+                wait_load(barV, tv);
+                if (ok) mma_tbv();
+            } else if (ok) {
+                mma_tbv();   // U = Tb (V - (k*gamma) S), the v tile holding the difference
+                commit_mma();
             }
+            wait_mma();
+            KDA_TC_PHASE(24);
+        }
+        if constexpr (kSummary) {
+            handoff();   // E
+            if (ctl) {
+                if (ok) mma_u();
+                wait_mma();
+            }
+        }
+        if (ctl && chunk + 1 < nchunks && ok) {   // v is consumed
+            issue_v(row0 + C);
+            issued(tv);
         }
         tc_fence_before();
         const int any_timeout = __syncthreads_or(!ok);   // F, uniform: every thread leaves together
@@ -1054,6 +1134,7 @@ kda_chunk_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_consta
         if (tka.issued) mbar_wait_ns(barKA, (tka.issued - 1) & 1u, kWaitNs);
         if (tv.issued) mbar_wait_ns(barV, (tv.issued - 1) & 1u, kWaitNs);
         if (mma_out) mbar_wait_ns(barM, mma_out_ph, kWaitNs);
+        if (z_out) mbar_wait_ns(barZ, z_out_ph, kWaitNs);
     }
     __syncthreads();
     if (kCtaStatus && tid == 0) status[(size_t)n * H + h] = *sFlag;
