@@ -385,7 +385,6 @@ def run_ours(args, w):
         segments = None
         algo_bytes = decode_bytes(w, n_sh)
         algo_flops = decode_flops(w, n_sh)
-        src_file = "kda_decode.cu"
     elif w.kind == "pooled":
         # a serving step: T tokens per sequence from and into pooled state slots
         out = torch.empty(w.B, w.T, w.H, w.dv, dtype=torch.bfloat16, device=dev)
@@ -394,11 +393,12 @@ def run_ours(args, w):
         def step():
             kda.kda_forward_indexed(inp["q"], inp["k"], inp["v"], inp["alpha"], inp["beta"], pool,
                                     inp["slots"], out=out, chunk=w.chunk)
-        kname = kda.kda_forward_kernel_name(w.dk, w.dv, w.chunk, inp["q"].dtype, out.dtype)
+        # steps of at most 16 tokens run on the token-sequential kernel (state on chip)
+        kname = ("decode_f32state_steps" if w.T <= 16 else
+                 kda.kda_forward_kernel_name(w.dk, w.dv, w.chunk, inp["q"].dtype, out.dtype))
         segments = 1
         algo_bytes = forward_bytes(w, n_th, n_sh, True)   # state read and written once
         algo_flops = forward_flops(w, n_th)
-        src_file = "kda_chunk_tc.cu"
     else:
         cu = inp.get("cu_seqlens")
         B, T = inp["q"].shape[0], inp["q"].shape[1]
@@ -427,13 +427,14 @@ def run_ours(args, w):
                 kda_forward_sequence_parallel(part["q"], part["k"], part["v"], part["alpha"],
                                               part["beta"], S0)
         kname = kda.kda_forward_kernel_name(w.dk, w.dv, w.chunk, inp["q"].dtype, out.dtype)
+        if args.fused:
+            kname += "_fused"   # its own compile-time variant (no DRAM-traffic record)
         # time segments per sequence of the tensor-core path (1: unsplit); with g > 1 a
         # step is three launches (segment maps, scan, forward) timed together
         segments = (kda.kda_forward_segments(nseq, -(-B * T // nseq), w.H)
-                    if kname == "chunk_tc_bf16" else 1)
+                    if kname.startswith("chunk_tc_bf16") else 1)
         algo_bytes = forward_bytes(w, n_th, n_sh, inp["S0"] is not None)
         algo_flops = forward_flops(w, n_th)
-        src_file = "kda_chunk_tc.cu" if kname == "chunk_tc_bf16" else "kda_chunk_simt.cu"
 
     warm = max(3, args.warmup)
     for _ in range(warm):
@@ -490,7 +491,7 @@ def run_ours(args, w):
             "steps": args.steps, "warmup": warm, "ms_per_step": ms_per_step,
             "higher_is_better": True, "scaling": "strong" if seqpar else "weak",
             "vs_baseline": None,
-            "dtype": "bf16" if kname == "chunk_tc_bf16" else "f32",
+            "dtype": "bf16" if kname.startswith("chunk_tc_bf16") else "f32",
             "data": "synthetic (seeded generators, the workload's shapes and distributions)",
             "config": dict(cfg,
                            l2="no flush: inputs %.2f GB per step > 126 MB L2"

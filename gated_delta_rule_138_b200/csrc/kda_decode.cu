@@ -21,12 +21,15 @@
 
 namespace kda {
 
-template <typename Tin, typename Tout, int DK, int DV>
-__global__ void __launch_bounds__(256)
+// kFused: alpha and beta arrive as logits and q, k unnormalised (a compile-time
+// variant, so that the plain step carries none of the transforms' code)
+template <typename Tin, typename Tout, int DK, int DV, bool kFused>
+__global__ void __launch_bounds__(256, 3)
 kda_decode_kernel(const Tin* __restrict__ q, const Tin* __restrict__ k,
                   const Tin* __restrict__ v, const Tin* __restrict__ alpha,
                   const Tin* __restrict__ beta, float* __restrict__ S, Tout* __restrict__ out,
-                  const int32_t* __restrict__ slots, int num_slots, int H, int T, int fused) {
+                  const int32_t* __restrict__ slots, int num_slots, int H, int T) {
+    constexpr bool fused = kFused;
     constexpr int NT = 256;
     constexpr int TX = DV / 4;       // threads across a row (float4 each)
     constexpr int TY = NT / TX;      // rows per pass
@@ -58,7 +61,7 @@ kda_decode_kernel(const Tin* __restrict__ q, const Tin* __restrict__ k,
     if (t > 0) __syncthreads();   // the previous token's update has read ga, kk and us
     // fused inputs: alpha and beta are logits, q and k are L2-normalised here
     float ikn = 1.0f, iqn = 1.0f;
-    if (fused) {
+    if constexpr (fused) {
         float pk = 0.0f, pq = 0.0f;
         if (tid < DK) {
             const float kv = to_f32(k[kb + tid]), qv = to_f32(q[kb + tid]);
@@ -148,9 +151,14 @@ static cudaError_t launch_decode_t(const void* q, const void* k, const void* v, 
                                    const void* beta, float* S, void* out, int64_t NH,
                                    cudaStream_t stream, const int32_t* slots, int num_slots, int H,
                                    int T, int fused) {
-    kda_decode_kernel<Tin, Tout, DK, DV><<<(unsigned)NH, 256, 0, stream>>>(
-        (const Tin*)q, (const Tin*)k, (const Tin*)v, (const Tin*)alpha, (const Tin*)beta, S,
-        (Tout*)out, slots, num_slots, H, T, fused);
+    if (fused)
+        kda_decode_kernel<Tin, Tout, DK, DV, true><<<(unsigned)NH, 256, 0, stream>>>(
+            (const Tin*)q, (const Tin*)k, (const Tin*)v, (const Tin*)alpha, (const Tin*)beta, S,
+            (Tout*)out, slots, num_slots, H, T);
+    else
+        kda_decode_kernel<Tin, Tout, DK, DV, false><<<(unsigned)NH, 256, 0, stream>>>(
+            (const Tin*)q, (const Tin*)k, (const Tin*)v, (const Tin*)alpha, (const Tin*)beta, S,
+            (Tout*)out, slots, num_slots, H, T);
     return cudaGetLastError();
 }
 
