@@ -58,6 +58,19 @@ kda_decode_kernel(const Tin* __restrict__ q, const Tin* __restrict__ k,
     for (int t = 0; t < T; ++t) {
     const size_t tok = ((size_t)n * T + t) * H + hh;   // (sequence, token, head)
     const size_t kb = tok * DK, vb = tok * DV;
+    if (t + 1 < T) {
+        // the next token's q, k, alpha and v rows (and beta) towards L2 while this one
+        // is worked on: one thread per 128-byte line, no registers held
+        const size_t nk = (tok + H) * DK, nv = (tok + H) * DV;
+        constexpr int LK = (DK * (int)sizeof(Tin) + 127) / 128, LV = (DV * (int)sizeof(Tin) + 127) / 128;
+        const char* line = nullptr;
+        if (tid < LK) line = reinterpret_cast<const char*>(q + nk) + 128 * tid;
+        else if (tid < 2 * LK) line = reinterpret_cast<const char*>(k + nk) + 128 * (tid - LK);
+        else if (tid < 3 * LK) line = reinterpret_cast<const char*>(alpha + nk) + 128 * (tid - 2 * LK);
+        else if (tid < 3 * LK + LV) line = reinterpret_cast<const char*>(v + nv) + 128 * (tid - 3 * LK);
+        else if (tid == 3 * LK + LV) line = reinterpret_cast<const char*>(beta + tok + H);
+        if (line) asm volatile("prefetch.global.L2 [%0];" :: "l"(line));
+    }
     if (t > 0) __syncthreads();   // the previous token's update has read ga, kk and us
     // fused inputs: alpha and beta are logits, q and k are L2-normalised here
     float ikn = 1.0f, iqn = 1.0f;
