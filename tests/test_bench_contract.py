@@ -1,0 +1,104 @@
+"""CPU checks of bench.py: the work model behind `roofline` and `tensor`, the
+DRAM-traffic record lookup, and the JSON line of the reference (oracle) arm.
+
+The byte and flop counts are the ones the measurement section states: per (token, head)
+q, k, alpha, v, beta read and o written once; per (sequence, head) S0 read and S_final
+written once; chunk-form flops 6 d_k d_v + 2 C (3 d_k + 2 d_v).
+"""
+import importlib.util
+import json
+import os
+import subprocess
+import sys
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def _bench():
+    spec = importlib.util.spec_from_file_location("bench_under_test", os.path.join(ROOT, "bench.py"))
+    mod = importlib.util.module_from_spec(spec)
+    spec.loader.exec_module(mod)
+    return mod
+
+
+def _workload(name):
+    sys.path.insert(0, ROOT)
+    from gated_delta_rule_138_b200 import inputs
+    return inputs.WORKLOADS[name]
+
+
+def test_forward_bytes_and_flops_of_the_default_workload():
+    b = _bench()
+    w = _workload(b.DEFAULT_WORKLOAD)
+    n_th, n_sh = w.B * w.T * w.H, w.B * w.H
+    # bf16 d_k = d_v = 128: 2 (3*128 + 128 + 1) + 2*128 = 1282 B per (token, head)
+    assert b.forward_bytes(w, 1, 0, True) == 1282
+    # fp32 S0 and S_final: 2 * 4 * 128 * 128 B per (sequence, head); without S0 only S_final
+    assert b.forward_bytes(w, 0, 1, True) == 131072
+    assert b.forward_bytes(w, 0, 1, False) == 65536
+    assert b.forward_bytes(w, n_th, n_sh, True) == 1377828864
+    assert b.forward_flops(w, 1) == 6 * 128 * 128 + 2 * 64 * (3 * 128 + 2 * 128) == 180224
+
+
+def test_decode_bytes():
+    b = _bench()
+    w = _workload("decode_N256_H32_d128")
+    # the fp32 state read and written once, the token's inputs and output once
+    assert b.decode_bytes(w, 1) == 8 * 128 * 128 + 2 * (3 * 128 + 128 + 1) + 2 * 128
+    assert b.decode_flops(w, 1) == 6 * 128 * 128
+
+
+def test_recorded_traffic_lookup():
+    b = _bench()
+    path = os.path.join(ROOT, "profiles", "dram_traffic.txt")
+    rows = [ln.split() for ln in open(path).read().splitlines()
+            if ln.strip() and not ln.startswith("#")]
+    assert rows, "no DRAM-traffic records"
+    for kernel, workload, files, digest, nbytes in rows:
+        got = b.recorded_traffic(kernel, workload)
+        # a record counts only while the kernel sources still hash to the recorded digest
+        if b.kernel_source_digest(files) == digest:
+            assert got == float(nbytes)
+        else:
+            assert got is None
+    # no record for a workload or kernel variant that was never captured
+    assert b.recorded_traffic("chunk_tc_bf16", "no_such_workload") is None
+    assert b.recorded_traffic("chunk_tc_bf16_fused", "bf16_B8_T4096_H32_d128") is None
+
+
+def _run_reference(extra_env=None):
+    env = dict(os.environ)
+    env.update(extra_env or {})
+    return subprocess.run([sys.executable, os.path.join(ROOT, "bench.py"), "--impl", "reference",
+                           "--workload", "fp32_T256_d64", "--steps", "1", "--warmup", "3"],
+                          cwd=ROOT, env=env, capture_output=True, text=True, timeout=600)
+
+
+def test_reference_arm_json_line():
+    r = _run_reference()
+    assert r.returncode == 0, r.stderr[-2000:]
+    lines = [ln for ln in r.stdout.splitlines() if ln.startswith("{")]
+    assert len(lines) == 1
+    d = json.loads(lines[0])
+    for key in ("metric", "value", "unit", "n_gpus", "steps", "warmup", "ms_per_step",
+                "higher_is_better", "scaling", "vs_baseline", "dtype", "data", "config",
+                "cpu_baseline", "e2e"):
+        assert key in d, key
+    assert d["impl"] == "reference"
+    assert d["steps"] == 1 and d["warmup"] == 3 and d["n_gpus"] == 1
+    assert d["value"] > 0 and d["higher_is_better"] is True
+    assert d["config"]["workload"] == "fp32_T256_d64"
+    cb = d["cpu_baseline"]
+    assert cb["kind"] == "oracle" and cb["cores"] >= 1 and cb["value"] == d["value"]
+    assert cb["sample"]
+    e = d["e2e"]
+    assert e["value"] == d["value"] and e["unit"] == d["unit"]
+    assert e["h2d_bytes_per_step"] == 0 and e["d2h_bytes_per_step"] == 0
+
+
+def test_reference_arm_other_ranks_do_no_work():
+    r = _run_reference({"RANK": "1", "WORLD_SIZE": "2"})
+    assert r.returncode == 0, r.stderr[-2000:]
+    assert not [ln for ln in r.stdout.splitlines() if ln.startswith("{")]
