@@ -1,7 +1,8 @@
 """KDA oracle -- TEST INFRASTRUCTURE ONLY.
 
 A plain fp64 CPU implementation of the KDA forward pass (token-by-token gated
-delta rule), used to check the CUDA path.  Only ``tests/``,
+delta rule) and of its reverse mode (the backward pass), used to check the CUDA
+path.  Only ``tests/``,
 ``__graft_entry__.smoke()`` and ``bench.py``'s CPU-baseline leg may import
 this package.  It shares no code with ``gated_delta_rule_138_b200`` and the
 product never imports it.
@@ -40,6 +41,14 @@ def _load(path=None):
             ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p, ctypes.c_int32,
             ctypes.c_int32, ctypes.c_int64, ctypes.c_int32, ctypes.c_int32,
             ctypes.c_int32, ctypes.c_void_p, ctypes.c_void_p, ctypes.c_int32]
+        lib.kda_oracle_backward.restype = ctypes.c_int
+        lib.kda_oracle_backward.argtypes = [
+            ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p,
+            ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p,
+            ctypes.c_void_p, ctypes.c_int32, ctypes.c_int32, ctypes.c_int64,
+            ctypes.c_int32, ctypes.c_int32, ctypes.c_int32, ctypes.c_void_p,
+            ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p,
+            ctypes.c_void_p, ctypes.c_int32]
         lib.kda_oracle_alpha_min.restype = ctypes.c_double
         lib.kda_oracle_alpha_min.argtypes = []
         _libs[key] = lib
@@ -92,6 +101,43 @@ def forward(q, k, v, alpha, beta, S0=None, cu_seqlens=None, nthreads=0, lib_path
     if rc != 0:
         raise ValueError("kda_oracle_forward rejected its arguments (rc=%d)" % rc)
     return out, S_final
+
+
+def backward(q, k, v, alpha, beta, dout, S0=None, dS_final=None, cu_seqlens=None,
+             nthreads=0, lib_path=None):
+    """Reverse mode of the token recurrence in fp64 (the backward pass).
+
+    Inputs as `forward`, plus dout (dL/d out, like v) and dS_final (dL/d S_final,
+    like S0, or None for zero).  The clamp passes the gradient where alpha lies
+    in [e^-5, 1] (bounds included) and blocks it outside.  Returns fp64
+    (dq, dk, dv, dalpha, dbeta, dS0), each shaped like its input (dS0 like S0,
+    [N, H, dk, dv], also when S0 is None).
+    """
+    q, k, v, alpha, beta, S0, dout, dS_final = (
+        _f32(x) for x in (q, k, v, alpha, beta, S0, dout, dS_final))
+    B, T, H, dk = q.shape
+    dv = v.shape[-1]
+    assert k.shape == q.shape and alpha.shape == q.shape
+    assert v.shape == (B, T, H, dv) and beta.shape == (B, T, H) and dout.shape == v.shape
+    if cu_seqlens is not None:
+        cu = np.ascontiguousarray(np.asarray(cu_seqlens, dtype=np.int32))
+        nseq = cu.shape[0] - 1
+        assert B == 1
+    else:
+        cu = None
+        nseq = B
+    for x in (S0, dS_final):
+        if x is not None:
+            assert x.shape == (nseq, H, dk, dv)
+    dq = np.zeros((B, T, H, dk)); dk_ = np.zeros((B, T, H, dk)); dal = np.zeros((B, T, H, dk))
+    dv_ = np.zeros((B, T, H, dv)); dbe = np.zeros((B, T, H)); dS0 = np.zeros((nseq, H, dk, dv))
+    rc = _load(lib_path).kda_oracle_backward(
+        _ptr(q), _ptr(k), _ptr(v), _ptr(alpha), _ptr(beta), _ptr(S0), _ptr(dout),
+        _ptr(dS_final), _ptr(cu), nseq, B, T, H, dk, dv, _ptr(dq), _ptr(dk_), _ptr(dv_),
+        _ptr(dal), _ptr(dbe), _ptr(dS0), int(nthreads))
+    if rc != 0:
+        raise ValueError("kda_oracle_backward rejected its arguments (rc=%d)" % rc)
+    return dq, dk_, dv_, dal, dbe, dS0
 
 
 def decode_steps(q, k, v, alpha, beta, S, nthreads=0):
