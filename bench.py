@@ -60,6 +60,22 @@ def forward_flops(w, n_token_heads: int) -> int:
     return (6 * w.dk * w.dv + 2 * w.chunk * (3 * w.dk + 2 * w.dv)) * n_token_heads
 
 
+def backward_bytes(w, n_token_heads: int, n_seq_heads: int, has_s0: bool) -> int:
+    """Algorithmic HBM bytes of one backward: q, k, alpha, v, beta and dout read,
+    fp32 dq, dk, dalpha, dv, dbeta written once per (token, head); S0 (if any)
+    and dS_final read and dS0 written once per (sequence, head)."""
+    ei = esize(w.dtype)
+    per_th = ei * (3 * w.dk + 2 * w.dv + 1) + 4 * (3 * w.dk + w.dv + 1)
+    per_sh = 4 * w.dk * w.dv * ((1 if has_s0 else 0) + 2)
+    return per_th * n_token_heads + per_sh * n_seq_heads
+
+
+def backward_flops(w, n_token_heads: int) -> int:
+    """Flops per (token, head) as the backward kernel executes them: two forward
+    recomputations (5 dk dv each) and the reverse step (21 dk dv)."""
+    return 31 * w.dk * w.dv * n_token_heads
+
+
 def decode_bytes(w, n_seq_heads: int) -> int:
     ei, eo = esize(w.dtype), esize(w.out_dtype)
     return n_seq_heads * (8 * w.dk * w.dv + ei * (3 * w.dk + w.dv + 1) + eo * w.dv)
@@ -415,6 +431,18 @@ def run_ours(args, w):
             def step():
                 kda.kda_forward_fused(inp["q"], inp["k"], inp["v"], inp["alpha"], inp["beta"],
                                       inp["S0"], cu_seqlens=cu, out=out, S_final=Sf, chunk=w.chunk)
+        if args.backward:
+            # gradients of the same forward: dout like out, dS_final like S_final
+            gb = torch.Generator(device=dev).manual_seed(int(w.seed) + 5)
+            dout = torch.randn(out.shape, generator=gb, device=dev).to(inp["q"].dtype)
+            dSf = torch.randn(Sf.shape, generator=gb, device=dev)
+            ws = torch.empty(kda.kda_backward_workspace_bytes(
+                B, T, w.H, w.dk, w.dv, None if cu is None else nseq), dtype=torch.uint8,
+                device=dev)
+
+            def step():
+                kda.kda_backward(inp["q"], inp["k"], inp["v"], inp["alpha"], inp["beta"], dout,
+                                 inp["S0"], dSf, cu_seqlens=cu, workspace=ws)
         if args.seqpar and w.kind == "forward":
             # this rank's time segment; maps exchanged through the process group
             from gated_delta_rule_138_b200.seqpar import kda_forward_sequence_parallel, split_time
@@ -429,12 +457,17 @@ def run_ours(args, w):
         kname = kda.kda_forward_kernel_name(w.dk, w.dv, w.chunk, inp["q"].dtype, out.dtype)
         if args.fused:
             kname += "_fused"   # its own compile-time variant (no DRAM-traffic record)
+        if args.backward:
+            kname = "backward_f32"
         # time segments per sequence of the tensor-core path (1: unsplit); with g > 1 a
         # step is three launches (segment maps, scan, forward) timed together
         segments = (kda.kda_forward_segments(nseq, -(-B * T // nseq), w.H)
                     if kname.startswith("chunk_tc_bf16") else 1)
         algo_bytes = forward_bytes(w, n_th, n_sh, inp["S0"] is not None)
         algo_flops = forward_flops(w, n_th)
+        if args.backward:
+            algo_bytes = backward_bytes(w, n_th, n_sh, inp["S0"] is not None)
+            algo_flops = backward_flops(w, n_th)
 
     warm = max(3, args.warmup)
     for _ in range(warm):
@@ -474,6 +507,7 @@ def run_ours(args, w):
     # end to end: pinned host inputs -> device -> kda_forward -> host results
     e2e = run_e2e(args, w, inp, dev, stream, world) \
         if w.kind in ("forward", "varlen") and args.e2e_steps > 0 and not seqpar \
+        and not args.backward \
         else None
 
     if rank == 0:
@@ -484,6 +518,8 @@ def run_ours(args, w):
         cfg = config_of(w, world)
         if args.fused:
             cfg["inputs"] = "raw: gate logits, unnormalised q and k (kda_forward_fused)"
+        if args.backward:
+            cfg["pass"] = "backward (kda_backward: dq, dk, dv, dalpha, dbeta, dS0 in fp32)"
         if seqpar:
             cfg["parallelism"] = "sequence x%d (time segments per rank, maps all-gathered)" % world
         line = {
@@ -584,6 +620,8 @@ def main():
     ap.add_argument("--fused", action="store_true",
                     help="forward workloads through kda_forward_fused (gates as logits, q and k "
                          "normalised inside the kernel)")
+    ap.add_argument("--backward", action="store_true",
+                    help="time kda_backward (all input gradients) on a forward workload")
     ap.add_argument("--seqpar", action="store_true",
                     help="split every sequence's time axis across the ranks (strong scaling)")
     ap.add_argument("--e2e-steps", type=int, default=10,

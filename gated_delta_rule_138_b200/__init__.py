@@ -1,4 +1,4 @@
-"""B200-native KDA (Kimi Delta Attention) forward pass and decode step.
+"""B200-native KDA (Kimi Delta Attention) forward pass, decode step and backward pass.
 
 The compute path is the C-ABI library ``libkda.so`` built from ``csrc/``
 (hand-written sm_100a CUDA kernels); ``kda.py`` is a thin ctypes binding with
@@ -11,7 +11,7 @@ from .kda import (KdaError, kda_forward, kda_decode_step, kda_status_string,  # 
                   kda_device_status, kda_forward_noalloc, kda_selftest_timeout,
                   kda_forward_segments, kda_segment_maps, kda_segment_scan,
                   kda_forward_indexed, kda_decode_step_indexed, kda_forward_fused,
-                  kda_decode_step_fused,
+                  kda_decode_step_fused, kda_backward, kda_backward_workspace_bytes,
                   library_path, load_library)
 
 __all__ = ["KdaError", "kda_forward", "kda_decode_step", "kda_status_string",
@@ -19,5 +19,5 @@ __all__ = ["KdaError", "kda_forward", "kda_decode_step", "kda_status_string",
            "kda_device_status", "kda_forward_noalloc", "kda_selftest_timeout",
            "kda_forward_segments", "kda_segment_maps", "kda_segment_scan",
            "kda_forward_indexed", "kda_decode_step_indexed", "kda_forward_fused",
-           "kda_decode_step_fused",
+           "kda_decode_step_fused", "kda_backward", "kda_backward_workspace_bytes",
            "library_path", "load_library"]

@@ -28,6 +28,12 @@ cudaError_t launch_chunk_tc(const void* q, const void* k, const void* v, const v
                             cudaStream_t stream, const int32_t* slots = nullptr, int num_slots = 0,
                             int fused = 0);
 size_t chunk_tc_segmented_workspace_floats(int64_t nseq, int H, int nseg);
+size_t backward_workspace_floats(bool packed, int64_t nseq, int64_t T, int H, int DK, int DV);
+cudaError_t launch_backward(int in_bf16, const void* q, const void* k, const void* v,
+                            const void* alpha, const void* beta, const float* S0, const void* dout,
+                            const float* dSf, const int32_t* cu, int64_t nseq, int64_t T, int H,
+                            int DK, int DV, float* dq, float* dk, float* dv, float* dalpha,
+                            float* dbeta, float* dS0, float* workspace, cudaStream_t s);
 cudaError_t launch_segment_maps(const void* k, const void* v, const void* alpha, const void* beta,
                                 const int32_t* cu, int nseq, float* maps, int64_t rows, int64_t T,
                                 int H, int* status, cudaStream_t stream);
@@ -477,6 +483,62 @@ kda_status_t kda_decode_step_fused(const void* q, const void* k, const void* v,
                                    kda_stream_t stream) {
     return decode_impl(q, k, v, alpha_logits, beta_logits, S, out, N, H, d_k, d_v, in_dtype,
                        out_dtype, stream, 1);
+}
+
+size_t kda_backward_workspace_bytes(int32_t B, int64_t T, int32_t H, int32_t d_k, int32_t d_v,
+                                    int32_t packed, int32_t num_seqs) {
+    if (B < 0 || T < 0 || H <= 0 || num_seqs < 0) return 0;
+    const int64_t nseq = packed ? (int64_t)num_seqs : (int64_t)B;
+    return sizeof(float) * kda::backward_workspace_floats(packed != 0, nseq, T, H, d_k, d_v);
+}
+
+kda_status_t kda_backward(const void* q, const void* k, const void* v, const void* alpha,
+                          const void* beta, const float* S0, const void* dout,
+                          const float* dS_final, const int32_t* cu_seqlens, int32_t num_seqs,
+                          float* dq, float* dk, float* dv, float* dalpha, float* dbeta,
+                          float* dS0, int32_t B, int64_t T, int32_t H, int32_t d_k, int32_t d_v,
+                          kda_dtype_t in_dtype, void* workspace, size_t workspace_bytes,
+                          kda_stream_t stream) {
+    if (B < 0 || T < 0 || H <= 0 || !is_dtype(in_dtype)) return KDA_ERR_INVALID_ARG;
+    if (cu_seqlens != nullptr && (B != 1 || num_seqs < 0)) return KDA_ERR_INVALID_ARG;
+    const int64_t nseq = cu_seqlens ? (int64_t)num_seqs : (int64_t)B;
+    const bool has_tokens = (int64_t)B * T > 0;
+    if (has_tokens && (!q || !k || !v || !alpha || !beta || !dout || !dq || !dk || !dv ||
+                       !dalpha || !dbeta))
+        return KDA_ERR_INVALID_ARG;
+    const int es = in_dtype == KDA_BF16 ? 2 : 4;
+    const void* elem[] = {q, k, v, alpha, beta, dout};
+    for (const void* p : elem)
+        if (!aligned_to(p, es)) return KDA_ERR_INVALID_ARG;
+    const void* f32[] = {dq, dk, dv, dalpha, dbeta};
+    for (const void* p : f32)
+        if (!aligned_to(p, 4)) return KDA_ERR_INVALID_ARG;
+    const void* vec[] = {S0, dS_final, dS0, workspace};
+    for (const void* p : vec)
+        if (p && !aligned16(p)) return KDA_ERR_INVALID_ARG;
+    if (!aligned_to(cu_seqlens, 4)) return KDA_ERR_INVALID_ARG;
+    if (!head_dim_ok(d_k) || !head_dim_ok(d_v)) return KDA_ERR_UNSUPPORTED;
+    if (nseq * H > 0x7fffffffLL) return KDA_ERR_UNSUPPORTED;
+    if (nseq == 0) return KDA_OK;
+    const size_t need = sizeof(float) * kda::backward_workspace_floats(cu_seqlens != nullptr, nseq,
+                                                                       T, H, d_k, d_v);
+    if (workspace && workspace_bytes < need) return KDA_ERR_INVALID_ARG;
+    g_last_error[0] = '\0';
+    const cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    float* ws = static_cast<float*>(workspace);
+    if (!ws) {
+        cudaError_t e = cudaMallocAsync(reinterpret_cast<void**>(&ws), need, s);
+        if (e != cudaSuccess) return cuda_status(e);
+    }
+    g_launches.fetch_add(1, std::memory_order_relaxed);
+    cudaError_t e = kda::launch_backward(in_dtype == KDA_BF16, q, k, v, alpha, beta, S0, dout,
+                                         dS_final, cu_seqlens, nseq, T, H, d_k, d_v, dq, dk, dv,
+                                         dalpha, dbeta, dS0, ws, s);
+    if (!workspace) {
+        const cudaError_t ef = cudaFreeAsync(ws, s);
+        if (e == cudaSuccess) e = ef;
+    }
+    return cuda_status(e);
 }
 
 }  // extern "C"

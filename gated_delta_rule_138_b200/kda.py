@@ -97,6 +97,11 @@ def load_library(build_if_missing: bool = True) -> ctypes.CDLL:
     lib.kda_decode_step_indexed.restype = ctypes.c_int
     lib.kda_decode_step_indexed.argtypes = [vp, vp, vp, vp, vp, vp, i32, vp, vp, i32, i32, i32, i32,
                                             ctypes.c_int, ctypes.c_int, vp]
+    lib.kda_backward.restype = ctypes.c_int
+    lib.kda_backward.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, vp, i32, vp, vp, vp, vp, vp, vp,
+                                 i32, i64, i32, i32, i32, ctypes.c_int, vp, ctypes.c_size_t, vp]
+    lib.kda_backward_workspace_bytes.restype = ctypes.c_size_t
+    lib.kda_backward_workspace_bytes.argtypes = [i32, i64, i32, i32, i32, i32, i32]
     _lib = lib
     return lib
 
@@ -208,6 +213,60 @@ def kda_forward(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, alpha: torch.
                          _dt(q), _dt(out), _stream(stream))
     _check("kda_forward", st)
     return out, S_final
+
+
+def kda_backward(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, alpha: torch.Tensor,
+                 beta: torch.Tensor, dout: torch.Tensor, S0: Optional[torch.Tensor] = None,
+                 dS_final: Optional[torch.Tensor] = None,
+                 cu_seqlens: Optional[torch.Tensor] = None, want_dS0: bool = True,
+                 workspace: Optional[torch.Tensor] = None, stream=None):
+    """Gradients of kda_forward through the C ABI (kda_backward).
+
+    Inputs as kda_forward plus dout (dL/d out, [B, T, H, d_v], the inputs' dtype)
+    and dS_final (dL/d S_final, fp32 [N, H, d_k, d_v], or None for zero).
+    Returns fp32 (dq, dk, dv, dalpha, dbeta, dS0 or None), shaped like the inputs.
+    workspace: optional uint8 device tensor of at least kda_backward_workspace_bytes.
+    """
+    lib = load_library()
+    B, T, H, dk = q.shape
+    dv = v.shape[-1]
+    if k.shape != q.shape or alpha.shape != q.shape or v.shape != (B, T, H, dv) \
+            or beta.shape != (B, T, H) or dout.shape != v.shape:
+        raise ValueError("inconsistent shapes")
+    if len({q.dtype, k.dtype, v.dtype, alpha.dtype, beta.dtype, dout.dtype}) != 1:
+        raise TypeError("q, k, v, alpha, beta, dout must share one dtype")
+    for name, t in (("q", q), ("k", k), ("v", v), ("alpha", alpha), ("beta", beta),
+                    ("dout", dout), ("S0", S0), ("dS_final", dS_final),
+                    ("cu_seqlens", cu_seqlens), ("workspace", workspace)):
+        _contig(name, t)
+    nseq = B if cu_seqlens is None else cu_seqlens.numel() - 1
+    if cu_seqlens is not None and cu_seqlens.dtype != torch.int32:
+        raise TypeError("cu_seqlens must be int32")
+    for name, t in (("S0", S0), ("dS_final", dS_final)):
+        if t is not None and (t.dtype != torch.float32 or tuple(t.shape) != (nseq, H, dk, dv)):
+            raise ValueError("%s must be fp32 [N, H, d_k, d_v]" % name)
+    f32 = dict(dtype=torch.float32, device=q.device)
+    dq, dk_, dal = (torch.empty(B, T, H, dk, **f32) for _ in range(3))
+    dv_ = torch.empty(B, T, H, dv, **f32)
+    dbe = torch.empty(B, T, H, **f32)
+    dS0 = torch.empty(nseq, H, dk, dv, **f32) if want_dS0 else None
+    st = lib.kda_backward(_ptr(q), _ptr(k), _ptr(v), _ptr(alpha), _ptr(beta), _ptr(S0),
+                          _ptr(dout), _ptr(dS_final), _ptr(cu_seqlens), int(nseq), _ptr(dq),
+                          _ptr(dk_), _ptr(dv_), _ptr(dal), _ptr(dbe), _ptr(dS0), int(B), int(T),
+                          int(H), int(dk), int(dv), _dt(q), _ptr(workspace),
+                          0 if workspace is None else workspace.numel() * workspace.element_size(),
+                          _stream(stream))
+    _check("kda_backward", st)
+    return dq, dk_, dv_, dal, dbe, dS0
+
+
+def kda_backward_workspace_bytes(B: int, T: int, H: int, d_k: int, d_v: int,
+                                 num_seqs: Optional[int] = None) -> int:
+    """Bytes of workspace kda_backward needs (num_seqs given: a packed batch)."""
+    lib = load_library()
+    packed = num_seqs is not None
+    return int(lib.kda_backward_workspace_bytes(int(B), int(T), int(H), int(d_k), int(d_v),
+                                                1 if packed else 0, int(num_seqs or 0)))
 
 
 def kda_segment_maps(k: torch.Tensor, v: torch.Tensor, alpha: torch.Tensor, beta: torch.Tensor,

@@ -322,6 +322,52 @@ kda_status_t kda_forward_noalloc(const void* q, const void* k, const void* v,
                                  int32_t chunk, kda_dtype_t in_dtype, kda_dtype_t out_dtype,
                                  kda_stream_t stream);
 
+/*
+ * kda_backward -- gradients of kda_forward's outputs with respect to all of
+ * its inputs (the backward pass, for training).  The pages print no backward;
+ * this is the reverse mode of the recurrence of the worldcybernews article
+ * "Kimi K3 Open Model Surpasses Closed GPT and Anthropic Systems on Independent
+ * Benchmarks", paragraph 2, as kda_forward computes it (a_t = clamp(alpha_t,
+ * e^-5, 1); S_t = (I - beta_t k_t k_t^T) Diag(a_t) S_{t-1} + beta_t k_t v_t^T;
+ * o_t = S_t^T q_t).  For a loss L, given dL/d out (`dout`) and dL/d S_final
+ * (`dS_final`, NULL = zero), it writes dL/dq, dL/dk, dL/dv, dL/dalpha,
+ * dL/dbeta and dL/dS0.  The clamp passes the gradient to alpha where alpha lies
+ * in [e^-5, 1] (bounds included) and blocks it outside.
+ *
+ *   q, k, alpha, v, beta, S0, cu_seqlens, num_seqs, B, T, H, d_k, d_v: as
+ *     kda_forward (device pointers, caller-owned; S0 NULL = zero state).
+ *   dout: like out, in in_dtype ([B, T, H, d_v]).
+ *   dq, dk, dalpha: fp32 [B, T, H, d_k]; dv: fp32 [B, T, H, d_v]; dbeta: fp32
+ *     [B, T, H]; all written for every token.  dS0: fp32 like S0 (NULL = not
+ *     wanted).  None of them may alias an input.
+ *   workspace: NULL, or device memory of at least kda_backward_workspace_bytes
+ *     (16-byte aligned, caller-owned, contents not preserved).  NULL: the call
+ *     allocates it stream-ordered (cudaMallocAsync) and frees it after the
+ *     kernel, on `stream`.
+ *   Supported: d_k, d_v in {64, 128}; in_dtype KDA_F32 or KDA_BF16; S0,
+ *     dS_final, dS0 and workspace 16-byte aligned.
+ *   The kernel keeps the state and its gradient in registers, one CTA per
+ *   (sequence, head), and recomputes states from checkpoints taken every 64
+ *   tokens: cost grows with the longest sequence, and the workspace holds
+ *   ceil(T / 64) + 64 states of d_k x d_v fp32 per (sequence, head).
+ *
+ *   Returns KDA_OK; KDA_ERR_INVALID_ARG (missing or misaligned pointer, bad
+ *   size, workspace too small); KDA_ERR_UNSUPPORTED (head dims, more than
+ *   2^31 - 1 (sequence, head) pairs); KDA_ERR_CUDA (launch or allocation
+ *   failure, reason in kda_last_error()).
+ */
+kda_status_t kda_backward(const void* q, const void* k, const void* v, const void* alpha,
+                          const void* beta, const float* S0, const void* dout,
+                          const float* dS_final, const int32_t* cu_seqlens, int32_t num_seqs,
+                          float* dq, float* dk, float* dv, float* dalpha, float* dbeta,
+                          float* dS0, int32_t B, int64_t T, int32_t H, int32_t d_k, int32_t d_v,
+                          kda_dtype_t in_dtype, void* workspace, size_t workspace_bytes,
+                          kda_stream_t stream);
+/* Workspace bytes kda_backward needs for these sizes (cu_seqlens given: packed
+ * = 1, num_seqs sequences in T packed tokens; else B sequences of T tokens). */
+size_t kda_backward_workspace_bytes(int32_t B, int64_t T, int32_t H, int32_t d_k, int32_t d_v,
+                                    int32_t packed, int32_t num_seqs);
+
 #ifdef __cplusplus
 }
 #endif

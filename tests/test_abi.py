@@ -161,3 +161,33 @@ def test_indexed_calls_reject_before_launch():
                                    1, 4, 1, 96, 128, 64, 1, 1, None) == 1   # no pool / slots
     assert lib.kda_forward_indexed(None, None, None, None, None, None, 4, None, None, 0, None,
                                    0, 4, 1, 96, 128, 64, 1, 1, None) == 2   # d_k = 96
+
+
+def test_backward_rejects_before_launch():
+    lib = kda.load_library()
+    p = ctypes.c_void_p(0x10000)
+    need = kda.kda_backward_workspace_bytes(2, 128, 4, 128, 128)
+
+    def call(B=2, T=128, H=4, dk=128, dv=128, q=p, S0=None, ws=p, ws_bytes=need, dt=1, cu=None,
+             nseq=0):
+        return lib.kda_backward(q, p, p, p, p, S0, p, None, cu, nseq, p, p, p, p, p, None,
+                                B, T, H, dk, dv, dt, ws, ws_bytes, None)
+    assert call(H=0) == 1
+    assert call(q=None) == 1
+    assert call(dt=7) == 1
+    assert call(S0=ctypes.c_void_p(0x10008)) == 1        # S0 read with 16-byte accesses
+    assert call(ws=ctypes.c_void_p(0x10004)) == 1        # workspace likewise
+    assert call(ws_bytes=need - 1) == 1                  # workspace too small
+    assert call(dk=32) == 2
+    assert call(B=0) == 0                                # nothing to do, nothing launched
+    assert call(B=2, cu=p, nseq=1) == 1                  # packed batches have B == 1
+
+
+def test_backward_workspace_sizes():
+    mat = 128 * 128 * 4
+    # dense: ceil(T / 64) checkpoints per (sequence, head) plus a 64-state slab
+    assert kda.kda_backward_workspace_bytes(8, 4096, 32, 128, 128) == (8 * 64 + 8 * 64) * 32 * mat
+    assert kda.kda_backward_workspace_bytes(1, 65, 1, 128, 128) == (2 + 64) * mat
+    # packed: floor(T / 64) + num_seqs checkpoints per head
+    assert kda.kda_backward_workspace_bytes(1, 1000, 2, 128, 128, num_seqs=3) == \
+        ((1000 // 64 + 3) * 2 + 3 * 2 * 64) * mat
