@@ -19,17 +19,19 @@
 // registers, d_k x d_v split as in the decode kernel (thread (tx, ty): rows
 // ty + TY i, columns 4 tx .. 4 tx + 3).  The reverse sweep needs S_{t-1} for t
 // descending, and the step is not invertible in floating point, so states are
-// recomputed: a forward sweep stores the state at every 64-token chunk start
-// (checkpoints); then, chunk by chunk from the last, the chunk's 64 states are
-// recomputed from its checkpoint into a scratch slab and read back in reverse.
-// Each thread reads back only what it wrote, so the slabs need no barriers.
+// recomputed: a forward sweep stores the state at every 16-token chunk start
+// (checkpoints); then, chunk by chunk from the last, the chunk's 16 states are
+// recomputed from its checkpoint into a scratch slab (1 MB per CTA at d = 128,
+// small enough to stay in L2) and read back in reverse.  Each thread reads back
+// only what it wrote, so the slabs need no barriers.  The token rows of the
+// next chunk to be worked on are prefetched into L2 one chunk ahead.
 #include "kda_common.cuh"
 
 namespace kda {
 namespace bwd {
 
 constexpr int NT = 256;
-constexpr int CK = 64;   // tokens between checkpoints
+constexpr int CK = 16;   // tokens between checkpoints
 
 template <typename Tin, int DK, int DV>
 __global__ void __launch_bounds__(NT, 1)
@@ -48,6 +50,9 @@ kda_backward_kernel(const Tin* __restrict__ q, const Tin* __restrict__ k, const 
     __shared__ float ga[DK], ka[DK], kk[DK], qq[DK], okm[DK];
     __shared__ float vv[DV], dov[DV], us[DV], xs[DV], dxs[DV];
     __shared__ float red[TY][DV];
+    // per-row partials over the TX threads of a row (dq; later dk and dalpha),
+    // padded so that a thread summing one row reads its own bank sequence
+    __shared__ float rowp[2][DK][TX + 1];
     __shared__ float dbp[NT / 32];
     __shared__ float sb;
 
@@ -66,6 +71,29 @@ kda_backward_kernel(const Tin* __restrict__ q, const Tin* __restrict__ k, const 
         return reinterpret_cast<float4*>(ckpt + ((size_t)(ck0 + ci) * H + h) * mat);
     };
     auto tok = [&](int64_t t) { return (bos + t) * H + h; };   // (token, head) row
+    // L2 prefetch of the rows of chunk ci (k, alpha, v, beta; with q and dout when
+    // `grads`): one thread per 128-byte line, no registers held
+    constexpr int LK = (DK * (int)sizeof(Tin) + 127) / 128, LV = (DV * (int)sizeof(Tin) + 127) / 128;
+    constexpr int LINES = 3 * LK + 2 * LV + 1;
+    auto prefetch_chunk = [&](int64_t ci, bool grads) {
+        if (ci < 0 || ci * CK >= len) return;
+        const int64_t t0 = ci * CK;
+        const int L = (int)(min(len, t0 + CK) - t0);
+        for (int e = tid; e < L * LINES; e += NT) {
+            const int j = e / LINES, l = e % LINES;
+            const int64_t r = tok(t0 + j);
+            const char* line = nullptr;
+            if (l < LK) line = reinterpret_cast<const char*>(k + r * DK) + 128 * l;
+            else if (l < 2 * LK) line = reinterpret_cast<const char*>(alpha + r * DK) + 128 * (l - LK);
+            else if (l < 3 * LK) {
+                if (grads) line = reinterpret_cast<const char*>(q + r * DK) + 128 * (l - 2 * LK);
+            } else if (l < 3 * LK + LV) line = reinterpret_cast<const char*>(v + r * DV) + 128 * (l - 3 * LK);
+            else if (l < 3 * LK + 2 * LV) {
+                if (grads) line = reinterpret_cast<const char*>(dout + r * DV) + 128 * (l - 3 * LK - LV);
+            } else line = reinterpret_cast<const char*>(beta + r);
+            if (line) asm volatile("prefetch.global.L2 [%0];" :: "l"(line));
+        }
+    };
 
     float4 s[RPT];
     {
@@ -133,7 +161,9 @@ kda_backward_kernel(const Tin* __restrict__ q, const Tin* __restrict__ k, const 
 
     // ---- forward sweep: a checkpoint at every chunk start
     const int64_t nck = (len + CK - 1) / CK;
+    prefetch_chunk(0, false);
     for (int64_t ci = 0; ci < nck; ++ci) {
+        prefetch_chunk(ci + 1, false);
         float4* ck = ck_at(ci);
 #pragma unroll
         for (int i = 0; i < RPT; ++i) slab(ck, i) = s[i];
@@ -149,15 +179,19 @@ kda_backward_kernel(const Tin* __restrict__ q, const Tin* __restrict__ k, const 
             g[i] = src ? src[(size_t)(ty + TY * i) * TX + tx] : make_float4(0.f, 0.f, 0.f, 0.f);
     }
 
-    // row sums over the TX threads that share a row (lanes of one warp)
-    auto row_sum = [&](float x) {
+    // row c of slot `slot` summed over its TX partials
+    auto row_sum = [&](int slot, int c) {
+        const float* p = rowp[slot][c];
+        float sum = 0.0f;
 #pragma unroll
-        for (int o = TX / 2; o > 0; o >>= 1) x += __shfl_xor_sync(0xffffffffu, x, o);
-        return x;
+        for (int j = 0; j < TX; ++j) sum += p[j];
+        return sum;
     };
 
     // ---- reverse sweep, chunk by chunk from the last
+    prefetch_chunk(nck - 1, true);
     for (int64_t ci = nck - 1; ci >= 0; --ci) {
+        prefetch_chunk(ci - 1, true);
         const float4* ck = ck_at(ci);
 #pragma unroll
         for (int i = 0; i < RPT; ++i) s[i] = ck[(size_t)(ty + TY * i) * TX + tx];
@@ -186,8 +220,7 @@ kda_backward_kernel(const Tin* __restrict__ q, const Tin* __restrict__ k, const 
                 float4 st;
                 st.x = fmaf(a, s[i].x, kc * u4.x); st.y = fmaf(a, s[i].y, kc * u4.y);
                 st.z = fmaf(a, s[i].z, kc * u4.z); st.w = fmaf(a, s[i].w, kc * u4.w);
-                const float dqc = row_sum(st.x * do4.x + st.y * do4.y + st.z * do4.z + st.w * do4.w);
-                if (tx == 0) dq[r * DK + c] = dqc;
+                rowp[0][c][tx] = st.x * do4.x + st.y * do4.y + st.z * do4.z + st.w * do4.w;
                 g[i].x = fmaf(qc, do4.x, g[i].x); g[i].y = fmaf(qc, do4.y, g[i].y);
                 g[i].z = fmaf(qc, do4.z, g[i].z); g[i].w = fmaf(qc, do4.w, g[i].w);
                 pdu.x = fmaf(g[i].x, kc, pdu.x); pdu.y = fmaf(g[i].y, kc, pdu.y);
@@ -195,6 +228,7 @@ kda_backward_kernel(const Tin* __restrict__ q, const Tin* __restrict__ k, const 
             }
             *reinterpret_cast<float4*>(&red[ty][4 * tx]) = pdu;
             __syncthreads();
+            for (int c = tid; c < DK; c += NT) dq[r * DK + c] = row_sum(0, c);
             // through u_t = b_t (v_t - x_t): dv_t, dx, db_t
             float db = 0.0f;
             if (tid < DV) {
@@ -222,17 +256,20 @@ kda_backward_kernel(const Tin* __restrict__ q, const Tin* __restrict__ k, const 
                 const int c = ty + TY * i;
                 const float a = ga[c], kc = kk[c];
                 const float4 sp = make_float4(a * s[i].x, a * s[i].y, a * s[i].z, a * s[i].w);
-                const float dkc = row_sum(g[i].x * u4.x + g[i].y * u4.y + g[i].z * u4.z + g[i].w * u4.w +
-                                          sp.x * dx4.x + sp.y * dx4.y + sp.z * dx4.z + sp.w * dx4.w);
+                rowp[0][c][tx] = g[i].x * u4.x + g[i].y * u4.y + g[i].z * u4.z + g[i].w * u4.w +
+                                 sp.x * dx4.x + sp.y * dx4.y + sp.z * dx4.z + sp.w * dx4.w;
                 float4 dsp;
                 dsp.x = fmaf(kc, dx4.x, g[i].x); dsp.y = fmaf(kc, dx4.y, g[i].y);
                 dsp.z = fmaf(kc, dx4.z, g[i].z); dsp.w = fmaf(kc, dx4.w, g[i].w);
-                const float dac = row_sum(dsp.x * s[i].x + dsp.y * s[i].y + dsp.z * s[i].z + dsp.w * s[i].w);
-                if (tx == 0) {
-                    dk[r * DK + c] = dkc;
-                    dalpha[r * DK + c] = okm[c] * dac;
-                }
+                rowp[1][c][tx] = dsp.x * s[i].x + dsp.y * s[i].y + dsp.z * s[i].z + dsp.w * s[i].w;
                 g[i] = make_float4(a * dsp.x, a * dsp.y, a * dsp.z, a * dsp.w);
+            }
+            __syncthreads();
+            // (slot 0 was last read for dq before the barrier of the db reduction)
+            for (int e = tid; e < 2 * DK; e += NT) {
+                const int c = e % DK;
+                if (e < DK) dk[r * DK + c] = row_sum(0, c);
+                else dalpha[r * DK + c] = okm[c] * row_sum(1, c);
             }
         }
     }
@@ -257,8 +294,8 @@ static cudaError_t launch_t(const void* q, const void* k, const void* v, const v
 
 }  // namespace bwd
 
-// Floats of workspace the backward needs: checkpoints (dense: nseq * ceil(T / 64)
-// per head; packed: floor(T / 64) + nseq per head) and one 64-state scratch slab
+// Floats of workspace the backward needs: checkpoints (dense: nseq * ceil(T / 16)
+// per head; packed: floor(T / 16) + nseq per head) and one 16-state scratch slab
 // per (sequence, head).
 size_t backward_workspace_floats(bool packed, int64_t nseq, int64_t T, int H, int DK, int DV) {
     const int64_t cks = packed ? T / bwd::CK + nseq : nseq * ((T + bwd::CK - 1) / bwd::CK);

@@ -185,9 +185,9 @@ def test_backward_rejects_before_launch():
 
 def test_backward_workspace_sizes():
     mat = 128 * 128 * 4
-    # dense: ceil(T / 64) checkpoints per (sequence, head) plus a 64-state slab
-    assert kda.kda_backward_workspace_bytes(8, 4096, 32, 128, 128) == (8 * 64 + 8 * 64) * 32 * mat
-    assert kda.kda_backward_workspace_bytes(1, 65, 1, 128, 128) == (2 + 64) * mat
-    # packed: floor(T / 64) + num_seqs checkpoints per head
+    # dense: ceil(T / 16) checkpoints per (sequence, head) plus a 16-state slab
+    assert kda.kda_backward_workspace_bytes(8, 4096, 32, 128, 128) == (8 * 256 + 8 * 16) * 32 * mat
+    assert kda.kda_backward_workspace_bytes(1, 17, 1, 128, 128) == (2 + 16) * mat
+    # packed: floor(T / 16) + num_seqs checkpoints per head
     assert kda.kda_backward_workspace_bytes(1, 1000, 2, 128, 128, num_seqs=3) == \
-        ((1000 // 64 + 3) * 2 + 3 * 2 * 64) * mat
+        ((1000 // 16 + 3) * 2 + 3 * 2 * 16) * mat
