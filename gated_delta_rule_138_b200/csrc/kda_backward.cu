@@ -47,9 +47,13 @@ kda_backward_kernel(const Tin* __restrict__ q, const Tin* __restrict__ k, const 
     constexpr int TY = NT / TX;     // rows per pass
     constexpr int RPT = DK / TY;    // rows per thread
     static_assert(DV % 4 == 0 && NT % TX == 0 && DK % TY == 0 && TX <= 32, "tile");
+    // (arrays read or written as float4 are declared 16-byte aligned)
     __shared__ float ga[DK], ka[DK], kk[DK], qq[DK], okm[DK];
-    __shared__ float vv[DV], dov[DV], us[DV], xs[DV], dxs[DV];
-    __shared__ float red[TY][DV];
+    __shared__ float vv[DV], xs[DV];
+    __shared__ __align__(16) float dov[DV];
+    __shared__ __align__(16) float us[DV];
+    __shared__ __align__(16) float dxs[DV];
+    __shared__ __align__(16) float red[TY][DV];
     // per-row partials over the TX threads of a row (dq; later dk and dalpha),
     // padded so that a thread summing one row reads its own bank sequence
     __shared__ float rowp[2][DK][TX + 1];

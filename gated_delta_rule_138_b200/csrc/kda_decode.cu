@@ -36,8 +36,10 @@ kda_decode_kernel(const Tin* __restrict__ q, const Tin* __restrict__ k,
     constexpr int RPT = DK / TY;     // rows per thread
     static_assert(DV % 4 == 0 && NT % TX == 0 && DK % TY == 0, "tile");
     __shared__ float ka[DK], qa[DK], kk[DK], ga[DK];
-    __shared__ float red_x[TY][DV], red_y[TY][DV];
-    __shared__ float us[DV];
+    // (arrays read or written as float4 are declared 16-byte aligned)
+    __shared__ __align__(16) float red_x[TY][DV];
+    __shared__ __align__(16) float red_y[TY][DV];
+    __shared__ __align__(16) float us[DV];
     __shared__ float kq_part[NT / 32], nk_part[NT / 32], nq_part[NT / 32];
 
     const int tid = threadIdx.x, tx = tid % TX, ty = tid / TX;
