@@ -1,0 +1,155 @@
+"""The chunk-parallel form of the backward pass, restated in fp64 numpy and
+checked against the oracle's token-by-token reverse mode.
+
+The pages give neither the chunk form nor any backward; the forward chunk form
+is the one of test_chunk_form.py (per chunk of C tokens with start state S0,
+a = clamp(alpha), g_r = sum_{s<=r} log a_s per key channel, gamma = e^g):
+
+    Kt = K * gamma,  Qt = Q * gamma,  Z = K / gamma,  Kh = K * gamma_C / gamma
+    A  = strict_lower(diag(beta) Kt Z^T),   P = lower(Qt Z^T),   T = (I + A)^-1
+    R  = V - Kt S0,  Y = diag(beta) R,  U = T Y
+    O  = Qt S0 + P U,   S_C = diag(gamma_C) S0 + Kh^T U
+
+Its reverse mode, chunk by chunk from the last, carrying only dS across chunk
+boundaries (the order a chunk-parallel backward kernel would use):
+
+    dU  = P^T dO + Kh dS_C;          dP = lower(dO U^T)
+    dQt = dO S0^T + dP Z;            dZ = dP^T Qt
+    dS0 = Qt^T dO + diag(gamma_C) dS_C;   dKh = U dS_C^T
+    dY  = T^T dU;  dT = dU Y^T;  dR = diag(beta) dY;  dbeta = rowsum(R * dY)
+    dA  = strict_lower(-T^T dT T^T)
+    dV  = dR;  dKt = -dR S0^T;  dS0 -= Kt^T dR
+    dM  = diag(beta) dA (M = Kt Z^T);  dbeta += rowsum(dA * M);  dKt += dM Z;  dZ += dM^T Kt
+    dK  = dKt * gamma + dZ / gamma + dKh * gamma_C / gamma;   dQ = dQt * gamma
+    dg  = dKt * Kt - dZ * Z + dQt * Qt - dKh * Kh;   dg[C-1] += sum_j dKh_j * Kh_j + gamma_C * rowsum(S0 * dS_C)
+    dlog a_s = sum_{r >= s} dg_r;    dalpha = dlog a / a where e^-5 <= alpha <= 1, else 0
+
+Plain gamma ratios are exact enough in fp64 (a 64-token product of gates >= e^-5
+stays above e^-320); a CUDA kernel would use the sub-chunk factorisation of
+test_chunk_form.py for the fp32 range.
+"""
+import numpy as np
+import pytest
+
+import oracle
+
+
+def _clamp(alpha):
+    lo = np.float32(np.exp(-5.0))
+    a32 = alpha.astype(np.float32)
+    a = np.clip(a32, lo, np.float32(1.0)).astype(np.float64)
+    mask = ((a32 >= lo) & (a32 <= np.float32(1.0))).astype(np.float64)
+    return a, mask
+
+
+def chunk_backward_one(q, k, v, alpha, beta, S0, dout, dSf, C):
+    """One (sequence, head): q, k, alpha [T, dk]; v, dout [T, dv]; beta [T];
+    S0, dSf [dk, dv].  Returns dq, dk, dv, dalpha, dbeta, dS0 (fp64)."""
+    T, dk = q.shape
+    dv = v.shape[1]
+    a_all, mask = _clamp(alpha)
+    q, k, v, beta, dout = (np.asarray(x, np.float64) for x in (q, k, v, beta, dout))
+    nck = (T + C - 1) // C
+
+    def chunk(ci):
+        t0 = ci * C
+        L = min(C, T - t0)
+        Q = np.zeros((C, dk)); K = np.zeros((C, dk)); V = np.zeros((C, dv))
+        a = np.ones((C, dk)); b = np.zeros(C); dO = np.zeros((C, dv))
+        Q[:L], K[:L], V[:L], a[:L], b[:L], dO[:L] = (q[t0:t0 + L], k[t0:t0 + L], v[t0:t0 + L],
+                                                     a_all[t0:t0 + L], beta[t0:t0 + L],
+                                                     dout[t0:t0 + L])
+        g = np.cumsum(np.log(a), axis=0)
+        gam = np.exp(g)
+        gC = gam[-1]
+        Kt, Qt, Z, Kh = K * gam, Q * gam, K / gam, K * (gC / gam)
+        lower = np.tril(np.ones((C, C)))
+        strict = np.tril(np.ones((C, C)), -1)
+        M = Kt @ Z.T
+        A = strict * (b[:, None] * M)
+        P = lower * (Qt @ Z.T)
+        Tm = np.linalg.inv(np.eye(C) + A)
+        return dict(L=L, t0=t0, Q=Q, K=K, V=V, a=a, b=b, dO=dO, gam=gam, gC=gC, Kt=Kt, Qt=Qt,
+                    Z=Z, Kh=Kh, M=M, A=A, P=P, T=Tm, lower=lower, strict=strict)
+
+    # forward over the chunks: the start state of each
+    S = np.asarray(S0, np.float64).copy()
+    starts = []
+    for ci in range(nck):
+        c = chunk(ci)
+        starts.append(S.copy())
+        R = c["V"] - c["Kt"] @ S
+        U = c["T"] @ (c["b"][:, None] * R)
+        S = c["gC"][:, None] * S + c["Kh"].T @ U
+
+    dq = np.zeros((T, dk)); dkk = np.zeros((T, dk)); dvv = np.zeros((T, dv))
+    dal = np.zeros((T, dk)); dbe = np.zeros(T)
+    dS = np.asarray(dSf, np.float64).copy()
+    for ci in range(nck - 1, -1, -1):
+        c = chunk(ci)
+        S0c = starts[ci]
+        R = c["V"] - c["Kt"] @ S0c
+        Y = c["b"][:, None] * R
+        U = c["T"] @ Y
+        dO, Tm = c["dO"], c["T"]
+        dU = c["P"].T @ dO + c["Kh"] @ dS
+        dP = c["lower"] * (dO @ U.T)
+        dQt = dO @ S0c.T + dP @ c["Z"]
+        dZ = dP.T @ c["Qt"]
+        dS0 = c["Qt"].T @ dO + c["gC"][:, None] * dS
+        dKh = U @ dS.T
+        dgC = c["gC"] * (S0c * dS).sum(1)
+        dY = Tm.T @ dU
+        dT = dU @ Y.T
+        dR = c["b"][:, None] * dY
+        db = (R * dY).sum(1)
+        dA = c["strict"] * (-(Tm.T @ dT @ Tm.T))
+        dV = dR
+        dKt = -dR @ S0c.T
+        dS0 -= c["Kt"].T @ dR
+        dM = c["b"][:, None] * dA
+        db += (dA * c["M"]).sum(1)
+        dKt += dM @ c["Z"]
+        dZ += dM.T @ c["Kt"]
+        gam, gC = c["gam"], c["gC"]
+        dK = dKt * gam + dZ / gam + dKh * (gC / gam)
+        dQ = dQt * gam
+        dg = dKt * c["Kt"] - dZ * c["Z"] + dQt * c["Qt"] - dKh * c["Kh"]
+        dg[-1] += (dKh * c["Kh"]).sum(0) + dgC
+        dloga = np.cumsum(dg[::-1], axis=0)[::-1]
+        L, t0 = c["L"], c["t0"]
+        dq[t0:t0 + L], dkk[t0:t0 + L], dvv[t0:t0 + L] = dQ[:L], dK[:L], dV[:L]
+        dbe[t0:t0 + L] = db[:L]
+        dal[t0:t0 + L] = (dloga[:L] / c["a"][:L]) * mask[t0:t0 + L]
+        dS = dS0
+    return dq, dkk, dvv, dal, dbe, dS
+
+
+def _rel(x, ref):
+    den = np.linalg.norm(ref.ravel())
+    return float(np.linalg.norm((x - ref).ravel()) / (den if den > 0 else 1.0))
+
+
+@pytest.mark.parametrize("C", [16, 32, 64])
+@pytest.mark.parametrize("T", [1, 40, 64, 150])
+def test_chunk_backward_equals_token_backward(C, T):
+    rng = np.random.default_rng(1000 + 7 * C + T)
+    dk, dv = 16, 12
+    f = lambda *s: rng.standard_normal(s).astype(np.float32)
+    q, k = f(T, dk), f(T, dk)
+    q /= np.linalg.norm(q, axis=1, keepdims=True)
+    k /= np.linalg.norm(k, axis=1, keepdims=True)
+    v, do = f(T, dv), f(T, dv)
+    al = np.exp(-np.log1p(np.exp(rng.standard_normal((T, dk))))).astype(np.float32)
+    al[:, 0] = 1.0                 # a channel on the upper bound
+    al[::7, 1] = 1e-4              # gates below the clamp floor (gradient blocked)
+    be = (1 / (1 + np.exp(-rng.standard_normal(T)))).astype(np.float32)
+    S0, dSf = f(dk, dv), f(dk, dv)
+    got = chunk_backward_one(q, k, v, al, be, S0, do, dSf, C)
+    x = lambda a: a[None, :, None]
+    ref = oracle.backward(x(q), x(k), x(v), x(al), be[None, :, None], x(do), S0[None, None],
+                          dSf[None, None])
+    names = ("dq", "dk", "dv", "dalpha", "dbeta", "dS0")
+    for name, g_, r in zip(names, got, ref):
+        r = r[0, :, 0] if name != "dS0" else r[0, 0]
+        assert _rel(g_, r) < 1e-9, (name, _rel(g_, r))
