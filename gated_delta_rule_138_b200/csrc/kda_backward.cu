@@ -19,10 +19,10 @@
 // registers, d_k x d_v split as in the decode kernel (thread (tx, ty): rows
 // ty + TY i, columns 4 tx .. 4 tx + 3).  The reverse sweep needs S_{t-1} for t
 // descending, and the step is not invertible in floating point, so states are
-// recomputed: a forward sweep stores the state at every 16-token chunk start
-// (checkpoints); then, chunk by chunk from the last, the chunk's 16 states are
-// recomputed from its checkpoint into a scratch slab (1 MB per CTA at d = 128,
-// small enough to stay in L2) and read back in reverse.  Each thread reads back
+// recomputed: a forward sweep stores the state at every 8-token chunk start
+// (checkpoints); then, chunk by chunk from the last, the chunk's 8 states are
+// recomputed from its checkpoint into a scratch slab (512 KB per CTA at d = 128:
+// the slabs of all resident CTAs fit in L2) and read back in reverse.  Each thread reads back
 // only what it wrote, so the slabs need no barriers.  The token rows of the
 // next chunk to be worked on are prefetched into L2 one chunk ahead.
 #include "kda_common.cuh"
@@ -31,7 +31,7 @@ namespace kda {
 namespace bwd {
 
 constexpr int NT = 256;
-constexpr int CK = 16;   // tokens between checkpoints
+constexpr int CK = 8;    // tokens between checkpoints
 
 template <typename Tin, int DK, int DV>
 __global__ void __launch_bounds__(NT, 1)
@@ -298,8 +298,8 @@ static cudaError_t launch_t(const void* q, const void* k, const void* v, const v
 
 }  // namespace bwd
 
-// Floats of workspace the backward needs: checkpoints (dense: nseq * ceil(T / 16)
-// per head; packed: floor(T / 16) + nseq per head) and one 16-state scratch slab
+// Floats of workspace the backward needs: checkpoints (dense: nseq * ceil(T / 8)
+// per head; packed: floor(T / 8) + nseq per head) and one 8-state scratch slab
 // per (sequence, head).
 size_t backward_workspace_floats(bool packed, int64_t nseq, int64_t T, int H, int DK, int DV) {
     const int64_t cks = packed ? T / bwd::CK + nseq : nseq * ((T + bwd::CK - 1) / bwd::CK);

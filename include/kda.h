@@ -347,9 +347,9 @@ kda_status_t kda_forward_noalloc(const void* q, const void* k, const void* v,
  *   Supported: d_k, d_v in {64, 128}; in_dtype KDA_F32 or KDA_BF16; S0,
  *     dS_final, dS0 and workspace 16-byte aligned.
  *   The kernel keeps the state and its gradient in registers, one CTA per
- *   (sequence, head), and recomputes states from checkpoints taken every 16
+ *   (sequence, head), and recomputes states from checkpoints taken every 8
  *   tokens: cost grows with the longest sequence, and the workspace holds
- *   ceil(T / 16) + 16 states of d_k x d_v fp32 per (sequence, head).
+ *   ceil(T / 8) + 8 states of d_k x d_v fp32 per (sequence, head).
  *
  *   Returns KDA_OK; KDA_ERR_INVALID_ARG (missing or misaligned pointer, bad
  *   size, workspace too small); KDA_ERR_UNSUPPORTED (head dims, more than

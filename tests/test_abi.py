@@ -185,9 +185,9 @@ def test_backward_rejects_before_launch():
 
 def test_backward_workspace_sizes():
     mat = 128 * 128 * 4
-    # dense: ceil(T / 16) checkpoints per (sequence, head) plus a 16-state slab
-    assert kda.kda_backward_workspace_bytes(8, 4096, 32, 128, 128) == (8 * 256 + 8 * 16) * 32 * mat
-    assert kda.kda_backward_workspace_bytes(1, 17, 1, 128, 128) == (2 + 16) * mat
-    # packed: floor(T / 16) + num_seqs checkpoints per head
+    # dense: ceil(T / 8) checkpoints per (sequence, head) plus an 8-state slab
+    assert kda.kda_backward_workspace_bytes(8, 4096, 32, 128, 128) == (8 * 512 + 8 * 8) * 32 * mat
+    assert kda.kda_backward_workspace_bytes(1, 9, 1, 128, 128) == (2 + 8) * mat
+    # packed: floor(T / 8) + num_seqs checkpoints per head
     assert kda.kda_backward_workspace_bytes(1, 1000, 2, 128, 128, num_seqs=3) == \
-        ((1000 // 16 + 3) * 2 + 3 * 2 * 16) * mat
+        ((1000 // 8 + 3) * 2 + 3 * 2 * 8) * mat
