@@ -42,6 +42,17 @@ def test_forward_bytes_and_flops_of_the_default_workload():
     assert b.forward_flops(w, 1) == 6 * 128 * 128 + 2 * 64 * (3 * 128 + 2 * 128) == 180224
 
 
+def test_backward_bytes_and_flops():
+    b = _bench()
+    w = _workload(b.DEFAULT_WORKLOAD)
+    # per (token, head): bf16 q, k, alpha, v, dout, beta read; fp32 dq, dk, dalpha, dv, dbeta written
+    assert b.backward_bytes(w, 1, 0, True) == 2 * (3 * 128 + 2 * 128 + 1) + 4 * (3 * 128 + 128 + 1)
+    # per (sequence, head): S0 and dS_final read, dS0 written (fp32)
+    assert b.backward_bytes(w, 0, 1, True) == 3 * 4 * 128 * 128
+    assert b.backward_bytes(w, 0, 1, False) == 2 * 4 * 128 * 128
+    assert b.backward_flops(w, 1) == 31 * 128 * 128
+
+
 def test_decode_bytes():
     b = _bench()
     w = _workload("decode_N256_H32_d128")
