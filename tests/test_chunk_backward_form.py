@@ -25,8 +25,9 @@ boundaries (the order a chunk-parallel backward kernel would use):
     dlog a_s = sum_{r >= s} dg_r;    dalpha = dlog a / a where e^-5 <= alpha <= 1, else 0
 
 Plain gamma ratios are exact enough in fp64 (a 64-token product of gates >= e^-5
-stays above e^-320); a CUDA kernel would use the sub-chunk factorisation of
-test_chunk_form.py for the fp32 range.
+stays above e^-320).  In fp32 a kernel takes the decay gradients of A and P from
+the tensor-core forward's bounded sub-chunk factors instead; the last test shows
+that form gives the same gradients.
 """
 import numpy as np
 import pytest
@@ -153,3 +154,63 @@ def test_chunk_backward_equals_token_backward(C, T):
     for name, g_, r in zip(names, got, ref):
         r = r[0, :, 0] if name != "dS0" else r[0, 0]
         assert _rel(g_, r) < 1e-9, (name, _rel(g_, r))
+
+
+def _decay_grads_gamma_form(K, Q, b, g, dA, dP):
+    """dg of A and P through plain gamma = e^g (the form above): X dX - Z dZ + Qt dQt."""
+    gam = np.exp(g)
+    X, Z, Qt = K * gam, K / gam, Q * gam
+    dX = b[:, None] * (dA @ Z)                      # A = strict(diag(b) X Z^T)
+    dZ = (b[:, None] * dA).T @ X + dP.T @ Qt        # and P = lower(Qt Z^T)
+    dQt = dP @ Z
+    return X * dX - Z * dZ + Qt * dQt
+
+
+def _decay_grads_factored(K, Q, b, g, dA, dP, sub=32):
+    """The same gradients from the tensor-core kernel's factors: sub-chunks I of `sub`
+    tokens with reference token ref_I = sub I + sub/2 - 1, left factors
+    lam_r = e^{g_r - g_ref(I(r))} and right factors rho^I_j = e^{g_ref(I) - g_j}
+    (j < end of I), so that D(r, j) = lam_r rho^{I(r)}_j.  With L = K lam, Lq = Q lam,
+    R^I = K rho^I:  dg_r = L_r dL_r + Lq_r dLq_r - sum_I R^I_r dR^I_r  (the reference's
+    own derivative cancels between left and right)."""
+    C = K.shape[0]
+    nsub = C // sub
+    ref = np.array([sub * (r // sub) + sub // 2 - 1 for r in range(C)])
+    lam = np.exp(g - g[ref])
+    L, Lq = K * lam, Q * lam
+    dg = np.zeros_like(g)
+    dL = np.zeros_like(K)
+    dLq = np.zeros_like(K)
+    for I in range(nsub):
+        rows = slice(sub * I, sub * (I + 1))
+        cols = slice(0, sub * (I + 1))                 # j < end of I
+        rho = np.exp(g[sub * I + sub // 2 - 1] - g[cols])
+        R = K[cols] * rho
+        dAI, dPI = dA[rows, cols], dP[rows, cols]
+        dL[rows] = b[rows, None] * (dAI @ R)
+        dLq[rows] = dPI @ R
+        dR = (b[rows, None] * dAI).T @ L[rows] + dPI.T @ Lq[rows]
+        dg[cols] -= R * dR
+        # every factor stays within the fp32 range (e^88): a row is at most sub/2 tokens
+        # from its reference and each gate is >= e^-5, so |log lam| <= 5 sub/2 = 80, and
+        # log rho <= 80 (tokens before the reference give rho <= 1)
+        assert np.all(np.abs(np.log(lam[rows])) <= 5.0 * sub / 2 + 1e-9)
+        assert np.all(np.log(rho) <= 5.0 * sub / 2 + 1e-9)
+    dg += L * dL + Lq * dLq
+    return dg
+
+
+@pytest.mark.parametrize("seed", [0, 1, 2])
+def test_factored_decay_gradients_equal_gamma_form(seed):
+    rng = np.random.default_rng(seed)
+    C, dk = 64, 24
+    K, Q = rng.standard_normal((C, dk)), rng.standard_normal((C, dk))
+    a = np.clip(np.exp(-np.log1p(np.exp(rng.standard_normal((C, dk))))), np.exp(-5.0), 1.0)
+    a[:, :3] = np.exp(-5.0)                         # channels decaying as fast as allowed
+    g = np.cumsum(np.log(a), axis=0)
+    b = rng.uniform(0, 1, C)
+    dA = np.tril(rng.standard_normal((C, C)), -1)
+    dP = np.tril(rng.standard_normal((C, C)))
+    want = _decay_grads_gamma_form(K, Q, b, g, dA, dP)
+    got = _decay_grads_factored(K, Q, b, g, dA, dP)
+    assert np.allclose(got, want, rtol=1e-9, atol=1e-9 * np.abs(want).max())
