@@ -291,7 +291,7 @@ kda_status_t kda_selftest_timeout(uint64_t limit_ns, kda_stream_t stream);
 
 /*
  * kda_forward_noalloc -- kda_forward's tensor-core path without any device
- * allocation.  The paper has no counterpart: this exists for callers that
+ * allocation.  The pages have no counterpart: this exists for callers that
  * cannot call cudaMalloc (for example a server or training loop that has
  * reserved the device memory for its own pool, or a latency-critical loop in
  * which an allocation may synchronise the device).  kda_forward allocates one
