@@ -153,7 +153,7 @@ class ClockSampler:
             except Exception:
                 self._h = pynvml.nvmlDeviceGetHandleByIndex(device_index)
             self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(self._h, pynvml.NVML_CLOCK_SM)
-        except Exception as exc:  # pragma: no cover - depends on the box
+        except Exception as exc:  # pragma: no cover - depends on the machine
             self.error = repr(exc)
         self._t = threading.Thread(target=self._run, daemon=True)
 

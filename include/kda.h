@@ -50,7 +50,7 @@ typedef enum {
 typedef enum {
     KDA_OK = 0,
     KDA_ERR_INVALID_ARG = 1,     /* a NULL, misaligned or inconsistent argument */
-    KDA_ERR_UNSUPPORTED = 2,     /* valid, but a size or dtype this build has no kernel for */
+    KDA_ERR_UNSUPPORTED = 2,     /* valid, but a size or dtype the library has no kernel for */
     KDA_ERR_CUDA = 3,            /* a CUDA runtime error (launch or device) */
     KDA_ERR_DEVICE_TIMEOUT = 4   /* a bounded device-side wait gave up */
 } kda_status_t;
