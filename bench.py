@@ -321,6 +321,38 @@ def time_oracle(w, inp, budget_s: float, cores: int):
             P = min(len(pairs), int(P * grow))
 
 
+def time_oracle_backward(w, inp, dout, dSf, budget_s: float, cores: int):
+    """Time the oracle's fp64 backward on a bounded sample of a dense forward workload:
+    the first P (sequence, head) pairs over their first Ts tokens (the oracle keeps
+    every state, so Ts stays at most 1024), grown until a run takes about `budget_s`.
+    Returns (tokens_per_s, seconds, description)."""
+    import numpy as np
+    import oracle
+    f = lambda t: t.detach().float().cpu().numpy()
+    B, T, H = inp["q"].shape[0], inp["q"].shape[1], w.H
+    pairs = [(b, h) for b in range(B) for h in range(H)]
+    P, Ts = min(len(pairs), max(1, cores)), min(T, 256)
+    while True:
+        sel = pairs[:P]
+        pick = lambda x: np.stack([f(x[b, :Ts, h]) for b, h in sel])[:, :, None]
+        s0 = (np.stack([f(inp["S0"][b, h]) for b, h in sel])[:, None]
+              if inp.get("S0") is not None else None)
+        dsf = np.stack([f(dSf[b, h]) for b, h in sel])[:, None]
+        t0 = time.perf_counter()
+        oracle.backward(pick(inp["q"]), pick(inp["k"]), pick(inp["v"]), pick(inp["alpha"]),
+                        np.stack([f(inp["beta"][b, :Ts, h]) for b, h in sel])[:, :, None],
+                        pick(dout), s0, dsf, nthreads=cores)
+        dt = time.perf_counter() - t0
+        if dt >= 0.5 * budget_s or (P == len(pairs) and Ts == min(T, 1024)):
+            desc = "%d (sequence, head) pairs x first %d tokens, backward" % (P, Ts)
+            return (P * Ts / H) / dt, dt, desc
+        grow = max(2.0, min(8.0, budget_s / max(dt, 1e-3)))
+        if Ts < min(T, 1024):
+            Ts = min(T, 1024, int(Ts * grow))
+        else:
+            P = min(len(pairs), int(P * grow))
+
+
 # ---------------------------------------------------------------- arms
 
 def run_reference(args, w):
@@ -545,10 +577,14 @@ def run_ours(args, w):
             "gpu_launches": int(launches),
             "e2e": e2e,
         }
-        if world == 1 and not args.no_cpu_baseline:
+        # (the backward's sample is taken over dense sequences only)
+        if world == 1 and not args.no_cpu_baseline and not (args.backward and w.kind != "forward"):
             import oracle
             cores = oracle.available_cores()
-            r, dt, desc = time_oracle(w, inp, args.cpu_budget, cores)
+            if args.backward:
+                r, dt, desc = time_oracle_backward(w, inp, dout, dSf, args.cpu_budget, cores)
+            else:
+                r, dt, desc = time_oracle(w, inp, args.cpu_budget, cores)
             line["cpu_baseline"] = {"value": r, "unit": "tokens/s", "cores": cores,
                                     "kind": "oracle", "sample": desc, "seconds": dt}
         print(json.dumps(line), flush=True)

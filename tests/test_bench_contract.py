@@ -53,6 +53,23 @@ def test_backward_bytes_and_flops():
     assert b.backward_flops(w, 1) == 31 * 128 * 128
 
 
+def test_oracle_backward_baseline_sample():
+    """The backward line's cpu_baseline times the oracle's backward (not its forward)
+    on a bounded sample of the workload."""
+    import torch
+    b = _bench()
+    w = _workload("fp32_T256_d64")
+    sys.path.insert(0, ROOT)
+    from gated_delta_rule_138_b200 import inputs
+    inp = inputs.draw_forward(2, 64, 3, 64, 64, "f32", 5, device="cpu", s0=True)
+    w = type(w)(**dict(w.__dict__, B=2, T=64, H=3))
+    g = torch.Generator().manual_seed(1)
+    dout = torch.randn(2, 64, 3, 64, generator=g)
+    dSf = torch.randn(2, 3, 64, 64, generator=g)
+    rate, secs, desc = b.time_oracle_backward(w, inp, dout, dSf, 0.01, 2)
+    assert rate > 0 and secs > 0 and "backward" in desc
+
+
 def test_decode_bytes():
     b = _bench()
     w = _workload("decode_N256_H32_d128")
