@@ -663,6 +663,8 @@ def main():
     ap.add_argument("--e2e-steps", type=int, default=10,
                     help="steps of the end-to-end (host buffers) measurement; 0 skips it")
     args = ap.parse_args()
+    if args.backward and (args.fused or args.seqpar):
+        ap.error("--backward times kda_backward alone (not with --fused or --seqpar)")
     from gated_delta_rule_138_b200 import inputs as gen
     w = gen.WORKLOADS[args.workload]
     if args.impl == "reference":
