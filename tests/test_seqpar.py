@@ -13,7 +13,7 @@ import gated_delta_rule_138_b200 as kda
 from gated_delta_rule_138_b200 import inputs as gen
 from gated_delta_rule_138_b200.seqpar import split_time
 
-from _parity import np32, oracle_forward, rel_l2
+from _parity import check_o, check_S, np32, oracle_forward
 
 pytestmark = pytest.mark.gpu
 DEV = "cuda"
@@ -37,8 +37,8 @@ def test_segment_maps_match_their_definition():
                           None)
     got = f(maps)
     assert np.abs(M).max() > 0.1          # a non-trivial map
-    assert rel_l2(got[..., :d], M) <= 2e-2
-    assert rel_l2(got[..., d:], N) <= 2e-2
+    check_S(got[..., :d], M, 2e-2)
+    check_S(got[..., d:], N, 2e-2)
 
 
 def test_segment_scan_composes_in_order():
@@ -52,7 +52,7 @@ def test_segment_scan_composes_in_order():
     m = maps.double().cpu().numpy()
     for i in range(G):
         ref = m[i, ..., :d] @ ref + m[i, ..., d:]
-    assert rel_l2(np32(out), ref) <= 1e-5
+    check_S(np32(out), ref, 1e-5)
     # no maps: a copy of S0; in place allowed
     same = kda.kda_segment_scan(maps[:0], S0.clone())
     torch.cuda.synchronize()
@@ -78,8 +78,8 @@ def test_ranks_emulated_in_one_process(world, T):
         outs.append(o)
     torch.cuda.synchronize()
     ro, rS = oracle_forward(inp)
-    assert rel_l2(np32(torch.cat(outs, dim=1)), ro) <= 2e-2
-    assert rel_l2(np32(S_end), rS) <= 2e-2
+    check_o(np32(torch.cat(outs, dim=1)), ro, 2e-2)
+    check_S(np32(S_end), rS, 2e-2)
 
 
 def _free_port():
@@ -122,5 +122,5 @@ def test_two_ranks_through_torch_distributed():
     inp = gen.draw_forward(1, T, 2, 128, 128, "bf16", 1320, device="cpu", s0=True)
     ro, rS = oracle_forward(inp)
     out = np.concatenate([res[r][0] for r in range(world)], axis=1)
-    assert rel_l2(out, ro) <= 2e-2
-    assert rel_l2(res[world - 1][1], rS) <= 2e-2
+    check_o(out, ro, 2e-2)
+    check_S(res[world - 1][1], rS, 2e-2)
