@@ -14,9 +14,13 @@
 // holds this array until the process exits.  Each CTA always writes its own
 // word (0 = finished, 1 = a bounded wait gave up), so nothing has to be cleared
 // before a call.  All calls on a device share the array and it keeps the last
-// call's contents; two calls that overlap on the GPU race on it.
+// call's contents; two calls that overlap on the GPU race on it.  The caller
+// learns of a timeout by reading the words back with kda_noalloc_status, which
+// allocates nothing either (a copy into caller-provided or stack host memory).
 #include <cstdio>
 #include <mutex>
+
+#include "kda_sm100.cuh"
 
 #include "../../include/kda.h"
 #include "kda_common.cuh"
@@ -40,7 +44,10 @@ int* g_addr[kMaxDevices] = {};
 
 // Device address of the scratch array for the current device.  In host code
 // the array's name is only a host-side stand-in, so the address is taken from
-// the runtime once per device (with that device current) and cached.
+// the runtime once per device (with that device current) and cached.  The
+// cache assumes the device context lives as long as the process: after a
+// cudaDeviceReset the module is loaded afresh and the cached address is stale,
+// so a program that resets a device must not call these entry points again.
 cudaError_t scratch_address(int** out) {
     int dev = 0;
     cudaError_t e = cudaGetDevice(&dev);
@@ -108,5 +115,55 @@ extern "C" kda_status_t kda_forward_noalloc(const void* q, const void* k, const 
     e = kda::launch_chunk_tc_cta_status(q, k, v, alpha, beta, S0, cu_seqlens, (int)nseq, out,
                                         S_final, rows, T, H, status,
                                         reinterpret_cast<cudaStream_t>(stream));
+    return e == cudaSuccess ? KDA_OK : fail_cuda(e);
+}
+
+namespace {
+// Waits, bounded by limit_ns, on an mbarrier that nothing arrives on, then
+// records the outcome in word `word` of the fixed array exactly as a forward
+// CTA whose wait gave up does (1).  No fault, no hang.
+__global__ void kda_noalloc_selftest_kernel(uint64_t limit_ns, int word) {
+    __shared__ uint64_t bar;
+    if (threadIdx.x == 0) {
+        kda::sm100::mbar_init(&bar, 1);
+        kda::sm100::mbar_fence_init();
+    }
+    __syncthreads();
+    const bool done = kda::sm100::mbar_wait_ns(&bar, 0, limit_ns);
+    if (threadIdx.x == 0) g_kda_noalloc_status[word] = done ? 0 : 1;
+}
+}  // namespace
+
+extern "C" kda_status_t kda_noalloc_status(int32_t num_words, int32_t* host_words,
+                                           kda_stream_t stream) {
+    if (num_words < 0 || num_words > KDA_NOALLOC_MAX_SEQ_HEADS) return KDA_ERR_INVALID_ARG;
+    int* unused = nullptr;
+    cudaError_t e = scratch_address(&unused);   // loads the module on this device if needed
+    if (e != cudaSuccess) return fail_cuda(e);
+    e = cudaStreamSynchronize(reinterpret_cast<cudaStream_t>(stream));
+    if (e != cudaSuccess) return fail_cuda(e);
+    bool any = false;
+    constexpr int kBlock = 1024;
+    int32_t buf[kBlock];
+    for (int32_t w0 = 0; w0 < num_words; w0 += kBlock) {
+        const int32_t n = num_words - w0 < kBlock ? num_words - w0 : kBlock;
+        int32_t* dst = host_words ? host_words + w0 : buf;
+        e = cudaMemcpyFromSymbol(dst, g_kda_noalloc_status, sizeof(int32_t) * (size_t)n,
+                                 sizeof(int32_t) * (size_t)w0, cudaMemcpyDeviceToHost);
+        if (e != cudaSuccess) return fail_cuda(e);
+        for (int32_t i = 0; i < n; ++i) any |= dst[i] != 0;
+    }
+    return any ? KDA_ERR_DEVICE_TIMEOUT : KDA_OK;
+}
+
+extern "C" kda_status_t kda_noalloc_selftest_timeout(uint64_t limit_ns, int32_t word,
+                                                     kda_stream_t stream) {
+    if (limit_ns == 0 || limit_ns > 10000000000ull) return KDA_ERR_INVALID_ARG;
+    if (word < 0 || word >= KDA_NOALLOC_MAX_SEQ_HEADS) return KDA_ERR_INVALID_ARG;
+    int* unused = nullptr;
+    cudaError_t e = scratch_address(&unused);
+    if (e != cudaSuccess) return fail_cuda(e);
+    kda_noalloc_selftest_kernel<<<1, 32, 0, reinterpret_cast<cudaStream_t>(stream)>>>(limit_ns, word);
+    e = cudaGetLastError();
     return e == cudaSuccess ? KDA_OK : fail_cuda(e);
 }

@@ -87,6 +87,10 @@ def load_library(build_if_missing: bool = True) -> ctypes.CDLL:
     lib.kda_selftest_timeout.argtypes = [ctypes.c_uint64, vp]
     lib.kda_forward_noalloc.restype = ctypes.c_int
     lib.kda_forward_noalloc.argtypes = lib.kda_forward.argtypes
+    lib.kda_noalloc_status.restype = ctypes.c_int
+    lib.kda_noalloc_status.argtypes = [i32, vp, vp]
+    lib.kda_noalloc_selftest_timeout.restype = ctypes.c_int
+    lib.kda_noalloc_selftest_timeout.argtypes = [ctypes.c_uint64, i32, vp]
     lib.kda_forward_fused.restype = ctypes.c_int
     lib.kda_forward_fused.argtypes = lib.kda_forward.argtypes
     lib.kda_decode_step_fused.restype = ctypes.c_int
@@ -330,6 +334,25 @@ def kda_forward_noalloc(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, alpha
                                  _dt(q), _dt(out), _stream(stream))
     _check("kda_forward_noalloc", st)
     return out, S_final
+
+
+def kda_noalloc_status(num_words: int, stream=None, check: bool = True) -> list:
+    """Synchronise `stream` and read the first num_words status words of
+    kda_forward_noalloc's fixed array (word n * H + h of the last call: 0 =
+    finished, 1 = that CTA's bounded wait gave up).  Raises KdaError
+    (KDA_ERR_DEVICE_TIMEOUT) if any is set and `check`; returns the words."""
+    words = (ctypes.c_int32 * max(int(num_words), 1))()
+    st = load_library().kda_noalloc_status(int(num_words), ctypes.cast(words, ctypes.c_void_p),
+                                           _stream(stream))
+    if st not in (0, 4) or (st == 4 and check):
+        _check("kda_noalloc_status", st)
+    return list(words)[:int(num_words)]
+
+
+def kda_noalloc_selftest_timeout(limit_ns: int, word: int, stream=None) -> None:
+    """A bounded wait that must give up, reported in word `word` of the fixed array."""
+    _check("kda_noalloc_selftest_timeout",
+           load_library().kda_noalloc_selftest_timeout(int(limit_ns), int(word), _stream(stream)))
 
 
 def kda_decode_step(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, alpha: torch.Tensor,

@@ -306,13 +306,17 @@ kda_status_t kda_selftest_timeout(uint64_t limit_ns, kda_stream_t stream);
  *   the library until the process exits).  More (sequence, head) pairs than
  *   that: KDA_ERR_UNSUPPORTED, with the reason in kda_last_error().
  *   Every call on a device shares the array, which keeps the last call's
- *   contents (0 = finished, 1 = a bounded device wait gave up); each CTA
- *   writes its own word, so nothing needs clearing first.  Calls whose
- *   kernels overlap on the GPU race on the array.
+ *   contents (word n * H + h: 0 = finished, 1 = a bounded device wait of that
+ *   (sequence, head) gave up and its out / S_final rows are not valid); each
+ *   CTA writes its own word, so nothing needs clearing first.  The call itself
+ *   returns KDA_OK once the kernel is launched: read the words back with
+ *   kda_noalloc_status to learn of a timeout.  Calls whose kernels overlap on
+ *   the GPU race on the array.
  *   The first call on a device looks up the array's device address
- *   (cudaGetSymbolAddress) with that device current; make that first call
- *   before any stream capture.  No cudaMalloc, cudaFree or other allocating
- *   routine is called.
+ *   (cudaGetSymbolAddress) with that device current and keeps it for the
+ *   life of the process; make that first call before any stream capture, and
+ *   do not use these entry points on a device after cudaDeviceReset.  No
+ *   cudaMalloc, cudaFree or other allocating routine is called.
  */
 kda_status_t kda_forward_noalloc(const void* q, const void* k, const void* v,
                                  const void* alpha, const void* beta, const float* S0,
@@ -321,6 +325,28 @@ kda_status_t kda_forward_noalloc(const void* q, const void* k, const void* v,
                                  int32_t B, int64_t T, int32_t H, int32_t d_k, int32_t d_v,
                                  int32_t chunk, kda_dtype_t in_dtype, kda_dtype_t out_dtype,
                                  kda_stream_t stream);
+
+/*
+ * Status words of kda_forward_noalloc (no counterpart on the pages; allocates
+ * nothing).  Synchronises `stream`, then copies the first num_words words
+ * (0 .. KDA_NOALLOC_MAX_SEQ_HEADS) of the fixed array of the current device
+ * into host_words (host memory the caller owns, num_words int32 values; NULL:
+ * the words are only inspected) and returns KDA_ERR_DEVICE_TIMEOUT if any of
+ * them is non-zero, KDA_OK if all are 0, KDA_ERR_INVALID_ARG for a bad count,
+ * KDA_ERR_CUDA on a runtime error.  After a kda_forward_noalloc call of
+ * N sequences and H heads, the first N * H words are that call's.
+ */
+kda_status_t kda_noalloc_status(int32_t num_words, int32_t* host_words, kda_stream_t stream);
+
+/*
+ * Self-test of kda_forward_noalloc's timeout report (no counterpart on the
+ * pages).  Launches one warp that waits, bounded by limit_ns nanoseconds
+ * (1 ns .. 10 s), on an mbarrier nothing arrives on, with the forward kernel's
+ * bounded wait, and writes the outcome into word `word` (0 ..
+ * KDA_NOALLOC_MAX_SEQ_HEADS - 1) of the fixed array as a forward CTA does
+ * (1 = gave up).  Nothing faults or hangs; allocates nothing.
+ */
+kda_status_t kda_noalloc_selftest_timeout(uint64_t limit_ns, int32_t word, kda_stream_t stream);
 
 /*
  * kda_backward -- gradients of kda_forward's outputs with respect to all of

@@ -191,3 +191,12 @@ def test_backward_workspace_sizes():
     # packed: floor(T / 8) + num_seqs checkpoints per head
     assert kda.kda_backward_workspace_bytes(1, 1000, 2, 128, 128, num_seqs=3) == \
         ((1000 // 8 + 3) * 2 + 3 * 2 * 8) * mat
+
+
+def test_noalloc_status_rejects_bad_counts_before_any_copy():
+    lib = kda.load_library()
+    assert lib.kda_noalloc_status(-1, None, None) == 1
+    assert lib.kda_noalloc_status(16384 + 1, None, None) == 1
+    assert lib.kda_noalloc_selftest_timeout(0, 0, None) == 1          # zero limit
+    assert lib.kda_noalloc_selftest_timeout(1000, -1, None) == 1      # word out of range
+    assert lib.kda_noalloc_selftest_timeout(1000, 16384, None) == 1
