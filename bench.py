@@ -3,8 +3,11 @@
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME] [--impl ours|reference]
 
-One step = one kda_forward call (the whole chunk-parallel forward, one kernel
-launch) over one batch of seeded synthetic inputs already resident in HBM.
+One step = one kda_forward call (the whole chunk-parallel forward) over one
+batch of seeded synthetic inputs already resident in HBM.  The default workload
+is the long-context one (B=1, H=32, T=2^20, d=128): few (sequence, head) pairs,
+so the forward splits every sequence into time segments (segment maps, scan,
+forward: three launches per step, timed together).
 For N > 1 (launched with torch.distributed.run, one process per GPU) every
 rank runs its own batch (independent sequences, no data-path collective:
 weak scaling); the time is the max over ranks and `value` counts all ranks'
@@ -35,7 +38,7 @@ if ROOT not in sys.path:
     sys.path.insert(0, ROOT)
 
 METRIC = "KDA fwd tokens/s and TFLOP/s (% roofline) at H=32, d=128, 1 B200"
-DEFAULT_WORKLOAD = "bf16_B8_T4096_H32_d128"
+DEFAULT_WORKLOAD = "bf16_B1_T1M_H32_d128"
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 
 
@@ -353,6 +356,71 @@ def time_oracle_backward(w, inp, dout, dSf, budget_s: float, cores: int):
             P = min(len(pairs), int(P * grow))
 
 
+# ---------------------------------------------------------------- parity on a sample
+
+def _parity_stats(x, ref, time_axis):
+    """Relative L2 of the whole sample, of its worst (sequence, head) slab and of
+    its worst row (token output, or key row of a state), in fp64."""
+    import numpy as np
+    x = np.asarray(x, np.float64)
+    ref = np.asarray(ref, np.float64)
+    err = x - ref
+    nrm = lambda a, ax: np.sqrt(np.sum(a * a, axis=ax, keepdims=True))
+    glob = float(np.linalg.norm(err) / max(np.linalg.norm(ref), 1e-300))
+    red = (x.ndim - 2, x.ndim - 1) if time_axis is None else (time_axis, x.ndim - 1)
+    s_num, s_den = nrm(err, red), nrm(ref, red)
+    worst_slab = float(np.max(s_num / np.maximum(s_den, 1e-300)))
+    floor = s_den / np.sqrt(x.shape[red[0]])          # rms row norm of the slab
+    worst_row = float(np.max(nrm(err, -1) / np.maximum(np.maximum(nrm(ref, -1), floor), 1e-300)))
+    return {"rel_l2": glob, "worst_head": worst_slab, "worst_row": worst_row}
+
+
+def bench_parity(w, inp, out, Sf, max_tokens=8192):
+    """The bench's own outputs against the oracle on sampled (sequence, head) pairs:
+    o over the first `max_tokens` tokens of each pair, S_final where the pair's
+    whole sequence fits in that budget.  Seconds of host time, not the tests."""
+    import numpy as np
+    import oracle
+    f = lambda t: t.detach().float().cpu().numpy()
+    if w.kind not in ("forward", "varlen"):
+        return None
+    if w.kind == "forward":
+        B, T = inp["q"].shape[0], inp["q"].shape[1]
+        # (batch row, first token, head, length, sequence index)
+        picks = [(0, 0, 0, T, 0), (B - 1, 0, w.H - 1, T, B - 1)]
+    else:
+        cu = f(inp["cu_seqlens"]).astype(np.int64)
+        lens = np.diff(cu)
+        picks = [(0, int(cu[n]), h, int(lens[n]), n)
+                 for n, h in ((int(np.argmin(lens)), 0), (int(np.argmax(lens)), w.H - 1))]
+    res = {"o": [], "S": []}
+    for bb, a, h, L, n in picks:
+        t1 = min(L, max_tokens)
+        sl = lambda x: f(x[bb:bb + 1, a:a + t1, h:h + 1])
+        S0 = inp.get("S0")
+        s0 = None if S0 is None else f(S0[n:n + 1, h:h + 1])
+        ro, rS = oracle.forward(sl(inp["q"]), sl(inp["k"]), sl(inp["v"]), sl(inp["alpha"]),
+                                sl(inp["beta"]), s0)
+        res["o"].append((f(out[bb:bb + 1, a:a + t1, h:h + 1]), ro))
+        if t1 == L:
+            res["S"].append((f(Sf[n:n + 1, h:h + 1]), rS))
+    pack = lambda pairs: (np.concatenate([p[0] for p in pairs], axis=2),
+                          np.concatenate([p[1] for p in pairs], axis=2))
+    line = {"sample": "%d (sequence, head) pairs, o over the first <= %d tokens%s"
+            % (len(picks), max_tokens, ", S_final" if res["S"] else "")}
+    # slabs are the sampled heads (axis 2 after concatenation)
+    xo, ro = pack(res["o"]) if w.kind == "forward" else (None, None)
+    if w.kind == "forward":
+        line["o"] = _parity_stats(xo, ro, 1)
+    else:
+        st = [_parity_stats(x, r, 1) for x, r in res["o"]]
+        line["o"] = {k: max(d[k] for d in st) for k in st[0]}
+    if res["S"]:
+        st = [_parity_stats(x, r, None) for x, r in res["S"]]
+        line["S_final"] = {k: max(d[k] for d in st) for k in st[0]}
+    return line
+
+
 # ---------------------------------------------------------------- arms
 
 def run_reference(args, w):
@@ -381,7 +449,7 @@ def run_reference(args, w):
         "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
         "ms_per_step": 1e3 * secs / max(1, args.steps), "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-        "config": config_of(w, args.gpus),
+        "config": dict(config_of(w, args.gpus), l2=l2_note(workload_bytes(w))),
         "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": cores, "kind": "oracle",
                          "sample": desc},
         "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0,
@@ -389,6 +457,23 @@ def run_reference(args, w):
     }
     print(json.dumps(line), flush=True)
     del torch
+
+
+def workload_bytes(w) -> int:
+    """Algorithmic bytes of one step of a named workload, from its definition alone."""
+    if w.kind == "decode":
+        return decode_bytes(w, w.B * w.H)
+    if w.kind == "varlen":
+        from gated_delta_rule_138_b200 import inputs as gen
+        total = int(sum(gen.varlen_lengths(w.nseq, w.min_len, w.max_len, w.seed + 999)))
+        return forward_bytes(w, total * w.H, w.nseq * w.H, w.s0)
+    if w.kind == "pooled":
+        return forward_bytes(w, w.B * w.T * w.H, w.B * w.H, True)
+    return forward_bytes(w, w.B * w.T * w.H, w.B * w.H, w.s0)
+
+
+def l2_note(algo_bytes) -> str:
+    return "no flush: inputs %.2f GB per step > 126 MB L2" % (algo_bytes / 1e9)
 
 
 def config_of(w, n_gpus):
@@ -561,9 +646,7 @@ def run_ours(args, w):
             "vs_baseline": None,
             "dtype": "bf16" if kname.startswith("chunk_tc_bf16") else "f32",
             "data": "synthetic (seeded generators, the workload's shapes and distributions)",
-            "config": dict(cfg,
-                           l2="no flush: inputs %.2f GB per step > 126 MB L2"
-                              % (algo_bytes / 1e9)),
+            "config": dict(cfg, l2=l2_note(algo_bytes)),
             "tflops": tflops,
             "roofline": {"bound": "hbm", "achieved": achieved, "peak": peaks["hbm_gbs"],
                          "unit": "GB/s", "frac": achieved / peaks["hbm_gbs"],
@@ -577,6 +660,9 @@ def run_ours(args, w):
             "gpu_launches": int(launches),
             "e2e": e2e,
         }
+        if w.kind in ("forward", "varlen") and not args.backward and not seqpar \
+                and not args.fused and not args.no_parity:
+            line["parity"] = bench_parity(w, inp, out, Sf)
         # (the backward's sample is taken over dense sequences only)
         if world == 1 and not args.no_cpu_baseline and not (args.backward and w.kind != "forward"):
             import oracle
@@ -593,36 +679,118 @@ def run_ours(args, w):
         dist.destroy_process_group()
 
 
+def e2e_pieces(w, B, T):
+    """How one step's batch is cut for the copy / compute / copy pipeline of the
+    end-to-end leg: (axis, piece length).  Independent sequences are cut along
+    the batch; a single long sequence along time, each piece starting from the
+    previous piece's S_final (kda_forward's S0 / S_final chaining)."""
+    if w.kind != "forward":
+        return None, 0
+    if B >= 2:
+        return 0, max(1, B // 4)
+    return 1, max(64, min(T, 1 << 17))
+
+
 def run_e2e(args, w, inp, dev, stream, world):
     """Same metric through the public API with host buffers: every step copies
-    its inputs from pinned host memory and reads its result back."""
+    its inputs from pinned host memory and reads its outputs (out and S_final)
+    back.  Host -> device copies, kda_forward calls and device -> host copies run
+    on three streams ordered by events over pieces of the batch (e2e_pieces):
+    piece j+1 is copied in and piece j-1 copied out while piece j computes, and
+    consecutive steps overlap the same way.  One cudaMemcpyAsync per tensor and
+    piece."""
     import torch
     import gated_delta_rule_138_b200 as kda
-    names = [n for n in ("q", "k", "v", "alpha", "beta", "S0", "cu_seqlens")
-             if inp.get(n) is not None]
+    names = [n for n in ("q", "k", "v", "alpha", "beta") if inp.get(n) is not None]
+    cu_d = inp.get("cu_seqlens")
+    B, T = inp["q"].shape[0], inp["q"].shape[1]
+    nseq = B if cu_d is None else cu_d.numel() - 1
+    odt = torch.bfloat16 if w.out_dtype == "bf16" else torch.float32
     try:
-        host = {n: inp[n].cpu().pin_memory() for n in names}
+        host = {n: torch.empty(inp[n].shape, dtype=inp[n].dtype, pin_memory=True).copy_(inp[n])
+                for n in names}
+        S0_h = (torch.empty(inp["S0"].shape, dtype=torch.float32, pin_memory=True).copy_(inp["S0"])
+                if inp.get("S0") is not None else None)
+        out_h = torch.empty(B, T, w.H, w.dv, dtype=odt, pin_memory=True)
+        Sf_h = torch.empty(nseq, w.H, w.dk, w.dv, dtype=torch.float32, pin_memory=True)
     except RuntimeError as exc:
         return {"value": None, "unit": "tokens/s", "note": "pinned host alloc failed: %s" % exc}
-    devb = {n: torch.empty_like(inp[n]) for n in names}
-    cu = devb.get("cu_seqlens")
-    B, T = inp["q"].shape[0], inp["q"].shape[1]
-    nseq = B if cu is None else cu.numel() - 1
-    out = torch.empty(B, T, w.H, w.dv, dtype=torch.bfloat16 if w.out_dtype == "bf16"
-                      else torch.float32, device=dev)
-    Sf = torch.empty(nseq, w.H, w.dk, w.dv, dtype=torch.float32, device=dev)
-    out_h = torch.empty(out.shape, dtype=out.dtype).pin_memory()
-    Sf_h = torch.empty(Sf.shape, dtype=Sf.dtype).pin_memory()
-    h2d = sum(host[n].numel() * host[n].element_size() for n in names)
-    d2h = out_h.numel() * out_h.element_size() + Sf_h.numel() * Sf_h.element_size()
+    axis, plen = e2e_pieces(w, B, T)
+    extent = B if axis == 0 else T
+    bounds = ([(0, extent)] if axis is None else
+              [(a, min(extent, a + plen)) for a in range(0, extent, plen)])
+    sl = lambda t, a, b: t if axis is None else (t[a:b] if axis == 0 else t[:, a:b])
+    nslot = 2
+    pb = bounds[0][1] - bounds[0][0]
+    shape_of = lambda t: ((pb,) + tuple(t.shape[1:]) if axis == 0 else
+                          (t.shape[0], pb) + tuple(t.shape[2:]) if axis == 1 else tuple(t.shape))
+    dslot = [{n: torch.empty(shape_of(inp[n]), dtype=inp[n].dtype, device=dev) for n in names}
+             for _ in range(nslot)]
+    oslot = [torch.empty(shape_of(out_h), dtype=odt, device=dev) for _ in range(nslot)]
+    cu = cu_d.clone() if cu_d is not None else None
+    # state chaining: batch pieces own their rows of S0 / S_final; time pieces pass S along
+    S0_d = torch.empty(nseq, w.H, w.dk, w.dv, dtype=torch.float32, device=dev) \
+        if S0_h is not None else None
+    Sbuf = [torch.empty(nseq, w.H, w.dk, w.dv, dtype=torch.float32, device=dev) for _ in range(2)]
+    s_in, s_out = torch.cuda.Stream(device=dev), torch.cuda.Stream(device=dev)
+    s_cmp = stream
+    ev = lambda: torch.cuda.Event()
+    h2d = sum(host[n].numel() * host[n].element_size() for n in names) + (
+        S0_h.numel() * 4 if S0_h is not None else 0)
+    d2h = out_h.numel() * out_h.element_size() + Sf_h.numel() * 4
+    slot_free = [None] * nslot      # compute of the slot's last piece has read its inputs
+    out_free = [None] * nslot       # its output copy has left the device buffer
+    sf_read = [None]                # the previous step's S_final copy has left Sbuf
+    cu_h = cu_d.cpu().pin_memory() if cu_d is not None else None
+    if cu_h is not None:
+        h2d += cu_h.numel() * 4
 
     def step():
-        for n in names:
-            devb[n].copy_(host[n], non_blocking=True)
-        kda.kda_forward(devb["q"], devb["k"], devb["v"], devb["alpha"], devb["beta"],
-                        devb.get("S0"), cu_seqlens=cu, out=out, S_final=Sf, chunk=w.chunk)
-        out_h.copy_(out, non_blocking=True)
-        Sf_h.copy_(Sf, non_blocking=True)
+        if sf_read[0] is not None:
+            s_cmp.wait_event(sf_read[0])
+        if cu_h is not None:
+            with torch.cuda.stream(s_in):
+                cu.copy_(cu_h, non_blocking=True)
+        if S0_d is not None or cu_h is not None:
+            if S0_d is not None:
+                with torch.cuda.stream(s_in):
+                    S0_d.copy_(S0_h, non_blocking=True)
+            e = ev(); e.record(s_in); s_cmp.wait_event(e)
+        S_prev = S0_d
+        last_sf = None
+        for j, (a, b) in enumerate(bounds):
+            k = j % nslot
+            d, o = dslot[k], oslot[k]
+            n_rows = b - a
+            with torch.cuda.stream(s_in):
+                if slot_free[k] is not None:
+                    s_in.wait_event(slot_free[k])
+                for n in names:
+                    sl(d[n], 0, n_rows).copy_(sl(host[n], a, b), non_blocking=True)
+                e_in = ev(); e_in.record(s_in)
+            s_cmp.wait_event(e_in)
+            if out_free[k] is not None:
+                s_cmp.wait_event(out_free[k])
+            with torch.cuda.stream(s_cmp):
+                dd = {n: sl(d[n], 0, n_rows) for n in names}
+                oo = sl(o, 0, n_rows)
+                if axis == 0:
+                    s0 = None if S0_d is None else S0_d[a:b]
+                    sf = Sbuf[0][a:b]
+                else:
+                    s0 = S_prev
+                    sf = Sbuf[j % 2]
+                kda.kda_forward(dd["q"], dd["k"], dd["v"], dd["alpha"], dd["beta"], s0,
+                                cu_seqlens=cu, out=oo, S_final=sf, chunk=w.chunk)
+                S_prev, last_sf = sf, sf
+                slot_free[k] = ev(); slot_free[k].record(s_cmp)
+            s_out.wait_event(slot_free[k])
+            with torch.cuda.stream(s_out):
+                sl(out_h, a, b).copy_(oo, non_blocking=True)
+                out_free[k] = ev(); out_free[k].record(s_out)
+        with torch.cuda.stream(s_out):
+            Sf_h.copy_(Sbuf[0] if axis == 0 else last_sf, non_blocking=True)
+            sf_read[0] = ev(); sf_read[0].record(s_out)
 
     n = max(1, min(args.steps, args.e2e_steps))
     for _ in range(2):
@@ -630,17 +798,22 @@ def run_e2e(args, w, inp, dev, stream, world):
     torch.cuda.synchronize()
     barrier(world)
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    e0.record(stream)
+    e0.record(s_cmp)
+    s_in.wait_event(e0)
+    s_out.wait_event(e0)
     for _ in range(n):
         step()
-    e1.record(stream)
+    for s_ in (s_in, s_out):
+        e = ev(); e.record(s_); s_cmp.wait_event(e)
+    e1.record(s_cmp)
     torch.cuda.synchronize()
     barrier(world)
     ms = max_over_ranks(e0.elapsed_time(e1), world)
     tokens, _, _ = counts(w, inp)
     total = sum_over_ranks(tokens * n, world)
     return {"value": total / (ms * 1e-3), "unit": "tokens/s", "h2d_bytes_per_step": int(h2d),
-            "d2h_bytes_per_step": int(d2h), "steps": n}
+            "d2h_bytes_per_step": int(d2h), "steps": n, "pieces": len(bounds),
+            "overlap": "h2d / compute / d2h streams, %d device slots" % nslot}
 
 
 def main():
@@ -653,6 +826,8 @@ def main():
     ap.add_argument("--cpu-budget", type=float, default=15.0,
                     help="seconds of oracle time for the cpu_baseline sample")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-parity", action="store_true",
+                    help="skip the oracle check of the bench's own outputs on sampled heads")
     ap.add_argument("--fused", action="store_true",
                     help="forward workloads through kda_forward_fused (gates as logits, q and k "
                          "normalised inside the kernel)")

@@ -29,9 +29,26 @@ def _workload(name):
     return inputs.WORKLOADS[name]
 
 
-def test_forward_bytes_and_flops_of_the_default_workload():
+def test_default_workload_is_the_long_context_one():
     b = _bench()
     w = _workload(b.DEFAULT_WORKLOAD)
+    assert (w.kind, w.B, w.T, w.H, w.dk, w.dv, w.chunk) == ("forward", 1, 1 << 20, 32, 128, 128, 64)
+    # 1282 B per (token, head) over 2^20 x 32 token-heads, S_final written (no S0)
+    assert b.forward_bytes(w, w.T * w.H, w.H, w.s0) == 1282 * (1 << 25) + 65536 * 32
+
+
+def test_e2e_pieces():
+    b = _bench()
+    w = _workload("bf16_B8_T4096_H32_d128")
+    assert b.e2e_pieces(w, 8, 4096) == (0, 2)           # batch rows, four pieces
+    w2 = _workload(b.DEFAULT_WORKLOAD)
+    assert b.e2e_pieces(w2, 1, 1 << 20) == (1, 1 << 17)  # time slices, S chained
+    assert b.e2e_pieces(_workload("varlen_64seq_H16_d128"), 1, 1000) == (None, 0)
+
+
+def test_forward_bytes_and_flops_of_the_batch_workload():
+    b = _bench()
+    w = _workload("bf16_B8_T4096_H32_d128")
     n_th, n_sh = w.B * w.T * w.H, w.B * w.H
     # bf16 d_k = d_v = 128: 2 (3*128 + 128 + 1) + 2*128 = 1282 B per (token, head)
     assert b.forward_bytes(w, 1, 0, True) == 1282
@@ -44,7 +61,7 @@ def test_forward_bytes_and_flops_of_the_default_workload():
 
 def test_backward_bytes_and_flops():
     b = _bench()
-    w = _workload(b.DEFAULT_WORKLOAD)
+    w = _workload("bf16_B8_T4096_H32_d128")
     # per (token, head): bf16 q, k, alpha, v, dout, beta read; fp32 dq, dk, dalpha, dv, dbeta written
     assert b.backward_bytes(w, 1, 0, True) == 2 * (3 * 128 + 2 * 128 + 1) + 4 * (3 * 128 + 128 + 1)
     # per (sequence, head): S0 and dS_final read, dS0 written (fp32)
