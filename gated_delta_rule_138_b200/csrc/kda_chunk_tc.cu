@@ -50,8 +50,11 @@
 // from its own start state.
 #include <cuda.h>
 
+#include <cstdlib>
+
 #include "kda_common.cuh"
 #include "kda_sm100.cuh"
+#include "kda_tc_maps.cuh"
 
 // Optional phase-boundary hook for profiling builds (no-op in the library).
 #ifndef KDA_TC_PHASE
@@ -1303,13 +1306,33 @@ static bool make_map(CUtensorMap* m, const void* base, int64_t rows, int H) {
 
 }  // namespace tc
 
-struct TcMaps {
-    CUtensorMap q, k, a, v, o;
-};
+cudaError_t launch_chunk_tc2(const void* q, const void* k, const void* v, const void* alpha,
+                             const void* beta, const float* S0, const int32_t* cu, int nseq,
+                             void* out, float* S_final, int64_t rows, int64_t T, int H, int* status,
+                             cudaStream_t stream, const int32_t* slots, int num_slots, int fused);
+cudaError_t launch_chunk_tc2_segments(const void* q, const void* k, const void* v, const void* alpha,
+                                      const void* beta, const float* start, const int32_t* cu,
+                                      int nseq, void* out, float* S_final, int64_t rows, int64_t T,
+                                      int H, int nseg, int* status, cudaStream_t stream, int fused);
+cudaError_t launch_chunk_tc2_cta_status(const void* q, const void* k, const void* v,
+                                        const void* alpha, const void* beta, const float* S0,
+                                        const int32_t* cu, int nseq, void* out, float* S_final,
+                                        int64_t rows, int64_t T, int H, int* status,
+                                        cudaStream_t stream);
 
-// out may be null (segment summaries write no output): its map then reuses v's.
-static bool make_maps(TcMaps* m, const void* q, const void* k, const void* v, const void* alpha,
-                      const void* out, int64_t rows, int H) {
+// Which forward kernel the tensor-core entry points use (KDA_TC_KERNEL=2: the
+// pipelined kernel of kda_chunk_tc2.cu; anything else: this file's kernel).
+static bool use_tc2() {
+    static int v = -1;
+    if (v < 0) {
+        const char* e = std::getenv("KDA_TC_KERNEL");
+        v = (e && e[0] == '2') ? 1 : 0;
+    }
+    return v == 1;
+}
+
+bool make_tc_maps(TcMaps* m, const void* q, const void* k, const void* v, const void* alpha,
+                  const void* out, int64_t rows, int H) {
     return tc::make_map(&m->q, q, rows, H) && tc::make_map(&m->k, k, rows, H) &&
            tc::make_map(&m->a, alpha, rows, H) && tc::make_map(&m->v, v, rows, H) &&
            tc::make_map(&m->o, out ? out : v, rows, H);
@@ -1334,8 +1357,11 @@ cudaError_t launch_chunk_tc(const void* q, const void* k, const void* v, const v
                             const void* beta, const float* S0, const int32_t* cu, int nseq,
                             void* out, float* S_final, int64_t rows, int64_t T, int H, int* status,
                             cudaStream_t stream, const int32_t* slots, int num_slots, int fused) {
+    if (use_tc2())
+        return launch_chunk_tc2(q, k, v, alpha, beta, S0, cu, nseq, out, S_final, rows, T, H, status,
+                                stream, slots, num_slots, fused);
     TcMaps m;
-    if (!make_maps(&m, q, k, v, alpha, out, rows, H)) return cudaErrorInvalidValue;
+    if (!make_tc_maps(&m, q, k, v, alpha, out, rows, H)) return cudaErrorInvalidValue;
     const tc::Segments whole{1, 1, nullptr, nullptr, slots, num_slots};
     return fused ? launch_tc_t<false, false, true>(m, beta, S0, cu, nseq, out, S_final, T, H, status,
                                                    whole, stream)
@@ -1360,7 +1386,7 @@ cudaError_t launch_chunk_tc_segmented(const void* q, const void* k, const void* 
                                       int* status, cudaStream_t stream, int fused) {
     if (nseg < 2 || nseq * (int64_t)nseg > 65535) return cudaErrorInvalidValue;
     TcMaps m;
-    if (!make_maps(&m, q, k, v, alpha, out, rows, H)) return cudaErrorInvalidValue;
+    if (!make_tc_maps(&m, q, k, v, alpha, out, rows, H)) return cudaErrorInvalidValue;
     float* maps = workspace;
     float* start = workspace + (size_t)nseq * H * (nseg - 1) * tc::DK * (tc::DK + tc::DV);
     const tc::Segments summary{nseg, nseg - 1, nullptr, maps};
@@ -1373,6 +1399,9 @@ cudaError_t launch_chunk_tc_segmented(const void* q, const void* k, const void* 
         S0, maps, start, nseg, H);
     e = cudaGetLastError();
     if (e != cudaSuccess) return e;
+    if (use_tc2())
+        return launch_chunk_tc2_segments(q, k, v, alpha, beta, start, cu, nseq, out, S_final, rows, T,
+                                         H, nseg, status, stream, fused);
     const tc::Segments fwd{nseg, nseg, start, nullptr};
     return fused ? launch_tc_t<false, false, true>(m, beta, nullptr, cu, nseq, out, S_final, T, H,
                                                    status, fwd, stream)
@@ -1386,7 +1415,7 @@ cudaError_t launch_segment_maps(const void* k, const void* v, const void* alpha,
                                 const int32_t* cu, int nseq, float* maps, int64_t rows, int64_t T,
                                 int H, int* status, cudaStream_t stream) {
     TcMaps m;
-    if (!make_maps(&m, k, k, v, alpha, nullptr, rows, H)) return cudaErrorInvalidValue;
+    if (!make_tc_maps(&m, k, k, v, alpha, nullptr, rows, H)) return cudaErrorInvalidValue;
     const tc::Segments one{1, 1, nullptr, maps};
     return launch_tc_t<false, true>(m, beta, nullptr, cu, nseq, nullptr, nullptr, T, H, status, one,
                                     stream);
@@ -1405,8 +1434,11 @@ cudaError_t launch_chunk_tc_cta_status(const void* q, const void* k, const void*
                                        const int32_t* cu, int nseq, void* out, float* S_final,
                                        int64_t rows, int64_t T, int H, int* status,
                                        cudaStream_t stream) {
+    if (use_tc2())
+        return launch_chunk_tc2_cta_status(q, k, v, alpha, beta, S0, cu, nseq, out, S_final, rows, T,
+                                           H, status, stream);
     TcMaps m;
-    if (!make_maps(&m, q, k, v, alpha, out, rows, H)) return cudaErrorInvalidValue;
+    if (!make_tc_maps(&m, q, k, v, alpha, out, rows, H)) return cudaErrorInvalidValue;
     const tc::Segments whole{1, 1, nullptr, nullptr};
     return launch_tc_t<true, false>(m, beta, S0, cu, nseq, out, S_final, T, H, status, whole,
                                     stream);
