@@ -16,25 +16,31 @@
 //   Tb = (I + A)^-1 diag(beta)
 //   Z = (k*gamma) S,   U = Tb (V - Z),   O = (q*gamma) S + P U,   S <- Diag(gamma_C) S + (k*eta)^T U
 //
-// Transposed, with S^T in TMEM (lane n = value column, columns = key channels):
+// Transposed, with S^T in TMEM (lane n = value column, columns = key channels), and
+// with gamma_r = lam_r Gamma_I for the tokens r of 32-token sub-chunk I (lam_r the
+// in-sub-chunk factor of the gate phase below, Gamma_I = gamma at the sub-chunk's
+// reference token, one value per key channel):
 //
-//   Z^T = S^T (k*gamma)^T            M=128 (n), N=64 (j), K=128 (c)   A: S^T bf16 (TMEM)
-//   O^T = S^T (q*gamma)^T            M=128, N=64 (r), K=128            A: S^T bf16 (TMEM)
-//   U^T = (V - Z)^T Tb^T             M=128, N=64, K=64 (j')            A: (V - Z)^T bf16 (TMEM)
-//   S^T <- S^T Diag(gamma_C) + U^T (k*eta)    M=128, N=128 (c), K=64   A: U^T bf16 (TMEM)
-//   O^T += U^T P^T                   M=128, N=64, K=64                 A: U^T bf16 (TMEM)
+//   Z^T[:, I] = (S^T Diag(Gamma_I)) (k*lam)_I^T     M=128 (n), N=32 (j), K=128 (c)
+//   O^T[:, I] = (S^T Diag(Gamma_I)) (q*lam)_I^T     M=128, N=32 (r), K=128
+//   U^T = V^T Tb^T - Z^T Tb^T                       M=128, N=64, K=64 (j'); V^T from shared memory
+//   S^T <- S^T Diag(gamma_C) + U^T (k*eta)          M=128, N=128 (c), K=64
+//   O^T += U^T P^T                                  M=128, N=64, K=64
 //
-// so the chain that carries the state from chunk to chunk moves no operand of its
-// own through shared memory: the B operands (k*gamma, q*gamma, Tb, k*eta, P) are
-// the state-independent products of the chunk, prepared one chunk ahead.
+// with every other A operand in TMEM: the two scaled bf16 copies of S^T, Z^T and U^T.
+// The chain that carries the state from chunk to chunk moves no operand of its own
+// through shared memory; its B operands are the chunk's state-independent products,
+// prepared one chunk ahead: k*lam and q*lam (also the left operands of [A/beta ; P],
+// written over k and q), Tb, P and k*eta = (k*rho^1) Diag(gamma_C / Gamma_1) (written
+// over alpha as k*rho^1, the right operand of [A/beta ; P], then rescaled).
 //
 // Warp roles (512 threads = four warpgroups, one CTA per SM):
-//   warps 0-7   prep: gate products, the seven bf16 operands, [A/beta ; P] (one
-//               tcgen05 MMA), the triangular solve, Tb; one of its threads issues
-//               its MMAs.  Works on chunk c+1 while the state chain runs chunk c.
-//   warps 8-11  the state chain, warp 8+q owning TMEM lane quarter q: the bf16 copy
-//               and decay of S^T, V - Z, U, and O^T out to global memory (through a
-//               staging tile and TMA stores; a partial last chunk row by row).
+//   warps 0-7   prep: gate products, the bf16 operands, [A/beta ; P] (one tcgen05
+//               MMA), the triangular solve, Tb, k*eta; one of its threads issues its
+//               MMAs.  Works on chunk c+1 while the state chain runs chunk c.
+//   warps 8-11  the state chain, warp 8+q owning TMEM lane quarter q: the scaled bf16
+//               copies and the decay of S^T, Z and U to bf16, and O^T out to global memory
+//               (transposed in registers by 8 x 8 shuffles, 16-byte stores).
 //   warp 12     one thread: every TMA load (k, q, alpha one stage per chunk parity;
 //               v) and the state chain's MMAs, in chunk order (warps 13-15 idle).
 // Registers are rebalanced per warpgroup (setmaxnreg): 168 for prep, 104 for the
@@ -53,8 +59,8 @@
 #include "kda_sm100.cuh"
 #include "kda_tc_maps.cuh"
 
-// Optional event hook for timing builds: (role, chunk, event) by one thread of the
-// role (no-op in the library).
+// Optional event hook for timing builds: (slot, chunk, event); slots 0-7 are the prep
+// warps, 8 the state chain, 9 the issuing thread (no-op in the library).
 #ifndef KDA_TC2_MARK
 #define KDA_TC2_MARK(role, chunk, event)
 #endif
@@ -77,27 +83,30 @@ constexpr int WARP_CTL = 12;
 constexpr uint64_t kWaitNs = 2000000000ull;    // 2 s per wait, then report a timeout
 
 // shared-memory map (bytes from the 1024-aligned base)
-constexpr uint32_t STAGE = 16384;              // per-parity stride of the k, q, alpha stages
-constexpr uint32_t OFF_K = 0;                  // k tile [64 j][128 c] x 2 stages -> k*gamma in place
-constexpr uint32_t OFF_Q = 32768;              // q tile x 2 stages -> q*gamma in place
-constexpr uint32_t OFF_A = 65536;              // alpha tile x 2 stages -> k*eta in place
-constexpr uint32_t OFF_V = 98304;              // v tile [64 j][128 n]
-constexpr uint32_t OFF_X = 114688;             // prep work region, 56 KB (below)
-constexpr uint32_t OFF_P = 172032;             // P [64 r][64 j] x 2 stages
-constexpr uint32_t OFF_TB = 188416;            // Tb [64 j][64 j'] x 2 stages
-constexpr uint32_t OFF_OST = 204800;           // O staging tile [64 r][128 n] (TMA store box layout)
+// A stage (one per chunk parity) holds the chunk's k, q and alpha tiles as TMA
+// delivers them, in the atoms the MMAs read afterwards:
+//   kq: per 64-channel atom a, rows 0-63 k then rows 64-127 q ([128][64] bf16, 16 KB
+//       at a * 16 KB): k*lam and q*lam in place, the M=128 left operand of [A/beta ; P]
+//   ar: per atom a, rows 0-31 k*rho^0, rows 32-95 alpha -> k*rho^1 -> k*eta
+//       ([96][64] bf16, 12 KB at a * 12 KB): the N=96 right operand of [A/beta ; P]
+constexpr uint32_t KQ_STAGE = 32768;
+constexpr uint32_t AR_STAGE = 24576;
+constexpr uint32_t OFF_KQ = 0;                 // 2 stages
+constexpr uint32_t OFF_AR = 65536;             // 2 stages
+constexpr uint32_t OFF_V = 114688;             // v tile [64 j][128 n] (two [64][64] atoms)
+constexpr uint32_t OFF_X = 131072;             // solve work region, 56 KB (below)
+constexpr uint32_t OFF_P = 188416;             // P [64 r][64 j] x 2 stages
+constexpr uint32_t OFF_TB = 204800;            // Tb [64 j][64 j'] x 2 stages
 constexpr uint32_t OFF_MISC = 221184;
 constexpr uint32_t MISC_PI = 0;                // float [8][128] octant gate products
-constexpr uint32_t MISC_GC = 4096;             // float [2][128] gamma_C per stage
-constexpr uint32_t MISC_BETA = 5120;           // float [2][64] beta per stage
-constexpr uint32_t MISC_BAR = 5632;            // mbarriers (enum below)
-constexpr uint32_t MISC_TMEM = 5760;
-constexpr uint32_t MISC_FLAG = 5764;
-constexpr uint32_t SMEM_BYTES = OFF_MISC + 5888 + 1024;   // + alignment slack
+constexpr uint32_t MISC_GAM = 4096;            // float [2 stages][4][128]: Gamma_0, Gamma_1, gamma_C, gamma_C/Gamma_1
+constexpr uint32_t MISC_BETA = 8192;           // float [2][64] beta per stage
+constexpr uint32_t MISC_BAR = 8704;            // mbarriers (enum below)
+constexpr uint32_t MISC_TMEM = 8832;
+constexpr uint32_t MISC_FLAG = 8836;
+constexpr uint32_t SMEM_BYTES = OFF_MISC + 9216 + 1024;   // + alignment slack
 
-// prep work region: the operands of [A/beta ; P], then (after that MMA) the solve
-constexpr uint32_t X_L = 0;        // [k*lam ; q*lam] [128][128] (two [128][64] atoms)
-constexpr uint32_t X_R = 32768;    // [k*rho^0 (32 rows) ; k*rho^1 (64 rows)] (two [96][64] atoms)
+// solve work region
 constexpr int AS = 68;             // row stride (floats) of the fp32 A and Tinv tiles
 constexpr uint32_t X_AM = 0;       // float A    [64][68]
 constexpr uint32_t X_TM = 17408;   // float Tinv [64][68]
@@ -114,7 +123,7 @@ enum Bar {
     B_PMMA = 7,       // prep's MMA groups
     B_RZ = 8,         // state -> issuer: S^T copied, issue Z^T
     B_RQ = 9,         //                 previous O^T read out, issue O^T
-    B_RU = 10,        //                 (V - Z)^T written, issue U^T
+    B_RU = 10,        //                 Z^T (bf16) written, issue U^T
     B_R3 = 11,        //                 U^T written, issue the state update and O^T += U^T P^T
     B_BZ = 12,        // issuer -> state: Z^T done
     B_BU = 13,        //                  U^T done
@@ -124,12 +133,12 @@ enum Bar {
 
 // TMEM columns
 constexpr uint32_t TS = 0;      // S^T fp32 [128 n][128 c]
-constexpr uint32_t TSB = 128;   // S^T bf16 pairs (64 columns)
-constexpr uint32_t TZ = 192;    // Z^T, then U^T, fp32 (64 columns)
-constexpr uint32_t TO = 256;    // O^T fp32 (64 columns)
-constexpr uint32_t TVB = 320;   // (V - Z)^T bf16 pairs (32 columns)
-constexpr uint32_t TUB = 352;   // U^T bf16 pairs (32 columns)
-constexpr uint32_t TP = 384;    // prep: [A/beta ; P] (96 columns), then the tf32 solve products
+constexpr uint32_t TSB0 = 128;  // S^T Diag(Gamma_0) bf16 pairs (64 columns)
+constexpr uint32_t TSB1 = 192;  // S^T Diag(Gamma_1) bf16 pairs (64 columns)
+constexpr uint32_t TZ = 256;    // Z^T, then U^T, fp32 (64 columns)
+constexpr uint32_t TO = 320;    // O^T fp32 (64 columns)
+constexpr uint32_t TVU = 384;   // Z^T, then U^T, bf16 pairs (32 columns)
+constexpr uint32_t TP = 416;    // prep: [A/beta ; P] (96 columns), then the tf32 solve products
 
 __device__ __forceinline__ uint32_t swz(uint32_t row, uint32_t chunk) {
     return row * 128u + (((chunk ^ row) & 7u) << 4);
@@ -173,22 +182,20 @@ template <bool kCtaStatus, bool kFused>
 __global__ void __launch_bounds__(NTHREADS, 1)
 kda_chunk_tc2_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                      const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmV,
-                     const __grid_constant__ CUtensorMap tmO, const __nv_bfloat16* __restrict__ beta, const float* S0,
+                     const __nv_bfloat16* __restrict__ beta, const float* S0,
                      const int32_t* __restrict__ cu_seqlens, __nv_bfloat16* __restrict__ out,
                      float* S_final, int64_t T, int H, int* status, const Segments seg) {
     extern __shared__ uint8_t smem_raw[];
     uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~static_cast<uintptr_t>(1023));
-    uint8_t* sK = sm + OFF_K;
-    uint8_t* sQ = sm + OFF_Q;
-    uint8_t* sAl = sm + OFF_A;
+    uint8_t* sKQ = sm + OFF_KQ;
+    uint8_t* sAR = sm + OFF_AR;
     uint8_t* sV = sm + OFF_V;
     uint8_t* sX = sm + OFF_X;
     uint8_t* sP = sm + OFF_P;
     uint8_t* sTB = sm + OFF_TB;
-    uint8_t* sOst = sm + OFF_OST;
     float* sPi = reinterpret_cast<float*>(sm + OFF_MISC + MISC_PI);
-    float* sGC = reinterpret_cast<float*>(sm + OFF_MISC + MISC_GC);
+    float* sGam = reinterpret_cast<float*>(sm + OFF_MISC + MISC_GAM);
     float* sBeta = reinterpret_cast<float*>(sm + OFF_MISC + MISC_BETA);
     uint64_t* bar = reinterpret_cast<uint64_t*>(sm + OFF_MISC + MISC_BAR);
     uint32_t* sTmem = reinterpret_cast<uint32_t*>(sm + OFF_MISC + MISC_TMEM);
@@ -267,9 +274,10 @@ kda_chunk_tc2_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_const
             mbar_arrive_expect_tx(bar + B_FULL + s, 3 * 16384);
 #pragma unroll
             for (int a = 0; a < 2; ++a) {
-                tma_load_2d(sK + s * STAGE + a * 8192, &tmK, bar + B_FULL + s, h * DK + 64 * a, row0);
-                tma_load_2d(sQ + s * STAGE + a * 8192, &tmQ, bar + B_FULL + s, h * DK + 64 * a, row0);
-                tma_load_2d(sAl + s * STAGE + a * 8192, &tmA, bar + B_FULL + s, h * DK + 64 * a, row0);
+                uint8_t* kq = sKQ + s * KQ_STAGE + a * 16384;
+                tma_load_2d(kq, &tmK, bar + B_FULL + s, h * DK + 64 * a, row0);
+                tma_load_2d(kq + 8192, &tmQ, bar + B_FULL + s, h * DK + 64 * a, row0);
+                tma_load_2d(sAR + s * AR_STAGE + a * 12288 + 4096, &tmA, bar + B_FULL + s, h * DK + 64 * a, row0);
             }
             ++issued_full[s];
         };
@@ -286,7 +294,8 @@ kda_chunk_tc2_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_const
             last_commit = b;
             last_commit_ph = ph;
         };
-        constexpr uint32_t id64 = idesc_bf16(128, 64);                  // both operands K-major
+        constexpr uint32_t id32 = idesc_bf16(128, 32);                  // both operands K-major
+        constexpr uint32_t id64 = idesc_bf16(128, 64);
         constexpr uint32_t id128mn = idesc_bf16(128, 128, false, true);  // B MN-major
         if (nchunks > 0) {
             issue_stage(0);
@@ -299,58 +308,73 @@ kda_chunk_tc2_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_const
             // Z^T = S^T (k*gamma)^T
             if (!wait_bar(B_RZ, ph)) break;
             tc_fence_after();
-            KDA_TC2_MARK(2, c, 0);
-            {
-                const uint32_t kg = smem_u32(sK + s * STAGE);
+            KDA_TC2_MARK(9, c, 0);
+            {   // sub-chunk I: Z^T columns j in [32 I, 32 I + 32) from k*lam rows 32 I ..
+                const uint32_t kq = smem_u32(sKQ + s * KQ_STAGE);
 #pragma unroll
-                for (int ks = 0; ks < 8; ++ks)
-                    mma_bf16_ts(tmem + TZ, tmem + TSB + 8 * ks,
-                                sdesc_sw128(kg + (ks >> 2) * 8192 + (ks & 3) * 32), id64, ks > 0);
+                for (int I = 0; I < 2; ++I)
+#pragma unroll
+                    for (int ks = 0; ks < 8; ++ks)
+                        mma_bf16_ts(tmem + TZ + 32 * I, tmem + (I ? TSB1 : TSB0) + 8 * ks,
+                                    sdesc_sw128(kq + (ks >> 2) * 16384 + I * 4096 + (ks & 3) * 32), id32,
+                                    ks > 0);
                 commit(B_BZ, ph);
             }
             // O^T = S^T (q*gamma)^T, once the previous chunk's O^T is read out
             if (!wait_bar(B_RQ, ph)) break;
             tc_fence_after();
-            KDA_TC2_MARK(2, c, 1);
-            {
-                const uint32_t qg = smem_u32(sQ + s * STAGE);
+            KDA_TC2_MARK(9, c, 1);
+            {   // from q*lam rows 32 I .. (the q half of each kq atom)
+                const uint32_t qg = smem_u32(sKQ + s * KQ_STAGE) + 8192;
 #pragma unroll
-                for (int ks = 0; ks < 8; ++ks)
-                    mma_bf16_ts(tmem + TO, tmem + TSB + 8 * ks,
-                                sdesc_sw128(qg + (ks >> 2) * 8192 + (ks & 3) * 32), id64, ks > 0);
+                for (int I = 0; I < 2; ++I)
+#pragma unroll
+                    for (int ks = 0; ks < 8; ++ks)
+                        mma_bf16_ts(tmem + TO + 32 * I, tmem + (I ? TSB1 : TSB0) + 8 * ks,
+                                    sdesc_sw128(qg + (ks >> 2) * 16384 + I * 4096 + (ks & 3) * 32), id32,
+                                    ks > 0);
             }
-            // U^T = (V - Z)^T Tb^T; the v tile is free again
+            // U^T = V^T Tb^T - Z^T Tb^T: the v tile as the MN-major A operand (M = 128 value
+            // columns, K = 64 tokens) from shared memory, then bf16(Z)^T from TMEM, negated
             if (!wait_bar(B_RU, ph)) break;
             tc_fence_after();
-            KDA_TC2_MARK(2, c, 2);
+            KDA_TC2_MARK(9, c, 2);
             {
-                const uint32_t tb = smem_u32(sTB + s * 8192);
+                constexpr uint32_t idv = idesc_bf16(128, 64, true, false);
+                constexpr uint32_t idneg = idesc_bf16(128, 64, false, false, true);
+                const uint32_t tb = smem_u32(sTB + s * 8192), v0 = smem_u32(sV);
 #pragma unroll
                 for (int ks = 0; ks < 4; ++ks)
-                    mma_bf16_ts(tmem + TZ, tmem + TVB + 8 * ks, sdesc_sw128(tb + ks * 32), id64, ks > 0);
+                    mma_bf16(tmem + TZ, sdesc_sw128(v0 + ks * 2048, 1024, 8192), sdesc_sw128(tb + ks * 32), idv,
+                             ks > 0);
+#pragma unroll
+                for (int ks = 0; ks < 4; ++ks)
+                    mma_bf16_ts(tmem + TZ, tmem + TVU + 8 * ks, sdesc_sw128(tb + ks * 32), idneg, 1);
                 commit(B_BU, ph);
             }
-            if (c + 1 < nchunks) issue_v(c + 1);
             // S^T += U^T (k*eta) (S^T already decayed) and O^T += U^T P^T
             if (!wait_bar(B_R3, ph)) break;
             tc_fence_after();
-            KDA_TC2_MARK(2, c, 3);
+            KDA_TC2_MARK(9, c, 3);
+            if (c + 1 < nchunks) issue_v(c + 1);   // U^T is done (the state waited for it): v is free
             {
-                const uint32_t kh = smem_u32(sAl + s * STAGE), p0 = smem_u32(sP + s * 8192);
+                // k*eta: rows 32..95 of the ar atoms, the MN-major B operand (N = 128 channels
+                // in two atoms 12 KB apart, K = 64 tokens)
+                const uint32_t kh = smem_u32(sAR + s * AR_STAGE) + 4096, p0 = smem_u32(sP + s * 8192);
 #pragma unroll
                 for (int ks = 0; ks < 4; ++ks)
-                    mma_bf16_ts(tmem + TS, tmem + TUB + 8 * ks, sdesc_sw128(kh + ks * 2048, 1024, 8192),
+                    mma_bf16_ts(tmem + TS, tmem + TVU + 8 * ks, sdesc_sw128(kh + ks * 2048, 1024, 12288),
                                 id128mn, 1);
 #pragma unroll
                 for (int ks = 0; ks < 4; ++ks)
-                    mma_bf16_ts(tmem + TO, tmem + TUB + 8 * ks, sdesc_sw128(p0 + ks * 32), id64, 1);
+                    mma_bf16_ts(tmem + TO, tmem + TVU + 8 * ks, sdesc_sw128(p0 + ks * 32), id64, 1);
                 commit(B_EMPTY + s, (uint32_t)(c >> 1) & 1u);
                 commit(B_BS, ph);
             }
             // the stage is free once these MMAs complete: load chunk c + 2 into it
             if (c + 2 < nchunks) {
                 if (!wait_bar(B_EMPTY + s, (uint32_t)(c >> 1) & 1u)) break;
-                KDA_TC2_MARK(2, c, 4);
+                KDA_TC2_MARK(9, c, 4);
                 issue_stage(c + 2);
             }
         }
@@ -385,15 +409,14 @@ kda_chunk_tc2_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_const
         for (int c = 0; c < nchunks; ++c) {
             const int s = c & 1;
             const int Lc = chunk_len(c);
-            uint8_t* sKc = sK + s * STAGE;
-            uint8_t* sQc = sQ + s * STAGE;
-            uint8_t* sAc = sAl + s * STAGE;
+            uint8_t* sKQc = sKQ + s * KQ_STAGE;
+            uint8_t* sARc = sAR + s * AR_STAGE;
             float* sBeta_s = sBeta + 64 * s;
-            float* sGC_s = sGC + 128 * s;
+            float* sGam_s = sGam + 512 * s;
             if (tid < C) sBeta_s[tid] = beta_next;
-            if (tid == 0) KDA_TC2_MARK(0, c, 0);
+            if (lane == 0) KDA_TC2_MARK(warp, c, 0);
             wait_bar(B_FULL + s, (uint32_t)(c >> 1) & 1u);
-            if (tid == 0) KDA_TC2_MARK(0, c, 1);
+            if (lane == 0) KDA_TC2_MARK(warp, c, 1);
 
             // ================= gate products and bf16 operands
             {
@@ -410,22 +433,27 @@ kda_chunk_tc2_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_const
                 // pi8: phi = phi8 * (O odd ? pi8_{O-1} : 1), psi = psi8 * (O even ? pi8_{O+1} : 1);
                 // those octant factors are folded into the per-thread scales below.
                 // Every tile touched here is row-major with 128-byte swizzled rows; a warp covers
-                // one token row of all 128 channels (8 bytes per thread).
+                // one token row of all 128 channels (8 bytes per thread).  Outputs: k*lam over
+                // k, q*lam over q, k*rho^1 over alpha, k*rho^0 in the rows before it.
                 const int cq = tid & 31, O = tid >> 5, Q = O >> 1, c0 = 4 * cq;
                 const uint32_t chk = (uint32_t)((c0 & 63) >> 3), inner = (uint32_t)((c0 & 7) << 1);
                 const uint32_t a64 = (uint32_t)(c0 >> 6);
-                auto in_off_of = [&](int r) {
-                    return a64 * 8192u + (uint32_t)r * 128u + (((chk ^ (uint32_t)r) & 7u) << 4) + inner;
+                auto sw_of = [&](int r) {
+                    return (uint32_t)r * 128u + (((chk ^ (uint32_t)r) & 7u) << 4) + inner;
                 };
+                uint8_t* kbase = sKQc + a64 * 16384u;           // k rows; q rows at + 8192
+                uint8_t* abase = sARc + a64 * 12288u;           // k*rho^0 rows; alpha rows at + 4096
                 float phi[8][4], psi[8][4];   // psi holds the clamped gates until the backward pass
 #pragma unroll
                 for (int i = 0; i < 8; ++i) {
                     const int r = 8 * O + i;
                     float a[4];
-                    unpack4_bf16(*reinterpret_cast<const uint2*>(sAc + in_off_of(r)), a);
+                    unpack4_bf16(*reinterpret_cast<const uint2*>(abase + 4096 + sw_of(r)), a);
 #pragma unroll
-                    for (int cc = 0; cc < 4; ++cc)
-                        psi[i][cc] = r < Lc ? clamp_gate(fused ? gate_from_logit(a[cc]) : a[cc]) : 1.0f;
+                    for (int cc = 0; cc < 4; ++cc) {
+                        const float g = clamp_gate(fused ? gate_from_logit(a[cc]) : a[cc]);
+                        psi[i][cc] = (Lc == C || r < Lc) ? g : 1.0f;
+                    }
                 }
                 {
                     float p[4] = {1.f, 1.f, 1.f, 1.f}, b[4] = {1.f, 1.f, 1.f, 1.f};
@@ -439,11 +467,12 @@ kda_chunk_tc2_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_const
                         for (int cc = 0; cc < 4; ++cc) { const float a = psi[i][cc]; psi[i][cc] = b[cc]; b[cc] *= a; }
                     *reinterpret_cast<float4*>(&sPi[O * DK + c0]) = make_float4(p[0], p[1], p[2], p[3]);
                 }
-                if (tid == 0) KDA_TC2_MARK(0, c, 2);
+                if (lane == 0) KDA_TC2_MARK(warp, c, 2);
                 prep_bar();
-                if (tid == 0) KDA_TC2_MARK(0, c, 3);
-                // per-thread scales: quarter products, gamma before / eta after this quarter
-                float dlf[4], bf[4], r0g[4], r1g[4], ag[4];
+                if (lane == 0) KDA_TC2_MARK(warp, c, 3);
+                // per-thread scales: quarter products; the sub-chunk reference products
+                // Gamma_0 = gamma_15, Gamma_1 = gamma_47, gamma_C and gamma_C / Gamma_1 per channel
+                float dlf[4], r0g[4], r1g[4];
                 {
                     float pq[4][4];   // [quarter][channel]
 #pragma unroll
@@ -464,7 +493,13 @@ kda_chunk_tc2_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_const
                             if (M > Q) aft *= pq[M][cc];
                             if (M == Q) own = pq[M][cc];
                         }
-                        if (O == 0) sGC_s[c0 + cc] = pq[0][cc] * pq[1][cc] * pq[2][cc] * pq[3][cc];
+                        if (O == 0) {
+                            const float g1 = pq[0][cc] * pq[1][cc] * pq[2][cc];
+                            sGam_s[c0 + cc] = pq[0][cc];
+                            sGam_s[128 + c0 + cc] = g1;
+                            sGam_s[256 + c0 + cc] = g1 * pq[3][cc];
+                            sGam_s[384 + c0 + cc] = pq[3][cc];
+                        }
                         const float fO = (O & 1) ? pov[cc] : 1.0f;
                         const float gO = (O & 1) ? 1.0f : pov[cc];
                         const float dl = (Q & 1) ? 1.0f : __frcp_rn(own);
@@ -472,10 +507,10 @@ kda_chunk_tc2_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_const
                         const float r1 = Q == 0 ? pq[1][cc] * pq[2][cc]
                                                 : (Q == 1 ? pq[2][cc] : (Q == 2 ? 1.0f : __frcp_rn(own)));
                         dlf[cc] = dl * fO;
-                        bf[cc] = bef * fO;
                         r0g[cc] = r0 * gO;
                         r1g[cc] = r1 * gO;
-                        ag[cc] = aft * gO;
+                        (void)bef;
+                        (void)aft;
                     }
                 }
                 // fused inputs: k and q rows L2-normalised in place (bf16), before any
@@ -485,10 +520,10 @@ kda_chunk_tc2_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_const
 #pragma unroll
                     for (int i = 0; i < 8; ++i) {
                         const int r = 8 * O + i;
-                        const uint32_t in_off = in_off_of(r);
+                        const uint32_t in_off = sw_of(r);
                         float k[4], q[4];
-                        unpack4_bf16(*reinterpret_cast<const uint2*>(sKc + in_off), k);
-                        unpack4_bf16(*reinterpret_cast<const uint2*>(sQc + in_off), q);
+                        unpack4_bf16(*reinterpret_cast<const uint2*>(kbase + in_off), k);
+                        unpack4_bf16(*reinterpret_cast<const uint2*>(kbase + 8192 + in_off), q);
                         float sk = k[0] * k[0] + k[1] * k[1] + k[2] * k[2] + k[3] * k[3];
                         float sq = q[0] * q[0] + q[1] * q[1] + q[2] * q[2] + q[3] * q[3];
 #pragma unroll
@@ -499,77 +534,60 @@ kda_chunk_tc2_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_const
                         const float ik = rsqrtf(fmaxf(sk, 1e-12f)), iq = rsqrtf(fmaxf(sq, 1e-12f));
 #pragma unroll
                         for (int cc = 0; cc < 4; ++cc) { k[cc] *= ik; q[cc] *= iq; }
-                        st4_bf16(sKc + in_off, k);
-                        st4_bf16(sQc + in_off, q);
+                        st4_bf16(kbase + in_off, k);
+                        st4_bf16(kbase + 8192 + in_off, q);
                     }
                 }
-                // each row's k and q are read before the previous row's stores: k*gamma,
-                // q*gamma and k*eta are written in place, so a load placed after a store
-                // could not be moved above it
-                uint2 kn = *reinterpret_cast<const uint2*>(sKc + in_off_of(8 * O));
-                uint2 qn = *reinterpret_cast<const uint2*>(sQc + in_off_of(8 * O));
+                // each row's k and q are read before the previous row's stores: k*lam and q*lam
+                // are written in place, so a load placed after a store could not be moved above it
+                uint2 kn = *reinterpret_cast<const uint2*>(kbase + sw_of(8 * O));
+                uint2 qn = *reinterpret_cast<const uint2*>(kbase + 8192 + sw_of(8 * O));
 #pragma unroll
                 for (int i = 0; i < 8; ++i) {
                     const int r = 8 * O + i;
-                    const uint32_t sw = (uint32_t)r * 128u + (((chk ^ (uint32_t)r) & 7u) << 4) + inner;
-                    const uint32_t in_off = a64 * 8192u + sw;    // 64-row tiles: q, k, alpha
+                    const uint32_t sw = sw_of(r);
                     float k[4], q[4];
                     unpack4_bf16(kn, k);
                     unpack4_bf16(qn, q);
                     if (i < 7) {
-                        kn = *reinterpret_cast<const uint2*>(sKc + in_off_of(r + 1));
-                        qn = *reinterpret_cast<const uint2*>(sQc + in_off_of(r + 1));
+                        kn = *reinterpret_cast<const uint2*>(kbase + sw_of(r + 1));
+                        qn = *reinterpret_cast<const uint2*>(kbase + 8192 + sw_of(r + 1));
                     }
                     if (r >= Lc) {
 #pragma unroll
                         for (int cc = 0; cc < 4; ++cc) { k[cc] = 0.0f; q[cc] = 0.0f; }
                     }
-                    float kp[4], qp[4], ks[4], w[4];
+                    float lam[4], w[4];
 #pragma unroll
-                    for (int cc = 0; cc < 4; ++cc) {
-                        kp[cc] = k[cc] * phi[i][cc];
-                        qp[cc] = q[cc] * phi[i][cc];
-                        ks[cc] = k[cc] * psi[i][cc];
-                    }
-                    uint8_t* lrow = sX + X_L + a64 * 16384u + sw;             // 128-row atoms
-                    uint8_t* rrow = sX + X_R + a64 * 12288u + sw;             // 96-row atoms
+                    for (int cc = 0; cc < 4; ++cc) lam[cc] = phi[i][cc] * dlf[cc];
 #pragma unroll
-                    for (int cc = 0; cc < 4; ++cc) w[cc] = kp[cc] * dlf[cc];
-                    st4_bf16(lrow, w);                                        // k*lam, row r
+                    for (int cc = 0; cc < 4; ++cc) w[cc] = k[cc] * lam[cc];
+                    st4_bf16(kbase + sw, w);                                  // k*lam over k, row r
 #pragma unroll
-                    for (int cc = 0; cc < 4; ++cc) w[cc] = qp[cc] * dlf[cc];
-                    st4_bf16(lrow + 64 * 128, w);                             // q*lam, row 64 + r
-#pragma unroll
-                    for (int cc = 0; cc < 4; ++cc) w[cc] = qp[cc] * bf[cc];
-                    st4_bf16(sQc + in_off, w);                                // q*gamma in place
+                    for (int cc = 0; cc < 4; ++cc) w[cc] = q[cc] * lam[cc];
+                    st4_bf16(kbase + 8192 + sw, w);                           // q*lam over q, row 64 + r
                     if (O < 4) {
 #pragma unroll
-                        for (int cc = 0; cc < 4; ++cc) w[cc] = ks[cc] * r0g[cc];
-                        st4_bf16(rrow, w);                                    // k*rho^0, row r < 32
+                        for (int cc = 0; cc < 4; ++cc) w[cc] = k[cc] * (psi[i][cc] * r0g[cc]);
+                        st4_bf16(abase + sw, w);                              // k*rho^0, row r < 32
                     }
 #pragma unroll
-                    for (int cc = 0; cc < 4; ++cc) w[cc] = ks[cc] * r1g[cc];
-                    st4_bf16(rrow + 32 * 128, w);                             // k*rho^1, row 32 + r
-#pragma unroll
-                    for (int cc = 0; cc < 4; ++cc) w[cc] = kp[cc] * bf[cc];
-                    st4_bf16(sKc + in_off, w);                                // k*gamma in place
-#pragma unroll
-                    for (int cc = 0; cc < 4; ++cc) w[cc] = ks[cc] * ag[cc];
-                    st4_bf16(sAc + in_off, w);                                // k*eta over alpha
+                    for (int cc = 0; cc < 4; ++cc) w[cc] = k[cc] * (psi[i][cc] * r1g[cc]);
+                    st4_bf16(abase + 4096 + sw, w);                           // k*rho^1 over alpha, row 32 + r
                 }
-                if (tid == 0) KDA_TC2_MARK(0, c, 4);
+                if (lane == 0) KDA_TC2_MARK(warp, c, 4);
             }
             fence_async_smem();
             tc_fence_before();
             prep_bar();
             tc_fence_after();
-            if (tid == 0) KDA_TC2_MARK(0, c, 5);
+            if (lane == 0) KDA_TC2_MARK(warp, c, 5);
 
             // ================= [A/beta ; P] = [k*lam ; q*lam] [k*rho^0 ; k*rho^1]^T   (M=128, N=96, K=128)
             //   rows 0..63 are A/beta rows r, rows 64..127 are P rows r.  Columns [0, 32) hold
             //   rho^0 (j < 32, valid for r < 32), columns [32, 96) hold rho^1 (j < 64, valid for r >= 32).
             if (tid == 0 && ok) {
-                const uint32_t l0 = smem_u32(sX + X_L), r0 = smem_u32(sX + X_R);
+                const uint32_t l0 = smem_u32(sKQc), r0 = smem_u32(sARc);
                 constexpr uint32_t idesc = idesc_bf16(128, 96);
 #pragma unroll
                 for (int ks = 0; ks < 8; ++ks)
@@ -582,7 +600,7 @@ kda_chunk_tc2_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_const
             if (wait_bar(B_PMMA, ph_p) && tid == 0) pmma_out = false;
             ph_p ^= 1u;
             tc_fence_after();
-            if (tid == 0) KDA_TC2_MARK(0, c, 6);
+            if (lane == 0) KDA_TC2_MARK(warp, c, 6);
 
             // ================= A (fp32, times beta_r, j < r) and P (bf16 K-major, j <= r)
             {
@@ -601,7 +619,7 @@ kda_chunk_tc2_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_const
 #pragma unroll
                     for (int i = 0; i < 32; ++i) v[i] = 0.0f;
                 }
-                if (tid == 0) KDA_TC2_MARK(0, c, 7);
+                if (lane == 0) KDA_TC2_MARK(warp, c, 7);
                 if (q4 < 2) {
                     float* Am = reinterpret_cast<float*>(sX + X_AM);
                     const float b = sBeta_s[r];
@@ -625,13 +643,14 @@ kda_chunk_tc2_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_const
                     }
                 }
             }
-            if (tid == 0) KDA_TC2_MARK(0, c, 8);
+            if (lane == 0) KDA_TC2_MARK(warp, c, 8);
             // beta of the next chunk, while the solve runs
             if (tid < C) {
                 const int64_t nxt = (int64_t)(c + 1) * C + tid;   // token index in the segment
                 beta_next = (c + 1 < nchunks && nxt < len) ? load_beta(nxt) : 0.0f;
             }
-            fence_async_smem();
+            // (no proxy fence here: P is read by an MMA only in the state chain, after the
+            // fence that precedes the stage hand-over; A is read by the CUDA cores)
             tc_fence_before();
             prep_bar();
             tc_fence_after();
@@ -639,7 +658,7 @@ kda_chunk_tc2_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_const
             // ================= Tinv = (I + A)^-1 by doubling: 16x16 blocks, then 32, then 64
             //   inv([[X, 0], [Y, Z]]) = [[X^-1, 0], [-Z^-1 Y X^-1, Z^-1]]
             {
-                if (tid == 0) KDA_TC2_MARK(0, c, 9);
+                if (lane == 0) KDA_TC2_MARK(warp, c, 9);
                 const float* Am = reinterpret_cast<const float*>(sX + X_AM);
                 float* Tm = reinterpret_cast<float*>(sX + X_TM);
                 float* Xs = reinterpret_cast<float*>(sX + X_XS);
@@ -680,9 +699,29 @@ kda_chunk_tc2_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_const
                     for (int c4 = 0; c4 < 2; ++c4)
                         *reinterpret_cast<float4*>(&Tm[r2 * AS + 32 + 16 * c4 + cq]) =
                             make_float4(0.f, 0.f, 0.f, 0.f);
+                    // k*eta = (k*rho^1) Diag(gamma_C / Gamma_1), in place (the [A/beta ; P] MMA
+                    // that read k*rho^1 is done).  Thread: atom, 16-byte chunk (8 channels), 8 rows.
+                    const int at = t >> 6, ch = t & 7, rg = (t >> 3) & 7;
+                    const float* ef = sGam_s + 384 + 64 * at + 8 * ch;
+                    const float4 e0 = *reinterpret_cast<const float4*>(ef);
+                    const float4 e1 = *reinterpret_cast<const float4*>(ef + 4);
+                    const float ev[8] = {e0.x, e0.y, e0.z, e0.w, e1.x, e1.y, e1.z, e1.w};
+                    uint8_t* kr = sARc + at * 12288 + 4096;
+#pragma unroll
+                    for (int i = 0; i < 8; ++i) {
+                        const uint32_t row = (uint32_t)(8 * rg + i);
+                        uint4* pr = reinterpret_cast<uint4*>(kr + row * 128u + ((((uint32_t)ch ^ row) & 7u) << 4));
+                        const uint4 raw = *pr;
+                        float x[8];
+                        unpack4_bf16(make_uint2(raw.x, raw.y), *reinterpret_cast<float(*)[4]>(&x[0]));
+                        unpack4_bf16(make_uint2(raw.z, raw.w), *reinterpret_cast<float(*)[4]>(&x[4]));
+#pragma unroll
+                        for (int e = 0; e < 8; ++e) x[e] *= ev[e];
+                        *pr = pack8(x);
+                    }
                 }
                 prep_bar();
-                if (tid == 0) KDA_TC2_MARK(0, c, 10);
+                if (lane == 0) KDA_TC2_MARK(warp, c, 10);
                 // 16 -> 32: blocks (1,0) and (3,2).  thread: block b, row r, columns m2, m2+1
                 {
                     const int b = tid >> 7, r = (tid >> 3) & 15, m2 = (tid & 7) * 2;
@@ -712,7 +751,7 @@ kda_chunk_tc2_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_const
                     *reinterpret_cast<float2*>(&Tm[(o1 + r) * AS + o0 + m2]) = make_float2(-y0, -y1);
                 }
                 prep_bar();
-                if (tid == 0) KDA_TC2_MARK(0, c, 11);
+                if (lane == 0) KDA_TC2_MARK(warp, c, 11);
                 // 32 -> 64 on the tensor cores (tf32): X^T = T0^T A10^T, then Y^T = X^T T1^T with
                 // X^T read back from TMEM by the second MMA; Tinv[32:64, 0:32] = -Y.  Operands:
                 // fp32 K-major tiles written here (T1 serves as the second product's B).
@@ -751,7 +790,7 @@ kda_chunk_tc2_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_const
                 if (wait_bar(B_PMMA, ph_p) && tid == 0) pmma_out = false;
                 ph_p ^= 1u;
                 tc_fence_after();
-                if (tid == 0) KDA_TC2_MARK(0, c, 12);
+                if (lane == 0) KDA_TC2_MARK(warp, c, 12);
                 // both products are done: Y^T = X^T T1^T is in TMEM (M=64 rows c = 16 q4 + lane,
                 // columns r'); Tinv[32 + r', c] = -Y[r', c]
                 if (q4 < 2) {
@@ -767,7 +806,7 @@ kda_chunk_tc2_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_const
                 }
                 tc_fence_before();
                 prep_bar();
-                if (tid == 0) KDA_TC2_MARK(0, c, 13);
+                if (lane == 0) KDA_TC2_MARK(warp, c, 13);
                 // Tb = Tinv diag(beta): the K-major B operand [64 j][64 j'] of U^T; zero above
                 // the diagonal
                 uint8_t* sTBc = sTB + s * 8192;
@@ -789,7 +828,7 @@ kda_chunk_tc2_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_const
             tc_fence_before();
             const bool stop = named_bar_or(1, NPREP, !ok || *sFlag != 0);
             if (stop) break;
-            if (tid == 0) KDA_TC2_MARK(0, c, 14);
+            if (lane == 0) KDA_TC2_MARK(warp, c, 14);
             if (tid == 0) mbar_arrive(bar + B_READY + s);
         }
         if (tid == 0 && pmma_out) mbar_wait_ns(bar + B_PMMA, pmma_ph, kWaitNs);
@@ -818,51 +857,57 @@ kda_chunk_tc2_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_const
             }
             tmem_wait_st();
         }
-        // O^T of chunk c from TMEM to out[row0 + r][h][n].  A full chunk goes through the
-        // staging tile (thread n writes column n of the row-major, 128-byte swizzled box;
-        // a warp's 32 columns of one row are 64 contiguous bytes) and two TMA stores
-        // issued by the elected thread; a partial last chunk is stored row by row.
-        bool ost_pending = false;   // (elected) a TMA store may still be reading the tile
+        // O^T of chunk c from TMEM to out[row0 + r][h][n].  Thread n holds column n of O for
+        // the 64 rows; each 8 x 8 block (8 rows x 8 consecutive columns of 8 lanes) is
+        // transposed by three xor-butterfly rounds of shuffles (rounds 4 and 2 swap whole
+        // bf16 pairs, round 1 swaps halves), after which lane i of the group holds 8
+        // consecutive columns of row i: one 16-byte store.  Rows past the chunk's length
+        // are not stored.
         auto store_o = [&](int c) {
             const int Lc = chunk_len(c);
             const int64_t row0 = bos + (int64_t)c * C;
-            if (Lc == C) {
-                // the previous store has read the tile (elected waits, the barrier publishes)
-                if (elected && ost_pending) bulk_wait_read_all();
-                state_bar();
-                const uint32_t ocol = (uint32_t)(nn >> 6) * 8192u + (uint32_t)(nn & 7) * 2u;
-                const uint32_t ochk = (uint32_t)((nn & 63) >> 3);
+            const int gi = lane & 7;
+            const bool b4 = (gi >> 2) & 1, b2 = (gi >> 1) & 1, b1 = gi & 1;
+            __nv_bfloat16* obase = out + ((size_t)row0 * H + h) * DV + (32 * q4 + (lane & ~7));
+            const size_t rs = (size_t)H * DV;
 #pragma unroll
-                for (int half = 0; half < 2; ++half) {
-                    uint32_t r[32];
-                    tmem_ld32(tmem + tlane + TO + 32 * half, r);
-                    tmem_wait_ld();
+            for (int half = 0; half < 2; ++half) {
+                uint32_t f[32];
+                tmem_ld32(tmem + tlane + TO + 32 * half, f);
+                tmem_wait_ld();
 #pragma unroll
-                    for (int i = 0; i < 32; ++i) {
-                        const uint32_t rr = (uint32_t)(32 * half + i);
-                        *reinterpret_cast<__nv_bfloat16*>(sOst + ocol + rr * 128u + (((ochk ^ rr) & 7u) << 4)) =
-                            __float2bfloat16_rn(u2f(r[i]));
+                for (int blk = 0; blk < 4; ++blk) {
+                    uint32_t p[4];
+#pragma unroll
+                    for (int u = 0; u < 4; ++u) p[u] = pack_bf16x2(u2f(f[8 * blk + 2 * u]), u2f(f[8 * blk + 2 * u + 1]));
+                    {   // rows 4..7 <-> lanes 4..7
+                        const uint32_t x0 = b4 ? p[0] : p[2], x1 = b4 ? p[1] : p[3];
+                        const uint32_t y0 = __shfl_xor_sync(0xffffffffu, x0, 4);
+                        const uint32_t y1 = __shfl_xor_sync(0xffffffffu, x1, 4);
+                        if (b4) { p[0] = y0; p[1] = y1; } else { p[2] = y0; p[3] = y1; }
                     }
-                }
-                fence_async_smem();
-                state_bar();
-                if (elected) {
-#pragma unroll
-                    for (int a = 0; a < 2; ++a) tma_store_2d(&tmO, sOst + a * 8192, h * DV + 64 * a, (int)row0);
-                    bulk_commit_group();
-                    ost_pending = true;
-                }
-            } else {
-                __nv_bfloat16* dst = out + ((size_t)row0 * H + h) * DV + nn;
-                const size_t rs = (size_t)H * DV;
-#pragma unroll
-                for (int half = 0; half < 2; ++half) {
-                    uint32_t r[32];
-                    tmem_ld32(tmem + tlane + TO + 32 * half, r);
-                    tmem_wait_ld();
-#pragma unroll
-                    for (int i = 0; i < 32; ++i)
-                        if (32 * half + i < Lc) dst[(size_t)(32 * half + i) * rs] = __float2bfloat16_rn(u2f(r[i]));
+                    {   // rows 2,3 <-> lanes 2,3 (within each half)
+                        const uint32_t x0 = b2 ? p[0] : p[1], x1 = b2 ? p[2] : p[3];
+                        const uint32_t y0 = __shfl_xor_sync(0xffffffffu, x0, 2);
+                        const uint32_t y1 = __shfl_xor_sync(0xffffffffu, x1, 2);
+                        if (b2) { p[0] = y0; p[2] = y1; } else { p[1] = y0; p[3] = y1; }
+                    }
+                    {   // odd rows <-> odd lanes: 16-bit halves
+                        const uint32_t x0 = b1 ? __byte_perm(p[0], p[1], 0x5410) : __byte_perm(p[0], p[1], 0x7632);
+                        const uint32_t x1 = b1 ? __byte_perm(p[2], p[3], 0x5410) : __byte_perm(p[2], p[3], 0x7632);
+                        const uint32_t y0 = __shfl_xor_sync(0xffffffffu, x0, 1);
+                        const uint32_t y1 = __shfl_xor_sync(0xffffffffu, x1, 1);
+                        if (b1) {
+                            p[0] = __byte_perm(y0, p[0], 0x7610); p[1] = __byte_perm(y0, p[1], 0x7632);
+                            p[2] = __byte_perm(y1, p[2], 0x7610); p[3] = __byte_perm(y1, p[3], 0x7632);
+                        } else {
+                            p[0] = __byte_perm(p[0], y0, 0x5410); p[1] = __byte_perm(p[1], y0, 0x7610);
+                            p[2] = __byte_perm(p[2], y1, 0x5410); p[3] = __byte_perm(p[3], y1, 0x7610);
+                        }
+                    }
+                    const int row = 32 * half + 8 * blk + gi;
+                    if (row < Lc)
+                        *reinterpret_cast<uint4*>(obase + (size_t)row * rs) = make_uint4(p[0], p[1], p[2], p[3]);
                 }
             }
         };
@@ -874,22 +919,35 @@ kda_chunk_tc2_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_const
             if (c > 0) wait_bar(B_BS, ph ^ 1u);
             ok = __all_sync(0xffffffffu, ok);   // the TMEM loads and stores below are warp-wide
             tc_fence_after();
-            if (elected) KDA_TC2_MARK(1, c, 0);
-            // ---- S^T to bf16 (the A operand of this chunk's products), and S^T <- S^T Diag(gamma_C)
+            if (elected) KDA_TC2_MARK(8, c, 0);
+            // ---- S^T Diag(Gamma_0) and S^T Diag(Gamma_1) to bf16 (the A operands of this chunk's
+            //      products), and S^T <- S^T Diag(gamma_C)
             if (ok) {
-                const float* g = sGC + 128 * s;
+                const float* g0 = sGam + 512 * s;
+                const float* g1 = g0 + 128;
+                const float* gc = g0 + 256;
 #pragma unroll
                 for (int p = 0; p < 4; ++p) {
                     uint32_t r[32];
                     tmem_ld32(tmem + tlane + TS + 32 * p, r);
                     tmem_wait_ld();
-                    uint32_t b[16];
+                    uint32_t b0[16], b1[16];
 #pragma unroll
-                    for (int i = 0; i < 16; ++i) b[i] = pack_bf16x2(u2f(r[2 * i]), u2f(r[2 * i + 1]));
-                    tmem_st16u(tmem + tlane + TSB + 16 * p, b);
+                    for (int i = 0; i < 16; i += 2) {
+                        const float4 a0 = *reinterpret_cast<const float4*>(g0 + 32 * p + 2 * i);
+                        const float4 a1 = *reinterpret_cast<const float4*>(g1 + 32 * p + 2 * i);
+                        const float x0 = u2f(r[2 * i]), x1 = u2f(r[2 * i + 1]);
+                        const float x2 = u2f(r[2 * i + 2]), x3 = u2f(r[2 * i + 3]);
+                        b0[i] = pack_bf16x2(x0 * a0.x, x1 * a0.y);
+                        b0[i + 1] = pack_bf16x2(x2 * a0.z, x3 * a0.w);
+                        b1[i] = pack_bf16x2(x0 * a1.x, x1 * a1.y);
+                        b1[i + 1] = pack_bf16x2(x2 * a1.z, x3 * a1.w);
+                    }
+                    tmem_st16u(tmem + tlane + TSB0 + 16 * p, b0);
+                    tmem_st16u(tmem + tlane + TSB1 + 16 * p, b1);
 #pragma unroll
                     for (int i = 0; i < 32; i += 4) {
-                        const float4 gg = *reinterpret_cast<const float4*>(g + 32 * p + i);
+                        const float4 gg = *reinterpret_cast<const float4*>(gc + 32 * p + i);
                         r[i] = __float_as_uint(u2f(r[i]) * gg.x);
                         r[i + 1] = __float_as_uint(u2f(r[i + 1]) * gg.y);
                         r[i + 2] = __float_as_uint(u2f(r[i + 2]) * gg.z);
@@ -902,22 +960,20 @@ kda_chunk_tc2_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_const
             tc_fence_before();
             if (named_bar_or(2, NSTATE, !ok || *sFlag != 0)) { broke = true; break; }
             if (elected) mbar_arrive(bar + B_RZ);
-            if (elected) KDA_TC2_MARK(1, c, 1);
+            if (elected) KDA_TC2_MARK(8, c, 1);
             // ---- the previous chunk's O^T leaves while Z^T is computed
             if (c > 0) store_o(c - 1);
             tc_fence_before();
             state_bar();
             if (elected) mbar_arrive(bar + B_RQ);
-            if (elected) KDA_TC2_MARK(1, c, 2);
+            if (elected) KDA_TC2_MARK(8, c, 2);
             // ---- (V - Z)^T: column n of the v tile minus row n of Z^T, as bf16 pairs
             wait_bar(B_VFULL, ph);
             wait_bar(B_BZ, ph);
             ok = __all_sync(0xffffffffu, ok);
             tc_fence_after();
-            if (elected) KDA_TC2_MARK(1, c, 3);
-            if (ok) {
-                const uint32_t vcol = (uint32_t)(nn >> 6) * 8192u + (uint32_t)(nn & 7) * 2u;
-                const uint32_t vchk = (uint32_t)((nn & 63) >> 3);
+            if (elected) KDA_TC2_MARK(8, c, 3);
+            if (ok) {   // Z^T to bf16 pairs, the A operand of the second U^T product
 #pragma unroll
                 for (int half = 0; half < 2; ++half) {
                     uint32_t z[32];
@@ -925,27 +981,20 @@ kda_chunk_tc2_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_const
                     tmem_wait_ld();
                     uint32_t b[16];
 #pragma unroll
-                    for (int i = 0; i < 16; ++i) {
-                        const uint32_t j0 = (uint32_t)(32 * half + 2 * i), j1 = j0 + 1;
-                        const float v0 = __bfloat162float(*reinterpret_cast<const __nv_bfloat16*>(
-                            sV + vcol + j0 * 128u + (((vchk ^ j0) & 7u) << 4)));
-                        const float v1 = __bfloat162float(*reinterpret_cast<const __nv_bfloat16*>(
-                            sV + vcol + j1 * 128u + (((vchk ^ j1) & 7u) << 4)));
-                        b[i] = pack_bf16x2(v0 - u2f(z[2 * i]), v1 - u2f(z[2 * i + 1]));
-                    }
-                    tmem_st16u(tmem + tlane + TVB + 16 * half, b);
+                    for (int i = 0; i < 16; ++i) b[i] = pack_bf16x2(u2f(z[2 * i]), u2f(z[2 * i + 1]));
+                    tmem_st16u(tmem + tlane + TVU + 16 * half, b);
                 }
                 tmem_wait_st();
             }
             tc_fence_before();
             state_bar();
             if (elected) mbar_arrive(bar + B_RU);
-            if (elected) KDA_TC2_MARK(1, c, 4);
+            if (elected) KDA_TC2_MARK(8, c, 4);
             // ---- U^T as bf16 pairs
             wait_bar(B_BU, ph);
             ok = __all_sync(0xffffffffu, ok);
             tc_fence_after();
-            if (elected) KDA_TC2_MARK(1, c, 5);
+            if (elected) KDA_TC2_MARK(8, c, 5);
             if (ok) {
 #pragma unroll
                 for (int half = 0; half < 2; ++half) {
@@ -955,14 +1004,14 @@ kda_chunk_tc2_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_const
                     uint32_t b[16];
 #pragma unroll
                     for (int i = 0; i < 16; ++i) b[i] = pack_bf16x2(u2f(u[2 * i]), u2f(u[2 * i + 1]));
-                    tmem_st16u(tmem + tlane + TUB + 16 * half, b);
+                    tmem_st16u(tmem + tlane + TVU + 16 * half, b);
                 }
                 tmem_wait_st();
             }
             tc_fence_before();
             if (named_bar_or(2, NSTATE, !ok || *sFlag != 0)) { broke = true; break; }
             if (elected) mbar_arrive(bar + B_R3);
-            if (elected) KDA_TC2_MARK(1, c, 6);
+            if (elected) KDA_TC2_MARK(8, c, 6);
         }
         // ---- the last chunk's O^T, then S_final (column n of S^T)
         if (!broke && nchunks > 0) {
@@ -982,7 +1031,6 @@ kda_chunk_tc2_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_const
                 for (int i = 0; i < 32; ++i) dst[(size_t)(32 * p + i) * DV] = u2f(r[i]);
             }
         }
-        if (elected && ost_pending) bulk_wait_all();   // every O store has completed
         if (!ok || broke) *sFlag = 1;
     }
 
@@ -1007,7 +1055,7 @@ static cudaError_t launch_tc2_t(const TcMaps& m, const void* beta, const float* 
     if (e != cudaSuccess) return e;
     dim3 grid(1, H, nseq * seg.per_seq);
     tc2::kda_chunk_tc2_kernel<kCtaStatus, kFused><<<grid, tc2::NTHREADS, tc2::SMEM_BYTES, stream>>>(
-        m.q, m.k, m.a, m.v, m.o, (const __nv_bfloat16*)beta, S0, cu, (__nv_bfloat16*)out, S_final, T, H,
+        m.q, m.k, m.a, m.v, (const __nv_bfloat16*)beta, S0, cu, (__nv_bfloat16*)out, S_final, T, H,
         status, seg);
     return cudaGetLastError();
 }
