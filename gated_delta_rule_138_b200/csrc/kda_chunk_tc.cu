@@ -50,8 +50,6 @@
 // from its own start state.
 #include <cuda.h>
 
-#include <cstdlib>
-
 #include "kda_common.cuh"
 #include "kda_sm100.cuh"
 #include "kda_tc_maps.cuh"
@@ -649,7 +647,8 @@ kda_chunk_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_consta
                 }
             }
         }
-        fence_async_smem();
+        // no proxy fence here: A is read by the CUDA cores, and P by an MMA only after the
+        // fenced hand-off that precedes the tf32 solve products
         tc_fence_before();
         sync_compute();
         KDA_TC_PHASE(3);
@@ -1306,31 +1305,6 @@ static bool make_map(CUtensorMap* m, const void* base, int64_t rows, int H) {
 
 }  // namespace tc
 
-cudaError_t launch_chunk_tc2(const void* q, const void* k, const void* v, const void* alpha,
-                             const void* beta, const float* S0, const int32_t* cu, int nseq,
-                             void* out, float* S_final, int64_t rows, int64_t T, int H, int* status,
-                             cudaStream_t stream, const int32_t* slots, int num_slots, int fused);
-cudaError_t launch_chunk_tc2_segments(const void* q, const void* k, const void* v, const void* alpha,
-                                      const void* beta, const float* start, const int32_t* cu,
-                                      int nseq, void* out, float* S_final, int64_t rows, int64_t T,
-                                      int H, int nseg, int* status, cudaStream_t stream, int fused);
-cudaError_t launch_chunk_tc2_cta_status(const void* q, const void* k, const void* v,
-                                        const void* alpha, const void* beta, const float* S0,
-                                        const int32_t* cu, int nseq, void* out, float* S_final,
-                                        int64_t rows, int64_t T, int H, int* status,
-                                        cudaStream_t stream);
-
-// Which forward kernel the tensor-core entry points use (KDA_TC_KERNEL=2: the
-// pipelined kernel of kda_chunk_tc2.cu; anything else: this file's kernel).
-static bool use_tc2() {
-    static int v = -1;
-    if (v < 0) {
-        const char* e = std::getenv("KDA_TC_KERNEL");
-        v = (e && e[0] == '2') ? 1 : 0;
-    }
-    return v == 1;
-}
-
 bool make_tc_maps(TcMaps* m, const void* q, const void* k, const void* v, const void* alpha,
                   const void* out, int64_t rows, int H) {
     return tc::make_map(&m->q, q, rows, H) && tc::make_map(&m->k, k, rows, H) &&
@@ -1357,9 +1331,6 @@ cudaError_t launch_chunk_tc(const void* q, const void* k, const void* v, const v
                             const void* beta, const float* S0, const int32_t* cu, int nseq,
                             void* out, float* S_final, int64_t rows, int64_t T, int H, int* status,
                             cudaStream_t stream, const int32_t* slots, int num_slots, int fused) {
-    if (use_tc2())
-        return launch_chunk_tc2(q, k, v, alpha, beta, S0, cu, nseq, out, S_final, rows, T, H, status,
-                                stream, slots, num_slots, fused);
     TcMaps m;
     if (!make_tc_maps(&m, q, k, v, alpha, out, rows, H)) return cudaErrorInvalidValue;
     const tc::Segments whole{1, 1, nullptr, nullptr, slots, num_slots};
@@ -1399,9 +1370,6 @@ cudaError_t launch_chunk_tc_segmented(const void* q, const void* k, const void* 
         S0, maps, start, nseg, H);
     e = cudaGetLastError();
     if (e != cudaSuccess) return e;
-    if (use_tc2())
-        return launch_chunk_tc2_segments(q, k, v, alpha, beta, start, cu, nseq, out, S_final, rows, T,
-                                         H, nseg, status, stream, fused);
     const tc::Segments fwd{nseg, nseg, start, nullptr};
     return fused ? launch_tc_t<false, false, true>(m, beta, nullptr, cu, nseq, out, S_final, T, H,
                                                    status, fwd, stream)
@@ -1434,9 +1402,6 @@ cudaError_t launch_chunk_tc_cta_status(const void* q, const void* k, const void*
                                        const int32_t* cu, int nseq, void* out, float* S_final,
                                        int64_t rows, int64_t T, int H, int* status,
                                        cudaStream_t stream) {
-    if (use_tc2())
-        return launch_chunk_tc2_cta_status(q, k, v, alpha, beta, S0, cu, nseq, out, S_final, rows, T,
-                                           H, status, stream);
     TcMaps m;
     if (!make_tc_maps(&m, q, k, v, alpha, out, rows, H)) return cudaErrorInvalidValue;
     const tc::Segments whole{1, 1, nullptr, nullptr};
