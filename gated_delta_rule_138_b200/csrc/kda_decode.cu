@@ -16,10 +16,15 @@
 // d_k x d_v slab with 16-byte loads and stores, keeping it in registers between
 // the reduction and the update.  A multi-token step (T tokens per sequence,
 // inputs [N, T, H, d]) keeps the state in registers across its T tokens: the
-// state is read and written once per step, not once per token.
+// state is read and written once per step, not once per token.  The token rows
+// (q, k, alpha, v, beta) of up to kStageTokens tokens are staged in shared memory
+// with 16-byte loads issued right behind the state loads, so that the token loop
+// waits on no global load.
 #include "kda_common.cuh"
 
 namespace kda {
+
+constexpr int kStageTokens = 16;   // token rows staged in shared memory at a time
 
 // kFused: alpha and beta arrive as logits and q, k unnormalised (a compile-time
 // variant, so that the plain step carries none of the transforms' code)
@@ -41,6 +46,10 @@ kda_decode_kernel(const Tin* __restrict__ q, const Tin* __restrict__ k,
     __shared__ __align__(16) float red_y[TY][DV];
     __shared__ __align__(16) float us[DV];
     __shared__ float kq_part[NT / 32], nk_part[NT / 32], nq_part[NT / 32];
+    // staged token rows: q, k, alpha [kStageTokens][DK] and v [kStageTokens][DV], then beta
+    constexpr int VE = 16 / (int)sizeof(Tin);            // elements per 16-byte load
+    __shared__ __align__(16) Tin tin[kStageTokens * (3 * DK + DV)];
+    __shared__ Tin tbeta[kStageTokens];
 
     const int tid = threadIdx.x, tx = tid % TX, ty = tid / TX;
     const size_t nh = blockIdx.x;                 // (sequence, head) flattened
@@ -57,29 +66,43 @@ kda_decode_kernel(const Tin* __restrict__ q, const Tin* __restrict__ k,
     for (int i = 0; i < RPT; ++i)
         s[i] = slot_ok ? Sv[(size_t)(ty + TY * i) * TX + tx] : make_float4(0.f, 0.f, 0.f, 0.f);
 
+    // a single-token step reads its rows straight from global memory (no staging,
+    // no extra barrier); longer steps stage them
+    const bool direct = T == 1;
     for (int t = 0; t < T; ++t) {
     const size_t tok = ((size_t)n * T + t) * H + hh;   // (sequence, token, head)
-    const size_t kb = tok * DK, vb = tok * DV;
-    if (t + 1 < T) {
-        // the next token's q, k, alpha and v rows (and beta) towards L2 while this one
-        // is worked on: one thread per 128-byte line, no registers held
-        const size_t nk = (tok + H) * DK, nv = (tok + H) * DV;
-        constexpr int LK = (DK * (int)sizeof(Tin) + 127) / 128, LV = (DV * (int)sizeof(Tin) + 127) / 128;
-        const char* line = nullptr;
-        if (tid < LK) line = reinterpret_cast<const char*>(q + nk) + 128 * tid;
-        else if (tid < 2 * LK) line = reinterpret_cast<const char*>(k + nk) + 128 * (tid - LK);
-        else if (tid < 3 * LK) line = reinterpret_cast<const char*>(alpha + nk) + 128 * (tid - 2 * LK);
-        else if (tid < 3 * LK + LV) line = reinterpret_cast<const char*>(v + nv) + 128 * (tid - 3 * LK);
-        else if (tid == 3 * LK + LV) line = reinterpret_cast<const char*>(beta + tok + H);
-        if (line) asm volatile("prefetch.global.L2 [%0];" :: "l"(line));
+    const size_t vb = tok * DV;
+    const int ts = t % kStageTokens;                     // staged slot of this token
+    if (!direct && ts == 0) {
+        // stage the token rows of tokens t .. t + nt - 1 with 16-byte loads (the barrier
+        // before: every thread is done with the previous batch)
+        if (t > 0) __syncthreads();
+        const int nt = T - t < kStageTokens ? T - t : kStageTokens;
+        constexpr int RK = DK / VE, RV = DV / VE, RT = 3 * RK + RV;   // 16-byte pieces per token
+        for (int e = tid; e < nt * RT; e += NT) {
+            const int tt = e / RT, w = e % RT;
+            const size_t tk = ((size_t)n * T + t + tt) * H + hh;
+            const Tin* src;
+            Tin* dst;
+            if (w < RK) { src = q + tk * DK + w * VE; dst = tin + tt * DK + w * VE; }
+            else if (w < 2 * RK) { src = k + tk * DK + (w - RK) * VE; dst = tin + (kStageTokens + tt) * DK + (w - RK) * VE; }
+            else if (w < 3 * RK) { src = alpha + tk * DK + (w - 2 * RK) * VE; dst = tin + (2 * kStageTokens + tt) * DK + (w - 2 * RK) * VE; }
+            else { src = v + tk * DV + (w - 3 * RK) * VE; dst = tin + 3 * kStageTokens * DK + tt * DV + (w - 3 * RK) * VE; }
+            *reinterpret_cast<uint4*>(dst) = __ldg(reinterpret_cast<const uint4*>(src));
+        }
+        if (tid < nt) tbeta[tid] = beta[((size_t)n * T + t + tid) * H + hh];
     }
-    if (t > 0) __syncthreads();   // the previous token's update has read ga, kk and us
+    if (!direct) __syncthreads();   // staged rows visible; the previous token's update has read ga, kk and us
+    const Tin* sq = direct ? q + tok * DK : tin + ts * DK;
+    const Tin* sk = direct ? k + tok * DK : tin + (kStageTokens + ts) * DK;
+    const Tin* sa = direct ? alpha + tok * DK : tin + (2 * kStageTokens + ts) * DK;
+    const Tin* sv = direct ? v + vb : tin + 3 * kStageTokens * DK + ts * DV;
     // fused inputs: alpha and beta are logits, q and k are L2-normalised here
     float ikn = 1.0f, iqn = 1.0f;
     if constexpr (fused) {
         float pk = 0.0f, pq = 0.0f;
         if (tid < DK) {
-            const float kv = to_f32(k[kb + tid]), qv = to_f32(q[kb + tid]);
+            const float kv = to_f32(sk[tid]), qv = to_f32(sq[tid]);
             pk = kv * kv;
             pq = qv * qv;
         }
@@ -98,9 +121,9 @@ kda_decode_kernel(const Tin* __restrict__ q, const Tin* __restrict__ k,
     }
     float kqp = 0.0f;
     if (tid < DK) {
-        const float ax = to_f32(alpha[kb + tid]);
+        const float ax = to_f32(sa[tid]);
         const float a = clamp_gate(fused ? gate_from_logit(ax) : ax);
-        const float kv = to_f32(k[kb + tid]) * ikn, qv = to_f32(q[kb + tid]) * iqn;
+        const float kv = to_f32(sk[tid]) * ikn, qv = to_f32(sq[tid]) * iqn;
         ga[tid] = a;
         ka[tid] = a * kv;
         qa[tid] = a * qv;
@@ -133,9 +156,9 @@ kda_decode_kernel(const Tin* __restrict__ q, const Tin* __restrict__ k,
         float kq = 0.0f;
 #pragma unroll
         for (int i = 0; i < NT / 32; ++i) kq += kq_part[i];
-        const float bx = to_f32(beta[tok]);
+        const float bx = to_f32(direct ? beta[tok] : tbeta[ts]);
         const float b = fused ? sigmoid_f(bx) : bx;
-        const float u = b * (to_f32(v[vb + tid]) - x);
+        const float u = b * (to_f32(sv[tid]) - x);
         us[tid] = u;
         out[vb + tid] = from_f32<Tout>(fmaf(u, kq, y));
     }
