@@ -34,6 +34,13 @@ cudaError_t launch_backward(int in_bf16, const void* q, const void* k, const voi
                             const float* dSf, const int32_t* cu, int64_t nseq, int64_t T, int H,
                             int DK, int DV, float* dq, float* dk, float* dv, float* dalpha,
                             float* dbeta, float* dS0, float* workspace, cudaStream_t s);
+size_t backward_tc_workspace_bytes(bool packed, int64_t nseq, int64_t T, int H);
+bool backward_tc_supported(bool bf16, int64_t nseq, int64_t T, int H, int DK, int DV, bool packed);
+cudaError_t launch_backward_tc(const void* q, const void* k, const void* v, const void* alpha,
+                               const void* beta, const float* S0, const void* dout,
+                               const float* dSf, const int32_t* cu, int64_t nseq, int64_t T, int H,
+                               float* dq, float* dk, float* dv, float* dalpha, float* dbeta,
+                               float* dS0, void* workspace, int* status, cudaStream_t s);
 cudaError_t launch_segment_maps(const void* k, const void* v, const void* alpha, const void* beta,
                                 const int32_t* cu, int nseq, float* maps, int64_t rows, int64_t T,
                                 int H, int* status, cudaStream_t stream);
@@ -489,7 +496,10 @@ size_t kda_backward_workspace_bytes(int32_t B, int64_t T, int32_t H, int32_t d_k
                                     int32_t packed, int32_t num_seqs) {
     if (B < 0 || T < 0 || H <= 0 || num_seqs < 0) return 0;
     const int64_t nseq = packed ? (int64_t)num_seqs : (int64_t)B;
-    return sizeof(float) * kda::backward_workspace_floats(packed != 0, nseq, T, H, d_k, d_v);
+    const size_t seq = sizeof(float) * kda::backward_workspace_floats(packed != 0, nseq, T, H, d_k, d_v);
+    // enough for either kernel: the dtype is not an argument here
+    const size_t tc = d_k == 128 && d_v == 128 ? kda::backward_tc_workspace_bytes(packed != 0, nseq, T, H) : 0;
+    return seq > tc ? seq : tc;
 }
 
 kda_status_t kda_backward(const void* q, const void* k, const void* v, const void* alpha,
@@ -520,20 +530,34 @@ kda_status_t kda_backward(const void* q, const void* k, const void* v, const voi
     if (!head_dim_ok(d_k) || !head_dim_ok(d_v)) return KDA_ERR_UNSUPPORTED;
     if (nseq * H > 0x7fffffffLL) return KDA_ERR_UNSUPPORTED;
     if (nseq == 0) return KDA_OK;
-    const size_t need = sizeof(float) * kda::backward_workspace_floats(cu_seqlens != nullptr, nseq,
-                                                                       T, H, d_k, d_v);
-    if (workspace && workspace_bytes < need) return KDA_ERR_INVALID_ARG;
+    const bool tc = kda::backward_tc_supported(in_dtype == KDA_BF16, nseq, T, H, d_k, d_v,
+                                               cu_seqlens != nullptr);
+    const size_t need =
+        tc ? kda::backward_tc_workspace_bytes(cu_seqlens != nullptr, nseq, T, H)
+           : sizeof(float) * kda::backward_workspace_floats(cu_seqlens != nullptr, nseq, T, H, d_k, d_v);
+    // a caller's workspace is held to the documented query (which covers either kernel)
+    if (workspace && workspace_bytes < kda_backward_workspace_bytes(
+                                           B, T, H, d_k, d_v, cu_seqlens != nullptr, num_seqs))
+        return KDA_ERR_INVALID_ARG;
     g_last_error[0] = '\0';
     const cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    int* status = nullptr;
+    if (tc) {
+        cudaError_t e = device_status_word(&status);
+        if (e != cudaSuccess) return cuda_status(e);
+    }
     float* ws = static_cast<float*>(workspace);
     if (!ws) {
         cudaError_t e = cudaMallocAsync(reinterpret_cast<void**>(&ws), need, s);
         if (e != cudaSuccess) return cuda_status(e);
     }
-    g_launches.fetch_add(1, std::memory_order_relaxed);
-    cudaError_t e = kda::launch_backward(in_dtype == KDA_BF16, q, k, v, alpha, beta, S0, dout,
-                                         dS_final, cu_seqlens, nseq, T, H, d_k, d_v, dq, dk, dv,
-                                         dalpha, dbeta, dS0, ws, s);
+    g_launches.fetch_add(tc ? 3 : 1, std::memory_order_relaxed);   // tensor cores: three kernels
+    cudaError_t e =
+        tc ? kda::launch_backward_tc(q, k, v, alpha, beta, S0, dout, dS_final, cu_seqlens, nseq, T, H,
+                                     dq, dk, dv, dalpha, dbeta, dS0, ws, status, s)
+           : kda::launch_backward(in_dtype == KDA_BF16, q, k, v, alpha, beta, S0, dout, dS_final,
+                                  cu_seqlens, nseq, T, H, d_k, d_v, dq, dk, dv, dalpha, dbeta, dS0,
+                                  ws, s);
     if (!workspace) {
         const cudaError_t ef = cudaFreeAsync(ws, s);
         if (e == cudaSuccess) e = ef;

@@ -53,6 +53,7 @@
 #include "kda_common.cuh"
 #include "kda_sm100.cuh"
 #include "kda_tc_maps.cuh"
+#include "kda_bwd_record.cuh"
 
 // Optional phase-boundary hook for profiling builds (no-op in the library).
 #ifndef KDA_TC_PHASE
@@ -159,6 +160,11 @@ struct Segments {
     // starts from zero and writes no state.  Null: slot n.
     const int32_t* slots;
     int num_slots;
+    // record mode (the backward's first pass): per-(chunk, head) records and per-chunk
+    // headers, chunks numbered across sequences in order
+    uint8_t* rec = nullptr;
+    bwdrec::Header* hdr = nullptr;
+    int64_t rec_chunks = 0;   // chunks the records hold (a malformed packed table is cut there)
 };
 
 // One TMA stream's bookkeeping: the parity a thread's next wait on it expects,
@@ -172,7 +178,10 @@ struct LoadTrack {
 // kSummary = true: the segment-map mode described at the top (q and out unused).
 // kFused = true: alpha and beta arrive as logits (alpha = 1/(1+e^x), beta =
 // sigmoid(x)) and q, k unnormalised (L2-normalised per token and head here).
-template <bool kCtaStatus, bool kSummary, bool kFused>
+// kRecord = true: the forward recurrence without outputs; every chunk's start state,
+// operand tiles, T, V - (k*gamma) S, U and gamma_C go to the backward's record of
+// (chunk, head) (kda_bwd_record.cuh), byte for byte as they sit in shared memory.
+template <bool kCtaStatus, bool kSummary, bool kFused, bool kRecord = false>
 __global__ void __launch_bounds__(NTHREADS, 1)
 kda_chunk_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                     const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmV,
@@ -209,13 +218,19 @@ kda_chunk_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_consta
     const int h = blockIdx.y;
     const int per_seq = seg.per_seq, gseg = (int)blockIdx.z % per_seq;
     __shared__ int s_seq;
+    __shared__ int64_t s_cbase;
     if (threadIdx.x < 32) {
         const int sq = longest_first_seq(cu_seqlens, (int)gridDim.z / per_seq,
                                          (int)blockIdx.z / per_seq, T);
-        if (threadIdx.x == 0) s_seq = sq;
+        const int64_t cb = kRecord ? chunks_before(cu_seqlens, sq, T, C) : 0;
+        if (threadIdx.x == 0) { s_seq = sq; s_cbase = cb; }
     }
     __syncthreads();
     const int n = s_seq;
+    // this CTA's record of chunk i (record mode)
+    auto rec_of = [&](int i) {
+        return seg.rec + ((size_t)(s_cbase + i) * H + h) * bwdrec::BYTES;
+    };
     int64_t bos, len;
     seq_range(cu_seqlens, n, T, bos, len);
     if (seg.nseg > 1) {   // this CTA's segment of the sequence
@@ -225,7 +240,9 @@ kda_chunk_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_consta
         bos += t0;
         len = t1 - t0;
     }
-    const int nchunks = (int)((len + C - 1) / C);
+    int nchunks = (int)((len + C - 1) / C);
+    if (kRecord && s_cbase + nchunks > seg.rec_chunks)
+        nchunks = (int)max((int64_t)0, seg.rec_chunks - s_cbase);
     const bool last_seg = gseg == seg.nseg - 1;
     const int slot = seg.slots ? seg.slots[n] : n;
     const bool slot_ok = !seg.slots || (slot >= 0 && slot < seg.num_slots);
@@ -369,6 +386,7 @@ kda_chunk_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_consta
 #pragma unroll
             for (int ch = 0; ch < 8; ++ch)
                 *reinterpret_cast<uint4*>(sS + hf * 16384 + swz(c, ch)) = pack8(&v[8 * ch]);
+            if constexpr (kRecord) return;   // no outputs
             tmem_ld64(tmem + tlane + TM_O + 64 * hf, v);
             const int r = 16 * q4 + lane;
             if (pLc == C) {
@@ -497,6 +515,8 @@ kda_chunk_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_consta
                         if (M == Q) own = pq[M][c];
                     }
                     if (O == 0) sGC[c0 + c] = pq[0][c] * pq[1][c] * pq[2][c] * pq[3][c];
+                    if (kRecord && O == 0)
+                        reinterpret_cast<float*>(rec_of(chunk) + bwdrec::GC)[c0 + c] = sGC[c0 + c];
                     const float fO = (O & 1) ? pov[c] : 1.0f;
                     const float gO = (O & 1) ? 1.0f : pov[c];
                     const float dl = (Q & 1) ? 1.0f : __frcp_rn(own);
@@ -809,6 +829,14 @@ kda_chunk_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_consta
                     v[i] = (jr >= m) ? Tm[jr * AS + m] * sBeta[m] : 0.0f;
                 }
                 *reinterpret_cast<uint4*>(sTB + swz(jr, ch)) = pack8(v);
+                if constexpr (kRecord) {   // T itself, in the same K-major layout
+#pragma unroll
+                    for (int i = 0; i < 8; ++i) {
+                        const int m = 8 * ch + i;
+                        v[i] = (jr >= m) ? Tm[jr * AS + m] : 0.0f;
+                    }
+                    *reinterpret_cast<uint4*>(rec_of(chunk) + bwdrec::T + swz(jr, ch)) = pack8(v);
+                }
             }
             KDA_TC_PHASE(12);
         }
@@ -949,7 +977,7 @@ kda_chunk_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_consta
         for (int ks = 0; ks < 8; ++ks)
             mma_bf16(tmem + TM_WK, sdesc_sw128(l0 + (ks >> 2) * 16384u + (ks & 3) * 32u),
                      sdesc_sw128(r0 + (ks >> 2) * 12288u + (ks & 3) * 32u), idesc, ks > 0);
-        commit_mma();
+        if constexpr (!kRecord) commit_mma();   // record mode commits after its copies
     };
     auto mma_z = [&]() {   // (k*gamma) S_start into U's columns (own barrier)
         const uint32_t kg = smem_u32(sKT), s0 = smem_u32(sS);
@@ -1024,12 +1052,14 @@ kda_chunk_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_consta
             for (int ks = 0; ks < 4; ++ks)
                 mma_bf16(tmem + TM_S, sdesc_sw128(kh + ks * 2048, 1024, 8192),
                          sdesc_sw128(u0 + ks * 2048, 1024, 8192), id_s, 1);
+            if constexpr (!kRecord) {
 #pragma unroll
-            for (int ks = 0; ks < 4; ++ks)
-                mma_bf16(tmem + TM_O, sdesc_sw128(p0 + ks * 32), sdesc_sw128(u0 + ks * 2048, 1024, 8192),
-                         idM64, 1);
+                for (int ks = 0; ks < 4; ++ks)
+                    mma_bf16(tmem + TM_O, sdesc_sw128(p0 + ks * 32),
+                             sdesc_sw128(u0 + ks * 2048, 1024, 8192), idM64, 1);
+            }
         }
-        commit_mma();
+        if constexpr (!kRecord) commit_mma();   // record mode commits after its copies
     };
     auto handoff = [&]() {
         tc_fence_before();
@@ -1045,13 +1075,31 @@ kda_chunk_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_consta
         if (ctl) {
             KDA_TC_PHASE(20);
             if (ok) {
+                if constexpr (kRecord) {   // start state and operand tiles to the record
+                    uint8_t* rp = rec_of(chunk);
+                    if (h == 0) {
+                        const int64_t rem = len - (int64_t)chunk * C;
+                        seg.hdr[s_cbase + chunk] = bwdrec::Header{row0, (int32_t)(rem < C ? rem : C), 0};
+                    }
+                    bulk_store(rp + bwdrec::S, sS, 32768);
+                    bulk_store(rp + bwdrec::L, sX + X_L, 32768);
+                    bulk_store(rp + bwdrec::R, sX + X_R, 24576);
+                    bulk_store(rp + bwdrec::QT, sQc, 16384);
+                    bulk_store(rp + bwdrec::KT, sKT, 16384);
+                    bulk_store(rp + bwdrec::KH, sKH, 16384);
+                    bulk_commit_group();
+                }
                 mma_ap();
                 if (!kSummary) {
                     mma_z();
-                    mma_qs(sQc);
+                    if (!kRecord) mma_qs(sQc);
+                }
+                if constexpr (kRecord) {   // the tiles are read before anyone may overwrite them
+                    bulk_wait_read_all();
+                    commit_mma();
                 }
             }
-            if (!kSummary && chunk > 0) store_o(sQ + ((chunk + 1) & 1) * 16384, row0 - C);
+            if (!kSummary && !kRecord && chunk > 0) store_o(sQ + ((chunk + 1) & 1) * 16384, row0 - C);
             if (chunk + 1 < nchunks && ok) {   // k and alpha are consumed
                 issue_ka(row0 + C);
                 issued(tka);
@@ -1071,6 +1119,10 @@ kda_chunk_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_consta
         }
         handoff();   // B
         if (ctl) {
+            if (kRecord && ok) {   // P (its read is waited for before the next commit)
+                bulk_store(rec_of(chunk) + bwdrec::P, sX + X_P, 8192);
+                bulk_commit_group();
+            }
             if (ok) {
                 mma_tf1();
                 mma_tf2();
@@ -1085,7 +1137,12 @@ kda_chunk_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_consta
                 wait_load(barV, tv);
                 if (ok) mma_tbv();
             } else if (ok) {
+                if constexpr (kRecord) {
+                    bulk_store(rec_of(chunk) + bwdrec::RV, sV, 16384);
+                    bulk_commit_group();
+                }
                 mma_tbv();   // U = Tb (V - (k*gamma) S), the v tile holding the difference
+                if constexpr (kRecord) bulk_wait_read_all();   // before the next v load
                 commit_mma();
             }
             wait_mma();
@@ -1109,7 +1166,17 @@ kda_chunk_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_consta
             broke = true;
             break;
         }
-        if (ctl && ok) mma_s();
+        if (ctl && ok) {
+            if constexpr (kRecord) {
+                bulk_store(rec_of(chunk) + bwdrec::U, sX + X_U, 16384);
+                bulk_commit_group();
+            }
+            mma_s();
+            if constexpr (kRecord) {
+                bulk_wait_read_all();
+                commit_mma();
+            }
+        }
     }
     if (ctl && nchunks > 0 && !broke) wait_mma();
 
@@ -1123,7 +1190,7 @@ kda_chunk_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_consta
     if (!ok) atomicExch(sFlag, 1);
     __syncthreads();
     if (!kSummary && ctl) {
-        if (nchunks > 0 && !broke && !*sFlag && last_Lc == C)
+        if (!kRecord && nchunks > 0 && !broke && !*sFlag && last_Lc == C)
             store_o(last_stage, bos + (int64_t)(nchunks - 1) * C);
         bulk_wait_all();   // every O store has completed before shared memory is released
     }
@@ -1312,16 +1379,16 @@ bool make_tc_maps(TcMaps* m, const void* q, const void* k, const void* v, const 
            tc::make_map(&m->o, out ? out : v, rows, H);
 }
 
-template <bool kCtaStatus, bool kSummary, bool kFused = false>
+template <bool kCtaStatus, bool kSummary, bool kFused = false, bool kRecord = false>
 static cudaError_t launch_tc_t(const TcMaps& m, const void* beta, const float* S0, const int32_t* cu,
                                int nseq, void* out, float* S_final, int64_t T, int H, int* status,
                                const tc::Segments& seg, cudaStream_t stream) {
-    cudaError_t e = cudaFuncSetAttribute(tc::kda_chunk_tc_kernel<kCtaStatus, kSummary, kFused>,
+    cudaError_t e = cudaFuncSetAttribute(tc::kda_chunk_tc_kernel<kCtaStatus, kSummary, kFused, kRecord>,
                                          cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          (int)tc::SMEM_BYTES);
     if (e != cudaSuccess) return e;
     dim3 grid(1, H, nseq * seg.per_seq);
-    tc::kda_chunk_tc_kernel<kCtaStatus, kSummary, kFused><<<grid, tc::NTHREADS, tc::SMEM_BYTES, stream>>>(
+    tc::kda_chunk_tc_kernel<kCtaStatus, kSummary, kFused, kRecord><<<grid, tc::NTHREADS, tc::SMEM_BYTES, stream>>>(
         m.q, m.k, m.a, m.v, m.o, (const __nv_bfloat16*)beta, S0, cu, (__nv_bfloat16*)out, S_final, T, H,
         status, seg);
     return cudaGetLastError();
@@ -1338,6 +1405,25 @@ cudaError_t launch_chunk_tc(const void* q, const void* k, const void* v, const v
                                                    whole, stream)
                  : launch_tc_t<false, false>(m, beta, S0, cu, nseq, out, S_final, T, H, status,
                                              whole, stream);
+}
+
+// The backward's first pass: the forward recurrence of whole sequences in record mode
+// (no outputs), filling rec (one kda_bwd_record.cuh record per (chunk, head), chunks
+// numbered across sequences in order) and hdr (one header per chunk; the caller
+// zeroes it first, so that unused entries read as empty).
+cudaError_t launch_chunk_tc_record(const void* q, const void* k, const void* v, const void* alpha,
+                                   const void* beta, const float* S0, const int32_t* cu, int nseq,
+                                   int64_t rows, int64_t T, int H, uint8_t* rec,
+                                   bwdrec::Header* hdr, int64_t rec_chunks, int* status,
+                                   cudaStream_t stream) {
+    TcMaps m;
+    if (!make_tc_maps(&m, q, k, v, alpha, nullptr, rows, H)) return cudaErrorInvalidValue;
+    tc::Segments whole{1, 1, nullptr, nullptr, nullptr, 0};
+    whole.rec = rec;
+    whole.hdr = hdr;
+    whole.rec_chunks = rec_chunks;
+    return launch_tc_t<false, false, false, true>(m, beta, S0, cu, nseq, nullptr, nullptr, T, H,
+                                                  status, whole, stream);
 }
 
 // Floats of workspace the split forward uses: the segment maps [M | N] and the

@@ -54,6 +54,22 @@ __device__ __forceinline__ void seq_range(const int32_t* __restrict__ cu_seqlens
     len = b - a;
 }
 
+// Chunks of C tokens before sequence n (the sum of ceil(len_m / C) over m < n),
+// computed by one whole warp; every lane returns the total.
+__device__ __forceinline__ int64_t chunks_before(const int32_t* __restrict__ cu, int n, int64_t T,
+                                                 int C) {
+    if (cu == nullptr) return (int64_t)n * ((T + C - 1) / C);
+    int64_t acc = 0;
+    for (int m = (int)(threadIdx.x & 31); m < n; m += 32) {
+        int64_t b, l;
+        seq_range(cu, m, T, b, l);
+        acc += (l + C - 1) / C;
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, o);
+    return acc;
+}
+
 // Longest-first schedule for packed batches: CTAs are launched in blockIdx.z
 // order, so z-th CTA column takes the sequence of rank z in decreasing length
 // (ties by index).  Each CTA ranks the lengths itself from cu_seqlens: no

@@ -226,6 +226,18 @@ __device__ __forceinline__ void tma_store_2d(const void* tmap, const void* src, 
         "cp.async.bulk.tensor.2d.global.shared::cta.tile.bulk_group [%0, {%1, %2}], [%3];"
         :: "l"(tmap), "r"(x), "r"(y), "r"(smem_u32(src)) : "memory");
 }
+// Untiled bulk copies of `bytes` contiguous bytes (both addresses 16-byte aligned,
+// bytes a multiple of 16): global -> shared with completion on `bar`, and
+// shared -> global in the current bulk group.
+__device__ __forceinline__ void bulk_load(void* dst, const void* src, uint32_t bytes, uint64_t* bar) {
+    asm volatile(
+        "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];"
+        :: "r"(smem_u32(dst)), "l"(src), "r"(bytes), "r"(smem_u32(bar)) : "memory");
+}
+__device__ __forceinline__ void bulk_store(void* dst, const void* src, uint32_t bytes) {
+    asm volatile("cp.async.bulk.global.shared::cta.bulk_group [%0], [%1], %2;"
+                 :: "l"(dst), "r"(smem_u32(src)), "r"(bytes) : "memory");
+}
 __device__ __forceinline__ void bulk_commit_group() {
     asm volatile("cp.async.bulk.commit_group;" ::: "memory");
 }
