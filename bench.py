@@ -79,6 +79,23 @@ def backward_flops(w, n_token_heads: int) -> int:
     return 31 * w.dk * w.dv * n_token_heads
 
 
+def backward_tc_flops(w, n_token_heads: int) -> int:
+    """Tensor-core backward (d_k = d_v = 128, C = 64): the MMA flops per chunk, per
+    (token, head).  Record pass: [A/beta ; P] (128 x 96 x 128), (k*gamma) S0
+    (64 x 128 x 128), U (64 x 128 x 64), the state update (128 x 128 x 64) and the
+    32 -> 64 solve step (2 x 64 x 32 x 32); state-gradient pass: dU (64 x 128 x 192),
+    dY (64 x 128 x 64), dS (128 x 128 x 128); chunk pass: [dY ; dO] U^T (128 x 64 x 128),
+    [A/beta ; P] (128 x 96 x 128), dS U^T (128 x 64 x 128), S0 [dR ; dO]^T, R^T G^T,
+    L^T G (128 x 128 x 128, 128 x 128 x 96, 128 x 128 x 128)."""
+    C = w.chunk
+    mnk = [(128, 96, 128), (64, 128, 128), (64, 128, 64), (128, 128, 64), (64, 32, 32), (64, 32, 32),
+           (64, 128, 192), (64, 128, 64), (128, 128, 128),
+           (128, 64, 128), (128, 96, 128), (128, 64, 128), (128, 128, 128), (128, 128, 96),
+           (128, 128, 128)]
+    per_chunk = sum(2 * m * n * k for m, n, k in mnk)
+    return per_chunk * n_token_heads // C
+
+
 def decode_bytes(w, n_seq_heads: int) -> int:
     ei, eo = esize(w.dtype), esize(w.out_dtype)
     return n_seq_heads * (8 * w.dk * w.dv + ei * (3 * w.dk + w.dv + 1) + eo * w.dv)
@@ -575,7 +592,8 @@ def run_ours(args, w):
         if args.fused:
             kname += "_fused"   # its own compile-time variant (no DRAM-traffic record)
         if args.backward:
-            kname = "backward_f32"
+            kname = ("backward_tc_bf16" if (w.dtype == "bf16" and w.dk == 128 and w.dv == 128)
+                     else "backward_f32")
         # time segments per sequence of the tensor-core path (1: unsplit); with g > 1 a
         # step is three launches (segment maps, scan, forward) timed together
         segments = (kda.kda_forward_segments(nseq, -(-B * T // nseq), w.H)
@@ -584,7 +602,8 @@ def run_ours(args, w):
         algo_flops = forward_flops(w, n_th)
         if args.backward:
             algo_bytes = backward_bytes(w, n_th, n_sh, inp["S0"] is not None)
-            algo_flops = backward_flops(w, n_th)
+            algo_flops = (backward_tc_flops(w, n_th) if kname == "backward_tc_bf16"
+                          else backward_flops(w, n_th))
 
     warm = max(3, args.warmup)
     for _ in range(warm):
@@ -837,11 +856,19 @@ def main():
                     help="split every sequence's time axis across the ranks (strong scaling)")
     ap.add_argument("--e2e-steps", type=int, default=10,
                     help="steps of the end-to-end (host buffers) measurement; 0 skips it")
+    ap.add_argument("--batch", type=int, default=0,
+                    help="a dense workload with this many sequences instead of its own B "
+                         "(smaller cases of the same kernels, for profiler captures)")
     args = ap.parse_args()
     if args.backward and (args.fused or args.seqpar):
         ap.error("--backward times kda_backward alone (not with --fused or --seqpar)")
     from gated_delta_rule_138_b200 import inputs as gen
     w = gen.WORKLOADS[args.workload]
+    if args.batch > 0:
+        if w.kind != "forward":
+            ap.error("--batch applies to the dense forward workloads")
+        import dataclasses
+        w = dataclasses.replace(w, B=args.batch, name="%s_batch%d" % (w.name, args.batch))
     if args.impl == "reference":
         run_reference(args, w)
     else:
