@@ -103,21 +103,29 @@ constexpr uint32_t OFF_KH = 40960;      // k*eta [64 j][128 c]
 constexpr uint32_t OFF_T = 57344;       // T [64 j][64 m]
 constexpr uint32_t OFF_QT = 65536;      // q*gamma [64 r][128 c]
 constexpr uint32_t OFF_KT = 81920;      // k*gamma [64 r][128 c]
-constexpr uint32_t OFF_DO = 98304;      // dO [64 r][128 n] (TMA)
+constexpr uint32_t OFF_DO = 98304;      // dO [64 r][128 n] (TMA), chunk parity 0; parity 1 at OFF_DO1
 constexpr uint32_t OFF_RV = 114688;     // R = V - (k*gamma) S0 [64 j][128 n]
 constexpr uint32_t OFF_DU = 131072;     // dU bf16 [64 j][128 n], MN-major B
 constexpr uint32_t OFF_MDR = 147456;    // -dR bf16 [64 r][128 n], MN-major B
 constexpr uint32_t OFF_DY = 163840;     // dY bf16 [64 m][128 n] (to the record)
-constexpr uint32_t OFF_MISC = 180224;
-constexpr uint32_t M_GC = 0;            // float [128]
-constexpr uint32_t M_BETA = 512;        // float [64]
-constexpr uint32_t M_DB = 768;          // float [64][2]
-constexpr uint32_t M_BAR = 1280;        // uint64 x4: loads A (P, k*eta), B (T), C (the rest), MMA
-constexpr uint32_t M_TMEM = 1312;
-constexpr uint32_t M_FLAG = 1316;
-constexpr uint32_t SMEM_BYTES = OFF_MISC + 1344 + 1024;
+constexpr uint32_t OFF_DO1 = 180224;
+constexpr uint32_t OFF_MISC = 196608;
+constexpr uint32_t M_GC = 0;            // float [2 parities][128]
+constexpr uint32_t M_BETA = 1024;       // float [64]
+constexpr uint32_t M_DB = 1280;         // float [64][2]
+constexpr uint32_t M_BAR = 1792;        // uint64 x4: loads A (P, k*eta, dO, gamma_C), B (T), C (q*gamma, k*gamma, R), MMA
+constexpr uint32_t M_TMEM = 1824;
+constexpr uint32_t M_FLAG = 1828;
+constexpr uint32_t SMEM_BYTES = OFF_MISC + 1856 + 1024;
 constexpr uint32_t TM_DS = 0, TM_DU = 128, TM_DY = 256;
 }  // namespace ds
+
+// 32 consecutive fp32 TMEM columns of this thread's lane
+__device__ __forceinline__ void tmem_ld32(uint32_t taddr, float (&v)[32]) {
+    tmem_ld16(taddr, *reinterpret_cast<float(*)[16]>(&v[0]));
+    tmem_ld16(taddr + 16, *reinterpret_cast<float(*)[16]>(&v[16]));
+    tmem_wait_ld();
+}
 
 __global__ void __launch_bounds__(NT + 32, 1)
 kda_bwd_dstate_kernel(const __grid_constant__ CUtensorMap tmDO, const __nv_bfloat16* __restrict__ beta,
@@ -159,6 +167,7 @@ kda_bwd_dstate_kernel(const __grid_constant__ CUtensorMap tmDO, const __nv_bfloa
     if (s_cbase + nchunks > rec_chunks)   // a malformed packed table: cut at the records' end
         nchunks = (int)max((int64_t)0, rec_chunks - s_cbase);
     auto rec_of = [&](int i) { return rec + ((size_t)(s_cbase + i) * H + h) * bwdrec::BYTES; };
+    auto dO_of = [&](int i) { return sm + ((i & 1) ? OFF_DO1 : OFF_DO); };
 
     if (tid == 0) {
         mbar_init(barA, 1);
@@ -219,11 +228,18 @@ kda_bwd_dstate_kernel(const __grid_constant__ CUtensorMap tmDO, const __nv_bfloa
         phM ^= 1u;
         tc_fence_after();
     };
+    // loads a chunk ahead where the buffers allow: A (needed first) lands while the
+    // previous chunk's dY and dS steps run
     auto issue_a = [&](int i) {
         uint8_t* rp = rec_of(i);
-        mbar_arrive_expect_tx(barA, 8192 + 16384);
+        const int64_t row0 = bos + (int64_t)i * C;
+        mbar_arrive_expect_tx(barA, 8192 + 16384 + 16384 + 512);
         bulk_load(sm + OFF_P, rp + bwdrec::P, 8192, barA);
         bulk_load(sm + OFF_KH, rp + bwdrec::KH, 16384, barA);
+        bulk_load(sGC + 128 * (i & 1), rp + bwdrec::GC, 512, barA);
+#pragma unroll
+        for (int a = 0; a < 2; ++a)
+            tma_load_2d(dO_of(i) + a * 8192, &tmDO, barA, h * DV + 64 * a, (int)row0);
         ++nA;
     };
     auto issue_b = [&](int i) {
@@ -233,15 +249,10 @@ kda_bwd_dstate_kernel(const __grid_constant__ CUtensorMap tmDO, const __nv_bfloa
     };
     auto issue_c = [&](int i) {
         uint8_t* rp = rec_of(i);
-        const int64_t row0 = bos + (int64_t)i * C;
-        mbar_arrive_expect_tx(barC, 4 * 16384 + 512);
+        mbar_arrive_expect_tx(barC, 3 * 16384);
         bulk_load(sm + OFF_QT, rp + bwdrec::QT, 16384, barC);
         bulk_load(sm + OFF_KT, rp + bwdrec::KT, 16384, barC);
         bulk_load(sm + OFF_RV, rp + bwdrec::RV, 16384, barC);
-        bulk_load(sGC, rp + bwdrec::GC, 512, barC);
-#pragma unroll
-        for (int a = 0; a < 2; ++a)
-            tma_load_2d(sm + OFF_DO + a * 8192, &tmDO, barC, h * DV + 64 * a, (int)row0);
         ++nC;
     };
     if (ctl && nchunks > 0) {
@@ -261,16 +272,15 @@ kda_bwd_dstate_kernel(const __grid_constant__ CUtensorMap tmDO, const __nv_bfloa
         float bval = 0.0f;
         if (compute && tid < C && tid < Lc) bval = __bfloat162float(beta[(size_t)(row0 + tid) * H + h]);
 
-        // ---- X1: the dS copy is in place; dU = P^T dO + (k*eta) dS
+        // ---- dU = P^T dO + (k*eta) dS (the dS copy is in place)
         if (ctl) {
             wait_bar(barA, phA);
-            wait_bar(barC, phC);
             if (ok) {
                 bulk_store(rec_of(i) + bwdrec::DS, sm + OFF_DS, 32768);
                 bulk_commit_group();
                 constexpr uint32_t id64 = idesc_bf16(64, 128, true, true);
                 constexpr uint32_t id64k = idesc_bf16(64, 128, false, true);
-                const uint32_t p0 = smem_u32(sm + OFF_P), d0 = smem_u32(sm + OFF_DO);
+                const uint32_t p0 = smem_u32(sm + OFF_P), d0 = smem_u32(dO_of(i));
                 const uint32_t kh = smem_u32(sm + OFF_KH), s0 = smem_u32(sm + OFF_DS);
 #pragma unroll
                 for (int ks = 0; ks < 4; ++ks)
@@ -282,45 +292,49 @@ kda_bwd_dstate_kernel(const __grid_constant__ CUtensorMap tmDO, const __nv_bfloa
                 commit();
             }
             wait_mma();
-            if (i > 0 && ok) issue_a(i - 1);   // P and k*eta are consumed
         }
         if (compute) {
-            wait_bar(barC, phC);   // gamma_C (and the tiles read below)
+            wait_bar(barA, phA);   // gamma_C
             wait_mma();
             const int c = 32 * q4 + lane;
             // dS <- Diag(gamma_C) dS in TMEM (the MMAs read the bf16 copy)
-            {
-                const float g = sGC[c];
-                const uint32_t ta = tmem + tlane + TM_DS + 64 * hf;
-                float v[64];
-                tmem_ld64(ta, v);
+            const float g = sGC[128 * (i & 1) + c];
 #pragma unroll
-                for (int k2 = 0; k2 < 64; ++k2) v[k2] *= g;
+            for (int p = 0; p < 2; ++p) {
+                const uint32_t ta = tmem + tlane + TM_DS + 64 * hf + 32 * p;
+                float v[32];
+                tmem_ld32(ta, v);
 #pragma unroll
-                for (int blk = 0; blk < 4; ++blk)
-                    tmem_st16(ta + 16 * blk, *reinterpret_cast<float(*)[16]>(&v[16 * blk]));
-                tmem_wait_st();
+                for (int k2 = 0; k2 < 32; ++k2) v[k2] *= g;
+                tmem_st16(ta, *reinterpret_cast<float(*)[16]>(&v[0]));
+                tmem_st16(ta + 16, *reinterpret_cast<float(*)[16]>(&v[16]));
             }
+            tmem_wait_st();
             // dU as the MN-major B operand: M=64 row j = 16 q4 + lane (lane < 16)
-            {
-                float v[64];
-                tmem_ld64(tmem + tlane + TM_DU + 64 * hf, v);
+#pragma unroll
+            for (int p = 0; p < 2; ++p) {
+                float v[32];
+                tmem_ld32(tmem + tlane + TM_DU + 64 * hf + 32 * p, v);
                 if (lane < 16) {
                     const int j = 16 * q4 + lane;
 #pragma unroll
-                    for (int ch = 0; ch < 8; ++ch)
-                        *reinterpret_cast<uint4*>(sm + OFF_DU + hf * 8192 + swz(j, ch)) = pack8(&v[8 * ch]);
+                    for (int ch = 0; ch < 4; ++ch)
+                        *reinterpret_cast<uint4*>(sm + OFF_DU + hf * 8192 + swz(j, 4 * p + ch)) =
+                            pack8(&v[8 * ch]);
                 }
             }
             if (tid < C) sBeta[tid] = bval;
         }
         fence_async_smem();
         tc_fence_before();
-        __syncthreads();   // X2
+        __syncthreads();
         tc_fence_after();
 
         // ---- dY = T^T dU
         if (ctl) {
+            // every thread has passed its wait on this chunk's A loads: P and k*eta are
+            // consumed, and the other dO and gamma_C buffers are free
+            if (i > 0 && ok) issue_a(i - 1);
             wait_bar(barB, phB);
             if (ok) {
                 constexpr uint32_t id64 = idesc_bf16(64, 128, true, true);
@@ -334,49 +348,55 @@ kda_bwd_dstate_kernel(const __grid_constant__ CUtensorMap tmDO, const __nv_bfloa
             if (i > 0 && ok) issue_b(i - 1);   // T is consumed
         }
         if (compute) {
+            wait_bar(barC, phC);   // R
             wait_mma();
-            float v[64];
-            tmem_ld64(tmem + tlane + TM_DY + 64 * hf, v);
-            if (lane < 16) {
-                const int m = 16 * q4 + lane;
-                const float b = sBeta[m];
-                // dV = dR = beta dY (fp32 out), -dR and dY as bf16 tiles, dbeta's first part
-                float part = 0.0f;
+            const int m = 16 * q4 + lane;
+            const float b = lane < 16 ? sBeta[m] : 0.0f;
+            float part = 0.0f;
 #pragma unroll
-                for (int ch = 0; ch < 8; ++ch) {
-                    float r8[8], w[8];
-                    unpack8(*reinterpret_cast<const uint4*>(sm + OFF_RV + hf * 8192 + swz(m, ch)), r8);
+            for (int p = 0; p < 2; ++p) {
+                float v[32];
+                tmem_ld32(tmem + tlane + TM_DY + 64 * hf + 32 * p, v);
+                if (lane < 16) {
+                    // dV = dR = beta dY (fp32 out), -dR and dY as bf16 tiles, dbeta's first part
 #pragma unroll
-                    for (int e = 0; e < 8; ++e) {
-                        part = fmaf(r8[e], v[8 * ch + e], part);
-                        w[e] = -b * v[8 * ch + e];
+                    for (int ch = 0; ch < 4; ++ch) {
+                        float r8[8], w[8];
+                        const uint32_t off = hf * 8192 + swz(m, 4 * p + ch);
+                        unpack8(*reinterpret_cast<const uint4*>(sm + OFF_RV + off), r8);
+#pragma unroll
+                        for (int e = 0; e < 8; ++e) {
+                            part = fmaf(r8[e], v[8 * ch + e], part);
+                            w[e] = -b * v[8 * ch + e];
+                        }
+                        *reinterpret_cast<uint4*>(sm + OFF_MDR + off) = pack8(w);
+                        *reinterpret_cast<uint4*>(sm + OFF_DY + off) = pack8(&v[8 * ch]);
                     }
-                    *reinterpret_cast<uint4*>(sm + OFF_MDR + hf * 8192 + swz(m, ch)) = pack8(w);
-                    *reinterpret_cast<uint4*>(sm + OFF_DY + hf * 8192 + swz(m, ch)) = pack8(&v[8 * ch]);
-                }
-                sDB[2 * m + hf] = part;
-                if (m < Lc) {
-                    float* dst = dv + ((size_t)(row0 + m) * H + h) * DV + 64 * hf;
+                    if (m < Lc) {
+                        float* dst = dv + ((size_t)(row0 + m) * H + h) * DV + 64 * hf + 32 * p;
 #pragma unroll
-                    for (int e = 0; e < 64; e += 4)
-                        *reinterpret_cast<float4*>(dst + e) =
-                            make_float4(b * v[e], b * v[e + 1], b * v[e + 2], b * v[e + 3]);
+                        for (int e = 0; e < 32; e += 4)
+                            *reinterpret_cast<float4*>(dst + e) =
+                                make_float4(b * v[e], b * v[e + 1], b * v[e + 2], b * v[e + 3]);
+                    }
                 }
             }
+            if (lane < 16) sDB[2 * m + hf] = part;
         }
         fence_async_smem();
         tc_fence_before();
-        __syncthreads();   // X3
+        __syncthreads();
         tc_fence_after();
 
         // ---- dS += (q*gamma)^T dO - (k*gamma)^T dR
         if (ctl) {
+            wait_bar(barC, phC);
             if (ok) {
                 bulk_store(rec_of(i) + bwdrec::DY, sm + OFF_DY, 16384);
                 bulk_commit_group();
                 constexpr uint32_t id128 = idesc_bf16(128, 128, true, true);
                 const uint32_t qt = smem_u32(sm + OFF_QT), kt = smem_u32(sm + OFF_KT);
-                const uint32_t d0 = smem_u32(sm + OFF_DO), r0 = smem_u32(sm + OFF_MDR);
+                const uint32_t d0 = smem_u32(dO_of(i)), r0 = smem_u32(sm + OFF_MDR);
 #pragma unroll
                 for (int ks = 0; ks < 4; ++ks)
                     mma_bf16(tmem + TM_DS, mnmaj(qt, 8192, ks), mnmaj(d0, 8192, ks), id128, 1);
@@ -387,7 +407,7 @@ kda_bwd_dstate_kernel(const __grid_constant__ CUtensorMap tmDO, const __nv_bfloa
                 commit();
             }
             wait_mma();
-            if (i > 0 && ok) issue_c(i - 1);   // q*gamma, k*gamma, dO, R, gamma_C are consumed
+            if (i > 0 && ok) issue_c(i - 1);   // q*gamma, k*gamma and R are consumed
         }
         if (compute) {
             if (tid < C && tid < Lc)
@@ -395,11 +415,15 @@ kda_bwd_dstate_kernel(const __grid_constant__ CUtensorMap tmDO, const __nv_bfloa
             wait_mma();
             // the new dS's bf16 copy for the next chunk's MMAs
             const int c = 32 * q4 + lane;
-            float v[64];
-            tmem_ld64(tmem + tlane + TM_DS + 64 * hf, v);
 #pragma unroll
-            for (int ch = 0; ch < 8; ++ch)
-                *reinterpret_cast<uint4*>(sm + OFF_DS + hf * 16384 + swz(c, ch)) = pack8(&v[8 * ch]);
+            for (int p = 0; p < 2; ++p) {
+                float v[32];
+                tmem_ld32(tmem + tlane + TM_DS + 64 * hf + 32 * p, v);
+#pragma unroll
+                for (int ch = 0; ch < 4; ++ch)
+                    *reinterpret_cast<uint4*>(sm + OFF_DS + hf * 16384 + swz(c, 4 * p + ch)) =
+                        pack8(&v[8 * ch]);
+            }
         }
         fence_async_smem();
         tc_fence_before();
@@ -428,18 +452,20 @@ kda_bwd_dstate_kernel(const __grid_constant__ CUtensorMap tmDO, const __nv_bfloa
     } else if (compute && dS0 && !broke) {
         const int c = 32 * q4 + lane;
         float* dst = dS0 + (((size_t)n * H + h) * DK + c) * DV + 64 * hf;
-        float v[64];
-        tmem_ld64(tmem + tlane + TM_DS + 64 * hf, v);
 #pragma unroll
-        for (int e = 0; e < 64; e += 4)
-            *reinterpret_cast<float4*>(dst + e) = make_float4(v[e], v[e + 1], v[e + 2], v[e + 3]);
+        for (int p = 0; p < 2; ++p) {
+            float v[32];
+            tmem_ld32(tmem + tlane + TM_DS + 64 * hf + 32 * p, v);
+#pragma unroll
+            for (int e = 0; e < 32; e += 4)
+                *reinterpret_cast<float4*>(dst + 32 * p + e) = make_float4(v[e], v[e + 1], v[e + 2], v[e + 3]);
+        }
     }
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
     if (warp == 0) tmem_dealloc(tmem, 512);
 }
-
 
 // ================================================================ chunk gradient pass
 //
@@ -697,41 +723,51 @@ kda_bwd_chunk_kernel(const __grid_constant__ CUtensorMap tmDO, const __grid_cons
         dbeta[(size_t)(row0 + tid) * H + h] += sDB[2 * tid] + sDB[2 * tid + 1];
     wait_mma();
 
-    // ---- per key channel c (TMEM lane c), tokens [32 hf, 32 hf + 32)
+    // ---- per key channel c (TMEM lane c), tokens [32 hf, 32 hf + 32).  Group 2 is done:
+    //      the stacked tile, S0 and G are free for fp32 tables [64 t][128 c].
     {
+        float* gT = reinterpret_cast<float*>(sm + OFF_STK);   // cumulative log-gates g_t
+        float* xT = reinterpret_cast<float*>(sm + OFF_S0);    // terms summed over r >= s
+        float* yT = reinterpret_cast<float*>(sm + OFF_G);     // terms summed over j < s
         const int c = 32 * q4 + lane;
         const int t0 = 32 * hf;
-        const int a_at = c >> 6;
-        const uint32_t cb = (uint32_t)(c & 7) * 2u, cc = (uint32_t)((c & 63) >> 3);
-        auto bf_at = [&](const uint8_t* tile, uint32_t atom, int row) {
-            return __bfloat162float(*reinterpret_cast<const __nv_bfloat16*>(
-                tile + (uint32_t)a_at * atom + swz((uint32_t)row, cc) + cb));
-        };
-        // cumulative log-gates of this channel: g_t = sum_{s <= t} log a_s (a = 1 past Lc)
-        float gown[32], g15 = 0.f, g47 = 0.f, g63 = 0.f;
+        // column c of row t in a tile of 128-byte swizzled rows: (t >> 3) * 1024 + roff[t & 7]
+        uint32_t roff[8];
+        {
+            const uint32_t cc = (uint32_t)((c & 63) >> 3), cb = (uint32_t)(c & 7) * 2u;
+#pragma unroll
+            for (int v = 0; v < 8; ++v) roff[v] = (uint32_t)v * 128u + (((cc ^ (uint32_t)v) & 7u) << 4) + cb;
+        }
+        const uint32_t at8 = (uint32_t)(c >> 6) * 8192u;    // 64-row tiles: alpha, q, k
+        const uint8_t* sAl = sm + OFF_AL + at8;
+        const uint8_t* sQ = sm + OFF_Q + at8;
+        const uint8_t* sK = sm + OFF_K + at8;
+        const uint8_t* sLt = sm + OFF_L + (uint32_t)(c >> 6) * 16384u;
+        const uint8_t* sRt = sm + OFF_R + (uint32_t)(c >> 6) * 12288u;
+        auto ld = [](const uint8_t* p) { return __bfloat162float(*reinterpret_cast<const __nv_bfloat16*>(p)); };
+        // g_t = sum_{s <= t} log a_s (a = 1 past the chunk's tokens), each thread up to its half's end
         {
             float g = 0.0f;
+            const int nb = 4 * (hf + 1);   // blocks of 8 tokens
+#pragma unroll 1
+            for (int u = 0; u < nb; ++u) {
 #pragma unroll
-            for (int t = 0; t < 32; ++t) {
-                const float a = t < Lc ? clamp_gate(bf_at(sm + OFF_AL, 8192, t)) : 1.0f;
-                g += __logf(a);
-                if (hf == 0) gown[t] = g;
-                if (t == 15) g15 = g;
+                for (int v = 0; v < 8; ++v) {
+                    const int t = 8 * u + v;
+                    const float a = t < Lc ? clamp_gate(ld(sAl + (uint32_t)u * 1024u + roff[v])) : 1.0f;
+                    g += __logf(a);
+                    if ((t >> 5) == hf) gT[t * 128 + c] = g;
+                }
             }
-#pragma unroll
-            for (int t = 32; t < C; ++t) {
-                const float a = t < Lc ? clamp_gate(bf_at(sm + OFF_AL, 8192, t)) : 1.0f;
-                g += __logf(a);
-                if (hf == 1) gown[t - 32] = g;
-                if (t == 47) g47 = g;
-            }
-            g63 = g;
         }
-        float X[32], Y[32];
+        __syncthreads();
+        const float g15 = gT[15 * 128 + c], g47 = gT[47 * 128 + c], g63 = gT[63 * 128 + c];
         const float dgc = sDGC[c] + sDGC[128 + c];
-#pragma unroll
+        float sx = 0.f, sy = 0.f;
+#pragma unroll 1
         for (int blk = 0; blk < 2; ++blk) {
-            const int tb = t0 + 16 * blk;   // first token of this block
+            const int tb = t0 + 16 * blk;   // first token of this block (a multiple of 16)
+            const uint32_t rb = (uint32_t)(tb >> 3) * 1024u;
             float mdkt[16], dqt[16], dl[16], dlq[16], drf[16], dkh[16];
             tmem_ld16(tmem + tlane + TM_ST + tb, mdkt);
             tmem_ld16(tmem + tlane + TM_ST + 64 + tb, dqt);
@@ -743,35 +779,41 @@ kda_bwd_chunk_kernel(const __grid_constant__ CUtensorMap tmDO, const __grid_cons
 #pragma unroll
             for (int i = 0; i < 16; ++i) {
                 const int t = tb + i;
-                const float gt = gown[16 * blk + i];
-                const float gref = t < 32 ? g15 : g47;
-                const float gam = __expf(gt), lam = __expf(gt - gref);
+                const uint32_t o = rb + (uint32_t)(i >> 3) * 1024u + roff[i & 7];
+                const float gt = gT[t * 128 + c];
+                const float gam = __expf(gt), lam = __expf(gt - (tb < 32 ? g15 : g47));
                 const float rho1 = __expf(g47 - gt), eta = __expf(g63 - gt);
                 const bool live = t < Lc;
-                const float kv = live ? bf_at(sm + OFF_K, 8192, t) : 0.0f;
-                const float qv = live ? bf_at(sm + OFF_Q, 8192, t) : 0.0f;
-                const float Lv = bf_at(sm + OFF_L, 16384, t), Lqv = bf_at(sm + OFF_L, 16384, 64 + t);
-                const float R1v = bf_at(sm + OFF_R, 12288, 32 + t);
+                const float kv = live ? ld(sK + o) : 0.0f;
+                const float qv = live ? ld(sQ + o) : 0.0f;
+                const float Lv = ld(sLt + o), Lqv = ld(sLt + 8192u + o);      // rows t, 64 + t
+                const float R1v = ld(sRt + 4096u + o);                         // row 32 + t
                 const float dkt = -mdkt[i];
                 const float dqv = gam * dqt[i] + lam * dlq[i];
-                float dkv = gam * dkt + eta * dkh[i] + lam * dl[i] + rho1 * drf[i];
-                float x = (kv * gam) * dkt + (qv * gam) * dqt[i] + Lv * dl[i] + Lqv * dlq[i] - R1v * drf[i];
-                Y[16 * blk + i] = (kv * eta) * dkh[i];
-                X[16 * blk + i] = x;
-                mdkt[i] = dkv;    // dk so far (rho^0 term below)
+                const float dkv = gam * dkt + eta * dkh[i] + lam * dl[i] + rho1 * drf[i];
+                const float x = (kv * gam) * dkt + (qv * gam) * dqt[i] + Lv * dl[i] + Lqv * dlq[i] -
+                                R1v * drf[i];
+                const float y = (kv * eta) * dkh[i];
+                xT[t * 128 + c] = x;
+                yT[t * 128 + c] = y;
+                sx += x;
+                sy += y;
+                mdkt[i] = dkv;   // dk so far (the rho^0 term below)
                 dqt[i] = dqv;
             }
-            if (tb < 32) {   // d(k*rho^0), rows t < 32
+            if (tb < 32) {   // d(k*rho^0), rows t < 32 (warp-uniform)
                 float dr0[16];
                 tmem_ld16(tmem + tlane + TM_RF + tb, dr0);
                 tmem_wait_ld();
 #pragma unroll
                 for (int i = 0; i < 16; ++i) {
                     const int t = tb + i;
-                    const float rho0 = __expf(g15 - gown[16 * blk + i]);
-                    const float R0v = bf_at(sm + OFF_R, 12288, t);
+                    const uint32_t o = rb + (uint32_t)(i >> 3) * 1024u + roff[i & 7];
+                    const float rho0 = __expf(g15 - gT[t * 128 + c]);
+                    const float x0 = ld(sRt + o) * dr0[i];
                     mdkt[i] += rho0 * dr0[i];
-                    X[16 * blk + i] -= R0v * dr0[i];
+                    xT[t * 128 + c] -= x0;
+                    sx -= x0;
                 }
             }
 #pragma unroll
@@ -784,28 +826,25 @@ kda_bwd_chunk_kernel(const __grid_constant__ CUtensorMap tmDO, const __grid_cons
                 }
             }
         }
-        // dlog a_s = sum_{r >= s} X_r + sum_{j < s} Y_j + dgc, across the two token halves
-        float sx = 0.f, sy = 0.f;
-#pragma unroll
-        for (int i = 0; i < 32; ++i) { sx += X[i]; sy += Y[i]; }
+        // dlog a_s = sum_{r >= s} x_r + sum_{j < s} y_j + dgc, across the two token halves
         sTot[(hf * 2 + 0) * 128 + c] = sx;
         sTot[(hf * 2 + 1) * 128 + c] = sy;
         __syncthreads();
-        float suf = hf == 0 ? sTot[(1 * 2 + 0) * 128 + c] : 0.0f;   // X of tokens 32..63
-        float pre = hf == 1 ? sTot[(0 * 2 + 1) * 128 + c] : 0.0f;   // Y of tokens 0..31
+        float suf = hf == 0 ? sTot[(1 * 2 + 0) * 128 + c] : 0.0f;        // x of tokens 32..63
+        float pre = (hf == 1 ? sTot[(0 * 2 + 1) * 128 + c] : 0.0f) + sy;  // y of tokens < t0 + 32
+#pragma unroll 1
+        for (int u = 3; u >= 0; --u) {
 #pragma unroll
-        for (int i = 0; i < 32; ++i) pre += Y[i];   // pre = Y of tokens < t0 + 32
-#pragma unroll
-        for (int i = 31; i >= 0; --i) {
-            const int t = t0 + i;
-            suf += X[i];
-            pre -= Y[i];   // Y of tokens < t
-            if (t < Lc) {
-                const float araw = bf_at(sm + OFF_AL, 8192, t);
-                const float a = clamp_gate(araw);
-                const bool pass = araw >= kAlphaMin && araw <= 1.0f;
-                const float dl = suf + pre + dgc;
-                dalpha[((size_t)(row0 + t) * H + h) * DK + c] = pass ? dl / a : 0.0f;
+            for (int v = 7; v >= 0; --v) {
+                const int t = t0 + 8 * u + v;
+                suf += xT[t * 128 + c];
+                pre -= yT[t * 128 + c];   // y of tokens < t
+                if (t < Lc) {
+                    const float araw = ld(sAl + (uint32_t)(t >> 3) * 1024u + roff[v]);
+                    const float a = clamp_gate(araw);
+                    const bool pass = araw >= kAlphaMin && araw <= 1.0f;
+                    dalpha[((size_t)(row0 + t) * H + h) * DK + c] = pass ? (suf + pre + dgc) / a : 0.0f;
+                }
             }
         }
     }
