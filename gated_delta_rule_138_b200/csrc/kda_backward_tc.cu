@@ -42,6 +42,11 @@
 #include "kda_sm100.cuh"
 #include "kda_tc_maps.cuh"
 
+// Optional phase-boundary hook of the chunk kernel for profiling builds (no-op in the library).
+#ifndef KDA_BWD_PHASE
+#define KDA_BWD_PHASE(i)
+#endif
+
 namespace kda {
 using namespace sm100;
 
@@ -135,8 +140,9 @@ kda_bwd_dstate_kernel(const __grid_constant__ CUtensorMap tmDO, const __nv_bfloa
                       int* status) {
     using namespace ds;
     extern __shared__ uint8_t smem_raw[];
-    uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
-                                             ~static_cast<uintptr_t>(1023));
+    // the 1024-aligned base as an offset into the shared array (the compiler keeps
+    // every access below a shared-memory one)
+    uint8_t* sm = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
     float* sGC = reinterpret_cast<float*>(sm + OFF_MISC + M_GC);
     float* sBeta = reinterpret_cast<float*>(sm + OFF_MISC + M_BETA);
     float* sDB = reinterpret_cast<float*>(sm + OFF_MISC + M_DB);
@@ -495,9 +501,9 @@ constexpr uint32_t M_BETA = 512;        // float [64]
 constexpr uint32_t M_DGC = 768;         // float [2][128] gamma_C * sum_n S0 dS, two halves
 constexpr uint32_t M_DB = 1792;         // float [64][2] dbeta's second part, two halves
 constexpr uint32_t M_TOT = 2304;        // float [2 halves][2 (X, Y)][128]
-constexpr uint32_t M_BAR = 4352;        // uint64 x2: loads, MMA
-constexpr uint32_t M_TMEM = 4368;
-constexpr uint32_t M_FLAG = 4372;
+constexpr uint32_t M_BAR = 4352;        // uint64 x3: loads A (group 1's operands), loads B, MMA
+constexpr uint32_t M_TMEM = 4376;
+constexpr uint32_t M_FLAG = 4380;
 constexpr uint32_t SMEM_BYTES = OFF_MISC + 4384 + 1024;
 constexpr uint32_t TM_G1 = 0, TM_AP = 64, TM_KH = 160, TM_ST = 224, TM_LF = 352, TM_RF = 0;
 }  // namespace ck
@@ -519,15 +525,17 @@ kda_bwd_chunk_kernel(const __grid_constant__ CUtensorMap tmDO, const __grid_cons
     const uint8_t* rp = rec + ((size_t)chunk * H + h) * bwdrec::BYTES;
 
     extern __shared__ uint8_t smem_raw[];
-    uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
-                                             ~static_cast<uintptr_t>(1023));
+    // the 1024-aligned base as an offset into the shared array (the compiler keeps
+    // every access below a shared-memory one)
+    uint8_t* sm = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
     float* sGC = reinterpret_cast<float*>(sm + OFF_MISC + M_GC);
     float* sBeta = reinterpret_cast<float*>(sm + OFF_MISC + M_BETA);
     float* sDGC = reinterpret_cast<float*>(sm + OFF_MISC + M_DGC);
     float* sDB = reinterpret_cast<float*>(sm + OFF_MISC + M_DB);
     float* sTot = reinterpret_cast<float*>(sm + OFF_MISC + M_TOT);
     uint64_t* barL = reinterpret_cast<uint64_t*>(sm + OFF_MISC + M_BAR);
-    uint64_t* barM = barL + 1;
+    uint64_t* barL2 = barL + 1;
+    uint64_t* barM = barL + 2;
     uint32_t* sTmem = reinterpret_cast<uint32_t*>(sm + OFF_MISC + M_TMEM);
     int* sFlag = reinterpret_cast<int*>(sm + OFF_MISC + M_FLAG);
 
@@ -537,6 +545,7 @@ kda_bwd_chunk_kernel(const __grid_constant__ CUtensorMap tmDO, const __grid_cons
 
     if (issuer) {
         mbar_init(barL, 1);
+        mbar_init(barL2, 1);
         mbar_init(barM, 1);
         mbar_fence_init();
         *sFlag = 0;
@@ -544,29 +553,32 @@ kda_bwd_chunk_kernel(const __grid_constant__ CUtensorMap tmDO, const __grid_cons
     if (warp == 0) tmem_alloc(sTmem, 512);
     tc_fence_before();
     __syncthreads();
+    KDA_BWD_PHASE(0);
     tc_fence_after();
     const uint32_t tmem = *sTmem;
     const uint32_t tlane = (uint32_t)(32 * q4) << 16;
 
     if (issuer) {
-        mbar_arrive_expect_tx(barL, 16384 + 16384 + 16384 + 32768 + 32768 + 32768 + 24576 + 512 +
-                                        3 * 16384);
-        // [dY ; dO]: dY's two 64-column atoms are rows 0..63 of the stacked atoms
-        bulk_load(sm + OFF_STK, rp + bwdrec::DY, 8192, barL);
+        // A: what group 1's first products read (dY, dO, U, dS); B: the rest
+        mbar_arrive_expect_tx(barL, 16384 + 16384 + 16384 + 32768);
+        bulk_load(sm + OFF_STK, rp + bwdrec::DY, 8192, barL);   // dY: rows 0..63 of both atoms
         bulk_load(sm + OFF_STK + 16384, rp + bwdrec::DY + 8192, 8192, barL);
 #pragma unroll
-        for (int a = 0; a < 2; ++a) {
+        for (int a = 0; a < 2; ++a)
             tma_load_2d(sm + OFF_STK + a * 16384 + 8192, &tmDO, barL, h * DV + 64 * a, (int)row0);
-            tma_load_2d(sm + OFF_AL + a * 8192, &tmA, barL, h * DK + 64 * a, (int)row0);
-            tma_load_2d(sm + OFF_Q + a * 8192, &tmQ, barL, h * DK + 64 * a, (int)row0);
-            tma_load_2d(sm + OFF_K + a * 8192, &tmK, barL, h * DK + 64 * a, (int)row0);
-        }
         bulk_load(sm + OFF_U, rp + bwdrec::U, 16384, barL);
-        bulk_load(sm + OFF_S0, rp + bwdrec::S, 32768, barL);
         bulk_load(sm + OFF_DS, rp + bwdrec::DS, 32768, barL);
-        bulk_load(sm + OFF_L, rp + bwdrec::L, 32768, barL);
-        bulk_load(sm + OFF_R, rp + bwdrec::R, 24576, barL);
-        bulk_load(sGC, rp + bwdrec::GC, 512, barL);
+        mbar_arrive_expect_tx(barL2, 32768 + 32768 + 24576 + 512 + 3 * 16384);
+        bulk_load(sm + OFF_S0, rp + bwdrec::S, 32768, barL2);
+        bulk_load(sm + OFF_L, rp + bwdrec::L, 32768, barL2);
+        bulk_load(sm + OFF_R, rp + bwdrec::R, 24576, barL2);
+        bulk_load(sGC, rp + bwdrec::GC, 512, barL2);
+#pragma unroll
+        for (int a = 0; a < 2; ++a) {
+            tma_load_2d(sm + OFF_AL + a * 8192, &tmA, barL2, h * DK + 64 * a, (int)row0);
+            tma_load_2d(sm + OFF_Q + a * 8192, &tmQ, barL2, h * DK + 64 * a, (int)row0);
+            tma_load_2d(sm + OFF_K + a * 8192, &tmK, barL2, h * DK + 64 * a, (int)row0);
+        }
     }
     float bval = 0.0f;
     if (tid < C && tid < Lc) bval = __bfloat162float(beta[(size_t)(row0 + tid) * H + h]);
@@ -584,22 +596,28 @@ kda_bwd_chunk_kernel(const __grid_constant__ CUtensorMap tmDO, const __grid_cons
         tc_fence_after();
     };
     if (!mbar_wait_ns(barL, phL, kWaitNs)) ok = false;
-    phL ^= 1u;
+    KDA_BWD_PHASE(1);
 
-    // ---- group 1
+    // ---- group 1: [dY ; dO] U^T and dS U^T on loads A, [A/beta ; P] once B has landed
     if (issuer && ok) {
         const uint32_t stk = smem_u32(sm + OFF_STK), u0 = smem_u32(sm + OFF_U);
-        const uint32_t l0 = smem_u32(sm + OFF_L), r0 = smem_u32(sm + OFF_R);
         const uint32_t ds0 = smem_u32(sm + OFF_DS);
 #pragma unroll
         for (int ks = 0; ks < 8; ++ks)
             mma_bf16(tmem + TM_G1, kmaj(stk, 16384, ks), kmaj(u0, 8192, ks), idesc_bf16(128, 64), ks > 0);
 #pragma unroll
         for (int ks = 0; ks < 8; ++ks)
-            mma_bf16(tmem + TM_AP, kmaj(l0, 16384, ks), kmaj(r0, 12288, ks), idesc_bf16(128, 96), ks > 0);
+            mma_bf16(tmem + TM_KH, kmaj(ds0, 16384, ks), kmaj(u0, 8192, ks), idesc_bf16(128, 64), ks > 0);
+    }
+    if (ok && !mbar_wait_ns(barL2, phL, kWaitNs)) ok = false;
+    phL ^= 1u;
+    if (issuer && ok) {
+        const uint32_t l0 = smem_u32(sm + OFF_L), r0 = smem_u32(sm + OFF_R);
 #pragma unroll
         for (int ks = 0; ks < 8; ++ks)
-            mma_bf16(tmem + TM_KH, kmaj(ds0, 16384, ks), kmaj(u0, 8192, ks), idesc_bf16(128, 64), ks > 0);
+            mma_bf16(tmem + TM_AP, kmaj(l0, 16384, ks), kmaj(r0, 12288, ks), idesc_bf16(128, 96), ks > 0);
+    }
+    if (issuer && ok) {   // one commit covers the group (MMAs of one thread complete in order)
         mma_commit(barM);
         mma_out = true;
         mma_out_ph = phM;
@@ -621,6 +639,7 @@ kda_bwd_chunk_kernel(const __grid_constant__ CUtensorMap tmDO, const __grid_cons
     }
     __syncthreads();   // dS is no longer read by the CUDA cores (G goes over it)
     wait_mma();
+    KDA_BWD_PHASE(2);
 
     // ---- G = [beta dA ; dP] in the column layout of [A/beta ; P]; dbeta's second part;
     //      [dY ; dO] -> [dR ; dO]
@@ -697,6 +716,7 @@ kda_bwd_chunk_kernel(const __grid_constant__ CUtensorMap tmDO, const __grid_cons
     fence_async_smem();
     tc_fence_before();
     __syncthreads();
+    KDA_BWD_PHASE(3);
     tc_fence_after();
 
     // ---- group 2
@@ -722,6 +742,7 @@ kda_bwd_chunk_kernel(const __grid_constant__ CUtensorMap tmDO, const __grid_cons
     if (tid < C && tid < Lc)
         dbeta[(size_t)(row0 + tid) * H + h] += sDB[2 * tid] + sDB[2 * tid + 1];
     wait_mma();
+    KDA_BWD_PHASE(4);
 
     // ---- per key channel c (TMEM lane c), tokens [32 hf, 32 hf + 32).  Group 2 is done:
     //      the stacked tile, S0 and G are free for fp32 tables [64 t][128 c].
@@ -745,105 +766,122 @@ kda_bwd_chunk_kernel(const __grid_constant__ CUtensorMap tmDO, const __grid_cons
         const uint8_t* sLt = sm + OFF_L + (uint32_t)(c >> 6) * 16384u;
         const uint8_t* sRt = sm + OFF_R + (uint32_t)(c >> 6) * 12288u;
         auto ld = [](const uint8_t* p) { return __bfloat162float(*reinterpret_cast<const __nv_bfloat16*>(p)); };
-        // g_t = sum_{s <= t} log a_s (a = 1 past the chunk's tokens), each thread up to its half's end
+        // g_t = sum_{s <= t} log a_s (a = 1 past the chunk's tokens): each half its own
+        // running sum; tokens 32..63 add the first half's total g_31 where they are read
         {
             float g = 0.0f;
-            const int nb = 4 * (hf + 1);   // blocks of 8 tokens
 #pragma unroll 1
-            for (int u = 0; u < nb; ++u) {
+            for (int u = 4 * hf; u < 4 * hf + 4; ++u) {
+                float lg[8];
 #pragma unroll
                 for (int v = 0; v < 8; ++v) {
                     const int t = 8 * u + v;
-                    const float a = t < Lc ? clamp_gate(ld(sAl + (uint32_t)u * 1024u + roff[v])) : 1.0f;
-                    g += __logf(a);
-                    if ((t >> 5) == hf) gT[t * 128 + c] = g;
+                    lg[v] = __logf(t < Lc ? clamp_gate(ld(sAl + (uint32_t)u * 1024u + roff[v])) : 1.0f);
+                }
+#pragma unroll
+                for (int v = 0; v < 8; ++v) {
+                    g += lg[v];
+                    gT[(8 * u + v) * 128 + c] = g;
                 }
             }
         }
         __syncthreads();
-        const float g15 = gT[15 * 128 + c], g47 = gT[47 * 128 + c], g63 = gT[63 * 128 + c];
+        KDA_BWD_PHASE(5);
+        const float g31 = gT[31 * 128 + c];
+        const float gadd = hf == 1 ? g31 : 0.0f;
+        const float g15 = gT[15 * 128 + c], g47 = gT[47 * 128 + c] + g31, g63 = gT[63 * 128 + c] + g31;
         const float dgc = sDGC[c] + sDGC[128 + c];
+        const size_t tstride = (size_t)H * DK;   // floats from one token's row to the next
+        float* dq_c = dq + ((size_t)(row0 + t0) * H + h) * DK + c;
+        float* dk_c = dk + ((size_t)(row0 + t0) * H + h) * DK + c;
         float sx = 0.f, sy = 0.f;
+        // per block of 8 tokens: every load first, then the arithmetic, then the stores
+        // (a table store followed by a load would otherwise order each token after the last)
 #pragma unroll 1
-        for (int blk = 0; blk < 2; ++blk) {
-            const int tb = t0 + 16 * blk;   // first token of this block (a multiple of 16)
+        for (int blk = 0; blk < 4; ++blk) {
+            const int tb = t0 + 8 * blk;   // first token of this block (a multiple of 8)
+            const bool sub0 = tb < 32;     // warp-uniform: sub-chunk 0 has the rho^0 operand
             const uint32_t rb = (uint32_t)(tb >> 3) * 1024u;
-            float mdkt[16], dqt[16], dl[16], dlq[16], drf[16], dkh[16];
-            tmem_ld16(tmem + tlane + TM_ST + tb, mdkt);
-            tmem_ld16(tmem + tlane + TM_ST + 64 + tb, dqt);
-            tmem_ld16(tmem + tlane + TM_LF + tb, dl);
-            tmem_ld16(tmem + tlane + TM_LF + 64 + tb, dlq);
-            tmem_ld16(tmem + tlane + TM_KH + tb, dkh);
-            tmem_ld16(tmem + tlane + TM_RF + 32 + tb, drf);   // d(k*rho^1), rows 32 + t
+            float mdkt[8], dqt[8], dl[8], dlq[8], drf[8], dkh[8], dr0[8];
+            tmem_ld8(tmem + tlane + TM_ST + tb, mdkt);
+            tmem_ld8(tmem + tlane + TM_ST + 64 + tb, dqt);
+            tmem_ld8(tmem + tlane + TM_LF + tb, dl);
+            tmem_ld8(tmem + tlane + TM_LF + 64 + tb, dlq);
+            tmem_ld8(tmem + tlane + TM_KH + tb, dkh);
+            tmem_ld8(tmem + tlane + TM_RF + 32 + tb, drf);   // d(k*rho^1), rows 32 + t
+            if (sub0) tmem_ld8(tmem + tlane + TM_RF + tb, dr0);   // d(k*rho^0), rows t < 32
+            float gt[8], kv[8], qv[8], Lv[8], Lqv[8], R1v[8], R0v[8];
+#pragma unroll
+            for (int i = 0; i < 8; ++i) {
+                const uint32_t o = rb + roff[i];
+                const bool live = tb + i < Lc;
+                gt[i] = gT[(tb + i) * 128 + c] + gadd;
+                kv[i] = live ? ld(sK + o) : 0.0f;
+                qv[i] = live ? ld(sQ + o) : 0.0f;
+                Lv[i] = ld(sLt + o);               // row t of [k*lam ; q*lam]
+                Lqv[i] = ld(sLt + 8192u + o);      // row 64 + t
+                R1v[i] = ld(sRt + 4096u + o);      // row 32 + t of [k*rho^0 ; k*rho^1]
+                R0v[i] = sub0 ? ld(sRt + o) : 0.0f;
+            }
             tmem_wait_ld();
+            if (!sub0) {
 #pragma unroll
-            for (int i = 0; i < 16; ++i) {
-                const int t = tb + i;
-                const uint32_t o = rb + (uint32_t)(i >> 3) * 1024u + roff[i & 7];
-                const float gt = gT[t * 128 + c];
-                const float gam = __expf(gt), lam = __expf(gt - (tb < 32 ? g15 : g47));
-                const float rho1 = __expf(g47 - gt), eta = __expf(g63 - gt);
-                const bool live = t < Lc;
-                const float kv = live ? ld(sK + o) : 0.0f;
-                const float qv = live ? ld(sQ + o) : 0.0f;
-                const float Lv = ld(sLt + o), Lqv = ld(sLt + 8192u + o);      // rows t, 64 + t
-                const float R1v = ld(sRt + 4096u + o);                         // row 32 + t
+                for (int i = 0; i < 8; ++i) dr0[i] = 0.0f;
+            }
+            const float gref = sub0 ? g15 : g47;
+            float x[8], y[8];
+#pragma unroll
+            for (int i = 0; i < 8; ++i) {
+                const float gam = __expf(gt[i]), lam = __expf(gt[i] - gref);
+                const float rho1 = __expf(g47 - gt[i]), eta = __expf(g63 - gt[i]);
+                const float rho0 = sub0 ? __expf(g15 - gt[i]) : 0.0f;
                 const float dkt = -mdkt[i];
-                const float dqv = gam * dqt[i] + lam * dlq[i];
-                const float dkv = gam * dkt + eta * dkh[i] + lam * dl[i] + rho1 * drf[i];
-                const float x = (kv * gam) * dkt + (qv * gam) * dqt[i] + Lv * dl[i] + Lqv * dlq[i] -
-                                R1v * drf[i];
-                const float y = (kv * eta) * dkh[i];
-                xT[t * 128 + c] = x;
-                yT[t * 128 + c] = y;
-                sx += x;
-                sy += y;
-                mdkt[i] = dkv;   // dk so far (the rho^0 term below)
-                dqt[i] = dqv;
-            }
-            if (tb < 32) {   // d(k*rho^0), rows t < 32 (warp-uniform)
-                float dr0[16];
-                tmem_ld16(tmem + tlane + TM_RF + tb, dr0);
-                tmem_wait_ld();
-#pragma unroll
-                for (int i = 0; i < 16; ++i) {
-                    const int t = tb + i;
-                    const uint32_t o = rb + (uint32_t)(i >> 3) * 1024u + roff[i & 7];
-                    const float rho0 = __expf(g15 - gT[t * 128 + c]);
-                    const float x0 = ld(sRt + o) * dr0[i];
-                    mdkt[i] += rho0 * dr0[i];
-                    xT[t * 128 + c] -= x0;
-                    sx -= x0;
-                }
+                x[i] = (kv[i] * gam) * dkt + (qv[i] * gam) * dqt[i] + Lv[i] * dl[i] + Lqv[i] * dlq[i] -
+                       R1v[i] * drf[i] - R0v[i] * dr0[i];
+                y[i] = (kv[i] * eta) * dkh[i];
+                dqt[i] = gam * dqt[i] + lam * dlq[i];
+                mdkt[i] = gam * dkt + eta * dkh[i] + lam * dl[i] + rho1 * drf[i] + rho0 * dr0[i];   // dk
             }
 #pragma unroll
-            for (int i = 0; i < 16; ++i) {
-                const int t = tb + i;
-                if (t < Lc) {
-                    const size_t o = ((size_t)(row0 + t) * H + h) * DK + c;
-                    dq[o] = dqt[i];
-                    dk[o] = mdkt[i];
+            for (int i = 0; i < 8; ++i) {
+                xT[(tb + i) * 128 + c] = x[i];
+                yT[(tb + i) * 128 + c] = y[i];
+                sx += x[i];
+                sy += y[i];
+                if (tb + i < Lc) {
+                    const size_t o = (size_t)(8 * blk + i) * tstride;
+                    dq_c[o] = dqt[i];
+                    dk_c[o] = mdkt[i];
                 }
             }
         }
+        KDA_BWD_PHASE(6);
         // dlog a_s = sum_{r >= s} x_r + sum_{j < s} y_j + dgc, across the two token halves
         sTot[(hf * 2 + 0) * 128 + c] = sx;
         sTot[(hf * 2 + 1) * 128 + c] = sy;
         __syncthreads();
         float suf = hf == 0 ? sTot[(1 * 2 + 0) * 128 + c] : 0.0f;        // x of tokens 32..63
         float pre = (hf == 1 ? sTot[(0 * 2 + 1) * 128 + c] : 0.0f) + sy;  // y of tokens < t0 + 32
+        float* da_c = dalpha + ((size_t)(row0 + t0) * H + h) * DK + c;
 #pragma unroll 1
         for (int u = 3; u >= 0; --u) {
+            float xs[8], ys[8], ar[8];
+#pragma unroll
+            for (int v = 0; v < 8; ++v) {
+                const int t = t0 + 8 * u + v;
+                xs[v] = xT[t * 128 + c];
+                ys[v] = yT[t * 128 + c];
+                ar[v] = ld(sAl + (uint32_t)(t >> 3) * 1024u + roff[v]);
+            }
 #pragma unroll
             for (int v = 7; v >= 0; --v) {
                 const int t = t0 + 8 * u + v;
-                suf += xT[t * 128 + c];
-                pre -= yT[t * 128 + c];   // y of tokens < t
+                suf += xs[v];
+                pre -= ys[v];   // y of tokens < t
                 if (t < Lc) {
-                    const float araw = ld(sAl + (uint32_t)(t >> 3) * 1024u + roff[v]);
-                    const float a = clamp_gate(araw);
-                    const bool pass = araw >= kAlphaMin && araw <= 1.0f;
-                    dalpha[((size_t)(row0 + t) * H + h) * DK + c] = pass ? (suf + pre + dgc) / a : 0.0f;
+                    const float a = clamp_gate(ar[v]);
+                    const bool pass = ar[v] >= kAlphaMin && ar[v] <= 1.0f;
+                    da_c[(size_t)(8 * u + v) * tstride] = pass ? (suf + pre + dgc) * __frcp_rn(a) : 0.0f;
                 }
             }
         }
@@ -851,8 +889,12 @@ kda_bwd_chunk_kernel(const __grid_constant__ CUtensorMap tmDO, const __grid_cons
 
     if (!ok) atomicExch(sFlag, 1);
     __syncthreads();
+    KDA_BWD_PHASE(7);
     if (*sFlag && issuer && mma_out) mbar_wait_ns(barM, mma_out_ph, kWaitNs);
-    if (*sFlag && issuer) mbar_wait_ns(barL, 0, kWaitNs);   // the one load phase
+    if (*sFlag && issuer) {   // the one phase of each load barrier
+        mbar_wait_ns(barL, 0, kWaitNs);
+        mbar_wait_ns(barL2, 0, kWaitNs);
+    }
     __syncthreads();
     if (*sFlag && tid == 0) atomicExch(status, 1);
     tc_fence_before();
