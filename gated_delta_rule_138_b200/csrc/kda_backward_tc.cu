@@ -790,6 +790,11 @@ kda_bwd_chunk_kernel(const __grid_constant__ CUtensorMap tmDO, const __grid_cons
         const float g31 = gT[31 * 128 + c];
         const float gadd = hf == 1 ? g31 : 0.0f;
         const float g15 = gT[15 * 128 + c], g47 = gT[47 * 128 + c] + g31, g63 = gT[63 * 128 + c] + g31;
+        // token t of sub-chunk I (reference ref_I): lam_t = e^{g_t - g_ref} is the one
+        // exponential; gamma_t = lam_t e^{g_ref}, rho^I_t = 1 / lam_t, eta_t = e^{g_63 - g_ref} / lam_t,
+        // and for t < 32 rho^1_t = e^{g_47 - g_15} rho^0_t (every factor within e^+-80)
+        const float gref_me = hf == 0 ? g15 : g47;   // (the half is the sub-chunk)
+        const float Gref = __expf(gref_me), Eref = __expf(g63 - gref_me), P10 = __expf(g47 - g15);
         const float dgc = sDGC[c] + sDGC[128 + c];
         const size_t tstride = (size_t)H * DK;   // floats from one token's row to the next
         float* dq_c = dq + ((size_t)(row0 + t0) * H + h) * DK + c;
@@ -828,13 +833,13 @@ kda_bwd_chunk_kernel(const __grid_constant__ CUtensorMap tmDO, const __grid_cons
 #pragma unroll
                 for (int i = 0; i < 8; ++i) dr0[i] = 0.0f;
             }
-            const float gref = sub0 ? g15 : g47;
             float x[8], y[8];
 #pragma unroll
             for (int i = 0; i < 8; ++i) {
-                const float gam = __expf(gt[i]), lam = __expf(gt[i] - gref);
-                const float rho1 = __expf(g47 - gt[i]), eta = __expf(g63 - gt[i]);
-                const float rho0 = sub0 ? __expf(g15 - gt[i]) : 0.0f;
+                const float lam = __expf(gt[i] - gref_me), rl = __fdividef(1.0f, lam);
+                const float gam = lam * Gref, eta = Eref * rl;
+                const float rho0 = sub0 ? rl : 0.0f;
+                const float rho1 = sub0 ? P10 * rl : rl;
                 const float dkt = -mdkt[i];
                 x[i] = (kv[i] * gam) * dkt + (qv[i] * gam) * dqt[i] + Lv[i] * dl[i] + Lqv[i] * dlq[i] -
                        R1v[i] * drf[i] - R0v[i] * dr0[i];
@@ -881,7 +886,7 @@ kda_bwd_chunk_kernel(const __grid_constant__ CUtensorMap tmDO, const __grid_cons
                 if (t < Lc) {
                     const float a = clamp_gate(ar[v]);
                     const bool pass = ar[v] >= kAlphaMin && ar[v] <= 1.0f;
-                    da_c[(size_t)(8 * u + v) * tstride] = pass ? (suf + pre + dgc) * __frcp_rn(a) : 0.0f;
+                    da_c[(size_t)(8 * u + v) * tstride] = pass ? __fdividef(suf + pre + dgc, a) : 0.0f;
                 }
             }
         }
