@@ -1080,18 +1080,14 @@ kda_chunk_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_consta
         if (ctl) {
             KDA_TC_PHASE(20);
             if (ok) {
-                if constexpr (kRecord) {   // start state and operand tiles to the record
+                if constexpr (kRecord) {   // the tiles the extraction overwrites go first
                     uint8_t* rp = rec_of(chunk);
                     if (h == 0) {
                         const int64_t rem = len - (int64_t)chunk * C;
                         seg.hdr[s_cbase + chunk] = bwdrec::Header{row0, (int32_t)(rem < C ? rem : C), 0};
                     }
-                    bulk_store(rp + bwdrec::S, sS, 32768);
                     bulk_store(rp + bwdrec::L, sX + X_L, 32768);
                     bulk_store(rp + bwdrec::R, sX + X_R, 24576);
-                    bulk_store(rp + bwdrec::QT, sQc, 16384);
-                    bulk_store(rp + bwdrec::KT, sKT, 16384);
-                    bulk_store(rp + bwdrec::KH, sKH, 16384);
                     bulk_commit_group();
                 }
                 mma_ap();
@@ -1124,8 +1120,13 @@ kda_chunk_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_consta
         }
         handoff();   // B
         if (ctl) {
-            if (kRecord && ok) {   // P (its read is waited for before the next commit)
-                bulk_store(rec_of(chunk) + bwdrec::P, sX + X_P, 8192);
+            if (kRecord && ok) {   // tiles that stay valid until the next chunk's gate phase
+                uint8_t* rp = rec_of(chunk);   // (their reads are waited for before later commits)
+                bulk_store(rp + bwdrec::P, sX + X_P, 8192);
+                bulk_store(rp + bwdrec::S, sS, 32768);
+                bulk_store(rp + bwdrec::QT, sQc, 16384);
+                bulk_store(rp + bwdrec::KT, sKT, 16384);
+                bulk_store(rp + bwdrec::KH, sKH, 16384);
                 bulk_commit_group();
             }
             if (ok) {

@@ -43,15 +43,19 @@ def _clamp(alpha):
     return a, mask
 
 
-def chunk_backward_one(q, k, v, alpha, beta, S0, dout, dSf, C, rnd=None, rnd_decay=None):
+def chunk_backward_one(q, k, v, alpha, beta, S0, dout, dSf, C, rnd=None, rnd_decay=None,
+                       rnd_elem=None):
     """One (sequence, head): q, k, alpha [T, dk]; v, dout [T, dv]; beta [T];
     S0, dSf [dk, dv].  Returns dq, dk, dv, dalpha, dbeta, dS0 (fp64).
 
     rnd / rnd_decay (default: none) round the operands of every matrix product, as a
     tensor-core kernel would stage them; rnd_decay applies to the products that feed
-    the decay gradient (dQt, dKt, dZ, dKh), rnd to all others."""
+    the decay gradient (dQt, dKt, dZ, dKh), rnd to all others.  rnd_elem (default:
+    none) rounds the operands Kt, Z, Qt, Kh where the decay gradient multiplies them
+    element-wise by their gradients."""
     r = rnd or (lambda x: x)
     r2 = rnd_decay or r
+    re_ = rnd_elem or (lambda x: x)
     T, dk = q.shape
     dv = v.shape[1]
     a_all, mask = _clamp(alpha)
@@ -121,8 +125,8 @@ def chunk_backward_one(q, k, v, alpha, beta, S0, dout, dSf, C, rnd=None, rnd_dec
         gam, gC = c["gam"], c["gC"]
         dK = dKt * gam + dZ / gam + dKh * (gC / gam)
         dQ = dQt * gam
-        dg = dKt * c["Kt"] - dZ * c["Z"] + dQt * c["Qt"] - dKh * c["Kh"]
-        dg[-1] += (dKh * c["Kh"]).sum(0) + dgC
+        dg = dKt * re_(c["Kt"]) - dZ * re_(c["Z"]) + dQt * re_(c["Qt"]) - dKh * re_(c["Kh"])
+        dg[-1] += (dKh * re_(c["Kh"])).sum(0) + dgC
         dloga = np.cumsum(dg[::-1], axis=0)[::-1]
         L, t0 = c["L"], c["t0"]
         dq[t0:t0 + L], dkk[t0:t0 + L], dvv[t0:t0 + L] = dQ[:L], dK[:L], dV[:L]
@@ -239,10 +243,12 @@ def _tf32(x):
 
 def test_operand_precision_budget():
     """Which operand precision a tensor-core form of this backward needs.  With every
-    product staged in bf16, dq, dk, dv, dbeta and dS0 stay near 3e-3 of the oracle but
-    dalpha does not: the decay gradient sums operand * operand-gradient products that
-    largely cancel.  Staging the products that feed it (dQt, dKt, dZ, dKh) in tf32
-    keeps every gradient inside the bf16 bar of 2e-2."""
+    product staged in bf16 and the element-wise decay terms taken against unrounded
+    operands, dq, dk, dv, dbeta and dS0 stay near 3e-3 of the oracle but dalpha does
+    not: the decay gradient sums operand * operand-gradient products that largely
+    cancel.  Staging the products that feed it (dQt, dKt, dZ, dKh) in tf32 keeps every
+    gradient inside the bf16 bar of 2e-2; so does rounding the element-wise operands
+    the way the MMA operands are rounded, with every product in bf16."""
     rng = np.random.default_rng(0)
     T, dk, dv = 256, 128, 128
     n = lambda *s: rng.standard_normal(s)
@@ -259,11 +265,17 @@ def test_operand_precision_budget():
                           dSf[None, None])
     ref = [r[0, :, 0] for r in ref[:5]] + [ref[5][0, 0]]
 
-    def errs(rnd, rnd_decay):
-        got = chunk_backward_one(q, k, v, al, be, S0, do, dSf, 64, rnd, rnd_decay)
+    def errs(rnd, rnd_decay, rnd_elem=None):
+        got = chunk_backward_one(q, k, v, al, be, S0, do, dSf, 64, rnd, rnd_decay, rnd_elem)
         return [_rel(g_, r) for g_, r in zip(got, ref)]
     all_bf16 = errs(_bf16, _bf16)
     mixed = errs(_bf16, _tf32)
     assert max(all_bf16[i] for i in (0, 1, 2, 4, 5)) < 1e-2
     assert max(mixed) < 2e-2, mixed
     assert all_bf16[3] > 3 * mixed[3], (all_bf16[3], mixed[3])   # dalpha: the sensitive one
+    # ... unless the element-wise products take the same bf16 operand values the MMAs
+    # read: each (r, j) pair's two ends then cancel exactly, and all-bf16 products keep
+    # every gradient, dalpha included, inside the bar (the tensor-core backward's choice)
+    consistent = errs(_bf16, _bf16, _bf16)
+    assert max(consistent) < 1e-2, consistent
+    assert consistent[3] < all_bf16[3] / 3, (consistent[3], all_bf16[3])
