@@ -535,10 +535,12 @@ kda_chunk_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_consta
                     ag[c] = aft * gO;
                 }
             }
-            // fused inputs: k and q rows L2-normalised in place (bf16), before any
-            // operand is formed.  A warp holds all 128 channels of its eight rows, four
-            // per lane, and each thread rewrites only the elements it reads again below.
+            // fused inputs: the L2 norms of this warp's eight k (and q) rows (a warp holds all
+            // 128 channels of its rows, four per lane); the operand loop below scales the rows
+            // as it reads them, so nothing is written back
+            float kinv[8], qinv[8];
             if constexpr (kFused) {
+                float sk[8], sq[8];
 #pragma unroll
                 for (int i = 0; i < 8; ++i) {
                     const int r = 8 * O + i;
@@ -546,18 +548,21 @@ kda_chunk_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_consta
                     float k[4], q[4] = {0.f, 0.f, 0.f, 0.f};
                     unpack4_bf16(*reinterpret_cast<const uint2*>(sK + in_off), k);
                     if (!kSummary) unpack4_bf16(*reinterpret_cast<const uint2*>(sQc + in_off), q);
-                    float sk = k[0] * k[0] + k[1] * k[1] + k[2] * k[2] + k[3] * k[3];
-                    float sq = q[0] * q[0] + q[1] * q[1] + q[2] * q[2] + q[3] * q[3];
+                    sk[i] = k[0] * k[0] + k[1] * k[1] + k[2] * k[2] + k[3] * k[3];
+                    sq[i] = q[0] * q[0] + q[1] * q[1] + q[2] * q[2] + q[3] * q[3];
+                }
 #pragma unroll
-                    for (int o = 16; o > 0; o >>= 1) {
-                        sk += __shfl_xor_sync(0xffffffffu, sk, o);
-                        sq += __shfl_xor_sync(0xffffffffu, sq, o);
+                for (int o = 16; o > 0; o >>= 1) {
+#pragma unroll
+                    for (int i = 0; i < 8; ++i) {
+                        sk[i] += __shfl_xor_sync(0xffffffffu, sk[i], o);
+                        if (!kSummary) sq[i] += __shfl_xor_sync(0xffffffffu, sq[i], o);
                     }
-                    const float ik = rsqrtf(fmaxf(sk, 1e-12f)), iq = rsqrtf(fmaxf(sq, 1e-12f));
+                }
 #pragma unroll
-                    for (int c = 0; c < 4; ++c) { k[c] *= ik; q[c] *= iq; }
-                    st4_bf16(sK + in_off, k);
-                    if (!kSummary) st4_bf16(sQc + in_off, q);
+                for (int i = 0; i < 8; ++i) {
+                    kinv[i] = rsqrtf(fmaxf(sk[i], 1e-12f));
+                    qinv[i] = rsqrtf(fmaxf(sq[i], 1e-12f));
                 }
             }
             // each row's k (and q) is read before the previous row's stores: q*gamma is
@@ -575,6 +580,10 @@ kda_chunk_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_consta
                 float k[4], q[4] = {0.f, 0.f, 0.f, 0.f};
                 unpack4_bf16(kn, k);
                 if (!kSummary) unpack4_bf16(qn, q);
+                if constexpr (kFused) {
+#pragma unroll
+                    for (int c = 0; c < 4; ++c) { k[c] *= kinv[i]; q[c] *= qinv[i]; }
+                }
                 if (i < 7) {
                     kn = *reinterpret_cast<const uint2*>(sK + in_off_of(r + 1));
                     if (!kSummary) qn = *reinterpret_cast<const uint2*>(sQc + in_off_of(r + 1));

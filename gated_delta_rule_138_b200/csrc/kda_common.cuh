@@ -21,9 +21,10 @@ __device__ __forceinline__ float clamp_gate(float a) {
 
 // Input-side transforms of the fused entry points (plain definitions):
 //   alpha = exp(-softplus(x)) = 1 / (1 + e^x),   beta = sigmoid(x) = 1 / (1 + e^-x).
-// exp overflows to +inf for large x and the reciprocal then gives 0, the limit.
-__device__ __forceinline__ float gate_from_logit(float x) { return __frcp_rn(1.0f + __expf(x)); }
-__device__ __forceinline__ float sigmoid_f(float x) { return __frcp_rn(1.0f + __expf(-x)); }
+// exp overflows to +inf for large x and the (fast, approximate) reciprocal then gives 0,
+// the limit.
+__device__ __forceinline__ float gate_from_logit(float x) { return __fdividef(1.0f, 1.0f + __expf(x)); }
+__device__ __forceinline__ float sigmoid_f(float x) { return __fdividef(1.0f, 1.0f + __expf(-x)); }
 
 template <typename T> __device__ __forceinline__ float to_f32(T x);
 template <> __device__ __forceinline__ float to_f32<float>(float x) { return x; }
