@@ -368,14 +368,27 @@ kda_status_t kda_noalloc_selftest_timeout(uint64_t limit_ns, int32_t word, kda_s
  *     wanted).  None of them may alias an input.
  *   workspace: NULL, or device memory of at least kda_backward_workspace_bytes
  *     (16-byte aligned, caller-owned, contents not preserved).  NULL: the call
- *     allocates it stream-ordered (cudaMallocAsync) and frees it after the
- *     kernel, on `stream`.
+ *     allocates what its kernels need stream-ordered (cudaMallocAsync) and
+ *     frees it after them, on `stream`.
  *   Supported: d_k, d_v in {64, 128}; in_dtype KDA_F32 or KDA_BF16; S0,
  *     dS_final, dS0 and workspace 16-byte aligned.
- *   The kernel keeps the state and its gradient in registers, one CTA per
- *   (sequence, head), and recomputes states from checkpoints taken every 8
- *   tokens: cost grows with the longest sequence, and the workspace holds
- *   ceil(T / 8) + 8 states of d_k x d_v fp32 per (sequence, head).
+ *   Two implementations, chosen by the arguments:
+ *   - in_dtype KDA_BF16 with d_k = d_v = 128 (and at most 65535 sequences):
+ *     the chunk-parallel form on the tensor cores (bf16 MMA operands, fp32
+ *     accumulation; errors of a few 1e-3 relative to an exact backward).  Three
+ *     kernels: the forward recurrence writes, per chunk of 64 tokens and head, a
+ *     record of its start state and operand tiles (about 233 KB); a reverse pass
+ *     per (sequence, head) carries dS_final back to dS0 and writes dv and part
+ *     of dbeta; a pass over all (chunk, head) pairs in parallel writes dq, dk,
+ *     dalpha and the rest of dbeta.  Workspace: the records, about 3.6 KB per
+ *     (token, head).  A bounded device wait that gives up sets the device status
+ *     word (kda_device_status).
+ *   - otherwise: the token-sequential reverse mode in fp32 (one CTA per
+ *     (sequence, head), state and gradient in registers, states recomputed from
+ *     checkpoints every 8 tokens; the workspace holds ceil(T / 8) + 8 states of
+ *     d_k x d_v fp32 per (sequence, head)).
+ *   Tokens of a packed batch outside [cu_seqlens[0], cu_seqlens[num_seqs]) are
+ *   not written.
  *
  *   Returns KDA_OK; KDA_ERR_INVALID_ARG (missing or misaligned pointer, bad
  *   size, workspace too small); KDA_ERR_UNSUPPORTED (head dims, more than
@@ -390,7 +403,9 @@ kda_status_t kda_backward(const void* q, const void* k, const void* v, const voi
                           kda_dtype_t in_dtype, void* workspace, size_t workspace_bytes,
                           kda_stream_t stream);
 /* Workspace bytes kda_backward needs for these sizes (cu_seqlens given: packed
- * = 1, num_seqs sequences in T packed tokens; else B sequences of T tokens). */
+ * = 1, num_seqs sequences in T packed tokens; else B sequences of T tokens).  The
+ * dtype is not an argument: for d_k = d_v = 128 the value covers both
+ * implementations (the larger of the two). */
 size_t kda_backward_workspace_bytes(int32_t B, int64_t T, int32_t H, int32_t d_k, int32_t d_v,
                                     int32_t packed, int32_t num_seqs);
 
