@@ -56,7 +56,9 @@ kda_decode_kernel(const Tin* __restrict__ q, const Tin* __restrict__ k,
     constexpr int NS = kMulti ? kStageTokens : 1;
     __shared__ __align__(16) Tin tin[NS * (3 * DK + DV)];
     __shared__ Tin tbeta[NS];
-    __shared__ float bga[NS][DK], bka[NS][DK], bqa[NS][DK], bkk[NS][DK], bkq[NS];
+    // (a*k, a*q, a, k) of key channel c in one 16-byte element: one load per row and pass
+    __shared__ __align__(16) float4 bcf[NS][DK];
+    __shared__ float bkq[NS];
 
     const int tid = threadIdx.x, tx = tid % TX, ty = tid / TX;
     const size_t nh = blockIdx.x;                 // (sequence, head) flattened
@@ -134,10 +136,7 @@ kda_decode_kernel(const Tin* __restrict__ q, const Tin* __restrict__ k,
                 const float ax = to_f32(ra[c]);
                 const float a = clamp_gate(fused ? gate_from_logit(ax) : ax);
                 const float kc = kv[j] * ikn, qc = qv[j] * iqn;
-                bga[tt][c] = a;
-                bka[tt][c] = a * kc;
-                bqa[tt][c] = a * qc;
-                bkk[tt][c] = kc;
+                bcf[tt][c] = make_float4(a * kc, a * qc, a, kc);
                 kqp = fmaf(kc, qc, kqp);
             }
 #pragma unroll
@@ -150,10 +149,6 @@ kda_decode_kernel(const Tin* __restrict__ q, const Tin* __restrict__ k,
     const Tin* sk = direct ? k + tok * DK : nullptr;
     const Tin* sa = direct ? alpha + tok * DK : nullptr;
     const Tin* sv = direct ? v + vb : tin + 3 * NS * DK + ts * DV;
-    const float* pka = ka;   // this token's a*k, a*q, a and k
-    const float* pqa = qa;
-    const float* pga = ga;
-    const float* pkk = kk;
     if constexpr (direct) {
         // fused inputs: alpha and beta are logits, q and k are L2-normalised here
         float ikn = 1.0f, iqn = 1.0f;
@@ -192,18 +187,21 @@ kda_decode_kernel(const Tin* __restrict__ q, const Tin* __restrict__ k,
         for (int o = 16; o > 0; o >>= 1) kqp += __shfl_xor_sync(0xffffffffu, kqp, o);
         if ((tid & 31) == 0) kq_part[tid >> 5] = kqp;
         __syncthreads();
-    } else {
-        pka = bka[ts];
-        pqa = bqa[ts];
-        pga = bga[ts];
-        pkk = bkk[ts];
     }
 
     float4 px = make_float4(0.f, 0.f, 0.f, 0.f), py = px;
 #pragma unroll
     for (int i = 0; i < RPT; ++i) {
         const int c = ty + TY * i;
-        const float wk = pka[c], wq = pqa[c];
+        float wk, wq;
+        if constexpr (direct) {
+            wk = ka[c];
+            wq = qa[c];
+        } else {
+            const float4 cf = bcf[ts][c];
+            wk = cf.x;
+            wq = cf.y;
+        }
         px.x = fmaf(s[i].x, wk, px.x); px.y = fmaf(s[i].y, wk, px.y);
         px.z = fmaf(s[i].z, wk, px.z); px.w = fmaf(s[i].w, wk, px.w);
         py.x = fmaf(s[i].x, wq, py.x); py.y = fmaf(s[i].y, wq, py.y);
@@ -236,8 +234,15 @@ kda_decode_kernel(const Tin* __restrict__ q, const Tin* __restrict__ k,
 #pragma unroll
     for (int i = 0; i < RPT; ++i) {
         const int c = ty + TY * i;
-        const float a = pga[c];
-        const float kc = pkk[c];
+        float a, kc;
+        if constexpr (direct) {
+            a = ga[c];
+            kc = kk[c];
+        } else {
+            const float4 cf = bcf[ts][c];
+            a = cf.z;
+            kc = cf.w;
+        }
         float4 r;
         r.x = fmaf(a, s[i].x, kc * u4.x);
         r.y = fmaf(a, s[i].y, kc * u4.y);
