@@ -18,6 +18,7 @@
 // learns of a timeout by reading the words back with kda_noalloc_status, which
 // allocates nothing either (a copy into caller-provided or stack host memory).
 #include <cstdio>
+#include <cstdlib>
 #include <mutex>
 
 #include "kda_sm100.cuh"
@@ -115,7 +116,12 @@ extern "C" kda_status_t kda_forward_noalloc(const void* q, const void* k, const 
     e = kda::launch_chunk_tc_cta_status(q, k, v, alpha, beta, S0, cu_seqlens, (int)nseq, out,
                                         S_final, rows, T, H, status,
                                         reinterpret_cast<cudaStream_t>(stream));
-    return e == cudaSuccess ? KDA_OK : fail_cuda(e);
+    if (e != cudaSuccess) return fail_cuda(e);
+    // KDA_DEBUG set: wait for the call and report its status words, as kda_forward does
+    // with its device status word
+    const char* dbg = std::getenv("KDA_DEBUG");
+    if (dbg && dbg[0] && dbg[0] != '0') return kda_noalloc_status((int32_t)(nseq * H), nullptr, stream);
+    return KDA_OK;
 }
 
 namespace {

@@ -312,6 +312,8 @@ kda_status_t kda_selftest_timeout(uint64_t limit_ns, kda_stream_t stream);
  *   returns KDA_OK once the kernel is launched: read the words back with
  *   kda_noalloc_status to learn of a timeout.  Calls whose kernels overlap on
  *   the GPU race on the array.
+ *   With the environment variable KDA_DEBUG set (not "0"), the call waits for
+ *   its kernel and returns what kda_noalloc_status reports for its words.
  *   The first call on a device looks up the array's device address
  *   (cudaGetSymbolAddress) with that device current and keeps it for the
  *   life of the process; make that first call before any stream capture, and
