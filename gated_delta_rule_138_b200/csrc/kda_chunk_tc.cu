@@ -638,19 +638,20 @@ kda_chunk_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_consta
         // ================= [A/beta ; P] = [k*lam ; q*lam] [k*rho^0 ; k*rho^1]^T   (M=128, N=96, K=128)
         //   rows 0..63 are A/beta rows r, rows 64..127 are P rows r.  Columns [0, 32) hold
         //   rho^0 (j < 32, valid for r < 32), columns [32, 96) hold rho^1 (j < 64, valid for r >= 32).
-        // meanwhile (forward mode): S <- Diag(gamma_C) S in TMEM -- the MMAs read the bf16
-        // copy, and only the state update, two hand-offs later, accumulates onto S
-        if constexpr (!kSummary) {
+        // meanwhile: S (summary: [M | N]) <- Diag(gamma_C) S in TMEM -- the MMAs read the
+        // bf16 copy, and only the state update, hand-offs later, accumulates onto S
+        {
             const int c = 32 * q4 + lane;
             const float g = sGC[c];
+            constexpr int ncol = kSummary ? 128 : 64;   // this thread's columns
 #pragma unroll
-            for (int blk = 0; blk < 4; ++blk) {
+            for (int blk = 0; blk < ncol / 16; ++blk) {
                 float w[16];
-                tmem_ld16(tmem + tlane + TM_S + 64 * hf + 16 * blk, w);
+                tmem_ld16(tmem + tlane + TM_S + ncol * hf + 16 * blk, w);
                 tmem_wait_ld();
 #pragma unroll
                 for (int i = 0; i < 16; ++i) w[i] *= g;
-                tmem_st16(tmem + tlane + TM_S + 64 * hf + 16 * blk, w);
+                tmem_st16(tmem + tlane + TM_S + ncol * hf + 16 * blk, w);
             }
             tmem_wait_st();
         }
@@ -903,23 +904,7 @@ kda_chunk_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_consta
         KDA_TC_PHASE(5);
         if constexpr (kSummary) {
         // ================= [U_M | U_N] = -W [M | N] + [0 | Tb V]   (M=64, N=256, K=128 (+64))
-        // meanwhile: [M | N] <- Diag(gamma_C) [M | N] in TMEM
-        {
-            const int c = 32 * q4 + lane;
-            const float g = sGC[c];
-#pragma unroll
-            for (int p = 0; p < 2; ++p) {
-                const uint32_t ta = tmem + tlane + TM_S + 128 * hf + 64 * p;
-                float v[64];
-                tmem_ld64(ta, v);
-#pragma unroll
-                for (int i = 0; i < 64; ++i) v[i] *= g;
-#pragma unroll
-                for (int blk = 0; blk < 4; ++blk)
-                    tmem_st16(ta + 16 * blk, *reinterpret_cast<float(*)[16]>(&v[16 * blk]));
-            }
-            tmem_wait_st();
-        }
+        // (the decay of [M | N] was applied beside the [A/beta ; P] product)
         wait_mma();
         if (tid < C) {
             const int64_t nxt = (int64_t)(chunk + 1) * C + tid;   // token index in the segment
