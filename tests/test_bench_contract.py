@@ -147,3 +147,13 @@ def test_reference_arm_other_ranks_do_no_work():
     r = _run_reference({"RANK": "1", "WORLD_SIZE": "2"})
     assert r.returncode == 0, r.stderr[-2000:]
     assert not [ln for ln in r.stdout.splitlines() if ln.startswith("{")]
+
+
+def test_batch_override_is_for_dense_forward_workloads_only():
+    """--batch (a smaller batch of the same kernels, for profiler captures) is refused
+    before any GPU work on workloads that are not dense forwards."""
+    r = subprocess.run([sys.executable, os.path.join(ROOT, "bench.py"), "--workload",
+                        "decode_N256_H32_d128", "--batch", "2"], capture_output=True, text=True,
+                       timeout=120)
+    assert r.returncode == 2
+    assert "--batch applies to the dense forward workloads" in r.stderr
