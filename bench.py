@@ -6,8 +6,10 @@
 One step = one kda_forward call (the whole chunk-parallel forward) over one
 batch of seeded synthetic inputs already resident in HBM.  The default workload
 is the long-context one (B=1, H=32, T=2^20, d=128): few (sequence, head) pairs,
-so the forward splits every sequence into time segments (segment maps, scan,
-forward: three launches per step, timed together).
+so the forward splits every sequence into time segments (one pass over every
+segment giving its state map, its zero-start outputs and map rows; the scan of
+the start states; the start states' share of the outputs: three launches per
+step, timed together).
 For N > 1 (launched with torch.distributed.run, one process per GPU) every
 rank runs its own batch (independent sequences, no data-path collective:
 weak scaling); the time is the max over ranks and `value` counts all ranks'
@@ -595,7 +597,7 @@ def run_ours(args, w):
             kname = ("backward_tc_bf16" if (w.dtype == "bf16" and w.dk == 128 and w.dv == 128)
                      else "backward_f32")
         # time segments per sequence of the tensor-core path (1: unsplit); with g > 1 a
-        # step is three launches (segment maps, scan, forward) timed together
+        # step is three launches (dual pass, scan, o += Qg S_g) timed together
         segments = (kda.kda_forward_segments(nseq, -(-B * T // nseq), w.H)
                     if kname.startswith("chunk_tc_bf16") else 1)
         algo_bytes = forward_bytes(w, n_th, n_sh, inp["S0"] is not None)

@@ -9,7 +9,7 @@ call does, and it raises if the library is missing.
 from .kda import (KdaError, kda_forward, kda_decode_step, kda_status_string,  # noqa: F401
                   kda_forward_workspace_bytes, kda_forward_kernel_name, kda_launch_count,
                   kda_device_status, kda_forward_noalloc, kda_selftest_timeout,
-                  kda_noalloc_status, kda_noalloc_selftest_timeout, kda_forward_segments, kda_segment_maps, kda_segment_scan,
+                  kda_noalloc_status, kda_noalloc_selftest_timeout, kda_forward_segments, kda_release_workspace, kda_segment_maps, kda_segment_scan,
                   kda_forward_indexed, kda_decode_step_indexed, kda_forward_fused,
                   kda_decode_step_fused, kda_backward, kda_backward_workspace_bytes,
                   library_path, load_library)
@@ -18,7 +18,7 @@ __all__ = ["KdaError", "kda_forward", "kda_decode_step", "kda_status_string",
            "kda_forward_workspace_bytes", "kda_forward_kernel_name", "kda_launch_count",
            "kda_device_status", "kda_forward_noalloc", "kda_selftest_timeout",
            "kda_noalloc_status", "kda_noalloc_selftest_timeout",
-           "kda_forward_segments", "kda_segment_maps", "kda_segment_scan",
+           "kda_forward_segments", "kda_release_workspace", "kda_segment_maps", "kda_segment_scan",
            "kda_forward_indexed", "kda_decode_step_indexed", "kda_forward_fused",
            "kda_decode_step_fused", "kda_backward", "kda_backward_workspace_bytes",
            "library_path", "load_library"]

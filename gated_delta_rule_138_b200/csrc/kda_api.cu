@@ -27,7 +27,7 @@ cudaError_t launch_chunk_tc(const void* q, const void* k, const void* v, const v
                             void* out, float* S_final, int64_t rows, int64_t T, int H, int* status,
                             cudaStream_t stream, const int32_t* slots = nullptr, int num_slots = 0,
                             int fused = 0);
-size_t chunk_tc_segmented_workspace_floats(int64_t nseq, int H, int nseg);
+size_t chunk_tc_segmented_workspace_bytes(int64_t nseq, int64_t rows, int H, int nseg);
 size_t backward_workspace_floats(bool packed, int64_t nseq, int64_t T, int H, int DK, int DV);
 cudaError_t launch_backward(int in_bf16, const void* q, const void* k, const void* v,
                             const void* alpha, const void* beta, const float* S0, const void* dout,
@@ -49,7 +49,7 @@ cudaError_t launch_apply_maps(const float* S0, const float* maps, int G, int nse
 cudaError_t launch_chunk_tc_segmented(const void* q, const void* k, const void* v,
                                       const void* alpha, const void* beta, const float* S0,
                                       const int32_t* cu, int nseq, void* out, float* S_final,
-                                      int64_t rows, int64_t T, int H, int nseg, float* workspace,
+                                      int64_t rows, int64_t T, int H, int nseg, void* workspace,
                                       int* status, cudaStream_t stream, int fused = 0);
 }  // namespace kda
 
@@ -97,13 +97,47 @@ cudaError_t device_status_word(int** out) {
     return cudaSuccess;
 }
 
+// One stream-ordered memory pool per GPU for the split forward's workspace.  It
+// keeps what it has reserved (no release threshold), so that repeated calls reuse
+// the same device memory instead of mapping it anew after every synchronisation;
+// kda_release_workspace hands it back.
+cudaMemPool_t g_pool[kMaxDevices] = {};
+
+cudaError_t workspace_pool(cudaMemPool_t* out) {
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return e;
+    if (dev < 0 || dev >= kMaxDevices) return cudaErrorInvalidDevice;
+    std::lock_guard<std::mutex> lock(g_status_mu);
+    if (!g_pool[dev]) {
+        cudaMemPoolProps props = {};
+        props.allocType = cudaMemAllocationTypePinned;
+        props.location.type = cudaMemLocationTypeDevice;
+        props.location.id = dev;
+        cudaMemPool_t pool = nullptr;
+        e = cudaMemPoolCreate(&pool, &props);
+        if (e != cudaSuccess) return e;
+        uint64_t keep = UINT64_MAX;
+        e = cudaMemPoolSetAttribute(pool, cudaMemPoolAttrReleaseThreshold, &keep);
+        if (e != cudaSuccess) { cudaMemPoolDestroy(pool); return e; }
+        g_pool[dev] = pool;
+    }
+    *out = g_pool[dev];
+    return cudaSuccess;
+}
+
 // Time segments per sequence for the tensor-core forward.  One CTA runs one
 // (sequence, head) segment on one SM and a segment costs in proportion to its
-// chunks; a split adds a summary pass (about 0.7 of a forward chunk) over all
-// but the last segment.  The cost, in units of the unsplit CTA's time, of g
-// segments is (waves of the forward + 0.7 waves of the summaries) / g, with
-// waves = ceil(CTAs / SMs); g = 1 costs ceil(units / SMs).  A small charge per
-// segment stands for the scan and launch overheads.  Segments keep >= 16 chunks.
+// chunks.  A split runs every segment in the dual mode (kSplitChunk of an unsplit
+// chunk: the 256-wide state and both output parts) and then a pass over the
+// outputs, o += Qg S_g, bound by memory: per (sequence, head) about kSplitPass of
+// the unsplit CTA's time (its traffic, 3 x 256 bytes per token, against a chunk's
+// time per token).  The cost, in units of the unsplit CTA's time, of g segments is
+// kSplitChunk * waves(units g) / g + kSplitPass * units / SMs + a small charge per
+// segment (the scan's chain, the launches), with waves = ceil(CTAs / SMs); g = 1
+// costs waves(units).  Segments keep >= 16 chunks.
+constexpr double kSplitChunk = 1.15;
+constexpr double kSplitPass = 0.15;
 int segments_for(int64_t nseq, int64_t tokens_per_seq, int64_t H, int sms) {
     const int64_t units = nseq * H;
     if (units <= 0 || sms <= 0) return 1;
@@ -112,7 +146,7 @@ int segments_for(int64_t nseq, int64_t tokens_per_seq, int64_t H, int sms) {
     double best = waves(units);
     int best_g = 1;
     for (int g = 2; g <= 64 && chunks >= (int64_t)g * 16 && nseq * g <= 65535; ++g) {
-        const double cost = (waves(units * g) + 0.7 * waves(units * (g - 1))) / g + 0.002 * g;
+        const double cost = kSplitChunk * waves(units * g) / g + kSplitPass * units / sms + 0.0002 * g;
         if (cost < best) {
             best = cost;
             best_g = g;
@@ -211,9 +245,22 @@ size_t kda_forward_workspace_bytes(int32_t B, int64_t T, int32_t H, int32_t d_k,
     size_t bytes = sizeof(int);  // the per-device status word, allocated once
     if (B > 0 && T > 0 && H > 0 && use_tc(d_k, d_v, chunk, KDA_BF16, KDA_BF16)) {
         const int nseg = segments_for(B, T, H, current_sms());
-        bytes += sizeof(float) * kda::chunk_tc_segmented_workspace_floats(B, H, nseg);
+        bytes += kda::chunk_tc_segmented_workspace_bytes(B, (int64_t)B * T, H, nseg);
     }
     return bytes;
+}
+
+kda_status_t kda_release_workspace(void) {
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return cuda_status(e);
+    if (dev < 0 || dev >= kMaxDevices) return KDA_OK;
+    cudaMemPool_t pool = nullptr;
+    {
+        std::lock_guard<std::mutex> lock(g_status_mu);
+        pool = g_pool[dev];
+    }
+    return pool ? cuda_status(cudaMemPoolTrimTo(pool, 0)) : KDA_OK;
 }
 
 int32_t kda_forward_segments(int32_t num_seqs, int64_t tokens_per_seq, int32_t H, int32_t num_sms) {
@@ -275,12 +322,15 @@ kda_status_t forward_impl(const void* q, const void* k, const void* v, const voi
         if (rows > 0x7fffffffLL) return KDA_ERR_UNSUPPORTED;  // TMA row coordinate is int32
         const int64_t per_seq = cu_seqlens ? (T + nseq - 1) / nseq : T;
         const int nseg = segments_for(nseq, per_seq, H, current_sms());
-        float* ws = nullptr;
+        void* ws = nullptr;
         if (nseg > 1) {
-            // stream-ordered workspace for the segment maps and start states; if it
-            // cannot be had, the unsplit kernel computes the same result
-            const size_t bytes = sizeof(float) * kda::chunk_tc_segmented_workspace_floats(nseq, H, nseg);
-            if (cudaMallocAsync(reinterpret_cast<void**>(&ws), bytes, s) != cudaSuccess) {
+            // stream-ordered workspace for the segment maps, start states and map rows,
+            // from this library's pool; if it cannot be had, the unsplit kernel computes
+            // the same result
+            const size_t bytes = kda::chunk_tc_segmented_workspace_bytes(nseq, rows, H, nseg);
+            cudaMemPool_t pool = nullptr;
+            if (workspace_pool(&pool) != cudaSuccess ||
+                cudaMallocFromPoolAsync(&ws, bytes, pool, s) != cudaSuccess) {
                 cudaGetLastError();
                 ws = nullptr;
             }

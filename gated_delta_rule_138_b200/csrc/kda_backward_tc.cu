@@ -109,16 +109,17 @@ constexpr uint32_t OFF_T = 57344;       // T [64 j][64 m]
 constexpr uint32_t OFF_QT = 65536;      // q*gamma [64 r][128 c]
 constexpr uint32_t OFF_KT = 81920;      // k*gamma [64 r][128 c]
 constexpr uint32_t OFF_DO = 98304;      // dO [64 r][128 n] (TMA), chunk parity 0; parity 1 at OFF_DO1
-constexpr uint32_t OFF_RV = 114688;     // R = V - (k*gamma) S0 [64 j][128 n]
+constexpr uint32_t OFF_RV = 114688;     // R = V - (k*gamma) S0 [64 j][128 n], chunk parity 0; 1 at OFF_RV1
 constexpr uint32_t OFF_DU = 131072;     // dU bf16 [64 j][128 n], MN-major B
 constexpr uint32_t OFF_MDR = 147456;    // -dR bf16 [64 r][128 n], MN-major B
 constexpr uint32_t OFF_DY = 163840;     // dY bf16 [64 m][128 n] (to the record)
 constexpr uint32_t OFF_DO1 = 180224;
-constexpr uint32_t OFF_MISC = 196608;
+constexpr uint32_t OFF_RV1 = 196608;
+constexpr uint32_t OFF_MISC = 212992;
 constexpr uint32_t M_GC = 0;            // float [2 parities][128]
 constexpr uint32_t M_BETA = 1024;       // float [64]
 constexpr uint32_t M_DB = 1280;         // float [64][2]
-constexpr uint32_t M_BAR = 1792;        // uint64 x4: loads A (P, k*eta, dO, gamma_C), B (T), C (q*gamma, k*gamma, R), MMA
+constexpr uint32_t M_BAR = 1792;        // uint64 x4: loads A (P, k*eta, dO, gamma_C, R), B (T), C (q*gamma, k*gamma), MMA
 constexpr uint32_t M_TMEM = 1824;
 constexpr uint32_t M_FLAG = 1828;
 constexpr uint32_t SMEM_BYTES = OFF_MISC + 1856 + 1024;
@@ -174,6 +175,7 @@ kda_bwd_dstate_kernel(const __grid_constant__ CUtensorMap tmDO, const __nv_bfloa
         nchunks = (int)max((int64_t)0, rec_chunks - s_cbase);
     auto rec_of = [&](int i) { return rec + ((size_t)(s_cbase + i) * H + h) * bwdrec::BYTES; };
     auto dO_of = [&](int i) { return sm + ((i & 1) ? OFF_DO1 : OFF_DO); };
+    auto rv_of = [&](int i) { return sm + ((i & 1) ? OFF_RV1 : OFF_RV); };
 
     if (tid == 0) {
         mbar_init(barA, 1);
@@ -239,9 +241,10 @@ kda_bwd_dstate_kernel(const __grid_constant__ CUtensorMap tmDO, const __nv_bfloa
     auto issue_a = [&](int i) {
         uint8_t* rp = rec_of(i);
         const int64_t row0 = bos + (int64_t)i * C;
-        mbar_arrive_expect_tx(barA, 8192 + 16384 + 16384 + 512);
+        mbar_arrive_expect_tx(barA, 8192 + 16384 + 16384 + 16384 + 512);
         bulk_load(sm + OFF_P, rp + bwdrec::P, 8192, barA);
         bulk_load(sm + OFF_KH, rp + bwdrec::KH, 16384, barA);
+        bulk_load(rv_of(i), rp + bwdrec::RV, 16384, barA);
         bulk_load(sGC + 128 * (i & 1), rp + bwdrec::GC, 512, barA);
 #pragma unroll
         for (int a = 0; a < 2; ++a)
@@ -255,10 +258,9 @@ kda_bwd_dstate_kernel(const __grid_constant__ CUtensorMap tmDO, const __nv_bfloa
     };
     auto issue_c = [&](int i) {
         uint8_t* rp = rec_of(i);
-        mbar_arrive_expect_tx(barC, 3 * 16384);
+        mbar_arrive_expect_tx(barC, 2 * 16384);
         bulk_load(sm + OFF_QT, rp + bwdrec::QT, 16384, barC);
         bulk_load(sm + OFF_KT, rp + bwdrec::KT, 16384, barC);
-        bulk_load(sm + OFF_RV, rp + bwdrec::RV, 16384, barC);
         ++nC;
     };
     if (ctl && nchunks > 0) {
@@ -339,7 +341,8 @@ kda_bwd_dstate_kernel(const __grid_constant__ CUtensorMap tmDO, const __nv_bfloa
         // ---- dY = T^T dU
         if (ctl) {
             // every thread has passed its wait on this chunk's A loads: P and k*eta are
-            // consumed, and the other dO and gamma_C buffers are free
+            // consumed, and the other dO, gamma_C and R buffers are free (the previous
+            // chunk's R was last read before its dS step)
             if (i > 0 && ok) issue_a(i - 1);
             wait_bar(barB, phB);
             if (ok) {
@@ -354,7 +357,6 @@ kda_bwd_dstate_kernel(const __grid_constant__ CUtensorMap tmDO, const __nv_bfloa
             if (i > 0 && ok) issue_b(i - 1);   // T is consumed
         }
         if (compute) {
-            wait_bar(barC, phC);   // R
             wait_mma();
             const int m = 16 * q4 + lane;
             const float b = lane < 16 ? sBeta[m] : 0.0f;
@@ -369,7 +371,7 @@ kda_bwd_dstate_kernel(const __grid_constant__ CUtensorMap tmDO, const __nv_bfloa
                     for (int ch = 0; ch < 4; ++ch) {
                         float r8[8], w[8];
                         const uint32_t off = hf * 8192 + swz(m, 4 * p + ch);
-                        unpack8(*reinterpret_cast<const uint4*>(sm + OFF_RV + off), r8);
+                        unpack8(*reinterpret_cast<const uint4*>(rv_of(i) + off), r8);
 #pragma unroll
                         for (int e = 0; e < 8; ++e) {
                             part = fmaf(r8[e], v[8 * ch + e], part);
@@ -413,7 +415,7 @@ kda_bwd_dstate_kernel(const __grid_constant__ CUtensorMap tmDO, const __nv_bfloa
                 commit();
             }
             wait_mma();
-            if (i > 0 && ok) issue_c(i - 1);   // q*gamma, k*gamma and R are consumed
+            if (i > 0 && ok) issue_c(i - 1);   // q*gamma and k*gamma are consumed
         }
         if (compute) {
             if (tid < C && tid < Lc)

@@ -87,10 +87,30 @@ constexpr uint32_t OFF_MISC = OFF_KH + 16384;
 constexpr uint32_t MISC_PI = 0;          // float [8][128] octant gate products
 constexpr uint32_t MISC_GC = 4096;       // float [128] gamma_C
 constexpr uint32_t MISC_BETA = 4608;     // float [64]
-constexpr uint32_t MISC_BAR = 4864;      // 5 x uint64 mbarriers: q, k+alpha, v, MMA, (k*gamma) S
-constexpr uint32_t MISC_TMEM = 4904;     // uint32 TMEM base
-constexpr uint32_t MISC_FLAG = 4908;     // int timeout seen
+constexpr uint32_t MISC_BAR = 4864;      // 6 x uint64 mbarriers: q, k+alpha (dual: k), v, MMA,
+                                         // (k*gamma) S, alpha (dual mode)
+constexpr uint32_t MISC_TMEM = 4912;     // uint32 TMEM base
+constexpr uint32_t MISC_FLAG = 4916;     // int timeout seen
 constexpr uint32_t SMEM_BYTES = OFF_MISC + 4928 + 1024;  // + alignment slack
+
+// The dual mode (a segment's map [M | N] and both parts of its outputs, see the
+// kernel) holds the 64 KB [M | N] copy and the q buffers at once: alpha and v take
+// turns in one buffer (alpha is consumed at a chunk's start, v only at its barrier
+// D), the work region ends at 64 KB, and the octant gate products live in its
+// first 4 KB (free from the previous chunk's barrier E to this chunk's operand loop).
+namespace dual {
+constexpr uint32_t OFF_S = 0;            // [M | N] bf16, four [128][64] atoms
+constexpr uint32_t OFF_Q = 65536;        // q, two buffers
+constexpr uint32_t OFF_K = 98304;
+constexpr uint32_t OFF_AV = 114688;      // alpha, then v
+constexpr uint32_t OFF_X = 131072;       // 64 KB work region
+constexpr uint32_t OFF_KT = 196608;
+constexpr uint32_t OFF_KH = 212992;
+constexpr uint32_t OFF_MISC = 229376 - 4096;   // the misc block without its first 4 KB (MISC_PI)
+constexpr uint32_t X_PI = 0;             // float [8][128] octant gate products
+constexpr uint32_t SMEM_BYTES = OFF_MISC + 4928 + 1024;
+static_assert(SMEM_BYTES <= 232448, "dual-mode shared memory");
+}  // namespace dual
 
 // work region X, by phase
 constexpr uint32_t X_L = 0;              // left rows [128][128]: k*lam rows 0..63, q*lam rows 64..127
@@ -104,7 +124,8 @@ constexpr uint32_t X_XS = 34816;         // float scratch [32][36]
 // fp32 K-major 128B-swizzled tiles (32 floats per row) for the tf32 MMAs of the 32 -> 64 step
 constexpr uint32_t X_T0T = 40960;        // Tinv[0:32, 0:32]^T   [64 rows (32 used)][32]
 constexpr uint32_t X_T1 = 49152;         // Tinv[32:64, 32:64]   [64 rows (32 used)][32]
-constexpr uint32_t X_A10 = 65536;        // A[32:64, 0:32]       [32][32]
+constexpr uint32_t X_A10 = 45056;        // A[32:64, 0:32]       [32][32]: the rows 32..63 of the
+                                         // T0^T tile, which its M=64 product reads but nobody uses
 constexpr uint32_t X_TB = 40960;         // Tb, K-major A [64 r][64 m] (after the solve)
 constexpr uint32_t X_WQ = 0;             // -W, K-major A [64][128] (two [64][64] atoms 8 KB apart)
 constexpr uint32_t X_U = 16384;          // U, MN-major B [64 j][128 n] (two [64][64] atoms);
@@ -128,6 +149,12 @@ __device__ __forceinline__ void st4_bf16(uint8_t* p, const float (&v)[4]) {
     *reinterpret_cast<uint2*>(p) = make_uint2(pack_bf16x2(v[0], v[1]), pack_bf16x2(v[2], v[3]));
 }
 
+// 32 consecutive fp32 columns of this thread's TMEM lane, one wait for both loads
+__device__ __forceinline__ void tmem_ld32(uint32_t taddr, float (&v)[32]) {
+    tmem_ld16(taddr, *reinterpret_cast<float(*)[16]>(&v[0]));
+    tmem_ld16(taddr + 16, *reinterpret_cast<float(*)[16]>(&v[16]));
+    tmem_wait_ld();
+}
 // 64 consecutive fp32 columns of this thread's TMEM lane, one wait for all four loads
 __device__ __forceinline__ void tmem_ld64(uint32_t taddr, float (&v)[64]) {
     tmem_ld16(taddr, *reinterpret_cast<float(*)[16]>(&v[0]));
@@ -160,6 +187,8 @@ struct Segments {
     // starts from zero and writes no state.  Null: slot n.
     const int32_t* slots;
     int num_slots;
+    // dual mode: the per-token map rows Qg [rows, H, DK] bf16 (see the kernel)
+    __nv_bfloat16* qg = nullptr;
     // record mode (the backward's first pass): per-(chunk, head) records and per-chunk
     // headers, chunks numbered across sequences in order
     uint8_t* rec = nullptr;
@@ -181,7 +210,13 @@ struct LoadTrack {
 // kRecord = true: the forward recurrence without outputs; every chunk's start state,
 // operand tiles, T, V - (k*gamma) S, U and gamma_C go to the backward's record of
 // (chunk, head) (kda_bwd_record.cuh), byte for byte as they sit in shared memory.
-template <bool kCtaStatus, bool kSummary, bool kFused, bool kRecord = false>
+// kDual = true (with kSummary): the summary recurrence on [M | N] from [I | 0] that also
+// forms the chunk outputs of that 256-wide state, [Qg | O0] = (q*gamma) [M | N] + P
+// [U_M | U_N]: O0 is the segment's output from a zero start state (written to out)
+// and Qg (written to seg.qg) the rows that carry its true start state S_g into it,
+// o = O0 + Qg S_g (the state map is affine, so the output is too).  One pass over a
+// segment then gives both its map and everything its outputs need but S_g.
+template <bool kCtaStatus, bool kSummary, bool kFused, bool kRecord = false, bool kDual = false>
 __global__ void __launch_bounds__(NTHREADS, 1)
 kda_chunk_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                     const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmV,
@@ -196,24 +231,28 @@ kda_chunk_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_consta
     uint8_t* sm = kFused ? reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                                       ~static_cast<uintptr_t>(1023))
                          : smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
-    uint8_t* sS = sm + OFF_S;
-    uint8_t* sQ = sm + OFF_Q;
-    uint8_t* sK = sm + OFF_K;
-    uint8_t* sAl = sm + OFF_AL;
-    uint8_t* sV = sm + OFF_V;
-    uint8_t* sX = sm + OFF_X;
-    uint8_t* sKT = sm + OFF_KT;
-    uint8_t* sKH = sm + OFF_KH;
-    float* sPi = reinterpret_cast<float*>(sm + OFF_MISC + MISC_PI);
-    float* sGC = reinterpret_cast<float*>(sm + OFF_MISC + MISC_GC);
-    float* sBeta = reinterpret_cast<float*>(sm + OFF_MISC + MISC_BETA);
-    uint64_t* barQ = reinterpret_cast<uint64_t*>(sm + OFF_MISC + MISC_BAR);
+    static_assert(!kDual || (kSummary && !kRecord), "the dual mode is a summary mode");
+    constexpr bool kQ = !kSummary || kDual;   // q is read and outputs are formed
+    constexpr uint32_t oMisc = kDual ? dual::OFF_MISC : OFF_MISC;
+    uint8_t* sS = sm + (kDual ? dual::OFF_S : OFF_S);
+    uint8_t* sQ = sm + (kDual ? dual::OFF_Q : OFF_Q);
+    uint8_t* sK = sm + (kDual ? dual::OFF_K : OFF_K);
+    uint8_t* sAl = sm + (kDual ? dual::OFF_AV : OFF_AL);
+    uint8_t* sV = sm + (kDual ? dual::OFF_AV : OFF_V);
+    uint8_t* sX = sm + (kDual ? dual::OFF_X : OFF_X);
+    uint8_t* sKT = sm + (kDual ? dual::OFF_KT : OFF_KT);
+    uint8_t* sKH = sm + (kDual ? dual::OFF_KH : OFF_KH);
+    float* sPi = reinterpret_cast<float*>(kDual ? sX + dual::X_PI : sm + OFF_MISC + MISC_PI);
+    float* sGC = reinterpret_cast<float*>(sm + oMisc + MISC_GC);
+    float* sBeta = reinterpret_cast<float*>(sm + oMisc + MISC_BETA);
+    uint64_t* barQ = reinterpret_cast<uint64_t*>(sm + oMisc + MISC_BAR);
     uint64_t* barKA = barQ + 1;
     uint64_t* barV = barQ + 2;
     uint64_t* barM = barQ + 3;
     uint64_t* barZ = barQ + 4;   // (k*gamma) S_start, forward mode
-    uint32_t* sTmem = reinterpret_cast<uint32_t*>(sm + OFF_MISC + MISC_TMEM);
-    int* sFlag = reinterpret_cast<int*>(sm + OFF_MISC + MISC_FLAG);
+    uint64_t* barAl = barQ + 5;  // alpha, dual mode
+    uint32_t* sTmem = reinterpret_cast<uint32_t*>(sm + oMisc + MISC_TMEM);
+    int* sFlag = reinterpret_cast<int*>(sm + oMisc + MISC_FLAG);
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const bool compute = warp < NT / 32;   // warps 0-7; warp 8 is the control warp
@@ -258,6 +297,7 @@ kda_chunk_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_consta
         mbar_init(barV, 1);
         mbar_init(barM, 1);
         mbar_init(barZ, 1);
+        mbar_init(barAl, 1);
         mbar_fence_init();
         *sFlag = 0;
     }
@@ -265,6 +305,7 @@ kda_chunk_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_consta
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
+    KDA_TC_PHASE(30);
     const uint32_t tmem = *sTmem;
     const uint32_t tlane = (uint32_t)(32 * q4) << 16;
 
@@ -314,13 +355,19 @@ kda_chunk_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_consta
         for (int a = 0; a < 2; ++a)
             tma_load_2d(sQ + buf * 16384 + a * 8192, &tmQ, barQ, h * DK + 64 * a, (int)row0);
     };
-    auto issue_ka = [&](int64_t row0) {
-        mbar_arrive_expect_tx(barKA, 2 * 16384);
+    auto issue_ka = [&](int64_t row0) {   // k and (but in the dual mode) alpha
+        mbar_arrive_expect_tx(barKA, kDual ? 16384 : 2 * 16384);
 #pragma unroll
         for (int a = 0; a < 2; ++a) {
             tma_load_2d(sK + a * 8192, &tmK, barKA, h * DK + 64 * a, (int)row0);
-            tma_load_2d(sAl + a * 8192, &tmA, barKA, h * DK + 64 * a, (int)row0);
+            if (!kDual) tma_load_2d(sAl + a * 8192, &tmA, barKA, h * DK + 64 * a, (int)row0);
         }
+    };
+    auto issue_al = [&](int64_t row0) {   // dual mode: alpha, into the buffer v leaves
+        mbar_arrive_expect_tx(barAl, 16384);
+#pragma unroll
+        for (int a = 0; a < 2; ++a)
+            tma_load_2d(sAl + a * 8192, &tmA, barAl, h * DK + 64 * a, (int)row0);
     };
     auto issue_v = [&](int64_t row0) {
         mbar_arrive_expect_tx(barV, 16384);
@@ -331,7 +378,7 @@ kda_chunk_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_consta
 
     bool ok = true;   // this thread has seen every wait complete
     // asynchronous work that a timed-out wait may leave in flight, drained before exit
-    LoadTrack tq, tka, tv;
+    LoadTrack tq, tka, tv, tal;
     uint32_t phM = 0, mma_out_ph = 0, phZ = 0, z_out_ph = 0;
     bool mma_out = false;   // (control thread) an MMA group committed and not yet waited for
     bool z_out = false;     // (control thread) the same for the (k*gamma) S group
@@ -372,11 +419,22 @@ kda_chunk_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_consta
     // chunk's U MMA needs them.  S goes to its bf16 copy, O to the output rows.
     // A full chunk's O is staged in the q buffer the next q load will use (row-major,
     // 128-byte swizzled, the TMA box layout) and written by one TMA store; a
-    // partial last chunk is stored row by row.
+    // partial last chunk is stored row by row.  The dual mode's [Qg | O0] (an M=64
+    // accumulator, N=256) leaves row by row: warps of column half 0 write Qg, half 1 O0.
     auto finish_prev = [&](int64_t prow0, int pLc, uint8_t* stage) {
         wait_mma();
         const int c = 32 * q4 + lane;
-        if constexpr (kSummary) {
+        if constexpr (kDual && !kFused) {   // (32-column pieces: fewer live registers)
+#pragma unroll
+            for (int p = 0; p < 4; ++p) {
+                float v[32];
+                tmem_ld32(tmem + tlane + TM_S + 128 * hf + 32 * p, v);
+#pragma unroll
+                for (int ch = 0; ch < 4; ++ch)
+                    *reinterpret_cast<uint4*>(sS + (2 * hf + (p >> 1)) * 16384 + swz(c, 4 * (p & 1) + ch)) =
+                        pack8(&v[8 * ch]);
+            }
+        } else if constexpr (kSummary) {
 #pragma unroll
             for (int p = 0; p < 2; ++p) {
                 float v[64];
@@ -384,6 +442,23 @@ kda_chunk_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_consta
 #pragma unroll
                 for (int ch = 0; ch < 8; ++ch)
                     *reinterpret_cast<uint4*>(sS + (2 * hf + p) * 16384 + swz(c, ch)) = pack8(&v[8 * ch]);
+            }
+        }
+        if constexpr (kSummary) {
+            if constexpr (kDual) {
+                const int r = 16 * q4 + lane;
+                __nv_bfloat16* dst_rows = hf == 0 ? seg.qg : out;
+                uint4* dst = reinterpret_cast<uint4*>(dst_rows + ((size_t)(prow0 + r) * H + h) * DK);
+                const bool wr = lane < 16 && r < pLc;
+#pragma unroll
+                for (int p = 0; p < 4; ++p) {   // (32-column pieces: fewer live registers)
+                    float v[32];
+                    tmem_ld32(tmem + tlane + TM_WK + 128 * hf + 32 * p, v);
+                    if (wr) {
+#pragma unroll
+                        for (int ch = 0; ch < 4; ++ch) dst[4 * p + ch] = pack8(&v[8 * ch]);
+                    }
+                }
             }
         } else {
             float v[64];
@@ -414,14 +489,19 @@ kda_chunk_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_consta
     };
 
     if (nchunks > 0 && ctl) {
-        if (!kSummary) {
+        if (kQ) {
             issue_q(bos, 0);
             issued(tq);
         }
         issue_ka(bos);
         issued(tka);
-        issue_v(bos);
-        issued(tv);
+        if (kDual) {   // v follows once the first chunk's gate phase has read alpha
+            issue_al(bos);
+            issued(tal);
+        } else {
+            issue_v(bos);
+            issued(tv);
+        }
     }
     fence_async_smem();
     tc_fence_before();
@@ -445,7 +525,8 @@ kda_chunk_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_consta
         uint8_t* sQc = sQ + (chunk & 1) * 16384;
         if (tid < C) sBeta[tid] = beta_next;
         wait_load(barKA, tka);
-        if (!kSummary) wait_load(barQ, tq);
+        if (kDual) wait_load(barAl, tal);
+        if (kQ) wait_load(barQ, tq);
         KDA_TC_PHASE(0);
 
         // ================= gate products and bf16 operands (all threads)
@@ -547,7 +628,7 @@ kda_chunk_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_consta
                     const uint32_t in_off = a64 * 8192u + (uint32_t)r * 128u + (((chk ^ (uint32_t)r) & 7u) << 4) + inner;
                     float k[4], q[4] = {0.f, 0.f, 0.f, 0.f};
                     unpack4_bf16(*reinterpret_cast<const uint2*>(sK + in_off), k);
-                    if (!kSummary) unpack4_bf16(*reinterpret_cast<const uint2*>(sQc + in_off), q);
+                    if (kQ) unpack4_bf16(*reinterpret_cast<const uint2*>(sQc + in_off), q);
                     sk[i] = k[0] * k[0] + k[1] * k[1] + k[2] * k[2] + k[3] * k[3];
                     sq[i] = q[0] * q[0] + q[1] * q[1] + q[2] * q[2] + q[3] * q[3];
                 }
@@ -556,7 +637,7 @@ kda_chunk_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_consta
 #pragma unroll
                     for (int i = 0; i < 8; ++i) {
                         sk[i] += __shfl_xor_sync(0xffffffffu, sk[i], o);
-                        if (!kSummary) sq[i] += __shfl_xor_sync(0xffffffffu, sq[i], o);
+                        if (kQ) sq[i] += __shfl_xor_sync(0xffffffffu, sq[i], o);
                     }
                 }
 #pragma unroll
@@ -570,8 +651,10 @@ kda_chunk_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_consta
             auto in_off_of = [&](int r) {
                 return a64 * 8192u + (uint32_t)r * 128u + (((chk ^ (uint32_t)r) & 7u) << 4) + inner;
             };
+            // dual mode: the gate products sit where the operand tiles go
+            if constexpr (kDual) sync_compute();
             uint2 kn = *reinterpret_cast<const uint2*>(sK + in_off_of(8 * O));
-            uint2 qn = kSummary ? make_uint2(0u, 0u) : *reinterpret_cast<const uint2*>(sQc + in_off_of(8 * O));
+            uint2 qn = !kQ ? make_uint2(0u, 0u) : *reinterpret_cast<const uint2*>(sQc + in_off_of(8 * O));
 #pragma unroll
             for (int i = 0; i < 8; ++i) {
                 const int r = 8 * O + i;
@@ -579,14 +662,14 @@ kda_chunk_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_consta
                 const uint32_t in_off = a64 * 8192u + sw;    // 64-row tiles: q, k, KT, KH
                 float k[4], q[4] = {0.f, 0.f, 0.f, 0.f};
                 unpack4_bf16(kn, k);
-                if (!kSummary) unpack4_bf16(qn, q);
+                if (kQ) unpack4_bf16(qn, q);
                 if constexpr (kFused) {
 #pragma unroll
                     for (int c = 0; c < 4; ++c) { k[c] *= kinv[i]; q[c] *= qinv[i]; }
                 }
                 if (i < 7) {
                     kn = *reinterpret_cast<const uint2*>(sK + in_off_of(r + 1));
-                    if (!kSummary) qn = *reinterpret_cast<const uint2*>(sQc + in_off_of(r + 1));
+                    if (kQ) qn = *reinterpret_cast<const uint2*>(sQc + in_off_of(r + 1));
                 }
                 if (r >= Lc) {
 #pragma unroll
@@ -604,7 +687,7 @@ kda_chunk_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_consta
 #pragma unroll
                 for (int c = 0; c < 4; ++c) w[c] = kp[c] * dlf[c];
                 st4_bf16(lrow, w);                                        // k*lam, row r
-                if (!kSummary) {
+                if (kQ) {
 #pragma unroll
                     for (int c = 0; c < 4; ++c) w[c] = qp[c] * dlf[c];
                     st4_bf16(lrow + 64 * 128, w);                         // q*lam, row 64 + r
@@ -666,7 +749,7 @@ kda_chunk_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_consta
             const bool lower = (q4 & 1) == 0;          // r < 32: group 1 columns
             const bool zero = lower && hf == 1;        // j >= 32 > r: all zero
             float v[32];
-            if (!zero && (q4 < 2 || !kSummary)) {
+            if (!zero && (q4 < 2 || kQ)) {
                 const uint32_t col = lower ? 0u : 32u + 32u * hf;
                 tmem_ld16(tmem + tlane + TM_WK + col, *reinterpret_cast<float(*)[16]>(&v[0]));
                 tmem_ld16(tmem + tlane + TM_WK + col + 16, *reinterpret_cast<float(*)[16]>(&v[16]));
@@ -687,7 +770,7 @@ kda_chunk_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_consta
                     f.w = (j0 + i + 3 < r) ? b * v[i + 3] : 0.0f;
                     *reinterpret_cast<float4*>(&Am[r * AS + j0 + i]) = f;
                 }
-            } else if (!kSummary) {
+            } else if (kQ) {
                 uint8_t* sP = sX + X_P;
 #pragma unroll
                 for (int c8 = 0; c8 < 4; ++c8) {
@@ -1039,7 +1122,7 @@ kda_chunk_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_consta
                      sdesc_sw128(s0 + 32768 + ks * 2048, 1024, 16384), idM64, 1);
         commit_mma();
     };
-    auto mma_s = [&]() {
+    auto mma_s = [&](uint8_t* sQc) {
         const uint32_t kh = smem_u32(sKH), u0 = smem_u32(sX + X_U);
         if constexpr (kSummary) {
             constexpr uint32_t idesc = idesc_bf16(128, 256, true, true);
@@ -1047,6 +1130,21 @@ kda_chunk_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_consta
             for (int ks = 0; ks < 4; ++ks)
                 mma_bf16(tmem + TM_S, sdesc_sw128(kh + ks * 2048, 1024, 8192),
                          sdesc_sw128(u0 + ks * 2048, 1024, 8192), idesc, 1);
+            if constexpr (kDual) {
+                // [Qg | O0] = (q*gamma) [M | N] + P [U_M | U_N]   (M=64, N=256) over the scratch
+                // and U columns, which the [U_M | U_N] extraction has emptied; [M | N] is read
+                // from its bf16 copy, still the chunk's start value
+                constexpr uint32_t id_o = idesc_bf16(64, 256, false, true);
+                const uint32_t qg = smem_u32(sQc), s0 = smem_u32(sS), p0 = smem_u32(sX + X_P);
+#pragma unroll
+                for (int ks = 0; ks < 8; ++ks)
+                    mma_bf16(tmem + TM_WK, sdesc_sw128(qg + (ks >> 2) * 8192 + (ks & 3) * 32),
+                             sdesc_sw128(s0 + ks * 2048, 1024, 16384), id_o, ks > 0);
+#pragma unroll
+                for (int ks = 0; ks < 4; ++ks)
+                    mma_bf16(tmem + TM_WK, sdesc_sw128(p0 + ks * 32),
+                             sdesc_sw128(u0 + ks * 2048, 1024, 8192), id_o, 1);
+            }
         } else {
             constexpr uint32_t id_s = idesc_bf16(128, 128, true, true);
             const uint32_t p0 = smem_u32(sX + X_P);
@@ -1102,6 +1200,14 @@ kda_chunk_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_consta
                 issue_ka(row0 + C);
                 issued(tka);
             }
+            if (kDual && ok) {
+                issue_v(row0);   // alpha has left the buffer v takes
+                issued(tv);
+                if (chunk + 1 < nchunks) {   // the other q buffer's O products are done
+                    issue_q(row0 + C, (chunk + 1) & 1);
+                    issued(tq);
+                }
+            }
             wait_mma();
             KDA_TC_PHASE(21);
             if (!kSummary) {
@@ -1139,6 +1245,7 @@ kda_chunk_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_consta
                 if (ok) mma_w();
                 wait_load(barV, tv);
                 if (ok) mma_tbv();
+                if (kDual && ok) commit_z();   // Tb V done: alpha may take the buffer
             } else if (ok) {
                 if constexpr (kRecord) {
                     bulk_store(rec_of(chunk) + bwdrec::RV, sV, 16384);
@@ -1149,6 +1256,13 @@ kda_chunk_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_consta
                 commit_mma();
             }
             wait_mma();
+            if constexpr (kDual) {
+                wait_z();
+                if (chunk + 1 < nchunks && ok) {
+                    issue_al(row0 + C);
+                    issued(tal);
+                }
+            }
             KDA_TC_PHASE(24);
         }
         if constexpr (kSummary) {
@@ -1158,7 +1272,7 @@ kda_chunk_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_consta
                 wait_mma();
             }
         }
-        if (ctl && chunk + 1 < nchunks && ok) {   // v is consumed
+        if (!kDual && ctl && chunk + 1 < nchunks && ok) {   // v is consumed
             issue_v(row0 + C);
             issued(tv);
         }
@@ -1174,7 +1288,7 @@ kda_chunk_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_consta
                 bulk_store(rec_of(chunk) + bwdrec::U, sX + X_U, 16384);
                 bulk_commit_group();
             }
-            mma_s();
+            mma_s(sQc);
             if constexpr (kRecord) {
                 bulk_wait_read_all();
                 commit_mma();
@@ -1205,6 +1319,7 @@ kda_chunk_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_consta
         if (tq.issued) mbar_wait_ns(barQ, (tq.issued - 1) & 1u, kWaitNs);
         if (tka.issued) mbar_wait_ns(barKA, (tka.issued - 1) & 1u, kWaitNs);
         if (tv.issued) mbar_wait_ns(barV, (tv.issued - 1) & 1u, kWaitNs);
+        if (tal.issued) mbar_wait_ns(barAl, (tal.issued - 1) & 1u, kWaitNs);
         if (mma_out) mbar_wait_ns(barM, mma_out_ph, kWaitNs);
         if (z_out) mbar_wait_ns(barZ, z_out_ph, kWaitNs);
     }
@@ -1247,12 +1362,14 @@ kda_chunk_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_consta
 
 // S_{g+1} = M_g S_g + N_g over the segments of one sequence, in fp32: one CTA
 // per (16 value columns, head, sequence), thread i owns row i of the state.
-// start[g = 0] receives S0 (or zeros), so the forward kernel never reads S0
-// itself and S_final may alias S0.
+// start[g = 0] receives S0 (or zeros), so no later kernel reads S0 and S_final
+// may alias S0.  maps holds nmaps maps per sequence: nseg - 1 (the last segment's
+// is not needed), or nseg, and then S_final (if not null) receives the state after
+// the last segment.
 constexpr int SCAN_COLS = 16;
 __global__ void __launch_bounds__(DK)
 kda_segment_scan_kernel(const float* S0, const float* __restrict__ maps, float* __restrict__ start,
-                        int nseg, int H) {
+                        int nseg, int nmaps, int H, float* S_final) {
     __shared__ __align__(16) float sS[DK][SCAN_COLS];
     const int cb = blockIdx.x, h = blockIdx.y, n = blockIdx.z, i = threadIdx.x;
     const size_t col = (size_t)SCAN_COLS * cb;
@@ -1263,17 +1380,17 @@ kda_segment_scan_kernel(const float* S0, const float* __restrict__ maps, float* 
         const float4 f = src ? *reinterpret_cast<const float4*>(src + c) : make_float4(0.f, 0.f, 0.f, 0.f);
         cur[c] = f.x; cur[c + 1] = f.y; cur[c + 2] = f.z; cur[c + 3] = f.w;
     }
-    for (int g = 0;; ++g) {
+    for (int g = 0; g < nseg; ++g) {
         float* dst = start + ((((size_t)n * nseg + g) * H + h) * DK + i) * DV + col;
 #pragma unroll
         for (int c = 0; c < SCAN_COLS; c += 4)
             *reinterpret_cast<float4*>(dst + c) = make_float4(cur[c], cur[c + 1], cur[c + 2], cur[c + 3]);
-        if (g == nseg - 1) break;
+        if (g == nmaps) break;
         __syncthreads();   // the previous step's reads of sS are done
 #pragma unroll
         for (int c = 0; c < SCAN_COLS; ++c) sS[i][c] = cur[c];
         __syncthreads();
-        const float* Mrow = maps + ((((size_t)n * (nseg - 1) + g) * H + h) * DK + i) * (DK + DV);
+        const float* Mrow = maps + ((((size_t)n * nmaps + g) * H + h) * DK + i) * (DK + DV);
 #pragma unroll
         for (int c = 0; c < SCAN_COLS; ++c) cur[c] = Mrow[DK + col + c];   // N_g
         for (int j = 0; j < DK; j += 4) {
@@ -1291,6 +1408,12 @@ kda_segment_scan_kernel(const float* S0, const float* __restrict__ maps, float* 
                 }
             }
         }
+    }
+    if (nmaps == nseg && S_final) {
+        float* dst = S_final + (((size_t)n * H + h) * DK + i) * DV + col;
+#pragma unroll
+        for (int c = 0; c < SCAN_COLS; c += 4)
+            *reinterpret_cast<float4*>(dst + c) = make_float4(cur[c], cur[c + 1], cur[c + 2], cur[c + 3]);
     }
 }
 
@@ -1341,6 +1464,193 @@ kda_apply_maps_kernel(const float* S0, const float* __restrict__ maps, int G, in
         *reinterpret_cast<float4*>(dst + c) = make_float4(cur[c], cur[c + 1], cur[c + 2], cur[c + 3]);
 }
 
+// o += Qg S_g over the tokens of segment g: the last step of the split forward, whose
+// dual-mode pass left each segment's zero-start output O0 in o and its map rows Qg.
+// One CTA per (slice of up to CR_TILES 128-token tiles of a segment, head, sequence *
+// nseg + g), 128 threads, thread 0 issuing every copy and product.  S_g (fp32, from
+// the scan) becomes a bf16 MN-major B operand once; each tile of Qg (K-major A) gives
+// one M=128, N=128, K=128 product in TMEM (two accumulators, so that the next tile's
+// product runs beside this tile's additions); thread t adds row t of it to row t of
+// the o tile in shared memory, and the tile leaves by TMA store.  Qg and o tiles
+// arrive by TMA in three stages each, issued two to three tiles ahead: the pass is
+// bound by memory (256 bytes read twice and written once per token and head).  A
+// segment's ragged last tile is written row by row (a TMA box would spill into the
+// next segment's rows, which another CTA writes).
+constexpr int CR_TILE = 128;
+constexpr int CR_TILES = 64;
+constexpr int CR_THREADS = 128;
+constexpr int CR_STAGES = 3;
+constexpr uint32_t CR_OFF_S = 0;          // S_g bf16 [128 c][128 n], two [128][64] atoms
+constexpr uint32_t CR_OFF_G = 32768;      // Qg tiles [128 t][128 c] (two [128][64] atoms), 3 stages
+constexpr uint32_t CR_OFF_O = CR_OFF_G + CR_STAGES * 32768;   // o tiles, same layout, 3 stages
+constexpr uint32_t CR_OFF_BAR = CR_OFF_O + CR_STAGES * 32768; // uint64 x8: Qg (3), o (3), MMA (2)
+constexpr uint32_t CR_OFF_TMEM = CR_OFF_BAR + 64;
+constexpr uint32_t CR_SMEM = CR_OFF_TMEM + 16 + 1024;
+static_assert(CR_SMEM <= 232448, "correction kernel shared memory");
+
+__global__ void __launch_bounds__(CR_THREADS, 1)
+kda_segment_correct_kernel(const __grid_constant__ CUtensorMap tmG, const __grid_constant__ CUtensorMap tmO,
+                           const float* __restrict__ start, const int32_t* __restrict__ cu_seqlens,
+                           int64_t T, int H, int nseg, int skip_first, __nv_bfloat16* __restrict__ out,
+                           int* status) {
+    const int h = blockIdx.y, z = blockIdx.z, n = z / nseg, g = z % nseg;
+    if (skip_first && g == 0) return;   // S_0 = 0: nothing to add
+    int64_t bos, len;
+    seq_range(cu_seqlens, n, T, bos, len);
+    const int64_t nch = (len + C - 1) / C, cps = (nch + nseg - 1) / nseg;
+    const int64_t t1 = min(min((int64_t)(g + 1) * cps, nch) * C, len);
+    const int64_t s0 = min(min((int64_t)g * cps, nch) * C, len) + (int64_t)blockIdx.x * CR_TILES * CR_TILE;
+    if (s0 >= t1) return;   // (uniform over the CTA)
+    const int ntiles = (int)min((int64_t)CR_TILES, (t1 - s0 + CR_TILE - 1) / CR_TILE);
+
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t* sm = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
+    uint64_t* barG = reinterpret_cast<uint64_t*>(sm + CR_OFF_BAR);
+    uint64_t* barO = barG + 3;
+    uint64_t* barM = barG + 6;
+    uint32_t* sTmem = reinterpret_cast<uint32_t*>(sm + CR_OFF_TMEM);
+    __shared__ int s_fail;
+    const int tid = threadIdx.x, warp = tid >> 5;
+    if (tid == 0) {
+        for (int i = 0; i < 8; ++i) mbar_init(barG + i, 1);
+        mbar_fence_init();
+        s_fail = 0;
+    }
+    if (warp == 0) tmem_alloc(sTmem, 256);
+    auto tile_row = [&](int i) { return (int)(bos + s0 + (int64_t)i * CR_TILE); };
+    auto load_tile = [&](const CUtensorMap* map, uint8_t* dst, uint64_t* bar, int i) {
+        mbar_arrive_expect_tx(bar, 32768);
+#pragma unroll
+        for (int a = 0; a < 2; ++a)
+#pragma unroll
+            for (int b = 0; b < 2; ++b)
+                tma_load_2d(dst + a * 16384 + b * 8192, map, bar, h * DK + 64 * a, tile_row(i) + 64 * b);
+    };
+    auto issue_g = [&](int i) { load_tile(&tmG, sm + CR_OFF_G + (i % 3) * 32768, barG + i % 3, i); };
+    auto issue_o = [&](int i) { load_tile(&tmO, sm + CR_OFF_O + (i % 3) * 32768, barO + i % 3, i); };
+    uint32_t ng[3] = {0, 0, 0}, no[3] = {0, 0, 0};   // (thread 0) loads issued per stage
+    __syncthreads();
+    if (tid == 0) {
+        for (int i = 0; i < ntiles && i < 3; ++i) {
+            issue_g(i);
+            ++ng[i];
+            issue_o(i);
+            ++no[i];
+        }
+    }
+    // S_g as bf16: thread c writes row c (both 64-column atoms)
+    {
+        const float* src = start + (((size_t)z * H + h) * DK + tid) * DV;
+#pragma unroll
+        for (int blk = 0; blk < DV / 8; ++blk) {
+            const float4 f0 = *reinterpret_cast<const float4*>(src + 8 * blk);
+            const float4 f1 = *reinterpret_cast<const float4*>(src + 8 * blk + 4);
+            const float v[8] = {f0.x, f0.y, f0.z, f0.w, f1.x, f1.y, f1.z, f1.w};
+            *reinterpret_cast<uint4*>(sm + CR_OFF_S + (blk >> 3) * 16384 + swz(tid, blk & 7)) = pack8(v);
+        }
+    }
+    fence_async_smem();
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = *sTmem;
+    const uint32_t tl = (uint32_t)(32 * warp) << 16;
+    bool ok = true;
+    bool mma_out = false;   // (thread 0) a product committed and not yet seen complete
+    uint32_t mma_ph = 0, mma_b = 0;
+    auto product = [&](int i) {   // thread 0: tile i's product into accumulator i & 1
+        if (ok && !mbar_wait_ns(barG + i % 3, (uint32_t)(i / 3) & 1u, kWaitNs)) ok = false;
+        tc_fence_after();
+        if (!ok) return;
+        constexpr uint32_t id = idesc_bf16(128, 128, false, true);
+        const uint32_t a0 = smem_u32(sm + CR_OFF_G + (i % 3) * 32768), b0 = smem_u32(sm + CR_OFF_S);
+#pragma unroll
+        for (int ks = 0; ks < 8; ++ks)
+            mma_bf16(tmem + 128 * (i & 1), sdesc_sw128(a0 + (ks >> 2) * 16384 + (ks & 3) * 32),
+                     sdesc_sw128(b0 + ks * 2048, 1024, 16384), id, ks > 0);
+        mma_commit(barM + (i & 1));
+        mma_out = true;
+        mma_ph = (uint32_t)(i >> 1) & 1u;
+        mma_b = (uint32_t)(i & 1);
+    };
+    if (tid == 0 && ntiles > 0) product(0);
+    for (int i = 0; i < ntiles; ++i) {
+        // tile i's product is done: its Qg stage is free, the next product may start
+        bool w = __syncthreads_and(ok) && mbar_wait_ns(barM + (i & 1), (uint32_t)(i >> 1) & 1u, kWaitNs);
+        tc_fence_after();
+        if (!__syncthreads_and(w)) { ok = false; break; }
+        if (tid == 0) {
+            mma_out = false;
+            if (i + 3 < ntiles) { issue_g(i + 3); ++ng[i % 3]; }
+            if (i + 1 < ntiles) product(i + 1);
+        }
+        // row tid of the product onto row tid of the o tile
+        w = mbar_wait_ns(barO + i % 3, (uint32_t)(i / 3) & 1u, kWaitNs);
+        if (!__syncthreads_and(w)) { ok = false; break; }
+        const int64_t t = s0 + (int64_t)i * CR_TILE + tid;
+        const bool full = s0 + (int64_t)(i + 1) * CR_TILE <= t1;
+        uint8_t* ot = sm + CR_OFF_O + (i % 3) * 32768;
+#pragma unroll
+        for (int p = 0; p < 4; ++p) {
+            float acc[32];
+            tmem_ld32(tmem + tl + 128 * (i & 1) + 32 * p, acc);
+#pragma unroll
+            for (int ch = 0; ch < 4; ++ch) {
+                uint8_t* cell = ot + (p >> 1) * 16384 + swz(tid, 4 * (p & 1) + ch);
+                const uint4 raw = *reinterpret_cast<const uint4*>(cell);
+                const uint32_t wds[4] = {raw.x, raw.y, raw.z, raw.w};
+                float v[8];
+#pragma unroll
+                for (int e = 0; e < 4; ++e) {
+                    const float2 f = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&wds[e]));
+                    v[2 * e] = f.x + acc[8 * ch + 2 * e];
+                    v[2 * e + 1] = f.y + acc[8 * ch + 2 * e + 1];
+                }
+                const uint4 res = pack8(v);
+                if (full) {
+                    *reinterpret_cast<uint4*>(cell) = res;
+                } else if (t < t1) {
+                    reinterpret_cast<uint4*>(out + ((size_t)(bos + t) * H + h) * DV)[8 * (p >> 1) + 4 * (p & 1) + ch] = res;
+                }
+            }
+        }
+        fence_async_smem();
+        tc_fence_before();
+        __syncthreads();
+        tc_fence_after();
+        if (tid == 0) {
+            if (full) {
+#pragma unroll
+                for (int a = 0; a < 2; ++a)
+#pragma unroll
+                    for (int b = 0; b < 2; ++b)
+                        tma_store_2d(&tmO, ot + a * 16384 + b * 8192, h * DV + 64 * a, tile_row(i) + 64 * b);
+                bulk_commit_group();
+            }
+            // the o stage of tile i - 1 has been read by its store: tile i + 2 goes there
+            if (i >= 1 && i + 2 < ntiles) {
+                if (full) bulk_wait_read_1();   // (the store just issued may still be reading)
+                else bulk_wait_read_all();
+                issue_o(i + 2);
+                ++no[(i + 2) % 3];
+            }
+        }
+    }
+    if (!ok && tid == 0) {   // let this CTA's own copies and product in flight finish (bounded)
+        s_fail = 1;
+        for (int st = 0; st < 3; ++st) {
+            if (ng[st]) mbar_wait_ns(barG + st, (ng[st] - 1) & 1u, kWaitNs);
+            if (no[st]) mbar_wait_ns(barO + st, (no[st] - 1) & 1u, kWaitNs);
+        }
+        if (mma_out) mbar_wait_ns(barM + mma_b, mma_ph, kWaitNs);
+    }
+    if (tid == 0) bulk_wait_all();   // every o store has completed before shared memory goes
+    tc_fence_before();
+    __syncthreads();
+    if (s_fail && tid == 0) atomicExch(status, 1);
+    if (warp == 0) tmem_dealloc(tmem, 256);
+}
+
 // ---------------------------------------------------------------- host side
 
 typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
@@ -1382,18 +1692,18 @@ bool make_tc_maps(TcMaps* m, const void* q, const void* k, const void* v, const 
            tc::make_map(&m->o, out ? out : v, rows, H);
 }
 
-template <bool kCtaStatus, bool kSummary, bool kFused = false, bool kRecord = false>
+template <bool kCtaStatus, bool kSummary, bool kFused = false, bool kRecord = false,
+          bool kDual = false>
 static cudaError_t launch_tc_t(const TcMaps& m, const void* beta, const float* S0, const int32_t* cu,
                                int nseq, void* out, float* S_final, int64_t T, int H, int* status,
                                const tc::Segments& seg, cudaStream_t stream) {
-    cudaError_t e = cudaFuncSetAttribute(tc::kda_chunk_tc_kernel<kCtaStatus, kSummary, kFused, kRecord>,
-                                         cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         (int)tc::SMEM_BYTES);
+    constexpr uint32_t smem = kDual ? tc::dual::SMEM_BYTES : tc::SMEM_BYTES;
+    auto* kern = tc::kda_chunk_tc_kernel<kCtaStatus, kSummary, kFused, kRecord, kDual>;
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
     dim3 grid(1, H, nseq * seg.per_seq);
-    tc::kda_chunk_tc_kernel<kCtaStatus, kSummary, kFused, kRecord><<<grid, tc::NTHREADS, tc::SMEM_BYTES, stream>>>(
-        m.q, m.k, m.a, m.v, m.o, (const __nv_bfloat16*)beta, S0, cu, (__nv_bfloat16*)out, S_final, T, H,
-        status, seg);
+    kern<<<grid, tc::NTHREADS, smem, stream>>>(m.q, m.k, m.a, m.v, m.o, (const __nv_bfloat16*)beta, S0,
+                                               cu, (__nv_bfloat16*)out, S_final, T, H, status, seg);
     return cudaGetLastError();
 }
 
@@ -1429,41 +1739,54 @@ cudaError_t launch_chunk_tc_record(const void* q, const void* k, const void* v, 
                                                   status, whole, stream);
 }
 
-// Floats of workspace the split forward uses: the segment maps [M | N] and the
-// segment start states.
-size_t chunk_tc_segmented_workspace_floats(int64_t nseq, int H, int nseg) {
+// Bytes of workspace the split forward uses: every segment's map [M | N] and start
+// state (fp32), and the map rows Qg of every token (bf16, like the output).
+size_t chunk_tc_segmented_workspace_bytes(int64_t nseq, int64_t rows, int H, int nseg) {
     if (nseg < 2) return 0;
-    return (size_t)nseq * H * ((size_t)(nseg - 1) * tc::DK * (tc::DK + tc::DV) +
-                               (size_t)nseg * tc::DK * tc::DV);
+    return sizeof(float) * (size_t)nseq * H * nseg * tc::DK * ((tc::DK + tc::DV) + tc::DV) +
+           sizeof(__nv_bfloat16) * (size_t)rows * H * tc::DK;
 }
 
-// The forward split along time into nseg segments per sequence: three launches
-// (segment maps, scan of the start states, forward of every segment).
+// The forward split along time into nseg segments per sequence: three launches.
+// (1) Every segment in the dual mode: its map [M | N], its output from a zero start
+// state (into out) and its map rows Qg; (2) the fp32 scan of the start states S_g,
+// which also gives S_final; (3) o += Qg S_g on the tensor cores.
 cudaError_t launch_chunk_tc_segmented(const void* q, const void* k, const void* v,
                                       const void* alpha, const void* beta, const float* S0,
                                       const int32_t* cu, int nseq, void* out, float* S_final,
-                                      int64_t rows, int64_t T, int H, int nseg, float* workspace,
+                                      int64_t rows, int64_t T, int H, int nseg, void* workspace,
                                       int* status, cudaStream_t stream, int fused) {
     if (nseg < 2 || nseq * (int64_t)nseg > 65535) return cudaErrorInvalidValue;
     TcMaps m;
     if (!make_tc_maps(&m, q, k, v, alpha, out, rows, H)) return cudaErrorInvalidValue;
-    float* maps = workspace;
-    float* start = workspace + (size_t)nseq * H * (nseg - 1) * tc::DK * (tc::DK + tc::DV);
-    const tc::Segments summary{nseg, nseg - 1, nullptr, maps};
-    cudaError_t e = fused ? launch_tc_t<false, true, true>(m, beta, nullptr, cu, nseq, nullptr,
-                                                           nullptr, T, H, status, summary, stream)
-                          : launch_tc_t<false, true>(m, beta, nullptr, cu, nseq, nullptr, nullptr, T,
-                                                     H, status, summary, stream);
+    float* maps = static_cast<float*>(workspace);
+    float* start = maps + (size_t)nseq * H * nseg * tc::DK * (tc::DK + tc::DV);
+    __nv_bfloat16* qg = reinterpret_cast<__nv_bfloat16*>(start + (size_t)nseq * H * nseg * tc::DK * tc::DV);
+    CUtensorMap tmG;
+    if (!tc::make_map(&tmG, qg, rows, H)) return cudaErrorInvalidValue;
+    tc::Segments dual{nseg, nseg, nullptr, maps};
+    dual.qg = qg;
+    cudaError_t e = fused ? launch_tc_t<false, true, true, false, true>(m, beta, nullptr, cu, nseq, out,
+                                                                        nullptr, T, H, status, dual, stream)
+                          : launch_tc_t<false, true, false, false, true>(m, beta, nullptr, cu, nseq, out,
+                                                                         nullptr, T, H, status, dual, stream);
     if (e != cudaSuccess) return e;
     tc::kda_segment_scan_kernel<<<dim3(tc::DV / tc::SCAN_COLS, H, nseq), tc::DK, 0, stream>>>(
-        S0, maps, start, nseg, H);
+        S0, maps, start, nseg, nseg, H, S_final);
     e = cudaGetLastError();
     if (e != cudaSuccess) return e;
-    const tc::Segments fwd{nseg, nseg, start, nullptr};
-    return fused ? launch_tc_t<false, false, true>(m, beta, nullptr, cu, nseq, out, S_final, T, H,
-                                                   status, fwd, stream)
-                 : launch_tc_t<false, false>(m, beta, nullptr, cu, nseq, out, S_final, T, H, status,
-                                             fwd, stream);
+    e = cudaFuncSetAttribute(tc::kda_segment_correct_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             (int)tc::CR_SMEM);
+    if (e != cudaSuccess) return e;
+    // slices per segment: a segment holds at most ceil(chunks / nseg) chunks of the longest
+    // sequence, which is at most T tokens (packed: the whole batch)
+    const int64_t cps = ((T + tc::C - 1) / tc::C + nseg - 1) / nseg;
+    const int64_t slice_tokens = (int64_t)tc::CR_TILES * tc::CR_TILE;
+    const int64_t nsl = (cps * tc::C + slice_tokens - 1) / slice_tokens;
+    const int slices = (int)(nsl > 1 ? nsl : 1);
+    tc::kda_segment_correct_kernel<<<dim3(slices, H, nseq * nseg), tc::CR_THREADS, tc::CR_SMEM, stream>>>(
+        tmG, m.o, start, cu, T, H, nseg, S0 == nullptr ? 1 : 0, static_cast<__nv_bfloat16*>(out), status);
+    return cudaGetLastError();
 }
 
 // Segment maps of whole sequences: maps [nseq][H][DK][DK + DV] fp32 with

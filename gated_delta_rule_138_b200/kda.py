@@ -83,6 +83,8 @@ def load_library(build_if_missing: bool = True) -> ctypes.CDLL:
     lib.kda_segment_scan.argtypes = [vp, vp, i32, vp, i32, i32, i32, i32, vp]
     lib.kda_forward_segments.restype = i32
     lib.kda_forward_segments.argtypes = [i32, i64, i32, i32]
+    lib.kda_release_workspace.restype = ctypes.c_int
+    lib.kda_release_workspace.argtypes = []
     lib.kda_selftest_timeout.restype = ctypes.c_int
     lib.kda_selftest_timeout.argtypes = [ctypes.c_uint64, vp]
     lib.kda_forward_noalloc.restype = ctypes.c_int
@@ -159,6 +161,12 @@ def kda_device_status(stream=None) -> None:
 def kda_forward_segments(num_seqs: int, tokens_per_seq: int, H: int, num_sms: int = 0) -> int:
     """Time segments per sequence the tensor-core forward uses (1 = unsplit)."""
     return int(load_library().kda_forward_segments(num_seqs, tokens_per_seq, H, num_sms))
+
+
+def kda_release_workspace() -> None:
+    """Hand back the device memory the current device's split-forward workspace
+    pool keeps between calls."""
+    _check("kda_release_workspace", load_library().kda_release_workspace())
 
 
 def kda_selftest_timeout(limit_ns: int = 1_000_000, stream=None) -> None:

@@ -223,26 +223,39 @@ const char* kda_status_string(kda_status_t status);
  * Bytes of device workspace kda_forward uses for a dense batch of these sizes:
  * the per-device status word (4 bytes, allocated on the first tensor-core call
  * on a device and kept until exit) plus, when the tensor-core path splits the
- * sequences along time (see kda_forward_segments), the segment maps and start
- * states: B * H * ((g - 1) * d_k * (d_k + d_v) + g * d_k * d_v) fp32 values for
- * g segments.  That part is allocated stream-ordered (cudaMallocAsync) on the
- * call's stream and freed (cudaFreeAsync) behind the call's kernels; if it
- * cannot be allocated the call runs unsplit.  Host-only.
+ * sequences along time (see kda_forward_segments), every segment's map and
+ * start state, B * H * g * d_k * (d_k + 2 d_v) fp32 values for g segments, and
+ * the map rows Qg of every token, B * T * H * d_k bf16 values (as large as the
+ * output).  That part is allocated stream-ordered on the call's stream from a
+ * memory pool of this library, which keeps what it has reserved for later calls
+ * (kda_release_workspace hands it back), and freed into that pool behind the
+ * call's kernels; if it cannot be allocated the call runs unsplit.  Host-only.
  */
 size_t kda_forward_workspace_bytes(int32_t B, int64_t T, int32_t H, int32_t d_k,
                                    int32_t d_v, int32_t chunk);
+
+/*
+ * Returns the device memory that the current device's workspace pool (see
+ * kda_forward_workspace_bytes) keeps between calls, except what work still
+ * queued on a stream uses.  Returns KDA_OK, or KDA_ERR_CUDA.  Later calls
+ * allocate again as needed.
+ */
+kda_status_t kda_release_workspace(void);
 
 /*
  * Time segments per sequence that kda_forward's tensor-core path uses for
  * num_seqs sequences of tokens_per_seq tokens (a packed batch uses its mean
  * length) and H heads on a GPU with num_sms SMs (0: the current device's, 148
  * if none is visible).  1 = each (sequence, head) runs whole on one CTA.  With
- * g > 1, every sequence's chunks are cut into g runs; a first kernel computes
- * each run's affine state map S_end = M S_start + N, a scan kernel chains the
- * start states in fp32, and the forward kernel runs all runs in parallel (the
- * article's paragraph 3: states reconstructed across chunks by a prefix scan).
- * The choice only balances the SMs: every g gives the same result up to
- * rounding.  Host-only.
+ * g > 1, every sequence's chunks are cut into g runs, all run in parallel by one
+ * kernel from a zero start: each run's affine state map S_end = M S_start + N,
+ * its output O0 from a zero start state and the rows Qg that carry the start
+ * state into the output (o = O0 + Qg S_start, the output being affine in the
+ * start state too); a scan kernel chains the start states in fp32 (and gives
+ * S_final), and a last kernel adds Qg S_start to the output (the article's
+ * paragraph 3: states reconstructed across chunks by a prefix scan).  The
+ * choice only balances the SMs: every g gives the same result up to rounding.
+ * Host-only.
  */
 int32_t kda_forward_segments(int32_t num_seqs, int64_t tokens_per_seq, int32_t H, int32_t num_sms);
 

@@ -90,6 +90,21 @@ def test_workspace_query_is_host_only():
     assert kda.kda_forward_workspace_bytes(8, 4096, 32, 128, 128, 64) >= 0
 
 
+def test_forward_workspace_covers_the_split():
+    """The split forward's workspace: per segment a map [M | N] and a start state
+    (fp32, d_k (d_k + 2 d_v) values per head and sequence) and, for every token, its
+    map row Qg (bf16, as large as the output); unsplit calls need only the status word."""
+    assert kda.kda_forward_segments(8, 4096, 32) == 1
+    assert kda.kda_forward_workspace_bytes(8, 4096, 32, 128, 128, 64) == 4
+    T = 1 << 20
+    g = kda.kda_forward_segments(1, T, 32)
+    assert g > 1
+    assert kda.kda_forward_workspace_bytes(1, T, 32, 128, 128, 64) == \
+        4 + 4 * g * 32 * 128 * (128 + 2 * 128) + 2 * T * 32 * 128
+    # the fp32 CUDA-core path never splits
+    assert kda.kda_forward_workspace_bytes(1, T, 32, 64, 64, 64) == 4
+
+
 def test_selftest_rejects_bad_limit():
     lib = kda.load_library()
     assert lib.kda_selftest_timeout(0, None) == 1
@@ -106,7 +121,8 @@ def test_time_segment_choice():
     assert seg(1, 64 * 32, 1, 148) == 2
     g = seg(1, 1 << 20, 32, 148)                 # 32 CTAs on 148 SMs, 16384 chunks each
     assert 4 <= g <= 64
-    assert (32 * g) % 148 > 100 or (32 * g) <= 148  # the last wave is mostly full
+    last = (32 * g) % 148
+    assert last == 0 or last > 100 or (32 * g) <= 148  # the last wave is mostly full
     assert seg(0, 100, 4, 148) == 1 and seg(1, 0, 4, 148) == 1
     for units_h in (1, 2, 4, 8, 16, 32, 64):
         assert 1 <= seg(1, 1 << 22, units_h, 148) <= 64

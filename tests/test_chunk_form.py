@@ -246,3 +246,35 @@ def test_time_segments_scan_equals_oracle(T, nseg, extreme):
         outs.append(o)
     np.testing.assert_allclose(np.concatenate(outs), ref_o[0, :, 0], rtol=1e-10, atol=1e-12)
     np.testing.assert_allclose(S_end, ref_S[0, 0], rtol=1e-10, atol=1e-12)
+
+
+@pytest.mark.parametrize("T,nseg,extreme", [(300, 3, False), (256, 4, True), (130, 5, False), (40, 5, False)])
+def test_split_forward_zero_start_outputs_and_map_rows(T, nseg, extreme):
+    """The split forward's one pass per segment: the chunk recurrence on the
+    widened state [M | N] from [I | 0], with values [0 | V], ends at the
+    segment's map and outputs [Qg | O0], O0 the outputs from a zero start state.
+    The output is affine in the start state like the state itself, so with the
+    start states chained by the maps, o = O0 + Qg S_g is the token recurrence's
+    output and the last map applied to the last start state its final state (the
+    prefix scan of the article's paragraph 3)."""
+    C, dk, dv = 16, 16, 8
+    q, k, v, al, be, S0 = (x.astype(np.float64) for x in _case(2100 + T, T, dk, dv, extreme))
+    ref_o, ref_S = oracle.forward(*(x[None, :, None].astype(np.float32) for x in (q, k, v, al, be)),
+                                  S0[None, None].astype(np.float32))
+    nch = -(-T // C)
+    cps = -(-nch // nseg)
+    bounds = [(min(g * cps * C, T), min((g + 1) * cps * C, T)) for g in range(nseg)]
+    start = S0
+    outs = []
+    for t0, t1 in bounds:
+        v_wide = np.concatenate([np.zeros((t1 - t0, dk)), v[t0:t1]], axis=1)
+        if t1 > t0:
+            o_wide, MN = chunk_forward_one(q[t0:t1], k[t0:t1], v_wide, al[t0:t1], be[t0:t1],
+                                           np.concatenate([np.eye(dk), np.zeros((dk, dv))], axis=1), C)
+            Qg, O0 = o_wide[:, :dk], o_wide[:, dk:]
+            outs.append(O0 + Qg @ start)
+        else:   # an empty segment: the identity map
+            MN = np.concatenate([np.eye(dk), np.zeros((dk, dv))], axis=1)
+        start = MN[:, :dk] @ start + MN[:, dk:]
+    np.testing.assert_allclose(np.concatenate(outs), ref_o[0, :, 0], rtol=1e-10, atol=1e-12)
+    np.testing.assert_allclose(start, ref_S[0, 0], rtol=1e-10, atol=1e-12)
