@@ -68,6 +68,11 @@ WORKLOADS = {
     "bf16_B1_T1M_H32_d128": Workload("bf16_B1_T1M_H32_d128", "forward", "bf16", H=32,
                                      dk=128, dv=128, B=1, T=1 << 20, s0=False,
                                      special_alpha=True, seed=1002),
+    # the same recipe on 65,536 tokens: a small case of the same time-split kernels (for
+    # profiling captures that must stay a few GB on the device)
+    "bf16_B1_T64K_H32_d128": Workload("bf16_B1_T64K_H32_d128", "forward", "bf16", H=32,
+                                      dk=128, dv=128, B=1, T=1 << 16, s0=False,
+                                      special_alpha=True, seed=1002),
     # single-token decode: 256 sequences x 32 heads, 128 consecutive steps
     "decode_N256_H32_d128": Workload("decode_N256_H32_d128", "decode", "bf16", H=32,
                                      dk=128, dv=128, B=256, steps=128, s0=True, seed=1003),
