@@ -105,6 +105,12 @@ def test_forward_workspace_covers_the_split():
     assert kda.kda_forward_workspace_bytes(1, T, 32, 64, 64, 64) == 4
 
 
+def test_release_workspace_answers_without_a_pool():
+    """Trimming the split forward's workspace pool launches nothing: OK when no pool
+    exists yet (or CUDA's error code when no device is visible), never a crash."""
+    assert kda.load_library().kda_release_workspace() in (0, 3)
+
+
 def test_selftest_rejects_bad_limit():
     lib = kda.load_library()
     assert lib.kda_selftest_timeout(0, None) == 1
