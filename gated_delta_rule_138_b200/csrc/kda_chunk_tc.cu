@@ -220,7 +220,8 @@ template <bool kCtaStatus, bool kSummary, bool kFused, bool kRecord = false, boo
 __global__ void __launch_bounds__(NTHREADS, 1)
 kda_chunk_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                     const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmV,
-                    const __grid_constant__ CUtensorMap tmO, const __nv_bfloat16* __restrict__ beta, const float* S0,
+                    const __grid_constant__ CUtensorMap tmO, const __grid_constant__ CUtensorMap tmG,
+                    const __nv_bfloat16* __restrict__ beta, const float* S0,
                     const int32_t* __restrict__ cu_seqlens, __nv_bfloat16* __restrict__ out,
                     float* S_final, int64_t T, int H, int* status, const Segments seg) {
     extern __shared__ uint8_t smem_raw[];
@@ -420,7 +421,9 @@ kda_chunk_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_consta
     // A full chunk's O is staged in the q buffer the next q load will use (row-major,
     // 128-byte swizzled, the TMA box layout) and written by one TMA store; a
     // partial last chunk is stored row by row.  The dual mode's [Qg | O0] (an M=64
-    // accumulator, N=256) leaves row by row: warps of column half 0 write Qg, half 1 O0.
+    // accumulator, N=256; warps of column half 0 hold Qg, half 1 O0) is staged the same
+    // way, O0 in that q buffer and Qg in the alpha / v buffer (alpha is read, v not yet
+    // loaded): both are free from here until the control thread's stores at barrier A.
     auto finish_prev = [&](int64_t prow0, int pLc, uint8_t* stage) {
         wait_mma();
         const int c = 32 * q4 + lane;
@@ -447,16 +450,30 @@ kda_chunk_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_consta
         if constexpr (kSummary) {
             if constexpr (kDual) {
                 const int r = 16 * q4 + lane;
-                __nv_bfloat16* dst_rows = hf == 0 ? seg.qg : out;
-                uint4* dst = reinterpret_cast<uint4*>(dst_rows + ((size_t)(prow0 + r) * H + h) * DK);
-                const bool wr = lane < 16 && r < pLc;
+                if (pLc == C) {
+                    uint8_t* stg = (hf == 0 ? sAl : stage) + r * 128;   // row r of both atoms
+                    const uint32_t rx = (uint32_t)(r & 7);
+#pragma unroll 1
+                    for (int p = 0; p < 4; ++p) {   // (32-column pieces: fewer live registers)
+                        float v[32];
+                        tmem_ld32(tmem + tlane + TM_WK + 128 * hf + 32 * p, v);
+                        if (lane < 16) {
 #pragma unroll
-                for (int p = 0; p < 4; ++p) {   // (32-column pieces: fewer live registers)
-                    float v[32];
-                    tmem_ld32(tmem + tlane + TM_WK + 128 * hf + 32 * p, v);
-                    if (wr) {
+                            for (int ch = 0; ch < 4; ++ch)
+                                *reinterpret_cast<uint4*>(stg + (p >> 1) * 8192 + (((4 * (p & 1) + ch) ^ rx) << 4)) =
+                                    pack8(&v[8 * ch]);
+                        }
+                    }
+                } else {
+                    uint4* dst = reinterpret_cast<uint4*>((hf == 0 ? seg.qg : out) + ((size_t)(prow0 + r) * H + h) * DK);
 #pragma unroll
-                        for (int ch = 0; ch < 4; ++ch) dst[4 * p + ch] = pack8(&v[8 * ch]);
+                    for (int p = 0; p < 4; ++p) {
+                        float v[32];
+                        tmem_ld32(tmem + tlane + TM_WK + 128 * hf + 32 * p, v);
+                        if (lane < 16 && r < pLc) {
+#pragma unroll
+                            for (int ch = 0; ch < 4; ++ch) dst[4 * p + ch] = pack8(&v[8 * ch]);
+                        }
                     }
                 }
             }
@@ -485,6 +502,14 @@ kda_chunk_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_consta
     auto store_o = [&](uint8_t* stage, int64_t prow0) {   // control thread, after a barrier
 #pragma unroll
         for (int a = 0; a < 2; ++a) tma_store_2d(&tmO, stage + a * 8192, h * DV + 64 * a, (int)prow0);
+        bulk_commit_group();
+    };
+    auto store_dual = [&](uint8_t* stage, int64_t prow0) {   // dual mode: O0 and Qg of a full chunk
+#pragma unroll
+        for (int a = 0; a < 2; ++a) {
+            tma_store_2d(&tmO, stage + a * 8192, h * DV + 64 * a, (int)prow0);
+            tma_store_2d(&tmG, sAl + a * 8192, h * DK + 64 * a, (int)prow0);
+        }
         bulk_commit_group();
     };
 
@@ -1201,9 +1226,15 @@ kda_chunk_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_consta
                 issued(tka);
             }
             if (kDual && ok) {
-                issue_v(row0);   // alpha has left the buffer v takes
+                // the previous chunk (full: only a segment's last chunk is not) leaves from
+                // its staging buffers; v and the next q go there once the stores have read them
+                if (chunk > 0) {
+                    store_dual(sQ + ((chunk + 1) & 1) * 16384, row0 - C);
+                    bulk_wait_read_all();
+                }
+                issue_v(row0);
                 issued(tv);
-                if (chunk + 1 < nchunks) {   // the other q buffer's O products are done
+                if (chunk + 1 < nchunks) {
                     issue_q(row0 + C, (chunk + 1) & 1);
                     issued(tq);
                 }
@@ -1306,9 +1337,11 @@ kda_chunk_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_consta
 
     if (!ok) atomicExch(sFlag, 1);
     __syncthreads();
-    if (!kSummary && ctl) {
-        if (!kRecord && nchunks > 0 && !broke && !*sFlag && last_Lc == C)
-            store_o(last_stage, bos + (int64_t)(nchunks - 1) * C);
+    if ((!kSummary || kDual) && ctl) {
+        if (!kRecord && nchunks > 0 && !broke && !*sFlag && last_Lc == C) {
+            if constexpr (kDual) store_dual(last_stage, bos + (int64_t)(nchunks - 1) * C);
+            else store_o(last_stage, bos + (int64_t)(nchunks - 1) * C);
+        }
         bulk_wait_all();   // every O store has completed before shared memory is released
     }
     if (*sFlag && ctl) {
@@ -1696,14 +1729,16 @@ template <bool kCtaStatus, bool kSummary, bool kFused = false, bool kRecord = fa
           bool kDual = false>
 static cudaError_t launch_tc_t(const TcMaps& m, const void* beta, const float* S0, const int32_t* cu,
                                int nseq, void* out, float* S_final, int64_t T, int H, int* status,
-                               const tc::Segments& seg, cudaStream_t stream) {
+                               const tc::Segments& seg, cudaStream_t stream,
+                               const CUtensorMap* tmG = nullptr) {
     constexpr uint32_t smem = kDual ? tc::dual::SMEM_BYTES : tc::SMEM_BYTES;
     auto* kern = tc::kda_chunk_tc_kernel<kCtaStatus, kSummary, kFused, kRecord, kDual>;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
     dim3 grid(1, H, nseq * seg.per_seq);
-    kern<<<grid, tc::NTHREADS, smem, stream>>>(m.q, m.k, m.a, m.v, m.o, (const __nv_bfloat16*)beta, S0,
-                                               cu, (__nv_bfloat16*)out, S_final, T, H, status, seg);
+    kern<<<grid, tc::NTHREADS, smem, stream>>>(m.q, m.k, m.a, m.v, m.o, tmG ? *tmG : m.o,
+                                               (const __nv_bfloat16*)beta, S0, cu, (__nv_bfloat16*)out,
+                                               S_final, T, H, status, seg);
     return cudaGetLastError();
 }
 
@@ -1767,9 +1802,11 @@ cudaError_t launch_chunk_tc_segmented(const void* q, const void* k, const void* 
     tc::Segments dual{nseg, nseg, nullptr, maps};
     dual.qg = qg;
     cudaError_t e = fused ? launch_tc_t<false, true, true, false, true>(m, beta, nullptr, cu, nseq, out,
-                                                                        nullptr, T, H, status, dual, stream)
+                                                                        nullptr, T, H, status, dual, stream,
+                                                                        &tmG)
                           : launch_tc_t<false, true, false, false, true>(m, beta, nullptr, cu, nseq, out,
-                                                                         nullptr, T, H, status, dual, stream);
+                                                                         nullptr, T, H, status, dual, stream,
+                                                                         &tmG);
     if (e != cudaSuccess) return e;
     tc::kda_segment_scan_kernel<<<dim3(tc::DV / tc::SCAN_COLS, H, nseq), tc::DK, 0, stream>>>(
         S0, maps, start, nseg, nseg, H, S_final);
