@@ -117,12 +117,40 @@ def load_peaks():
         return dict(FALLBACK_PEAKS), "fallback"
 
 
+def code_only(src: str) -> str:
+    """C/C++/CUDA source without its comments, whitespace runs collapsed to one
+    space: what the compiler sees, so that a record survives edits to comments only."""
+    out, i, n = [], 0, len(src)
+    while i < n:
+        c = src[i]
+        if c in "\"'":   # a string or character literal, kept whole
+            j = i + 1
+            while j < n and src[j] != c:
+                j += 2 if src[j] == "\\" else 1
+            out.append(src[i:j + 1])
+            i = j + 1
+        elif src.startswith("//", i):
+            j = src.find("\n", i)
+            i = n if j < 0 else j
+        elif src.startswith("/*", i):
+            j = src.find("*/", i + 2)
+            i = n if j < 0 else j + 2
+            out.append(" ")
+        else:
+            out.append(c)
+            i += 1
+    return " ".join("".join(out).split())
+
+
 def kernel_source_digest(names: str) -> str:
-    """sha256 (16 hex digits) of the concatenated csrc files, comma-separated."""
+    """sha256 (16 hex digits) of the code (comments and whitespace runs aside, see
+    code_only) of the comma-separated csrc files, in order."""
     h = hashlib.sha256()
     for name in names.split(","):
-        with open(os.path.join(ROOT, "gated_delta_rule_138_b200", "csrc", name), "rb") as fh:
-            h.update(fh.read())
+        with open(os.path.join(ROOT, "gated_delta_rule_138_b200", "csrc", name),
+                  encoding="utf-8") as fh:
+            h.update(code_only(fh.read()).encode("utf-8"))
+        h.update(b"\0")
     return h.hexdigest()[:16]
 
 

@@ -45,9 +45,11 @@
 // segment the state map is affine, S_end = M S_start + N with M (d_k x d_k) and
 // N (d_k x d_v); per chunk M_c = Diag(gamma_C) - (k*eta)^T W and
 // N_c = (k*eta)^T Tb V.  The same kernel in "summary" mode runs the chunk
-// recurrence on [M | N] from [I | 0] (no outputs); a small scan kernel chains
-// S_{g+1} = M_g S_g + N_g in fp32; the forward kernel then runs every segment
-// from its own start state.
+// recurrence on [M | N] from [I | 0] without outputs (the maps of whole
+// sequences); in "dual" mode it also forms that widened state's outputs
+// [Qg | O0], whence o = O0 + Qg S_start.  The split forward runs every segment
+// in the dual mode, chains S_{g+1} = M_g S_g + N_g in fp32 with a small scan
+// kernel, and adds Qg S_g to the outputs with a last tensor-core kernel.
 #include <cuda.h>
 
 #include "kda_common.cuh"
@@ -181,6 +183,8 @@ struct Segments {
     int nseg;             // segments per sequence (1: whole sequences)
     int per_seq;          // segment CTAs per sequence in this launch
     const float* start;   // forward with nseg > 1: start states [nseq * nseg, H, DK, DV]
+                          // (a form no entry point launches now: the split forward takes
+                          // the dual mode and adds the start states' share afterwards)
     float* maps;          // summary: [M | N] fp32 [nseq * per_seq, H, DK, DK + DV]
     // state slots (whole sequences only): sequence n reads S0 and writes S_final at
     // slot slots[n] of a pool of num_slots states; a slot outside [0, num_slots)

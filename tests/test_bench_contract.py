@@ -157,3 +157,16 @@ def test_batch_override_is_for_dense_forward_workloads_only():
                        timeout=120)
     assert r.returncode == 2
     assert "--batch applies to the dense forward workloads" in r.stderr
+
+
+def test_traffic_records_are_keyed_to_code_not_comments():
+    """A DRAM-traffic record stays valid across edits to comments and whitespace only,
+    and goes stale on any change to the code itself (string and character literals
+    included)."""
+    a = "int f(int x) { return x + 1; }  // one\n/* two */ const char* s = \"a // b\";\n"
+    b = "int f(int x) {\n  return x + 1;   /* edited */ }\nconst char* s = \"a // b\";  // new\n"
+    code_only = _bench().code_only
+    assert code_only(a) == code_only(b)
+    assert code_only(a) != code_only(a.replace("x + 1", "x + 2"))
+    assert code_only(a) != code_only(a.replace("a // b", "a // c"))
+    assert code_only("char c = '/'; // x\n") == "char c = '/';"
