@@ -38,7 +38,9 @@
 // gate phase has consumed them, q (double buffered) after the [A/beta ; P] MMA,
 // v once U has consumed it.  O leaves through TMA stores from a staging tile.
 // TMEM (512 columns): S fp32 [0,128), O [128,256), scratch accumulators
-// [256,384), U [384,512) (first (k*gamma) S_start, then U).
+// [256,384), U [384,512) (first (k*gamma) S_start, then U).  Summary and dual
+// modes: [M | N] fp32 [0,256); [256,512) holds in turn [A/beta ; P], the solve
+// products, W, [U_M | U_N] and (dual) [Qg | O0].
 //
 // Long sequences with few (sequence, head) pairs are also split along time
 // into segments (the prefix scan of paragraph 3, within one GPU).  Over a
@@ -1076,13 +1078,18 @@ kda_chunk_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_consta
     // group in order.  Groups without a commit ride on the next group's commit (the
     // tensor pipe runs one thread's MMAs in issue order).
     //   barrier A (operands of [A/beta ; P]):  [A/beta ; P] (commit); forward: (k*gamma) S_start
-    //                                            (own barrier), then (q*gamma) S_start
+    //                                            (own barrier), then (q*gamma) S_start; dual:
+    //                                            the previous chunk's [Qg | O0] stores, then the
+    //                                            loads of this chunk's v and the next q there
     //   barrier B (tf32 solve operands):          the two chained 32 -> 64 solve products
     //                                            (the second reads the first from TMEM; commit)
     //   barrier D (Tb):                          forward: U = Tb (V - (k*gamma) S) (commit);
     //                                            summary: W = Tb (k*gamma) (commit), then Tb V
+    //                                            (dual: its own commit, then the next alpha load)
     //   barrier E (-W, summary only):            [U_M | U_N] += -W [M | N] (commit)
-    //   barrier F (U):                           S += (k*eta)^T U and O += P U (commit)
+    //   barrier F (U):                           S += (k*eta)^T U and O += P U (commit); dual:
+    //                                            [M | N] += (k*eta)^T [U_M | U_N] and
+    //                                            [Qg | O0] = (q*gamma) [M | N] + P [U_M | U_N]
     const uint32_t idM64 = idesc_bf16(64, 128, false, true);   // M=64, N=128, B MN-major
     auto mma_ap = [&]() {
         const uint32_t l0 = smem_u32(sX + X_L), r0 = smem_u32(sX + X_R);
