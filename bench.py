@@ -422,6 +422,22 @@ def _parity_stats(x, ref, time_axis):
     return {"rel_l2": glob, "worst_head": worst_slab, "worst_row": worst_row}
 
 
+def parity_ok(par, bar):
+    """False if a sampled comparison is not finite or exceeds its bar (global and
+    worst-slab errors within `bar`, worst row within 5 x `bar`, as in the tests)."""
+    import math
+    for key in ("o", "S_final"):
+        st = (par or {}).get(key)
+        if not st:
+            continue
+        vals = (st["rel_l2"], st["worst_head"], st["worst_row"])
+        if not all(math.isfinite(v) for v in vals):
+            return False
+        if vals[0] > bar or vals[1] > bar or vals[2] > 5 * bar:
+            return False
+    return True
+
+
 def bench_parity(w, inp, out, Sf, max_tokens=8192):
     """The bench's own outputs against the oracle on sampled (sequence, head) pairs:
     o over the first `max_tokens` tokens of each pair, S_final where the pair's
@@ -544,6 +560,7 @@ def run_ours(args, w):
 
     rank, world, local = dist_setup(args.gpus)
     dev = torch.device("cuda", local)
+    parity_failed = False
     from gated_delta_rule_138_b200 import ranks
     inp = make_inputs(w, dev, ranks.rank_seed_offset(rank))
     tokens, n_th, n_sh = counts(w, inp)
@@ -711,7 +728,12 @@ def run_ours(args, w):
         }
         if w.kind in ("forward", "varlen") and not args.backward and not seqpar \
                 and not args.fused and not args.no_parity:
-            line["parity"] = bench_parity(w, inp, out, Sf)
+            par = bench_parity(w, inp, out, Sf)
+            if par is not None:
+                par["bar"] = 2e-2 if w.dtype == "bf16" else 1e-5
+                par["ok"] = parity_ok(par, par["bar"])
+                parity_failed = not par["ok"]
+            line["parity"] = par
         # (the backward's sample is taken over dense sequences only)
         if world == 1 and not args.no_cpu_baseline and not (args.backward and w.kind != "forward"):
             import oracle
@@ -726,6 +748,9 @@ def run_ours(args, w):
     if world > 1:
         import torch.distributed as dist
         dist.destroy_process_group()
+    if parity_failed:   # the line stands as printed; the run does not pass
+        print("bench: the sampled outputs fail the oracle check (parity.ok false)", file=sys.stderr)
+        sys.exit(3)
 
 
 def e2e_pieces(w, B, T):

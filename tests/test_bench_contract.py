@@ -170,3 +170,17 @@ def test_traffic_records_are_keyed_to_code_not_comments():
     assert code_only(a) != code_only(a.replace("x + 1", "x + 2"))
     assert code_only(a) != code_only(a.replace("a // b", "a // c"))
     assert code_only("char c = '/'; // x\n") == "char c = '/';"
+
+
+def test_parity_verdict_fails_on_nan_and_on_the_bars():
+    """The bench's own oracle check fails the run (after printing its line) when a
+    sampled comparison is not finite or over the bars the tests use."""
+    ok = _bench().parity_ok
+    good = {"o": {"rel_l2": 3e-3, "worst_head": 3e-3, "worst_row": 5e-3}}
+    assert ok(good, 2e-2) and ok(None, 2e-2) and ok({"sample": "x"}, 2e-2)
+    nan = float("nan")
+    assert not ok({"o": {"rel_l2": nan, "worst_head": nan, "worst_row": nan}}, 2e-2)
+    assert not ok({"o": {"rel_l2": 3e-2, "worst_head": 3e-3, "worst_row": 5e-3}}, 2e-2)
+    assert not ok({"o": {"rel_l2": 3e-3, "worst_head": 3e-3, "worst_row": 0.11}}, 2e-2)
+    assert ok({"o": {"rel_l2": 3e-3, "worst_head": 3e-3, "worst_row": 0.09}}, 2e-2)
+    assert not ok(dict(good, S_final={"rel_l2": 1e-4, "worst_head": 1e-4, "worst_row": nan}), 2e-2)
